@@ -1,0 +1,361 @@
+#!/usr/bin/env python
+"""Benchmark of the streaming int4 MoE stack on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Default workload ``decode_b1_l40``: one decode step = one token of one stream through all
+40 MoE layers (d=2048, 256 experts + 1 shared, I=512, top-4, int4 affine g64, LoRA r=16
+on the shared expert, 33 linear prerouter heads whose predictions are the next step's
+routing).  Weights and inputs are seeded synthetic draws (``synth``); the expert weights
+(18.1 GB) exceed L2, and each step reads ~406 MB of them.
+
+Prints one JSON line.  ``value`` is tokens/s with inputs resident in HBM; ``e2e`` is the
+same metric through the C ABI with the step's inputs copied from pinned host memory and
+its outputs copied back inside the timed region.  With N > 1 (torchrun) every rank runs
+an independent replica (the path has no exchange step) and ``value`` is the sum over
+ranks divided by the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (float64 numpy) on bounded samples of the same
+workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(PEAKS_FALLBACK, source="fallback")
+
+
+# ---------------------------------------------------------------------------------------
+# algorithmic bytes of one decode step (what the kernels must read at least once)
+# ---------------------------------------------------------------------------------------
+def step_bytes(dims, idx, B):
+    """idx [L, B, k] routing of the step.  Returns (expert bytes, all bytes)."""
+    blob = synth.blob_bytes(dims.d, dims.I)
+    d, E, I, r = dims.d, dims.E, dims.I, dims.r
+    expert = other = 0
+    heads = set(dims.head_layers)
+    for n in range(dims.L):
+        u = len(set(idx[n].reshape(-1).tolist()))
+        expert += (u + 1) * blob                            # routed uniques + shared expert
+        predicted = n > 0 and (n - 1) in heads
+        other += (B * dims.k * d * 2) if predicted else E * d * 2   # router rows
+        other += E * d * 2 if n in heads else 0                     # head
+        other += (2 * r * d + 2 * I * r + r * I + d * r) * 2        # LoRA
+        other += d * 2                                               # gamma
+        other += B * d * 2 * 2                                       # h in, y out (bf16)
+    return expert, expert + other
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                rows.append(p)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        for r in rows:
+            for name, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                               r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------------------
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle timing (baseline / reference arm)
+# ---------------------------------------------------------------------------------------
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_decode_sample(dims, seed, n_layers: int, step: int = 0):
+    """Time the oracle on one token of one stream through the first `n_layers` layers
+    (own-router routing, as at step 0).  Returns seconds."""
+    import oracle as O
+    hs = synth.hidden(seed, step, dims.L, 1, dims.d)
+    t0 = time.perf_counter()
+    for n in range(n_layers):
+        dense = synth.layer_dense(seed, n, dims)
+        out = O.moe_layer(hs[n], dense, lambda e, n=n: synth.expert_blob(seed, n, e, dims),
+                          synth.shared_blob(seed, n, dims), dims)
+        if n in dims.head_layers:
+            O.prerouter_head(out["x"][0], dense, dims)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(dims, seed, budget_s=20.0):
+    """The oracle as it stands on a bounded sample: whole layers of one token, as many as
+    fit the budget; tokens/s is extrapolated to the 40-layer stack."""
+    t1 = oracle_decode_sample(dims, seed, 1)
+    n = int(max(1, min(dims.L, budget_s / max(t1, 1e-3))))
+    t = oracle_decode_sample(dims, seed, n)
+    per_token = t * dims.L / n
+    return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"1 token (B=1) through {n} of {dims.L} layers, own-router routing; "
+                      f"time scaled x{dims.L / n:.2f} to the full stack (incl. weight generation per layer)"}
+
+
+def run_reference(args, dims, seed, ws, rank):
+    if rank != 0:
+        return
+    per_step_layers = None
+    times = []
+    for i in range(args.warmup + args.steps):
+        if per_step_layers is None:
+            t1 = oracle_decode_sample(dims, seed, 1)
+            # keep the whole run within ~3 minutes
+            per_step_layers = int(max(1, min(dims.L, 180.0 / max(1, args.warmup + args.steps) / max(t1, 1e-3))))
+        t = oracle_decode_sample(dims, seed, per_step_layers, step=i)
+        if i >= args.warmup:
+            times.append(t * dims.L / per_step_layers)
+    per_token = sum(times) / len(times)
+    v = 1.0 / per_token
+    sample = (f"each step: 1 token (B=1) through {per_step_layers} of {dims.L} layers, "
+              f"time scaled to the full stack")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_token * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "layers": dims.L, "batch": 1, "d": dims.d, "experts": dims.E},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+def run_decode(args, dims, seed, B, ws, rank, local):
+    import torch
+    import int4_expert_streaming_prerouter_b200 as e0
+    from synth.device import layer_tensors, bf16_tensor
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    t0 = time.time()
+    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, max(B, 1))
+    lys, hds = [], []
+    for n in range(dims.L):
+        ly, hd = layer_tensors(seed, n, dims, dev)
+        lys.append(ly)
+        hds.append(hd)
+    ctx.register_model(lys, hds)
+    setup_s = time.time() - t0
+    steps, warm = args.steps, args.warmup
+    total = steps + warm
+    # every step has its own generated inputs, resident before the timed region
+    h_all = torch.stack([bf16_tensor(synth.hidden(seed, t, dims.L, B, dims.d), dev) for t in range(total)])
+    y = torch.empty((dims.L, B, dims.d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for t in range(warm):
+        ctx.stack_decode(h_all[t], t, y_out=y)
+    ctx.sync_status()
+    launches0 = ctx.stats()["kernel_launches"]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    routes = []
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for t in range(warm, total):
+            ctx.stack_decode(h_all[t], t, y_out=y)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ctx.sync_status()
+    ms = ev0.elapsed_time(ev1)
+    launches = ctx.stats()["kernel_launches"] - launches0
+    idx, _ = ctx.get_routing(B)
+    exp_b, all_b = step_bytes(dims, idx, B)
+    ms_max = max_over_ranks(ms, ws)
+    tokens = sum_over_ranks(B * steps, ws)
+    value = tokens / (ms_max / 1e3)
+
+    # end-to-end through the C ABI with host buffers: inputs H2D and outputs D2H per step
+    h_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
+    h_host.copy_(h_all[warm:].cpu())
+    y_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
+    h_dev = torch.empty_like(h_all[0])
+    torch.cuda.synchronize()
+    nxt = total          # continue the same decode sequence
+    barrier(ws)
+    e0_, e1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0_.record(stream)
+    for t in range(steps):
+        h_dev.copy_(h_host[t], non_blocking=True)
+        ctx.stack_decode(h_dev, nxt + t, y_out=y)
+        y_host[t].copy_(y, non_blocking=True)
+    e1_.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_ms = max_over_ranks(e0_.elapsed_time(e1_), ws)
+    e2e_value = tokens / (e2e_ms / 1e3)
+
+    pk = peaks()
+    step_ms = ms / steps
+    achieved = exp_b / (step_ms / 1e3) / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": steps, "warmup": warm,
+        "ms_per_step": ms_max / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 weights, fp32 accumulate", "data": "synthetic (seeded; see DESIGN.md input recipe)",
+        "config": {"workload": args.workload, "layers": dims.L, "batch": B, "d": dims.d, "experts": dims.E,
+                   "d_ff": dims.I, "top_k": dims.k, "lora_rank": dims.r, "heads": len(dims.head_layers),
+                   "parallelism": f"replicas x{ws}", "l2": "inputs larger than L2 (18.1 GB of expert weights)"},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(h_dev.numel() * 2),
+                "d2h_bytes_per_step": int(y.numel() * 2)},
+        "gpu_launches": int(launches),
+        "hbm": {"expert_bytes_per_step": exp_b, "all_bytes_per_step": all_b,
+                "expert_GBps": achieved, "all_GBps": all_b / (step_ms / 1e3) / 1e9,
+                "frac_of_measured": achieved / pk["hbm_gbs"], "frac_of_8TBps": achieved / 8000.0},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "whole decode step (all kernels of one token), expert bytes only",
+                     "peak_source": pk["source"]},
+        "clocks": clk.summary(),
+        "setup_s": setup_s,
+    }
+    return out, ctx
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--workload", default="decode_b1_l40")
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = synth.WORKLOADS[args.workload]
+    dims, seed = wl["dims"], wl["seed"]
+    ws, rank, local = dist_init() if args.impl == "ours" else (int(os.environ.get("WORLD_SIZE", "1")),
+                                                                int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        run_reference(args, dims, seed, ws, rank)
+        return
+    B = args.batch or (wl["batch"] if isinstance(wl.get("batch"), int) else 8)
+    out, ctx = run_decode(args, dims, seed, B, ws, rank, local)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(dims, seed)
+        print(json.dumps(out), flush=True)
+    ctx.close()
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * e0moe.h -- C ABI of the B200 (sm_100a) streaming int4 MoE block with a prerouter.
+ *
+ * What the calls compute (sources are named by page title and section; no page prints
+ * code):
+ *   [G] "The Other Half of the Memory Wall: Serving 35B MoEs from SSD with Trained
+ *       Routing Prediction" (reading guide): "Temel fikirler", "Yöntem / Ön
+ *       Yönlendirici Başlık Mimarisi", "Yöntem / Birleştirilmemiş Adaptör Yürütme",
+ *       "Yöntem / Üç Aşamalı Eğitim", "Temel terimler", "Sorular".
+ *   [A] "Edge0 serve un MoE da 35B a 20 token al secondo in 3 GiB" (ai.info), section
+ *       "La versione da 35B usa 256 esperti distribuiti su 40 livelli".
+ *
+ * Conventions for every call:
+ *   - Every function returns an int status (E0_OK or a negative E0_ERR_*); the message
+ *     of the last failure on the calling host thread is e0_last_error().  Nothing here
+ *     aborts, traps or prints.
+ *   - The caller owns every device buffer and the pinned host expert store; pointers are
+ *     plain device (or pinned host) addresses and are only read during the enqueued work.
+ *     The library owns only the opaque e0_ctx (its workspaces, routing tables, slot table,
+ *     side stream and events), created by e0_create and released by e0_destroy.
+ *   - Work is enqueued on the caller's CUDA stream (passed as void*, a cudaStream_t) and
+ *     is asynchronous.  Errors found on the device (an expert index out of range, a
+ *     duplicated index, a slot-table tag that does not match the expert a kernel expects)
+ *     are latched in a device error word; e0_sync_status() synchronises and reports it.
+ *   - Layouts are row-major and contiguous.  bf16 is IEEE bfloat16.  One expert is one
+ *     contiguous blob (the int4 affine group-64 format of [G] "Temel fikirler" and [A]):
+ *         gate.codes [I, d/2] u8 | gate.scale [I, d/64] bf16 | gate.min [I, d/64] bf16 |
+ *         up.codes   [I, d/2]    | up.scale   [I, d/64]      | up.min   [I, d/64]      |
+ *         down.codes [d, I/2]    | down.scale [d, I/64]      | down.min [d, I/64]
+ *     code element 2i is the low nibble of byte i, w = scale * q + min, q = 0..15; groups
+ *     of 64 run along K (the input dimension).  1,769,472 bytes at d=2048, I=512.
+ *   - Supported sizes: d % 256 == 0 (d <= 4096), I % 128 == 0 (I <= 4096), 1 <= k <= 8,
+ *     k <= E <= 256, r <= 32, group == 64, head_hidden % 8 == 0, E % 4 == 0 when
+ *     head_onehot = 1.  Weight matrices, blobs and the host store are 16-byte aligned.
+ */
+#ifndef E0MOE_H
+#define E0MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  E0_OK = 0,
+  E0_ERR_INVALID_ARG = -1,   /* rejected before anything was enqueued */
+  E0_ERR_CUDA = -2,          /* a CUDA runtime call failed (message names it) */
+  E0_ERR_OOM = -3,           /* a workspace allocation failed */
+  E0_ERR_STAGING = -4,       /* an expert copy into the HBM pool could not be issued */
+  E0_ERR_SLOT_MISMATCH = -5, /* a kernel found a pool slot holding another expert */
+  E0_ERR_TIMEOUT = -6,       /* a bounded device-side wait gave up */
+  E0_ERR_DEVICE = -7         /* a kernel rejected its data (index out of range, duplicate) */
+};
+
+typedef struct e0_ctx e0_ctx;
+
+/* Model geometry.  head_hidden = 0 selects the linear head l(u); > 0 adds
+ * fc2(gelu_erf(fc1 u + b1)) + b2 ([G] "Ön Yönlendirici Başlık Mimarisi").
+ * head_onehot = 1 makes the head input u = [x; onehot_k(cur); onehot_k(prev)] (width
+ * d + 2E); 0 makes u = x.  lora_scale is alpha / r of [G] "Birleştirilmemiş Adaptör
+ * Yürütme".  rms_eps is the RMSNorm epsilon. */
+typedef struct {
+  int d_model, n_experts, d_ff, top_k, group, lora_rank, head_hidden, head_onehot;
+  float rms_eps, lora_scale;
+} e0_dims;
+
+/* One layer's weights (device pointers, all owned by the caller).
+ * experts  [E][blob]  routed experts; may be NULL for a layer served only from the
+ *                     streaming pool (e0_stream_register).
+ * shared   [blob]     the always-on shared expert ([A]).
+ * lora_*   bf16: Ag, Au [r, d]; Bg, Bu [I, r]; Ad [r, I]; Bd [d, r]  (NULL: no LoRA).  The
+ *          delta is unmerged: g += c Bg (Ag x), u += c Bu (Au x), y_s += c Bd (Ad a_s)
+ *          ([G] "Birleştirilmemiş Adaptör Yürütme"; on the shared expert only, as
+ *          "Üç Aşamalı Eğitim" places it).
+ * router_w bf16 [E, d];  norm_w bf16 [d] (RMSNorm gamma). */
+typedef struct {
+  const void *experts;
+  const void *shared;
+  const void *lora_Ag, *lora_Bg, *lora_Au, *lora_Bu, *lora_Ad, *lora_Bd;
+  const void *router_w;
+  const void *norm_w;
+} e0_layer;
+
+/* One layer's prerouter head (device pointers; w_lin NULL = the layer has no head).
+ * w_lin bf16 [E, d (+2E)]; fc1_w bf16 [H, d (+2E)], fc1_b [H], fc2_w [E, H], fc2_b [E]
+ * (fc* only when head_hidden > 0). */
+typedef struct {
+  const void *w_lin, *fc1_w, *fc1_b, *fc2_w, *fc2_b;
+} e0_head;
+
+/* Counters of the streaming tier and the decode loop (host-side accounting). */
+typedef struct {
+  uint64_t steps;              /* e0_moe_stack_decode calls */
+  uint64_t staged_experts;     /* expert blobs copied into the pool */
+  uint64_t staged_bytes;       /* host-link bytes issued by the staging copies */
+  uint64_t prefetched_experts; /* of which issued from a prediction (one token ahead) */
+  uint64_t ondemand_experts;   /* of which issued after the layer's own router ran */
+  uint64_t dropped;            /* routed experts that were not staged (always 0) */
+  double   stage_ms;           /* sum of copy durations (side-stream event pairs) */
+  double   exposed_wait_ms;    /* compute-stream time spent waiting on staging */
+  uint64_t kernel_launches;    /* kernels this context has launched */
+} e0_stats;
+
+/* Create a context on the current CUDA device.  n_layers >= 1; max_tokens bounds T of
+ * every call (and B of decode).  Allocates the workspaces.  Errors: INVALID_ARG (sizes
+ * outside the supported set), OOM, CUDA. */
+int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_ctx **out);
+
+/* Release the context and everything it allocated (synchronises its streams). */
+int e0_destroy(e0_ctx *ctx);
+
+/* Record the weights of all layers.  layers[n_layers]; heads[n_layers] or NULL (no
+ * heads).  Only the pointers are stored; the buffers must stay valid while the context
+ * uses them.  Heads on layer N predict layer N+1 ([G] "Ön Yönlendirici Başlık
+ * Mimarisi"; 33 heads on 40 layers per [A]). */
+int e0_register_model(e0_ctx *ctx, const e0_layer *layers, const e0_head *heads);
+
+/* One MoE block on T tokens of `layer` ([G] "Temel fikirler"; [A]):
+ *   x = bf16(RMSNorm(h)), logits = W_r x (fp32), S = top-k(logits) (descending, ties to
+ *   the lower index) or route_idx, w = softmax(logits[S]) over the selection,
+ *   y = sum_j w_j E_{S_j}(x) + E_shared(x) with the shared expert's unmerged LoRA.
+ * h        [T, d] bf16 device.
+ * route_idx NULL, or [T, k] int32 device: the routing to use ("prediction as routing");
+ *          a row whose first entry is -1 uses the layer's own router.
+ * y_bf16   [T, d] bf16 device (required);  y_f32 [T, d] fp32 or NULL.
+ * idx_out  [T, k] int32 or NULL;  gate_out [T, k] fp32 or NULL.
+ * Errors: INVALID_ARG (layer, T, NULL h/y), DEVICE (latched: route index out of range or
+ * duplicated within a token). */
+int e0_moe_layer_forward(e0_ctx *ctx, int layer, const void *h, int T, const int32_t *route_idx,
+                         void *y_bf16, float *y_f32, int32_t *idx_out, float *gate_out,
+                         void *stream);
+
+/* The prerouter head of `layer` on normed inputs ([G] "Ön Yönlendirici Başlık
+ * Mimarisi"): z = l(u) (+ fc2(gelu_erf(fc1 u + b1)) + b2), u = [x; onehot(cur);
+ * onehot(prev)]; pred = top-k(z) is layer+1's routing at the next token.
+ * x [T, d] bf16 device; cur_idx, prev_idx [T, k] int32 device or NULL (zero one-hot);
+ * pred_idx [T, k] int32 device (required); logits_out [T, E] fp32 or NULL.
+ * Errors: INVALID_ARG (no head on `layer`, sizes). */
+int e0_prerouter_predict(e0_ctx *ctx, int layer, const void *x, int T, const int32_t *cur_idx,
+                         const int32_t *prev_idx, int32_t *pred_idx, float *logits_out,
+                         void *stream);
+
+/* Streaming tier ([G] "Temel fikirler": weights stay off the GPU, only the working set
+ * is resident; "Temel terimler": staged decode with a fixed-slot double buffer and a
+ * GPU slot table).  host_blob: pinned host memory [L][E][expert_bytes] (caller-owned,
+ * must stay valid).  Allocates the HBM pool of pool_layers x slots_per_layer blobs
+ * (pool_layers >= 2, slots_per_layer >= k * max_tokens is not required: slots_per_layer
+ * must be >= the number of distinct experts a layer routes to in one step).
+ * Errors: INVALID_ARG, OOM. */
+int e0_stream_register(e0_ctx *ctx, const void *host_blob, size_t expert_bytes, int pool_layers,
+                       int slots_per_layer);
+
+/* Stage the experts host_idx[0..n) of `layer` into the layer's pool slot set: waits (on
+ * the side stream) until the previous user of that slot set has finished on
+ * compute_stream, issues one cudaMemcpyAsync per expert blob, writes the slot table and
+ * records the "ready" event that the consuming layer waits on.  host_idx is host memory.
+ * Errors: INVALID_ARG, STAGING (a copy could not be issued). */
+int e0_stage_experts(e0_ctx *ctx, int layer, const int32_t *host_idx, int n, void *compute_stream);
+
+/* One decode step of B streams through all layers.
+ * h_in [L, B, d] bf16 device (each layer's generated MoE input); y_out [L, B, d] bf16;
+ * y_f32 [L, B, d] fp32 or NULL.  Routing of layer N at step t: the head prediction of
+ * layer N-1 made at step t-1 when layer N-1 has a head and t > 0, else the layer's own
+ * router ([G] "Temel fikirler", "Sorular").  Every head runs and writes step t+1's
+ * routing into the context.  step == 0 starts a new sequence.  streaming = 1 serves the
+ * routed experts from the pool (e0_stream_register), 0 from the resident weights.
+ * chained = 1 feeds bf16(h_N + y_{N-1}) to layer N (a dependency check); 0 feeds h_N.
+ * Errors: INVALID_ARG, STAGING, CUDA; DEVICE/SLOT_MISMATCH are latched. */
+int e0_moe_stack_decode(e0_ctx *ctx, const void *h_in, int B, int step, void *y_out, float *y_f32,
+                        int streaming, int chained, void *stream);
+
+/* Routing the last e0_moe_stack_decode used and predicted, copied to host memory:
+ * idx [L, B, k] (routing used at that step), pred [L, B, k] (next step's routing; -1 for
+ * layers without a head).  Synchronises the context's last stream. */
+int e0_get_routing(e0_ctx *ctx, int B, int32_t *idx_host, int32_t *pred_host);
+
+int e0_get_stats(e0_ctx *ctx, e0_stats *out);
+
+/* Synchronise the last stream used and return E0_OK or the latched device error
+ * (DEVICE, SLOT_MISMATCH, TIMEOUT); the error word is cleared. */
+int e0_sync_status(e0_ctx *ctx);
+
+/* Host-side fault injection for tests (no GPU fault is involved):
+ * e0_debug_fail_staging_after(ctx, n): the (n+1)-th next staging copy is refused, so the
+ *   staging call returns E0_ERR_STAGING.
+ * e0_debug_set_slot_tag(ctx, set, slot, expert): the next slot-table write of pool set
+ *   `set` tags `slot` with `expert`; the expert kernels must then latch SLOT_MISMATCH. */
+int e0_debug_fail_staging_after(e0_ctx *ctx, int n);
+int e0_debug_set_slot_tag(e0_ctx *ctx, int pool_set, int slot, int expert);
+
+/* Message of the last failing call on this host thread ("" if none). */
+const char *e0_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* E0MOE_H */

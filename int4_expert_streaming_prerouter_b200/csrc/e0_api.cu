@@ -1,0 +1,709 @@
+// C ABI of libe0moe.so: context, weight registration, argument checks, launches of the
+// MoE-block kernels, the decode loop with prediction-as-routing, and the streaming tier
+// (pinned host store -> HBM slot pool on a side stream).  Declarations and the meaning
+// of every argument are in include/e0moe.h.
+#include "e0moe.h"
+#include "e0_kernels.cuh"
+#include "e0_decode.cuh"
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+using namespace e0;
+
+static thread_local std::string g_err;
+
+static int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define CK(call)                                                                         \
+  do {                                                                                   \
+    cudaError_t e_ = (call);                                                             \
+    if (e_ != cudaSuccess) return fail(E0_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define CKL(what)                                                                        \
+  do {                                                                                   \
+    C->stats.kernel_launches++;                                                          \
+    cudaError_t e_ = cudaGetLastError();                                                 \
+    if (e_ != cudaSuccess) return fail(E0_ERR_CUDA, "launch %s: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+
+// ---------------------------------------------------------------------------------------
+// Context
+// ---------------------------------------------------------------------------------------
+struct StreamPool {
+  uint8_t *mem = nullptr;            // [pool_layers][slots][blob]
+  int nsets = 0, slots = 0;
+  size_t bytes = 0;
+  const uint8_t *host = nullptr;     // pinned [L][E][blob]
+  int32_t *slot_of = nullptr;        // [nsets][E]
+  int32_t *slot_tag = nullptr;       // [nsets][slots]
+  cudaStream_t side = nullptr;
+  std::vector<cudaEvent_t> ready, freed;   // per pool set
+  // event quadruples (copy start/end on the side stream, wait start/end on the compute
+  // stream), one per staging round, reused round-robin and accounted on reuse
+  struct Rec { cudaEvent_t c0, c1, w0, w1; int state; };
+  std::vector<Rec> ring;
+  int ring_pos = 0;
+  std::vector<int> set_rec;                // per pool set: ring entry of its current round
+  int fail_after = -1;                     // host-side fault injection for tests
+  int corrupt_set = -1, corrupt_slot = 0, corrupt_tag = 0;  // one-shot wrong slot tag
+};
+
+struct e0_ctx {
+  e0_dims dims{};
+  int L = 0, maxT = 0, dev = 0, nsm = 0;
+  Blob bl{};
+  std::vector<e0_layer> layers;
+  std::vector<e0_head> heads;
+  bool registered = false;
+  // workspaces (device)
+  uint16_t *xb = nullptr;
+  float *xf = nullptr, *logits = nullptr, *hlog = nullptr, *lt = nullptr, *gates = nullptr;
+  int32_t *idx = nullptr;
+  uint16_t *a = nullptr;
+  int32_t *plan_mem = nullptr;
+  Plan plan{};
+  float *yscratch = nullptr;         // [2][maxT][d] fp32 outputs for chained decode
+  float *h1pre = nullptr, *h1 = nullptr;  // [maxT][H] full-head hidden layer
+  int32_t *pred_tab = nullptr;       // [2][L+1][maxT][k]  routing predicted for layer l
+  int32_t *hist_tab = nullptr;       // [2][L][maxT][k]    routing used by layer l
+  int *err = nullptr;
+  int32_t *host_idx = nullptr;       // pinned scratch for routing read-backs
+  cudaStream_t last = nullptr;
+  int last_step = -1, last_B = 0;
+  DecodeState dec{};
+  StreamPool pool;
+  e0_stats stats{};
+};
+
+extern "C" const char *e0_last_error(void) { return g_err.c_str(); }
+
+static bool supported(const e0_dims &D) {
+  return D.d_model > 0 && D.d_model % 256 == 0 && D.d_model <= 4096 && D.d_ff > 0 &&
+         D.d_ff % 128 == 0 && D.d_ff <= 4096 && D.top_k >= 1 && D.top_k <= kMaxK &&
+         D.n_experts >= D.top_k && D.n_experts <= kMaxE && D.group == 64 && D.lora_rank >= 0 &&
+         D.lora_rank <= kMaxR && D.head_hidden >= 0 && D.head_hidden % 8 == 0 && D.head_hidden <= 16384 &&
+         (D.head_onehot == 0 || (D.head_onehot == 1 && D.n_experts % 4 == 0));
+}
+
+template <typename T>
+static int dalloc(T **p, size_t n) {
+  if (cudaMalloc((void **)p, n * sizeof(T) + 16) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(E0_ERR_OOM, "cudaMalloc of %zu bytes failed", n * sizeof(T));
+  }
+  return E0_OK;
+}
+
+extern "C" int e0_destroy(e0_ctx *C) {
+  if (!C) return E0_OK;
+  cudaDeviceSynchronize();
+  void *bufs[] = {C->xb, C->xf, C->logits, C->hlog, C->lt, C->gates, C->idx, C->a, C->plan_mem,
+                  C->yscratch, C->pred_tab, C->hist_tab, C->err, C->h1pre, C->h1, C->pool.mem, C->pool.slot_of,
+                  C->pool.slot_tag};
+  for (void *b : bufs)
+    if (b) cudaFree(b);
+  decode_free(C->dec);
+  if (C->host_idx) cudaFreeHost(C->host_idx);
+  for (auto *v : {&C->pool.ready, &C->pool.freed})
+    for (auto e : *v) cudaEventDestroy(e);
+  for (auto &r : C->pool.ring)
+    for (auto e : {r.c0, r.c1, r.w0, r.w1}) cudaEventDestroy(e);
+  if (C->pool.side) cudaStreamDestroy(C->pool.side);
+  delete C;
+  return E0_OK;
+}
+
+extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_ctx **out) {
+  if (!dims || !out || n_layers < 1 || max_tokens < 1 || max_tokens > (1 << 16))
+    return fail(E0_ERR_INVALID_ARG, "e0_create: bad arguments");
+  if (!supported(*dims))
+    return fail(E0_ERR_INVALID_ARG,
+                "e0_create: unsupported dims (need d%%256==0, I%%128==0, k<=8, k<=E<=256, r<=32, group 64)");
+  *out = nullptr;
+  e0_ctx *C = new e0_ctx();
+  C->dims = *dims;
+  C->L = n_layers;
+  C->maxT = max_tokens;
+  cudaGetDevice(&C->dev);
+  cudaDeviceGetAttribute(&C->nsm, cudaDevAttrMultiProcessorCount, C->dev);
+  C->bl = blob_of(dims->d_model, dims->d_ff);
+  const size_t T = max_tokens, d = dims->d_model, E = dims->n_experts, I = dims->d_ff,
+               k = dims->top_k, r = dims->lora_rank > 0 ? dims->lora_rank : 1;
+  int rc = E0_OK;
+  if ((rc = dalloc(&C->xb, T * d)) || (rc = dalloc(&C->xf, T * d)) || (rc = dalloc(&C->logits, T * E)) ||
+      (rc = dalloc(&C->hlog, T * E)) || (rc = dalloc(&C->lt, T * 3 * r)) || (rc = dalloc(&C->gates, T * k)) ||
+      (rc = dalloc(&C->idx, T * k)) || (rc = dalloc(&C->a, T * (k + 1) * I)) ||
+      (rc = dalloc(&C->plan_mem, 1 + E + E + 1 + T * k)) || (rc = dalloc(&C->yscratch, 2 * T * d)) ||
+      (rc = dalloc(&C->pred_tab, 2 * (n_layers + 1) * T * k)) ||
+      (rc = dalloc(&C->hist_tab, 2 * n_layers * T * k)) || (rc = dalloc(&C->err, 4)) ||
+      (dims->head_hidden > 0 && ((rc = dalloc(&C->h1pre, T * dims->head_hidden)) ||
+                                 (rc = dalloc(&C->h1, T * dims->head_hidden))))) {
+    e0_destroy(C);
+    return rc;
+  }
+  C->plan.U = C->plan_mem;
+  C->plan.uexp = C->plan_mem + 1;
+  C->plan.ustart = C->plan_mem + 1 + E;
+  C->plan.assign = C->plan_mem + 2 + 2 * E;
+  cudaMemset(C->pred_tab, 0xFF, 2 * (n_layers + 1) * T * k * sizeof(int32_t));
+  cudaMemset(C->hist_tab, 0xFF, 2 * n_layers * T * k * sizeof(int32_t));
+  cudaMemset(C->err, 0, 16);
+  if (cudaMallocHost((void **)&C->host_idx, (n_layers + 2) * T * k * sizeof(int32_t)) != cudaSuccess) {
+    e0_destroy(C);
+    return fail(E0_ERR_OOM, "pinned scratch allocation failed");
+  }
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    e0_destroy(C);
+    return fail(E0_ERR_CUDA, "e0_create: %s", cudaGetErrorString(e));
+  }
+  *out = C;
+  return E0_OK;
+}
+
+extern "C" int e0_register_model(e0_ctx *C, const e0_layer *layers, const e0_head *heads) {
+  if (!C || !layers) return fail(E0_ERR_INVALID_ARG, "e0_register_model: NULL argument");
+  for (int l = 0; l < C->L; l++) {
+    const e0_layer &Y = layers[l];
+    if (!Y.shared || !Y.router_w || !Y.norm_w)
+      return fail(E0_ERR_INVALID_ARG, "layer %d: shared, router_w and norm_w are required", l);
+    const bool any = Y.lora_Ag || Y.lora_Bg || Y.lora_Au || Y.lora_Bu || Y.lora_Ad || Y.lora_Bd;
+    const bool all = Y.lora_Ag && Y.lora_Bg && Y.lora_Au && Y.lora_Bu && Y.lora_Ad && Y.lora_Bd;
+    if (any && (!all || C->dims.lora_rank < 1))
+      return fail(E0_ERR_INVALID_ARG, "layer %d: LoRA needs all six matrices and lora_rank >= 1", l);
+    if (((uintptr_t)Y.shared | (uintptr_t)Y.experts | (uintptr_t)Y.router_w | (uintptr_t)Y.lora_Ag |
+         (uintptr_t)Y.lora_Au) & 15)
+      return fail(E0_ERR_INVALID_ARG, "layer %d: weight pointers must be 16-byte aligned", l);
+    if (heads && heads[l].w_lin) {
+      if (C->dims.head_hidden > 0 && !(heads[l].fc1_w && heads[l].fc1_b && heads[l].fc2_w && heads[l].fc2_b))
+        return fail(E0_ERR_INVALID_ARG, "layer %d: head_hidden > 0 needs fc1/fc2 weights", l);
+      if (((uintptr_t)heads[l].w_lin | (uintptr_t)heads[l].fc1_w | (uintptr_t)heads[l].fc2_w) & 15)
+        return fail(E0_ERR_INVALID_ARG, "layer %d: head weights must be 16-byte aligned", l);
+    }
+  }
+  C->layers.assign(layers, layers + C->L);
+  C->heads.assign(C->L, e0_head{});
+  if (heads) C->heads.assign(heads, heads + C->L);
+  C->registered = true;
+  C->dec.valid = false;
+  return E0_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// One layer, split in two halves so that the streaming tier can stage experts between
+// the routing decision and the expert kernels.
+// ---------------------------------------------------------------------------------------
+struct LayerCall {
+  int l, T;
+  const uint16_t *h;
+  const float *chain;
+  const int32_t *route;
+  int full_mode;
+  int32_t *idx;            // [T,k] routing (written by k_route)
+  float *gates;
+  int32_t *hist;           // copy of idx for the next step's one-hot, or nullptr
+  bool head;
+  const int32_t *prev;     // [T,k] or nullptr
+  int32_t *pred;           // [T,k]
+  uint16_t *y;
+  float *yf;
+};
+
+static inline int grid_for(int warps_needed, int cap) {
+  int b = (warps_needed + 7) / 8;
+  return b < 1 ? 1 : (b > cap ? cap : b);
+}
+
+static int layer_pre(e0_ctx *C, const LayerCall &K, cudaStream_t s) {
+  const e0_dims &D = C->dims;
+  const e0_layer &Y = C->layers[K.l];
+  const e0_head &H = C->heads[K.l];
+  k_norm<<<K.T, 256, 0, s>>>(K.h, K.chain, (const uint16_t *)Y.norm_w, D.d_model, D.rms_eps, C->xb, C->xf);
+  CKL("k_norm");
+  RowsArgs R{};
+  R.xf = C->xf; R.T = K.T; R.d = D.d_model; R.E = D.n_experts; R.k = D.top_k;
+  R.Wr = (const uint16_t *)Y.router_w; R.logits = C->logits; R.route = K.route; R.full_mode = K.full_mode;
+  R.Wh = (K.head && H.w_lin) ? (const uint16_t *)H.w_lin : nullptr;
+  R.ldh = D.d_model + (D.head_onehot ? 2 * D.n_experts : 0);
+  R.hlog = C->hlog;
+  R.Ag = (const uint16_t *)Y.lora_Ag; R.Au = (const uint16_t *)Y.lora_Au; R.r = D.lora_rank; R.lt = C->lt;
+  R.err = C->err;
+  const int nTT = (K.T + kRowTile - 1) / kRowTile;
+  const int J = D.n_experts * nTT + K.T * D.top_k + (R.Wh ? D.n_experts * nTT : 0) + (R.Ag ? 2 * D.lora_rank * nTT : 0);
+  k_rows<<<grid_for(J, 8 * C->nsm), 256, 0, s>>>(R);
+  CKL("k_rows");
+  RouteArgs A{};
+  A.logits = C->logits; A.T = K.T; A.E = D.n_experts; A.k = D.top_k; A.route = K.route; A.full_mode = K.full_mode;
+  A.idx = K.idx; A.gates = K.gates; A.hist = K.hist;
+  A.hlog = R.Wh ? C->hlog : nullptr; A.Wh = R.Wh; A.ldh = R.ldh; A.d = D.d_model; A.onehot = D.head_onehot;
+  A.prev = K.prev; A.pred = K.pred; A.err = C->err;
+  k_route<<<(K.T + 7) / 8, 256, 0, s>>>(A);
+  CKL("k_route");
+  return E0_OK;
+}
+
+static int layer_post(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cudaStream_t s) {
+  const e0_dims &D = C->dims;
+  const e0_layer &Y = C->layers[K.l];
+  k_plan<<<1, 1024, 0, s>>>(K.idx, K.T * D.top_k, D.n_experts, C->plan);
+  CKL("k_plan");
+  GateUpArgs G{};
+  G.xf = C->xf; G.T = K.T; G.d = D.d_model; G.I = D.d_ff; G.k = D.top_k; G.r = D.lora_rank; G.c = D.lora_scale;
+  G.src = src; G.shared = (const uint8_t *)Y.shared; G.bl = C->bl; G.P = C->plan;
+  G.Bg = (const uint16_t *)Y.lora_Bg; G.Bu = (const uint16_t *)Y.lora_Bu; G.lt = C->lt; G.a = C->a;
+  const int items = (std::min(D.n_experts, K.T * D.top_k) + 1) * D.d_ff;
+  k_gateup<<<grid_for(items, 4 * C->nsm), 256, 0, s>>>(G);
+  CKL("k_gateup");
+  if (Y.lora_Ad) {
+    k_lora_t<<<(K.T * D.lora_rank + 7) / 8, 256, 0, s>>>((const uint16_t *)Y.lora_Ad, C->a, K.T, D.d_ff,
+                                                          D.top_k, D.lora_rank, C->lt);
+    CKL("k_lora_t");
+  }
+  DownArgs W{};
+  W.T = K.T; W.d = D.d_model; W.I = D.d_ff; W.k = D.top_k; W.r = D.lora_rank; W.c = D.lora_scale;
+  W.src = src; W.shared = (const uint8_t *)Y.shared; W.bl = C->bl; W.idx = K.idx; W.gates = K.gates; W.a = C->a;
+  W.Bd = (const uint16_t *)Y.lora_Bd; W.lt = C->lt; W.y = K.y; W.yf = K.yf;
+  k_down<<<grid_for(K.T * D.d_model, 4 * C->nsm), 256, 0, s>>>(W);
+  CKL("k_down");
+  return E0_OK;
+}
+
+static ExpertSrc resident_src(e0_ctx *C, int l) {
+  ExpertSrc s{};
+  s.resident = (const uint8_t *)C->layers[l].experts;
+  s.stride = C->bl.bytes;
+  s.err = C->err;
+  return s;
+}
+
+static ExpertSrc pool_src(e0_ctx *C, int l) {
+  ExpertSrc s{};
+  const int p = l % C->pool.nsets;
+  s.pool = C->pool.mem + (size_t)p * C->pool.slots * C->bl.bytes;
+  s.stride = C->bl.bytes;
+  s.slot_of = C->pool.slot_of + (size_t)p * C->dims.n_experts;
+  s.slot_tag = C->pool.slot_tag + (size_t)p * C->pool.slots;
+  s.err = C->err;
+  return s;
+}
+
+extern "C" int e0_moe_layer_forward(e0_ctx *C, int layer, const void *h, int T, const int32_t *route_idx,
+                                    void *y_bf16, float *y_f32, int32_t *idx_out, float *gate_out,
+                                    void *stream) {
+  if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
+  if (layer < 0 || layer >= C->L || T < 1 || T > C->maxT || !h || !y_bf16)
+    return fail(E0_ERR_INVALID_ARG, "e0_moe_layer_forward: bad layer/T/pointers (T=%d, max %d)", T, C->maxT);
+  if (!C->layers[layer].experts)
+    return fail(E0_ERR_INVALID_ARG, "layer %d has no resident experts", layer);
+  cudaStream_t s = (cudaStream_t)stream;
+  C->last = s;
+  LayerCall K{};
+  K.l = layer; K.T = T; K.h = (const uint16_t *)h; K.route = route_idx;
+  K.full_mode = route_idx ? 2 : 1;
+  K.idx = idx_out ? idx_out : C->idx;
+  K.gates = gate_out ? gate_out : C->gates;
+  K.y = (uint16_t *)y_bf16; K.yf = y_f32;
+  int rc = layer_pre(C, K, s);
+  if (rc) return rc;
+  return layer_post(C, K, resident_src(C, layer), s);
+}
+
+// The prerouter head of `layer` on C->xf ([G] "Ön Yönlendirici Başlık Mimarisi"):
+// z = l(u) (+ fc2(gelu_erf(fc1 u + b1)) + b2), pred = top-k(z).
+static int run_head(e0_ctx *C, int layer, int T, const int32_t *cur, const int32_t *prev, int32_t *pred,
+                    float *logits_out, cudaStream_t s) {
+  const e0_dims &D = C->dims;
+  const e0_head &H = C->heads[layer];
+  const int in = D.d_model + (D.head_onehot ? 2 * D.n_experts : 0);
+  if (D.head_hidden > 0) {
+    MatRowsArgs M{};
+    M.W = (const uint16_t *)H.fc1_w; M.ldw = in; M.rows = D.head_hidden; M.K = D.d_model;
+    M.X = C->xf; M.ldx = D.d_model; M.T = T; M.out = C->h1pre; M.ldo = D.head_hidden;
+    k_mat_rows<<<grid_for(D.head_hidden * ((T + kRowTile - 1) / kRowTile), 8 * C->nsm), 256, 0, s>>>(M);
+    CKL("k_mat_rows(fc1)");
+    const int n = T * D.head_hidden;
+    k_head_hidden<<<(n + 255) / 256, 256, 0, s>>>(C->h1pre, (const uint16_t *)H.fc1_w, (const uint16_t *)H.fc1_b, T,
+                                                  D.head_hidden, in, D.d_model, D.n_experts, D.top_k,
+                                                  D.head_onehot, cur, prev, C->h1);
+    CKL("k_head_hidden");
+    MatRowsArgs F{};
+    F.W = (const uint16_t *)H.fc2_w; F.ldw = D.head_hidden; F.rows = D.n_experts; F.K = D.head_hidden;
+    F.X = C->h1; F.ldx = D.head_hidden; F.T = T; F.bias = (const uint16_t *)H.fc2_b; F.out = C->hlog;
+    F.ldo = D.n_experts;
+    k_mat_rows<<<grid_for(D.n_experts * ((T + kRowTile - 1) / kRowTile), 8 * C->nsm), 256, 0, s>>>(F);
+    CKL("k_mat_rows(fc2)");
+  }
+  RowsArgs R{};
+  R.xf = C->xf; R.T = T; R.d = D.d_model; R.E = D.n_experts; R.k = D.top_k;
+  R.Wr = nullptr; R.Wh = (const uint16_t *)H.w_lin; R.ldh = in;
+  R.hlog = C->hlog; R.hacc = D.head_hidden > 0; R.err = C->err;
+  k_rows<<<grid_for(D.n_experts * ((T + kRowTile - 1) / kRowTile), 8 * C->nsm), 256, 0, s>>>(R);
+  CKL("k_rows(head)");
+  RouteArgs A{};
+  A.logits = nullptr; A.T = T; A.E = D.n_experts; A.k = D.top_k;
+  A.hlog = C->hlog; A.Wh = R.Wh; A.ldh = in; A.d = D.d_model; A.onehot = D.head_onehot;
+  A.prev = prev; A.cur = cur; A.pred = pred; A.hz_out = logits_out; A.err = C->err;
+  k_route<<<(T + 7) / 8, 256, 0, s>>>(A);
+  CKL("k_route(head)");
+  return E0_OK;
+}
+
+__global__ void k_bf16_to_f32(const uint16_t *__restrict__ x, float *__restrict__ y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = bf(x[i]);
+}
+
+extern "C" int e0_prerouter_predict(e0_ctx *C, int layer, const void *x, int T, const int32_t *cur_idx,
+                                    const int32_t *prev_idx, int32_t *pred_idx, float *logits_out,
+                                    void *stream) {
+  if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
+  if (layer < 0 || layer >= C->L || T < 1 || T > C->maxT || !x || !pred_idx)
+    return fail(E0_ERR_INVALID_ARG, "e0_prerouter_predict: bad layer/T/pointers");
+  const e0_head &H = C->heads[layer];
+  if (!H.w_lin) return fail(E0_ERR_INVALID_ARG, "layer %d has no prerouter head", layer);
+  const e0_dims &D = C->dims;
+  cudaStream_t s = (cudaStream_t)stream;
+  C->last = s;
+  const int n = T * D.d_model;
+  k_bf16_to_f32<<<(n + 255) / 256, 256, 0, s>>>((const uint16_t *)x, C->xf, n);
+  CKL("k_bf16_to_f32");
+  return run_head(C, layer, T, cur_idx, prev_idx, pred_idx, logits_out, s);
+}
+
+// ---------------------------------------------------------------------------------------
+// Streaming tier
+// ---------------------------------------------------------------------------------------
+extern "C" int e0_stream_register(e0_ctx *C, const void *host_blob, size_t expert_bytes, int pool_layers,
+                                  int slots_per_layer) {
+  if (!C || !host_blob) return fail(E0_ERR_INVALID_ARG, "e0_stream_register: NULL argument");
+  if (expert_bytes != (size_t)C->bl.bytes)
+    return fail(E0_ERR_INVALID_ARG, "expert_bytes %zu != blob size %lld", expert_bytes, C->bl.bytes);
+  if (pool_layers < 2 || slots_per_layer < C->dims.top_k || slots_per_layer > C->dims.n_experts)
+    return fail(E0_ERR_INVALID_ARG, "pool needs >= 2 layer sets and k <= slots <= E");
+  if ((uintptr_t)host_blob & 15) return fail(E0_ERR_INVALID_ARG, "host store must be 16-byte aligned");
+  StreamPool &P = C->pool;
+  if (P.mem) return fail(E0_ERR_INVALID_ARG, "a host store is already registered");
+  int rc;
+  if ((rc = dalloc(&P.mem, (size_t)pool_layers * slots_per_layer * expert_bytes)) ||
+      (rc = dalloc(&P.slot_of, (size_t)pool_layers * C->dims.n_experts)) ||
+      (rc = dalloc(&P.slot_tag, (size_t)pool_layers * slots_per_layer)))
+    return rc;
+  CK(cudaMemset(P.slot_of, 0xFF, (size_t)pool_layers * C->dims.n_experts * 4));
+  CK(cudaMemset(P.slot_tag, 0xFF, (size_t)pool_layers * slots_per_layer * 4));
+  P.nsets = pool_layers;
+  P.slots = slots_per_layer;
+  P.bytes = expert_bytes;
+  P.host = (const uint8_t *)host_blob;
+  CK(cudaStreamCreateWithFlags(&P.side, cudaStreamNonBlocking));
+  for (auto *v : {&P.ready, &P.freed}) {
+    v->resize(pool_layers);
+    for (auto &e : *v) CK(cudaEventCreate(&e));
+  }
+  P.ring.resize(4 * (size_t)C->L + 8);
+  for (auto &r : P.ring) {
+    for (auto *e : {&r.c0, &r.c1, &r.w0, &r.w1}) CK(cudaEventCreate(e));
+    r.state = 0;
+  }
+  P.set_rec.assign(pool_layers, -1);
+  CK(cudaDeviceSynchronize());
+  return E0_OK;
+}
+
+// Write a slot set's table: slot s holds expert L.e[s]; slot_of maps expert -> slot.
+// (bad_slot, bad_tag) is a host-armed corruption used by the fault tests (-1: none).
+__global__ void k_set_slots(int32_t *slot_of, int32_t *slot_tag, int E, int slots, SlotList L, int bad_slot,
+                            int bad_tag) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) slot_of[e] = -1;
+  __syncthreads();
+  for (int s = threadIdx.x; s < slots; s += blockDim.x) {
+    const int e = s < L.n ? L.e[s] : -1;
+    slot_tag[s] = (s == bad_slot) ? bad_tag : e;
+    if (e >= 0) slot_of[e] = s;
+  }
+}
+
+// Add one staging round's copy time and compute-stream wait time to the stats.
+static void account_rec(e0_ctx *C, StreamPool::Rec &r) {
+  if (!r.state) return;
+  float ms = 0.f;
+  cudaEventSynchronize(r.c1);
+  if (cudaEventElapsedTime(&ms, r.c0, r.c1) == cudaSuccess) C->stats.stage_ms += ms;
+  if (r.state == 2) {
+    cudaEventSynchronize(r.w1);
+    if (cudaEventElapsedTime(&ms, r.w0, r.w1) == cudaSuccess) C->stats.exposed_wait_ms += ms;
+  }
+  cudaGetLastError();
+  r.state = 0;
+}
+
+static int stage_impl(e0_ctx *C, int layer, const int32_t *host_idx, int n, cudaStream_t compute,
+                      bool prefetch) {
+  StreamPool &P = C->pool;
+  if (!P.mem) return fail(E0_ERR_INVALID_ARG, "no host store registered");
+  if (layer < 0 || layer >= C->L || n < 1 || !host_idx) return fail(E0_ERR_INVALID_ARG, "stage: bad arguments");
+  SlotList lst{};
+  for (int i = 0; i < n; i++) {
+    const int e = host_idx[i];
+    if (e < 0 || e >= C->dims.n_experts) return fail(E0_ERR_INVALID_ARG, "stage: expert %d out of range", e);
+    bool dup = false;
+    for (int q = 0; q < lst.n; q++) dup |= lst.e[q] == e;
+    if (dup) continue;
+    if (lst.n >= P.slots || lst.n >= kMaxSlots)
+      return fail(E0_ERR_INVALID_ARG, "stage: more distinct experts than pool slots (%d)", P.slots);
+    lst.e[lst.n++] = e;
+  }
+  const int p = layer % P.nsets;
+  StreamPool::Rec &rec = P.ring[P.ring_pos];
+  account_rec(C, rec);
+  P.set_rec[p] = P.ring_pos;
+  P.ring_pos = (P.ring_pos + 1) % (int)P.ring.size();
+  // the previous user of this slot set must be done (event recorded after its kernels)
+  CK(cudaStreamWaitEvent(P.side, P.freed[p], 0));
+  CK(cudaEventRecord(rec.c0, P.side));
+  uint8_t *dst = P.mem + (size_t)p * P.slots * P.bytes;
+  for (int s = 0; s < lst.n; s++) {
+    const uint8_t *src = P.host + ((size_t)layer * C->dims.n_experts + lst.e[s]) * P.bytes;
+    if (P.fail_after == 0) {
+      P.fail_after = -1;
+      return fail(E0_ERR_STAGING, "staging copy of layer %d expert %d refused (injected)", layer, lst.e[s]);
+    }
+    if (P.fail_after > 0) P.fail_after--;
+    cudaError_t e = cudaMemcpyAsync(dst + (size_t)s * P.bytes, src, P.bytes, cudaMemcpyHostToDevice, P.side);
+    if (e != cudaSuccess)
+      return fail(E0_ERR_STAGING, "staging copy of layer %d expert %d: %s", layer, lst.e[s], cudaGetErrorString(e));
+  }
+  int bad_slot = -1, bad_tag = 0;
+  if (P.corrupt_set == p) {
+    bad_slot = P.corrupt_slot;
+    bad_tag = P.corrupt_tag;
+    P.corrupt_set = -1;
+  }
+  k_set_slots<<<1, 256, 0, P.side>>>(P.slot_of + (size_t)p * C->dims.n_experts, P.slot_tag + (size_t)p * P.slots,
+                                     C->dims.n_experts, P.slots, lst, bad_slot, bad_tag);
+  CKL("k_set_slots");
+  CK(cudaEventRecord(rec.c1, P.side));
+  CK(cudaEventRecord(P.ready[p], P.side));
+  rec.state = 1;
+  C->stats.staged_experts += lst.n;
+  C->stats.staged_bytes += (uint64_t)lst.n * P.bytes;
+  (prefetch ? C->stats.prefetched_experts : C->stats.ondemand_experts) += lst.n;
+  (void)compute;
+  return E0_OK;
+}
+
+extern "C" int e0_stage_experts(e0_ctx *C, int layer, const int32_t *host_idx, int n, void *compute_stream) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  return stage_impl(C, layer, host_idx, n, (cudaStream_t)compute_stream, true);
+}
+
+// The compute stream waits for a layer's staged experts; the wait is bracketed by events
+// so that the exposed (stalled) time can be accounted.
+static int wait_ready(e0_ctx *C, int layer, cudaStream_t s) {
+  StreamPool &P = C->pool;
+  const int p = layer % P.nsets;
+  if (P.set_rec[p] < 0) return fail(E0_ERR_STAGING, "layer %d was never staged", layer);
+  StreamPool::Rec &rec = P.ring[P.set_rec[p]];
+  CK(cudaEventRecord(rec.w0, s));
+  CK(cudaStreamWaitEvent(s, P.ready[p], 0));
+  CK(cudaEventRecord(rec.w1, s));
+  if (rec.state == 1) rec.state = 2;
+  return E0_OK;
+}
+
+static int release_set(e0_ctx *C, int layer, cudaStream_t s) {
+  CK(cudaEventRecord(C->pool.freed[layer % C->pool.nsets], s));
+  return E0_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Decode over the stack
+// ---------------------------------------------------------------------------------------
+static inline int32_t *pred_at(e0_ctx *C, int parity, int layer) {
+  return C->pred_tab + ((size_t)parity * (C->L + 1) + layer) * C->maxT * C->dims.top_k;
+}
+static inline int32_t *hist_at(e0_ctx *C, int parity, int layer) {
+  return C->hist_tab + ((size_t)parity * C->L + layer) * C->maxT * C->dims.top_k;
+}
+
+static int host_read_idx(e0_ctx *C, int32_t *host, const int32_t *dev, int n, cudaStream_t s) {
+  CK(cudaMemcpyAsync(host, dev, n * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return E0_OK;
+}
+
+static int unique_list(const int32_t *v, int n, int32_t *out) {
+  int m = 0;
+  for (int i = 0; i < n; i++) {
+    bool seen = false;
+    for (int q = 0; q < m; q++) seen |= out[q] == v[i];
+    if (!seen) out[m++] = v[i];
+  }
+  return m;
+}
+
+static int stack_decode_general(e0_ctx *C, const uint16_t *h_in, int B, int step, uint16_t *y_out,
+                                float *y_f32, int streaming, int chained, cudaStream_t s) {
+  const e0_dims &D = C->dims;
+  const int k = D.top_k, L = C->L;
+  const size_t ld = (size_t)B * D.d_model;
+  const int cur = step & 1, prv = cur ^ 1;
+  std::vector<int32_t> uniq(B * k);
+  for (int l = 0; l < L; l++) {
+    const bool predicted = step > 0 && l > 0 && C->heads[l - 1].w_lin != nullptr;
+    LayerCall K{};
+    K.l = l; K.T = B; K.h = h_in + l * ld;
+    float *yf_l = y_f32 ? y_f32 + l * ld : C->yscratch + (size_t)(l & 1) * C->maxT * D.d_model;
+    K.chain = (chained && l > 0) ? (y_f32 ? y_f32 + (l - 1) * ld : C->yscratch + (size_t)((l - 1) & 1) * C->maxT * D.d_model)
+                                 : nullptr;
+    K.route = predicted ? pred_at(C, prv, l) : nullptr;
+    K.full_mode = predicted ? 0 : 1;
+    K.idx = hist_at(C, cur, l);
+    K.gates = C->gates;
+    K.hist = nullptr;
+    const bool has_head = C->heads[l].w_lin != nullptr;
+    K.head = has_head && D.head_hidden == 0;   // the linear head is fused into the routing kernel
+    K.prev = step > 0 ? hist_at(C, prv, l) : nullptr;
+    K.pred = pred_at(C, cur, l + 1);
+    K.y = y_out + l * ld;
+    K.yf = yf_l;
+    if (streaming) {
+      if (predicted) {
+        // the prediction made one token earlier is already on the host: stage now
+        const int n = unique_list(C->host_idx + (size_t)l * C->maxT * k, B * k, uniq.data());
+        int rc = stage_impl(C, l, uniq.data(), n, s, true);
+        if (rc) return rc;
+      }
+      int rc = layer_pre(C, K, s);
+      if (rc) return rc;
+      if (has_head && !K.head && (rc = run_head(C, l, B, K.idx, K.prev, K.pred, nullptr, s))) return rc;
+      if (!predicted) {
+        // reactive layer: the routing exists only now; read it back and stage on demand
+        int32_t *scratch = C->host_idx + (size_t)(L + 1) * C->maxT * k;
+        if ((rc = host_read_idx(C, scratch, K.idx, B * k, s))) return rc;
+        const int n = unique_list(scratch, B * k, uniq.data());
+        if ((rc = stage_impl(C, l, uniq.data(), n, s, false))) return rc;
+      }
+      if ((rc = wait_ready(C, l, s))) return rc;
+      if ((rc = layer_post(C, K, pool_src(C, l), s))) return rc;
+      if ((rc = release_set(C, l, s))) return rc;
+    } else {
+      int rc = layer_pre(C, K, s);
+      if (rc) return rc;
+      if (has_head && !K.head && (rc = run_head(C, l, B, K.idx, K.prev, K.pred, nullptr, s))) return rc;
+      if ((rc = layer_post(C, K, resident_src(C, l), s))) return rc;
+    }
+  }
+  if (streaming) {
+    // next step's predicted routing, for the staging decisions of the next call
+    int rc = host_read_idx(C, C->host_idx, pred_at(C, cur, 0), (L + 1) * C->maxT * k, s);
+    if (rc) return rc;
+  }
+  return E0_OK;
+}
+
+static bool decode_supported(const DecodeState &, const e0_dims &, int, int) { return false; }
+static int decode_persistent(DecodeState &, e0_ctx *, const uint16_t *, int, int, uint16_t *, float *, int,
+                             cudaStream_t) {
+  return E0_ERR_INVALID_ARG;
+}
+
+extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step, void *y_out, float *y_f32,
+                                   int streaming, int chained, void *stream) {
+  if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
+  if (!h_in || !y_out || B < 1 || B > C->maxT || step < 0)
+    return fail(E0_ERR_INVALID_ARG, "e0_moe_stack_decode: bad arguments (B=%d, max %d)", B, C->maxT);
+  if (step > 0 && (C->last_step != step - 1 || C->last_B != B))
+    return fail(E0_ERR_INVALID_ARG, "step %d does not follow step %d with the same B", step, C->last_step);
+  if (streaming && !C->pool.mem) return fail(E0_ERR_INVALID_ARG, "streaming decode needs e0_stream_register");
+  if (streaming && C->pool.slots < std::min(B * C->dims.top_k, C->dims.n_experts))
+    return fail(E0_ERR_INVALID_ARG, "pool has %d slots per layer, a step may route to %d experts", C->pool.slots,
+                std::min(B * C->dims.top_k, C->dims.n_experts));
+  if (!streaming)
+    for (int l = 0; l < C->L; l++)
+      if (!C->layers[l].experts) return fail(E0_ERR_INVALID_ARG, "layer %d has no resident experts", l);
+  cudaStream_t s = (cudaStream_t)stream;
+  C->last = s;
+  int rc;
+  if (!streaming && decode_supported(C->dec, C->dims, C->L, B))
+    rc = decode_persistent(C->dec, C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, chained, s);
+  else
+    rc = stack_decode_general(C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, streaming, chained, s);
+  if (rc) return rc;
+  C->last_step = step;
+  C->last_B = B;
+  C->stats.steps++;
+  return E0_OK;
+}
+
+extern "C" int e0_get_routing(e0_ctx *C, int B, int32_t *idx_host, int32_t *pred_host) {
+  if (!C || C->last_step < 0 || B != C->last_B) return fail(E0_ERR_INVALID_ARG, "no decode step with this B");
+  CK(cudaStreamSynchronize(C->last));
+  const int k = C->dims.top_k, cur = C->last_step & 1;
+  for (int l = 0; l < C->L; l++) {
+    if (idx_host) CK(cudaMemcpy(idx_host + (size_t)l * B * k, hist_at(C, cur, l), (size_t)B * k * 4, cudaMemcpyDeviceToHost));
+    if (pred_host) {
+      if (C->heads[l].w_lin)
+        CK(cudaMemcpy(pred_host + (size_t)l * B * k, pred_at(C, cur, l + 1), (size_t)B * k * 4, cudaMemcpyDeviceToHost));
+      else
+        for (int i = 0; i < B * k; i++) pred_host[(size_t)l * B * k + i] = -1;
+    }
+  }
+  return E0_OK;
+}
+
+extern "C" int e0_get_stats(e0_ctx *C, e0_stats *out) {
+  if (!C || !out) return fail(E0_ERR_INVALID_ARG, "NULL argument");
+  if (C->pool.mem) {
+    cudaStreamSynchronize(C->pool.side);
+    if (C->last) cudaStreamSynchronize(C->last);
+    for (auto &r : C->pool.ring) account_rec(C, r);
+  }
+  *out = C->stats;
+  return E0_OK;
+}
+
+extern "C" int e0_sync_status(e0_ctx *C) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  if (C->last) CK(cudaStreamSynchronize(C->last));
+  if (C->pool.side) CK(cudaStreamSynchronize(C->pool.side));
+  int err = 0;
+  CK(cudaMemcpy(&err, C->err, sizeof(int), cudaMemcpyDeviceToHost));
+  CK(cudaMemset(C->err, 0, sizeof(int)));
+  if (err & DERR_SLOT) return fail(E0_ERR_SLOT_MISMATCH, "a kernel found a pool slot holding another expert");
+  if (err & DERR_TIMEOUT) return fail(E0_ERR_TIMEOUT, "a bounded device wait gave up");
+  if (err & (DERR_INDEX | DERR_DUP))
+    return fail(E0_ERR_DEVICE, "routing rejected on the device (%s)",
+                (err & DERR_INDEX) ? "expert index out of range" : "duplicate expert in a token");
+  return E0_OK;
+}
+
+// Host-side fault injection for the staging tests: the n-th next staging copy fails.
+extern "C" int e0_debug_fail_staging_after(e0_ctx *C, int n) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  C->pool.fail_after = n;
+  return E0_OK;
+}
+
+// Arm a one-shot wrong tag: the next staging into `pool_set` tags `slot` with `expert`
+// (tests: the kernels must report the mismatch instead of reading the wrong blob).
+extern "C" int e0_debug_set_slot_tag(e0_ctx *C, int pool_set, int slot, int expert) {
+  if (!C || !C->pool.mem || pool_set < 0 || pool_set >= C->pool.nsets || slot < 0 || slot >= C->pool.slots)
+    return fail(E0_ERR_INVALID_ARG, "bad slot");
+  C->pool.corrupt_set = pool_set;
+  C->pool.corrupt_slot = slot;
+  C->pool.corrupt_tag = expert;
+  return E0_OK;
+}

@@ -1,0 +1,153 @@
+"""GPU parity of the decode loop over the stack (prediction-as-routing) against the oracle,
+on a small stack in full and on the full-size 40-layer model on sampled outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from synth import Dims
+from synth.device import bf16_tensor, layer_tensors
+from parity import bf16_bits_to_np, check_bf16, check_y, choose_following, idx_ok
+
+pytestmark = pytest.mark.gpu
+
+SMALL = Dims(d=256, E=16, I=128, k=4, r=8, L=4, head_layers=(0, 1, 2))
+
+
+def build(dims, seed, max_tokens, resident=True):
+    import int4_expert_streaming_prerouter_b200 as e0
+    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, max_tokens,
+                     head_hidden=dims.head_hidden, head_onehot=dims.head_onehot)
+    lys, hds = zip(*[layer_tensors(seed, n, dims, "cuda", resident=resident) for n in range(dims.L)])
+    ctx.register_model(list(lys), list(hds))
+    return ctx, lys, hds
+
+
+def run_steps(ctx, dims, seed, B, S, chained=False, streaming=False):
+    ys, y32s, idxs, preds = [], [], [], []
+    for t in range(S):
+        h = bf16_tensor(synth.hidden(seed, t, dims.L, B, dims.d), "cuda")
+        y32 = torch.empty((dims.L, B, dims.d), dtype=torch.float32, device="cuda")
+        y = ctx.stack_decode(h, t, y_f32=y32, chained=chained, streaming=streaming)
+        ctx.sync_status()
+        idx, pred = ctx.get_routing(B)
+        ys.append(bf16_bits_to_np(y))
+        y32s.append(y32.cpu().numpy().astype(np.float64))
+        idxs.append(idx)
+        preds.append(pred)
+    return np.stack(ys), np.stack(y32s), np.stack(idxs), np.stack(preds)
+
+
+def oracle_steps(dims, seed, B, S, gpu_idx, gpu_pred, chained=False):
+    hs = np.stack([synth.hidden(seed, t, dims.L, B, dims.d) for t in range(S)])
+    dense = {n: synth.layer_dense(seed, n, dims) for n in range(dims.L)}
+    cache = {}
+
+    def expert(n, e):
+        if (n, e) not in cache:
+            cache[(n, e)] = synth.expert_blob(seed, n, e, dims)
+        return cache[(n, e)]
+
+    sets = {}
+    for t in range(S):
+        for n in range(dims.L):
+            for b in range(B):
+                sets[("route", t, n, b)] = gpu_idx[t, n, b]
+                sets[("head", t, n, b)] = gpu_pred[t, n, b]
+    return O.stack_decode(hs, dense.__getitem__, expert, lambda n: synth.shared_blob(seed, n, dims), dims,
+                          chained=chained, choose=choose_following(sets))
+
+
+def compare_steps(dims, gpu, ref, chained=False):
+    yb, y32, idx, pred = gpu
+    S, L, B = idx.shape[:3]
+    assert np.array_equal(idx, ref["idx"]), "routing differs beyond admissible near ties"
+    for n in range(L):
+        if n in dims.head_layers:
+            assert np.array_equal(pred[:, n], ref["pred"][:, n])
+        else:
+            assert np.all(pred[:, n] == -1)
+    for t in range(S):
+        for n in range(L):
+            check_y(y32[t, n], ref["y"][t, n], f"step {t} layer {n}")
+            check_bf16(yb[t, n], ref["y"][t, n], f"step {t} layer {n}")
+
+
+@pytest.mark.parametrize("B", [1, 5])
+def test_small_stack_decode_matches_oracle(cuda_ok, B):
+    ctx, _, _ = build(SMALL, 60 + B, 16)
+    S = 4
+    gpu = run_steps(ctx, SMALL, 60 + B, B, S)
+    ref = oracle_steps(SMALL, 60 + B, B, S, gpu[2], gpu[3])
+    compare_steps(SMALL, gpu, ref)
+    # prediction is the routing: every predicted layer at t > 0 used the t-1 prediction
+    for t in range(1, S):
+        for n in range(1, SMALL.L):
+            assert np.array_equal(gpu[2][t, n], gpu[3][t - 1, n - 1])
+    ctx.close()
+
+
+def test_small_stack_chained_matches_oracle(cuda_ok):
+    ctx, _, _ = build(SMALL, 70, 8)
+    gpu = run_steps(ctx, SMALL, 70, 2, 3, chained=True)
+    ref = oracle_steps(SMALL, 70, 2, 3, gpu[2], gpu[3], chained=True)
+    compare_steps(SMALL, gpu, ref, chained=True)
+    ctx.close()
+
+
+def test_onehot_head_stack(cuda_ok):
+    dims = Dims(d=256, E=16, I=128, k=4, r=8, L=3, head_layers=(0, 1), head_onehot=1)
+    ctx, _, _ = build(dims, 71, 8)
+    gpu = run_steps(ctx, dims, 71, 3, 4)
+    ref = oracle_steps(dims, 71, 3, 4, gpu[2], gpu[3])
+    compare_steps(dims, gpu, ref)
+    ctx.close()
+
+
+def test_step_sequence_is_enforced(cuda_ok):
+    import int4_expert_streaming_prerouter_b200 as e0
+    ctx, _, _ = build(SMALL, 72, 8)
+    h = bf16_tensor(synth.hidden(72, 0, SMALL.L, 2, SMALL.d), "cuda")
+    with pytest.raises(e0.E0Error):
+        ctx.stack_decode(h, 3)
+    ctx.stack_decode(h, 0)
+    with pytest.raises(e0.E0Error):
+        ctx.stack_decode(h[:, :1].contiguous(), 1)   # B changed mid-sequence
+    ctx.close()
+
+
+# ---------------------------------------------------------------------------------------
+# full-size model (40 layers, d=2048, E=256, I=512, r=16, heads on 0..32), batch 1
+# ---------------------------------------------------------------------------------------
+FULL = synth.WORKLOADS["decode_b1_l40"]["dims"]
+
+
+@pytest.fixture(scope="module")
+def full_model(cuda_ok):
+    ctx, lys, hds = build(FULL, 1, 64)
+    yield ctx
+    ctx.close()
+
+
+def test_full_size_decode_b1_sampled(full_model):
+    """Two steps of the 40-layer stack at B=1 in the bench's launch configuration: every
+    layer's routing and head prediction exactly, and y on every layer of both steps."""
+    S = 2
+    gpu = run_steps(full_model, FULL, 1, 1, S)
+    ref = oracle_steps(FULL, 1, 1, S, gpu[2], gpu[3])
+    compare_steps(FULL, gpu, ref)
+
+
+def test_full_size_decode_b8_sampled_layers(full_model):
+    """B=8 streams, one step, every layer's routing; y checked on a sample of layers."""
+    B, dims = 8, FULL
+    gpu = run_steps(full_model, dims, 2, B, 1)
+    hs = synth.hidden(2, 0, dims.L, B, dims.d)
+    for n in (0, 1, 17, 33, 34, 39):
+        dense = synth.layer_dense(2, n, dims)
+        ref = O.moe_layer(hs[n], dense, lambda e: synth.expert_blob(2, n, e, dims), synth.shared_blob(2, n, dims),
+                          dims, choose=lambda t, c, a: next((x for x in a if np.array_equal(x, gpu[2][0, n, t])), c))
+        for b in range(B):
+            assert idx_ok(gpu[2][0, n, b], ref["logits"][b], ref["idx"][b], dims.k)
+        check_y(gpu[1][0, n], ref["y"], f"layer {n}")

@@ -1,0 +1,230 @@
+"""GPU parity of one MoE block and of the prerouter head against the CPU oracle.
+
+Every input is drawn by ``synth`` from a seed; the oracle never sees a GPU value except
+where a near tie (fp32 logit gap < 1e-5) admits several routings, and then only to pick
+which of the oracle's own admissible routings to follow.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from synth import Dims
+from synth.device import bf16_tensor, layer_tensors
+from parity import bf16_bits_to_np, check_bf16, check_y, idx_ok
+
+pytestmark = pytest.mark.gpu
+
+CFG1 = synth.WORKLOADS["layer_d256_e16"]["dims"]     # d=256, E=16, I=128, k=4, r=8
+
+
+def make_ctx(dims: Dims, seed: int, max_tokens: int, layers=None, lora=True):
+    import int4_expert_streaming_prerouter_b200 as e0
+    layers = range(dims.L) if layers is None else layers
+    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, max_tokens,
+                     head_hidden=dims.head_hidden, head_onehot=dims.head_onehot,
+                     eps=dims.eps, lora_scale=dims.lora_scale)
+    lys, hds = [], []
+    for n in range(dims.L):
+        ly, hd = layer_tensors(seed, n, dims, "cuda", lora=lora)
+        lys.append(ly)
+        hds.append(hd)
+    ctx.register_model(lys, hds)
+    return ctx, lys, hds
+
+
+def run_layer(ctx, dims, seed, layer, h_bits, route=None):
+    T = h_bits.shape[0]
+    h = bf16_tensor(h_bits, "cuda")
+    y32 = torch.empty((T, dims.d), dtype=torch.float32, device="cuda")
+    idx = torch.empty((T, dims.k), dtype=torch.int32, device="cuda")
+    gates = torch.empty((T, dims.k), dtype=torch.float32, device="cuda")
+    r = None if route is None else torch.from_numpy(np.asarray(route, np.int32)).cuda()
+    y = ctx.moe_layer_forward(layer, h, route_idx=r, y_f32=y32, idx=idx, gates=gates)
+    ctx.sync_status()
+    return (bf16_bits_to_np(y), y32.cpu().numpy().astype(np.float64), idx.cpu().numpy(),
+            gates.cpu().numpy().astype(np.float64))
+
+
+def oracle_layer(dims, seed, layer, h_bits, route=None, gpu_idx=None):
+    dense = synth.layer_dense(seed, layer, dims)
+    cache = {}
+
+    def blob(e):
+        if e not in cache:
+            cache[e] = synth.expert_blob(seed, layer, e, dims)
+        return cache[e]
+
+    choose = None
+    if gpu_idx is not None:
+        def choose(t, canonical, alts):
+            for a in alts:
+                if np.array_equal(a, gpu_idx[t]):
+                    return a
+            return canonical
+    return O.moe_layer(h_bits, dense, blob, synth.shared_blob(seed, layer, dims), dims,
+                       route_idx=route, choose=choose)
+
+
+def compare(dims, out_gpu, ref, what):
+    yb, y32, idx, gates = out_gpu
+    for t in range(idx.shape[0]):
+        assert idx_ok(idx[t], ref["logits"][t], ref["idx"][t], dims.k), (what, t, idx[t], ref["idx"][t])
+    check_y(y32, ref["y"], what)
+    check_bf16(yb, ref["y"], what)
+    assert np.allclose(gates, ref["gates"], rtol=1e-5, atol=1e-6), what
+
+
+@pytest.fixture(scope="module")
+def cfg1(cuda_ok):
+    ctx, lys, hds = make_ctx(CFG1, 0, 256)
+    yield ctx
+    ctx.close()
+
+
+def test_layer_d256_e16_single_token(cfg1):
+    h = synth.hidden(0, 0, 1, 1, CFG1.d)[0]
+    out = run_layer(cfg1, CFG1, 0, 0, h)
+    ref = oracle_layer(CFG1, 0, 0, h, gpu_idx=out[2])
+    compare(CFG1, out, ref, "T=1")
+
+
+@pytest.mark.parametrize("T", [2, 3, 17, 64, 255])
+def test_layer_ragged_token_counts(cfg1, T):
+    h = synth.hidden(100 + T, 0, 1, T, CFG1.d)[0]
+    out = run_layer(cfg1, CFG1, 0, 0, h)
+    ref = oracle_layer(CFG1, 0, 0, h, gpu_idx=out[2])
+    compare(CFG1, out, ref, f"T={T}")
+
+
+def test_prediction_as_routing_and_own_router_rows(cfg1):
+    """route_idx given: rows use it, rows starting with -1 use the layer's own router."""
+    T = 9
+    h = synth.hidden(7, 0, 1, T, CFG1.d)[0]
+    rng = np.random.default_rng(7)
+    route = np.stack([rng.permutation(CFG1.E)[:CFG1.k] for _ in range(T)]).astype(np.int32)
+    route[[0, 4]] = -1
+    out = run_layer(cfg1, CFG1, 0, 0, h, route=route)
+    ref = oracle_layer(CFG1, 0, 0, h, route=route, gpu_idx=out[2])
+    for t in range(T):
+        if route[t, 0] >= 0:
+            assert np.array_equal(out[2][t], route[t])
+    compare(CFG1, out, ref, "routed")
+
+
+def test_all_tokens_on_one_expert_set_and_idle_experts(cfg1):
+    T = 33
+    h = synth.hidden(8, 0, 1, T, CFG1.d)[0]
+    route = np.tile(np.array([5, 2, 11, 7], np.int32), (T, 1))
+    out = run_layer(cfg1, CFG1, 0, 0, h, route=route)
+    ref = oracle_layer(CFG1, 0, 0, h, route=route)
+    compare(CFG1, out, ref, "one set")
+
+
+def test_lora_branch_is_applied_with_large_B(cuda_ok):
+    """B ~ N(0,1) makes the LoRA delta large, so a dropped branch cannot hide."""
+    dims = CFG1
+    import int4_expert_streaming_prerouter_b200 as e0
+    dense = synth.layer_dense(21, 0, dims)
+    rng = np.random.default_rng(21)
+    for key, shape in (("lora_Bg", (dims.I, dims.r)), ("lora_Bu", (dims.I, dims.r)), ("lora_Bd", (dims.d, dims.r))):
+        dense[key] = synth.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32))
+    ly, hd = layer_tensors(21, 0, dims, "cuda", dense=dense)
+    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, 1, 8)
+    ctx.register_model([ly], [hd])
+    h = synth.hidden(21, 0, 1, 4, dims.d)[0]
+    out = run_layer(ctx, dims, 21, 0, h)
+    ref = O.moe_layer(h, dense, lambda e: synth.expert_blob(21, 0, e, dims), synth.shared_blob(21, 0, dims), dims)
+    compare(dims, out, ref, "large LoRA B")
+    ctx.close()
+
+
+@pytest.mark.parametrize("k", [1, 2, 8])
+def test_routing_widths(cuda_ok, k):
+    dims = Dims(d=256, E=16, I=128, k=k, r=8, L=1, head_layers=(0,))
+    ctx, _, _ = make_ctx(dims, 30 + k, 16)
+    h = synth.hidden(30 + k, 0, 1, 5, dims.d)[0]
+    out = run_layer(ctx, dims, 30 + k, 0, h)
+    ref = oracle_layer(dims, 30 + k, 0, h, gpu_idx=out[2])
+    compare(dims, out, ref, f"k={k}")
+    ctx.close()
+
+
+def test_wide_layer_d2048_e256(cuda_ok):
+    """The full-size geometry (d=2048, E=256, I=512, r=16) on one layer, several tokens."""
+    dims = Dims(d=2048, E=256, I=512, k=4, r=16, L=1, head_layers=(0,))
+    ctx, _, _ = make_ctx(dims, 40, 16)
+    h = synth.hidden(40, 0, 1, 6, dims.d)[0]
+    out = run_layer(ctx, dims, 40, 0, h)
+    ref = oracle_layer(dims, 40, 0, h, gpu_idx=out[2])
+    compare(dims, out, ref, "d2048")
+    ctx.close()
+
+
+def test_no_lora_layer(cuda_ok):
+    dims = CFG1
+    ctx, _, _ = make_ctx(dims, 41, 8, lora=False)
+    h = synth.hidden(41, 0, 1, 3, dims.d)[0]
+    out = run_layer(ctx, dims, 41, 0, h)
+    dense = synth.layer_dense(41, 0, dims)
+    for key in ("lora_Bg", "lora_Bu", "lora_Bd"):
+        dense[key] = np.zeros_like(dense[key])
+    ref = O.moe_layer(h, dense, lambda e: synth.expert_blob(41, 0, e, dims), synth.shared_blob(41, 0, dims), dims)
+    compare(dims, out, ref, "no LoRA")
+    ctx.close()
+
+
+# ---------------------------------------------------------------------------------------
+# prerouter head
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("onehot,hidden", [(0, 0), (1, 0), (1, 256), (0, 64)])
+def test_prerouter_head(cuda_ok, onehot, hidden):
+    dims = Dims(d=256, E=16, I=128, k=4, r=8, L=2, head_layers=(0,), head_onehot=onehot, head_hidden=hidden)
+    ctx, _, _ = make_ctx(dims, 50, 16)
+    T = 7
+    rng = np.random.default_rng(50)
+    x_bits = O.f64_to_bf16_bits(O.round_bf16(rng.standard_normal((T, dims.d))))
+    cur = np.stack([rng.permutation(dims.E)[:dims.k] for _ in range(T)]).astype(np.int32)
+    prev = np.stack([rng.permutation(dims.E)[:dims.k] for _ in range(T)]).astype(np.int32)
+    prev[2] = -1
+    logits = torch.empty((T, dims.E), dtype=torch.float32, device="cuda")
+    pred = ctx.prerouter_predict(0, bf16_tensor(x_bits, "cuda"), cur=torch.from_numpy(cur).cuda(),
+                                 prev=torch.from_numpy(prev).cuda(), logits=logits)
+    ctx.sync_status()
+    pred = pred.cpu().numpy()
+    lg = logits.cpu().numpy().astype(np.float64)
+    dense = synth.layer_dense(50, 0, dims)
+    for t in range(T):
+        z, p = O.prerouter_head(O.bf16_to_f64(x_bits[t]), dense, dims, cur[t], prev[t] if prev[t, 0] >= 0 else None)
+        assert np.allclose(lg[t], z, rtol=1e-5, atol=2e-6)
+        assert idx_ok(pred[t], z, p, dims.k), (t, pred[t], p)
+    ctx.close()
+
+
+def test_layer_rejects_bad_arguments(cfg1):
+    import int4_expert_streaming_prerouter_b200 as e0
+    h = torch.zeros((1, CFG1.d), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(e0.E0Error) as ei:
+        cfg1.moe_layer_forward(5, h)
+    assert ei.value.status == "INVALID_ARG"
+    big = torch.zeros((300, CFG1.d), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(e0.E0Error):
+        cfg1.moe_layer_forward(0, big)
+
+
+def test_out_of_range_and_duplicate_routes_are_flagged(cfg1):
+    import int4_expert_streaming_prerouter_b200 as e0
+    h = bf16_tensor(synth.hidden(9, 0, 1, 2, CFG1.d)[0], "cuda")
+    bad = torch.tensor([[1, 2, 3, 99], [0, 1, 2, 3]], dtype=torch.int32, device="cuda")
+    cfg1.moe_layer_forward(0, h, route_idx=bad)
+    with pytest.raises(e0.E0Error) as ei:
+        cfg1.sync_status()
+    assert ei.value.status == "DEVICE"
+    dup = torch.tensor([[1, 1, 3, 4], [0, 1, 2, 3]], dtype=torch.int32, device="cuda")
+    cfg1.moe_layer_forward(0, h, route_idx=dup)
+    with pytest.raises(e0.E0Error) as ei:
+        cfg1.sync_status()
+    assert ei.value.status == "DEVICE"
+    cfg1.moe_layer_forward(0, h)
+    cfg1.sync_status()          # the error word was cleared
