@@ -190,6 +190,16 @@ int e0_sync_status(e0_ctx *ctx);
 int e0_debug_fail_staging_after(e0_ctx *ctx, int n);
 int e0_debug_set_slot_tag(e0_ctx *ctx, int pool_set, int slot, int expert);
 
+/* Test hooks of the one-launch decode path (B = 1, resident experts, linear heads):
+ * e0_debug_decode_stall(ctx, cta, timeout_ns): in the next decode step CTA `cta` waits for
+ *   a word that nothing writes, and every device wait of that launch gives up after
+ *   timeout_ns; the step must end with E0_ERR_TIMEOUT from e0_sync_status (the context
+ *   stays usable).  timeout_ns = 0 restores the default budget (2 s).
+ * e0_debug_force_general(ctx, on): 1 sends every decode step through the per-layer
+ *   kernels instead of the one-launch kernel (for comparisons); 0 restores the default. */
+int e0_debug_decode_stall(e0_ctx *ctx, int cta, unsigned long long timeout_ns);
+int e0_debug_force_general(e0_ctx *ctx, int on);
+
 /* Message of the last failing call on this host thread ("" if none). */
 const char *e0_last_error(void);
 

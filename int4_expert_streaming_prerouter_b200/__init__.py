@@ -74,6 +74,8 @@ _SIGS = {
     "e0_last_error": (ctypes.c_char_p, []),
     "e0_debug_fail_staging_after": (_I, [_P, _I]),
     "e0_debug_set_slot_tag": (_I, [_P, _I, _I, _I]),
+    "e0_debug_decode_stall": (_I, [_P, _I, ctypes.c_ulonglong]),
+    "e0_debug_force_general": (_I, [_P, _I]),
 }
 
 
@@ -226,3 +228,9 @@ class Context:
 
     def debug_set_slot_tag(self, pool_set, slot, expert):
         _check(lib().e0_debug_set_slot_tag(self._h, pool_set, slot, expert))
+
+    def debug_decode_stall(self, cta, timeout_ns):
+        _check(lib().e0_debug_decode_stall(self._h, cta, timeout_ns))
+
+    def debug_force_general(self, on: bool):
+        _check(lib().e0_debug_force_general(self._h, int(on)))

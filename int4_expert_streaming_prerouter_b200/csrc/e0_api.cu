@@ -61,6 +61,27 @@ struct StreamPool {
   int corrupt_set = -1, corrupt_slot = 0, corrupt_tag = 0;  // one-shot wrong slot tag
 };
 
+// Persistent decode kernel state: device copy of the layer table, tagged exchange buffers
+// and the launch epoch (tags are unique per launch and layer).
+struct DecodeState {
+  bool ready = false;
+  DecLayer *d_layers = nullptr;
+  unsigned long long *tbuf = nullptr;   // one allocation for every tagged buffer
+  unsigned long long *t_y = nullptr, *t_a = nullptr, *t_lora = nullptr, *t_tdp = nullptr,
+                     *t_rsel = nullptr, *t_rlog = nullptr, *t_hlog = nullptr;
+  uint32_t epoch = 0;
+  int G = 0;
+  size_t smem = 0;
+  int stall_cta = -1;
+  unsigned long long timeout_ns = 2000000000ull;
+};
+
+static void decode_free(DecodeState &S) {
+  if (S.d_layers) cudaFree(S.d_layers);
+  if (S.tbuf) cudaFree(S.tbuf);
+  S = DecodeState{};
+}
+
 struct e0_ctx {
   e0_dims dims{};
   int L = 0, maxT = 0, dev = 0, nsm = 0;
@@ -83,6 +104,7 @@ struct e0_ctx {
   int32_t *host_idx = nullptr;       // pinned scratch for routing read-backs
   cudaStream_t last = nullptr;
   int last_step = -1, last_B = 0;
+  bool force_general = false;        // route decode through the general per-layer kernels
   DecodeState dec{};
   StreamPool pool;
   e0_stats stats{};
@@ -198,7 +220,7 @@ extern "C" int e0_register_model(e0_ctx *C, const e0_layer *layers, const e0_hea
   C->heads.assign(C->L, e0_head{});
   if (heads) C->heads.assign(heads, heads + C->L);
   C->registered = true;
-  C->dec.valid = false;
+  C->dec.ready = false;
   return E0_OK;
 }
 
@@ -614,10 +636,127 @@ static int stack_decode_general(e0_ctx *C, const uint16_t *h_in, int B, int step
   return E0_OK;
 }
 
-static bool decode_supported(const DecodeState &, const e0_dims &, int, int) { return false; }
-static int decode_persistent(DecodeState &, e0_ctx *, const uint16_t *, int, int, uint16_t *, float *, int,
-                             cudaStream_t) {
-  return E0_ERR_INVALID_ARG;
+// ---------------------------------------------------------------------------------------
+// Persistent decode path (one stream, resident experts, linear heads)
+// ---------------------------------------------------------------------------------------
+template <int D, int I>
+static size_t dec_smem() { return sizeof(DecSmem<D, I>); }
+
+static bool decode_geometry(const e0_dims &Dm, int *which) {
+  if (Dm.d_model == 2048 && Dm.d_ff == 512) *which = 0;
+  else if (Dm.d_model == 256 && Dm.d_ff == 128) *which = 1;
+  else return false;
+  return true;
+}
+
+static bool decode_supported(e0_ctx *C, int B) {
+  const e0_dims &D = C->dims;
+  int which;
+  if (B != 1 || D.head_hidden != 0 || !decode_geometry(D, &which) || C->L > 64) return false;
+  for (int l = 0; l < C->L; l++)
+    if (!C->layers[l].experts) return false;
+  // CTAs holding shared-expert rows each publish r partials of t_d
+  const int G = C->nsm, N = (D.top_k + 1) * D.d_ff;
+  int ncta = 0;
+  for (int c = 0; c < G; c++) {
+    int a, b;
+    split_range(N, G, c, a, b);
+    if (b > a && b > D.top_k * D.d_ff) ncta++;
+  }
+  return ncta * std::max(D.lora_rank, 1) <= kTdpMax;
+}
+
+static int decode_prepare(e0_ctx *C) {
+  DecodeState &S = C->dec;
+  if (S.ready) return E0_OK;
+  const e0_dims &D = C->dims;
+  const int L = C->L, E = D.n_experts, k = D.top_k, r = std::max(D.lora_rank, 1);
+  S.G = C->nsm;
+  std::vector<DecLayer> h(L);
+  for (int l = 0; l < L; l++) {
+    const e0_layer &Y = C->layers[l];
+    h[l] = DecLayer{(const uint8_t *)Y.experts, (const uint8_t *)Y.shared,
+                    (const uint16_t *)Y.lora_Ag, (const uint16_t *)Y.lora_Bg, (const uint16_t *)Y.lora_Au,
+                    (const uint16_t *)Y.lora_Bu, (const uint16_t *)Y.lora_Ad, (const uint16_t *)Y.lora_Bd,
+                    (const uint16_t *)Y.router_w, (const uint16_t *)Y.norm_w,
+                    (const uint16_t *)C->heads[l].w_lin};
+  }
+  if (!S.d_layers) {
+    int rc = dalloc(&S.d_layers, L);
+    if (rc) return rc;
+  }
+  CK(cudaMemcpy(S.d_layers, h.data(), L * sizeof(DecLayer), cudaMemcpyHostToDevice));
+  if (!S.tbuf) {
+    const size_t n_y = (size_t)L * D.d_model, n_a = (size_t)L * (k + 1) * D.d_ff, n_l = (size_t)L * 2 * r,
+                 n_t = (size_t)L * S.G * r, n_s = (size_t)L * k, n_r = (size_t)L * E, n_h = (size_t)L * E;
+    const size_t tot = n_y + n_a + n_l + n_t + n_s + n_r + n_h;
+    int rc = dalloc(&S.tbuf, tot);
+    if (rc) return rc;
+    CK(cudaMemset(S.tbuf, 0, tot * 8));
+    unsigned long long *p = S.tbuf;
+    S.t_y = p; p += n_y;
+    S.t_a = p; p += n_a;
+    S.t_lora = p; p += n_l;
+    S.t_tdp = p; p += n_t;
+    S.t_rsel = p; p += n_s;
+    S.t_rlog = p; p += n_r;
+    S.t_hlog = p;
+  }
+  int which;
+  decode_geometry(D, &which);
+  const void *fn = which == 0 ? (const void *)k_decode<2048, 512> : (const void *)k_decode<256, 128>;
+  S.smem = which == 0 ? dec_smem<2048, 512>() : dec_smem<256, 128>();
+  CK(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S.smem));
+  int per_sm = 0;
+  CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kDecThreads, S.smem));
+  if (per_sm < 1) return fail(E0_ERR_CUDA, "decode kernel does not fit on an SM (%zu B smem)", S.smem);
+  S.ready = true;
+  return E0_OK;
+}
+
+static int decode_persistent(e0_ctx *C, const uint16_t *h, int step, uint16_t *y, float *yf, int chained,
+                             cudaStream_t s) {
+  int rc = decode_prepare(C);
+  if (rc) return rc;
+  DecodeState &S = C->dec;
+  const e0_dims &D = C->dims;
+  const int cur = step & 1, prv = cur ^ 1;
+  DecodeParams P{};
+  P.layers = S.d_layers;
+  P.L = C->L; P.E = D.n_experts; P.k = D.top_k; P.r = D.lora_rank;
+  P.ldh = D.d_model + (D.head_onehot ? 2 * D.n_experts : 0);
+  P.onehot = D.head_onehot; P.G = S.G;
+  P.eps = D.rms_eps; P.c = D.lora_scale;
+  P.h = h; P.y = y; P.yf = yf; P.chained = chained;
+  P.epoch = ++S.epoch;
+  P.step0 = step == 0;
+  P.pred_in = step > 0 ? pred_at(C, prv, 0) : nullptr;
+  P.pred_out = pred_at(C, cur, 0);
+  P.hist_out = hist_at(C, cur, 0);
+  P.hist_prev = step > 0 ? hist_at(C, prv, 0) : nullptr;
+  P.maxT = C->maxT;
+  P.t_y = S.t_y; P.t_a = S.t_a; P.t_lora = S.t_lora; P.t_tdp = S.t_tdp;
+  P.t_rsel = S.t_rsel; P.t_rlog = S.t_rlog; P.t_hlog = S.t_hlog;
+  P.err = C->err;
+  P.timeout_ns = S.timeout_ns;
+  P.stall_cta = S.stall_cta;
+  S.stall_cta = -1;
+  int which;
+  decode_geometry(D, &which);
+  const void *fn = which == 0 ? (const void *)k_decode<2048, 512> : (const void *)k_decode<256, 128>;
+  void *args[] = {&P};
+  CK(cudaLaunchCooperativeKernel(fn, dim3(S.G), dim3(kDecThreads), args, S.smem, s));
+  C->stats.kernel_launches++;
+  return E0_OK;
+}
+
+// Test hook: make CTA `cta` of the next persistent decode launch wait on a word nobody
+// writes, with a wait budget of `timeout_ns`; the launch must come back with TIMEOUT.
+extern "C" int e0_debug_decode_stall(e0_ctx *C, int cta, unsigned long long timeout_ns) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  C->dec.stall_cta = cta;
+  C->dec.timeout_ns = timeout_ns ? timeout_ns : 2000000000ull;
+  return E0_OK;
 }
 
 extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step, void *y_out, float *y_f32,
@@ -637,8 +776,8 @@ extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step,
   cudaStream_t s = (cudaStream_t)stream;
   C->last = s;
   int rc;
-  if (!streaming && decode_supported(C->dec, C->dims, C->L, B))
-    rc = decode_persistent(C->dec, C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, chained, s);
+  if (!streaming && !C->force_general && decode_supported(C, B))
+    rc = decode_persistent(C, (const uint16_t *)h_in, step, (uint16_t *)y_out, y_f32, chained, s);
   else
     rc = stack_decode_general(C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, streaming, chained, s);
   if (rc) return rc;
@@ -694,6 +833,13 @@ extern "C" int e0_sync_status(e0_ctx *C) {
 extern "C" int e0_debug_fail_staging_after(e0_ctx *C, int n) {
   if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
   C->pool.fail_after = n;
+  return E0_OK;
+}
+
+// Select the decode implementation: 1 = general per-layer kernels only (comparisons).
+extern "C" int e0_debug_force_general(e0_ctx *C, int on) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  C->force_general = on != 0;
   return E0_OK;
 }
 

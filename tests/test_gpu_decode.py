@@ -142,12 +142,71 @@ def test_full_size_decode_b1_sampled(full_model):
 def test_full_size_decode_b8_sampled_layers(full_model):
     """B=8 streams, one step, every layer's routing; y checked on a sample of layers."""
     B, dims = 8, FULL
-    gpu = run_steps(full_model, dims, 2, B, 1)
+    gpu = run_steps(full_model, dims, 2, B, 1)       # inputs from seed 2, weights from seed 1
     hs = synth.hidden(2, 0, dims.L, B, dims.d)
     for n in (0, 1, 17, 33, 34, 39):
-        dense = synth.layer_dense(2, n, dims)
-        ref = O.moe_layer(hs[n], dense, lambda e: synth.expert_blob(2, n, e, dims), synth.shared_blob(2, n, dims),
+        dense = synth.layer_dense(1, n, dims)
+        ref = O.moe_layer(hs[n], dense, lambda e: synth.expert_blob(1, n, e, dims), synth.shared_blob(1, n, dims),
                           dims, choose=lambda t, c, a: next((x for x in a if np.array_equal(x, gpu[2][0, n, t])), c))
         for b in range(B):
             assert idx_ok(gpu[2][0, n, b], ref["logits"][b], ref["idx"][b], dims.k)
         check_y(gpu[1][0, n], ref["y"], f"layer {n}")
+
+
+# ---------------------------------------------------------------------------------------
+# the one-launch decode kernel (B = 1) against the per-layer kernels and the oracle
+# ---------------------------------------------------------------------------------------
+def test_one_launch_decode_equals_general_path_small(cuda_ok):
+    ctx, _, _ = build(SMALL, 90, 4)
+    ref, _, _ = build(SMALL, 90, 4)
+    ref.debug_force_general(True)
+    for t in range(5):
+        h = bf16_tensor(synth.hidden(91, t, SMALL.L, 1, SMALL.d), "cuda")
+        ya32 = torch.empty((SMALL.L, 1, SMALL.d), dtype=torch.float32, device="cuda")
+        yb32 = torch.empty_like(ya32)
+        ctx.stack_decode(h, t, y_f32=ya32)
+        ref.stack_decode(h, t, y_f32=yb32)
+        ctx.sync_status()
+        ref.sync_status()
+        ia, pa = ctx.get_routing(1)
+        ib, pb = ref.get_routing(1)
+        assert np.array_equal(ia, ib) and np.array_equal(pa, pb)
+        for n in range(SMALL.L):
+            check_y(ya32[n].cpu().numpy(), yb32[n].cpu().numpy().astype(np.float64), f"t{t} l{n}")
+    ctx.close()
+    ref.close()
+
+
+def test_one_launch_decode_chained_b1(cuda_ok):
+    ctx, _, _ = build(SMALL, 92, 4)
+    gpu = run_steps(ctx, SMALL, 92, 1, 3, chained=True)
+    ref = oracle_steps(SMALL, 92, 1, 3, gpu[2], gpu[3], chained=True)
+    compare_steps(SMALL, gpu, ref, chained=True)
+    ctx.close()
+
+
+def test_one_launch_decode_onehot_head_b1(cuda_ok):
+    dims = Dims(d=256, E=16, I=128, k=4, r=8, L=3, head_layers=(0, 1), head_onehot=1)
+    ctx, _, _ = build(dims, 93, 4)
+    gpu = run_steps(ctx, dims, 93, 1, 4)
+    ref = oracle_steps(dims, 93, 1, 4, gpu[2], gpu[3])
+    compare_steps(dims, gpu, ref)
+    ctx.close()
+
+
+def test_one_launch_decode_bounded_wait_reports_timeout(cuda_ok):
+    """A CTA that waits on a word nothing writes gives up after the budget; the launch ends,
+    the status is TIMEOUT, and the context decodes correctly afterwards."""
+    import int4_expert_streaming_prerouter_b200 as e0
+    ctx, _, _ = build(SMALL, 94, 4)
+    h = bf16_tensor(synth.hidden(94, 0, SMALL.L, 1, SMALL.d), "cuda")
+    ctx.debug_decode_stall(0, 20_000_000)          # 20 ms budget
+    ctx.stack_decode(h, 0)
+    with pytest.raises(e0.E0Error) as ei:
+        ctx.sync_status()
+    assert ei.value.status == "TIMEOUT"
+    ctx.debug_decode_stall(-1, 0)
+    gpu = run_steps(ctx, SMALL, 94, 1, 2)
+    ref = oracle_steps(SMALL, 94, 1, 2, gpu[2], gpu[3])
+    compare_steps(SMALL, gpu, ref)
+    ctx.close()
