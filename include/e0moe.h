@@ -198,6 +198,9 @@ int e0_debug_set_slot_tag(e0_ctx *ctx, int pool_set, int slot, int expert);
  * e0_debug_force_general(ctx, on): 1 sends every decode step through the per-layer
  *   kernels instead of the one-launch kernel (for comparisons); 0 restores the default. */
 int e0_debug_decode_stall(e0_ctx *ctx, int cta, unsigned long long timeout_ns);
+/* Profiling: the following one-launch decode steps write %globaltimer stamps (uint64,
+ * [grid][L][16], caller-owned device buffer; NULL stops it).  Returns the grid size. */
+int e0_debug_decode_trace(e0_ctx *ctx, unsigned long long *buf);
 int e0_debug_force_general(e0_ctx *ctx, int on);
 
 /* Message of the last failing call on this host thread ("" if none). */

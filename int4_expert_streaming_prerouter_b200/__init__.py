@@ -76,6 +76,7 @@ _SIGS = {
     "e0_debug_set_slot_tag": (_I, [_P, _I, _I, _I]),
     "e0_debug_decode_stall": (_I, [_P, _I, ctypes.c_ulonglong]),
     "e0_debug_force_general": (_I, [_P, _I]),
+    "e0_debug_decode_trace": (_I, [_P, _P]),
 }
 
 
@@ -231,6 +232,10 @@ class Context:
 
     def debug_decode_stall(self, cta, timeout_ns):
         _check(lib().e0_debug_decode_stall(self._h, cta, timeout_ns))
+
+    def debug_decode_trace(self, buf):
+        """buf: int64 CUDA tensor [grid, L, 16] or None; returns the grid size."""
+        return lib().e0_debug_decode_trace(self._h, _ptr(buf))
 
     def debug_force_general(self, on: bool):
         _check(lib().e0_debug_force_general(self._h, int(on)))

@@ -67,13 +67,14 @@ struct DecodeState {
   bool ready = false;
   DecLayer *d_layers = nullptr;
   unsigned long long *tbuf = nullptr;   // one allocation for every tagged buffer
-  unsigned long long *t_y = nullptr, *t_a = nullptr, *t_lora = nullptr, *t_tdp = nullptr,
-                     *t_rsel = nullptr, *t_rlog = nullptr, *t_hlog = nullptr;
+  unsigned long long *t_y = nullptr, *t_blk = nullptr, *t_rlog = nullptr, *t_hlog = nullptr;
+  int blk = 0;
   uint32_t epoch = 0;
   int G = 0;
   size_t smem = 0;
   int stall_cta = -1;
   unsigned long long timeout_ns = 2000000000ull;
+  unsigned long long *trace = nullptr;   // profiling timeline (caller-owned), or nullptr
 };
 
 static void decode_free(DecodeState &S) {
@@ -652,18 +653,16 @@ static bool decode_geometry(const e0_dims &Dm, int *which) {
 static bool decode_supported(e0_ctx *C, int B) {
   const e0_dims &D = C->dims;
   int which;
-  if (B != 1 || D.head_hidden != 0 || !decode_geometry(D, &which) || C->L > 64) return false;
+  if (B != 1 || D.head_hidden != 0 || !decode_geometry(D, &which) || C->L > 64 || D.lora_rank % 8 != 0 ||
+      D.top_k > kDecMaxK)
+    return false;
   for (int l = 0; l < C->L; l++)
     if (!C->layers[l].experts) return false;
-  // CTAs holding shared-expert rows each publish r partials of t_d
-  const int G = C->nsm, N = (D.top_k + 1) * D.d_ff;
-  int ncta = 0;
-  for (int c = 0; c < G; c++) {
-    int a, b;
-    split_range(N, G, c, a, b);
-    if (b > a && b > D.top_k * D.d_ff) ncta++;
-  }
-  return ncta * std::max(D.lora_rank, 1) <= kTdpMax;
+  // a CTA's gate/up rows and down rows must fit its scratch and the task segment table
+  const int G = C->nsm;
+  const int gu_rows = ((D.top_k + 1) * D.d_ff + G - 1) / G, dn_rows = (D.d_model + G - 1) / G;
+  return 2 * gu_rows <= 64 * (kMaxK + 1) && dn_rows * (D.top_k + 1) <= 64 * (kMaxK + 1) &&
+         kGuPiece0 + 6 * kMaxPieces <= kMaxSeg && gu_rows * kMaxPieces >= 1;
 }
 
 static int decode_prepare(e0_ctx *C) {
@@ -687,18 +686,15 @@ static int decode_prepare(e0_ctx *C) {
   }
   CK(cudaMemcpy(S.d_layers, h.data(), L * sizeof(DecLayer), cudaMemcpyHostToDevice));
   if (!S.tbuf) {
-    const size_t n_y = (size_t)L * D.d_model, n_a = (size_t)L * (k + 1) * D.d_ff, n_l = (size_t)L * 2 * r,
-                 n_t = (size_t)L * S.G * r, n_s = (size_t)L * k, n_r = (size_t)L * E, n_h = (size_t)L * E;
-    const size_t tot = n_y + n_a + n_l + n_t + n_s + n_r + n_h;
+    S.blk = ((k + 2) * D.d_ff + 2 * r + k + 7) / 8 * 8;
+    const size_t n_y = (size_t)L * D.d_model, n_b = (size_t)L * S.blk, n_r = (size_t)L * E, n_h = (size_t)L * E;
+    const size_t tot = n_y + n_b + n_r + n_h;
     int rc = dalloc(&S.tbuf, tot);
     if (rc) return rc;
     CK(cudaMemset(S.tbuf, 0, tot * 8));
     unsigned long long *p = S.tbuf;
     S.t_y = p; p += n_y;
-    S.t_a = p; p += n_a;
-    S.t_lora = p; p += n_l;
-    S.t_tdp = p; p += n_t;
-    S.t_rsel = p; p += n_s;
+    S.t_blk = p; p += n_b;
     S.t_rlog = p; p += n_r;
     S.t_hlog = p;
   }
@@ -735,11 +731,11 @@ static int decode_persistent(e0_ctx *C, const uint16_t *h, int step, uint16_t *y
   P.hist_out = hist_at(C, cur, 0);
   P.hist_prev = step > 0 ? hist_at(C, prv, 0) : nullptr;
   P.maxT = C->maxT;
-  P.t_y = S.t_y; P.t_a = S.t_a; P.t_lora = S.t_lora; P.t_tdp = S.t_tdp;
-  P.t_rsel = S.t_rsel; P.t_rlog = S.t_rlog; P.t_hlog = S.t_hlog;
+  P.t_y = S.t_y; P.t_blk = S.t_blk; P.blk = S.blk; P.t_rlog = S.t_rlog; P.t_hlog = S.t_hlog;
   P.err = C->err;
   P.timeout_ns = S.timeout_ns;
   P.stall_cta = S.stall_cta;
+  P.trace = S.trace;
   S.stall_cta = -1;
   int which;
   decode_geometry(D, &which);
@@ -834,6 +830,14 @@ extern "C" int e0_debug_fail_staging_after(e0_ctx *C, int n) {
   if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
   C->pool.fail_after = n;
   return E0_OK;
+}
+
+// Profiling: the next persistent decode launches write %globaltimer stamps into `buf`
+// ([grid][L][16] uint64, caller-owned device memory; NULL turns it off).  Returns the grid.
+extern "C" int e0_debug_decode_trace(e0_ctx *C, unsigned long long *buf) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  C->dec.trace = buf;
+  return C->nsm;
 }
 
 // Select the decode implementation: 1 = general per-layer kernels only (comparisons).
