@@ -182,6 +182,30 @@ int e0_get_stats(e0_ctx *ctx, e0_stats *out);
  * (DEVICE, SLOT_MISMATCH, TIMEOUT); the error word is cleared. */
 int e0_sync_status(e0_ctx *ctx);
 
+/* One MoE block, like e0_moe_layer_forward, for callers that cannot allocate device memory:
+ * a serving runtime that fixes its memory plan at start-up and forbids allocation later,
+ * code that runs while another component owns the device allocator, or code that must not
+ * risk the device synchronisation an allocation can cause.  No context is needed and
+ * nothing is allocated (no cudaMalloc, cudaFree or allocating library call).  The pages
+ * have no counterpart of this call.
+ * dims, layer   host structs as for e0_create / e0_register_model (layer->experts required).
+ * h, T, route_idx, y_bf16, y_f32, idx_out, gate_out   as for e0_moe_layer_forward.
+ * dev_status    device int or NULL: the kernels OR their error bits into it (1 = index out
+ *               of range, 2 = duplicated index); the caller zeroes it.  With NULL, device
+ *               errors are not reported.
+ * Scratch: one fixed 4 MiB device array inside the library (every GPU that loads the
+ * library holds it until the process exits).  A call whose intermediates do not fit is
+ * rejected with E0_ERR_INVALID_ARG and a message naming the bytes needed (at d = 2048,
+ * E = 256, I = 512, k = 4, r = 16 the limit is about T = 200 tokens).  The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress); make that first
+ * call outside any stream capture.  All calls share the one array and each overwrites it:
+ * calls on one device whose work overlaps on the GPU (for example on two streams)
+ * race and give wrong results, so serialise them.
+ * Errors: INVALID_ARG (arguments, sizes beyond the maximum), CUDA. */
+int e0_moe_layer_forward_noalloc(const e0_dims *dims, const e0_layer *layer, const void *h, int T,
+                                 const int32_t *route_idx, void *y_bf16, float *y_f32, int32_t *idx_out,
+                                 float *gate_out, int *dev_status, void *stream);
+
 /* Host-side fault injection for tests (no GPU fault is involved):
  * e0_debug_fail_staging_after(ctx, n): the (n+1)-th next staging copy is refused, so the
  *   staging call returns E0_ERR_STAGING.

@@ -72,6 +72,8 @@ _SIGS = {
     "e0_get_stats": (_I, [_P, ctypes.POINTER(Stats)]),
     "e0_sync_status": (_I, [_P]),
     "e0_last_error": (ctypes.c_char_p, []),
+    "e0_moe_layer_forward_noalloc": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Layer), _P, _I, _P, _P, _P, _P,
+                                          _P, _P, _P]),
     "e0_debug_fail_staging_after": (_I, [_P, _I]),
     "e0_debug_set_slot_tag": (_I, [_P, _I, _I, _I]),
     "e0_debug_decode_stall": (_I, [_P, _I, ctypes.c_ulonglong]),
@@ -116,6 +118,23 @@ def _stream(stream) -> int:
 
 def make_dims(d, E, I, k, r, head_hidden=0, head_onehot=0, eps=1e-6, lora_scale=1.0) -> Dims:
     return Dims(d, E, I, k, 64, r, head_hidden, head_onehot, eps, lora_scale)
+
+
+def moe_layer_forward_noalloc(dims: Dims, layer: dict, h, route_idx=None, y=None, y_f32=None, idx=None,
+                              gates=None, dev_status=None, stream=None):
+    """One MoE block without any device allocation by the library (see the C header).
+    `layer` is a dict of torch tensors as for Context.register_model."""
+    import torch
+    L = Layer()
+    for f, _ in Layer._fields_:
+        setattr(L, f, _ptr(layer.get(f)))
+    T = h.shape[0]
+    if y is None:
+        y = torch.empty((T, dims.d_model), dtype=torch.bfloat16, device=h.device)
+    _check(lib().e0_moe_layer_forward_noalloc(ctypes.byref(dims), ctypes.byref(L), _ptr(h), T, _ptr(route_idx),
+                                              _ptr(y), _ptr(y_f32), _ptr(idx), _ptr(gates), _ptr(dev_status),
+                                              _stream(stream)))
+    return y
 
 
 class Context:

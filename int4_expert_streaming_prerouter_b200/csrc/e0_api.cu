@@ -857,3 +857,127 @@ extern "C" int e0_debug_set_slot_tag(e0_ctx *C, int pool_set, int slot, int expe
   C->pool.corrupt_tag = expert;
   return E0_OK;
 }
+
+// ---------------------------------------------------------------------------------------
+// One MoE block without any allocation.
+//
+// Some callers cannot call cudaMalloc: a serving runtime that fixes its whole memory plan at
+// start-up and forbids allocation afterwards, code that runs while another component owns
+// the device allocator, or code that must not trigger the implicit device synchronisation
+// an allocation can cause.  This entry point needs no context and allocates nothing: its
+// intermediates live in one file-scope device array of fixed size, which every GPU that
+// loads this library holds until the process exits.
+// ---------------------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+static constexpr int kNoAllocMaxDevices = 64;
+// Device address of g_noalloc_scratch per device (the host-side symbol is not an address a
+// kernel may use), and the SM count, filled by the first call on each device.
+static unsigned char *g_noalloc_dev[kNoAllocMaxDevices];
+static int g_noalloc_nsm[kNoAllocMaxDevices];
+
+static size_t noalloc_align(size_t v) { return (v + 255) & ~(size_t)255; }
+
+extern "C" int e0_moe_layer_forward_noalloc(const e0_dims *dims, const e0_layer *layer, const void *h, int T,
+                                            const int32_t *route_idx, void *y_bf16, float *y_f32,
+                                            int32_t *idx_out, float *gate_out, int *dev_status, void *stream) {
+  if (!dims || !layer || !h || !y_bf16 || T < 1) return fail(E0_ERR_INVALID_ARG, "noalloc forward: bad arguments");
+  if (!supported(*dims) || dims->head_hidden < 0)
+    return fail(E0_ERR_INVALID_ARG, "noalloc forward: unsupported dims");
+  const e0_layer &Y = *layer;
+  if (!Y.experts || !Y.shared || !Y.router_w || !Y.norm_w)
+    return fail(E0_ERR_INVALID_ARG, "noalloc forward: experts, shared, router_w and norm_w are required");
+  const bool any = Y.lora_Ag || Y.lora_Bg || Y.lora_Au || Y.lora_Bu || Y.lora_Ad || Y.lora_Bd;
+  const bool all = Y.lora_Ag && Y.lora_Bg && Y.lora_Au && Y.lora_Bu && Y.lora_Ad && Y.lora_Bd;
+  if (any && (!all || dims->lora_rank < 1))
+    return fail(E0_ERR_INVALID_ARG, "noalloc forward: LoRA needs all six matrices and lora_rank >= 1");
+  const e0_dims &D = *dims;
+  const size_t d = D.d_model, E = D.n_experts, I = D.d_ff, k = D.top_k, r = D.lora_rank > 0 ? D.lora_rank : 1;
+  // scratch layout (each region 256-byte aligned)
+  size_t off = 0;
+  const size_t o_err = off;    off += noalloc_align(sizeof(int));
+  const size_t o_xb = off;     off += noalloc_align((size_t)T * d * 2);
+  const size_t o_xf = off;     off += noalloc_align((size_t)T * d * 4);
+  const size_t o_log = off;    off += noalloc_align((size_t)T * E * 4);
+  const size_t o_lt = off;     off += noalloc_align((size_t)T * 3 * r * 4);
+  const size_t o_idx = off;    off += noalloc_align((size_t)T * k * 4);
+  const size_t o_gate = off;   off += noalloc_align((size_t)T * k * 4);
+  const size_t o_a = off;      off += noalloc_align((size_t)T * (k + 1) * I * 2);
+  const size_t o_plan = off;   off += noalloc_align((1 + 2 * E + 1 + (size_t)T * k) * 4);
+  if (off > kNoAllocScratchBytes)
+    return fail(E0_ERR_INVALID_ARG,
+                "noalloc forward: T=%d needs %zu bytes of scratch, the fixed maximum is %zu bytes", T, off,
+                kNoAllocScratchBytes);
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(E0_ERR_INVALID_ARG, "noalloc forward: device %d", dev);
+  if (!g_noalloc_dev[dev]) {
+    // one-time set-up on this device (must not run inside a stream capture)
+    void *p = nullptr;
+    CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    int nsm = 0;
+    CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    g_noalloc_nsm[dev] = nsm;
+    g_noalloc_dev[dev] = (unsigned char *)p;
+  }
+  unsigned char *base = g_noalloc_dev[dev];
+  const int nsm = g_noalloc_nsm[dev];
+  cudaStream_t s = (cudaStream_t)stream;
+  int *err = dev_status ? dev_status : (int *)(base + o_err);
+  if (!dev_status) CK(cudaMemsetAsync(err, 0, sizeof(int), s));
+  uint16_t *xb = (uint16_t *)(base + o_xb);
+  float *xf = (float *)(base + o_xf), *logits = (float *)(base + o_log), *lt = (float *)(base + o_lt);
+  int32_t *idx = idx_out ? idx_out : (int32_t *)(base + o_idx);
+  float *gates = gate_out ? gate_out : (float *)(base + o_gate);
+  uint16_t *a = (uint16_t *)(base + o_a);
+  int32_t *pm = (int32_t *)(base + o_plan);
+  Plan plan{pm, pm + 1, pm + 1 + E, pm + 2 + 2 * E};
+  const int full_mode = route_idx ? 2 : 1;
+#define NOALLOC_CKL(what)                                                                    \
+  do {                                                                                     \
+    cudaError_t e_ = cudaGetLastError();                                                   \
+    if (e_ != cudaSuccess) return fail(E0_ERR_CUDA, "launch %s: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+  k_norm<<<T, 256, 0, s>>>((const uint16_t *)h, nullptr, (const uint16_t *)Y.norm_w, D.d_model, D.rms_eps, xb, xf);
+  NOALLOC_CKL("k_norm");
+  RowsArgs R{};
+  R.xf = xf; R.T = T; R.d = D.d_model; R.E = D.n_experts; R.k = D.top_k;
+  R.Wr = (const uint16_t *)Y.router_w; R.logits = logits; R.route = route_idx; R.full_mode = full_mode;
+  R.Wh = nullptr; R.hlog = nullptr;
+  R.Ag = (const uint16_t *)Y.lora_Ag; R.Au = (const uint16_t *)Y.lora_Au; R.r = D.lora_rank; R.lt = lt; R.err = err;
+  const int nTT = (T + kRowTile - 1) / kRowTile;
+  const int J = D.n_experts * nTT + T * D.top_k + (R.Ag ? 2 * D.lora_rank * nTT : 0);
+  k_rows<<<grid_for(J, 8 * nsm), 256, 0, s>>>(R);
+  NOALLOC_CKL("k_rows");
+  RouteArgs A{};
+  A.logits = logits; A.T = T; A.E = D.n_experts; A.k = D.top_k; A.route = route_idx; A.full_mode = full_mode;
+  A.idx = idx; A.gates = gates; A.err = err;
+  k_route<<<(T + 7) / 8, 256, 0, s>>>(A);
+  NOALLOC_CKL("k_route");
+  k_plan<<<1, 1024, 0, s>>>(idx, T * D.top_k, D.n_experts, plan);
+  NOALLOC_CKL("k_plan");
+  ExpertSrc src{};
+  src.resident = (const uint8_t *)Y.experts;
+  src.stride = blob_of(D.d_model, D.d_ff).bytes;
+  src.err = err;
+  GateUpArgs G{};
+  G.xf = xf; G.T = T; G.d = D.d_model; G.I = D.d_ff; G.k = D.top_k; G.r = D.lora_rank; G.c = D.lora_scale;
+  G.src = src; G.shared = (const uint8_t *)Y.shared; G.bl = blob_of(D.d_model, D.d_ff); G.P = plan;
+  G.Bg = (const uint16_t *)Y.lora_Bg; G.Bu = (const uint16_t *)Y.lora_Bu; G.lt = lt; G.a = a;
+  const int items = (std::min(D.n_experts, T * D.top_k) + 1) * D.d_ff;
+  k_gateup<<<grid_for(items, 4 * nsm), 256, 0, s>>>(G);
+  NOALLOC_CKL("k_gateup");
+  if (Y.lora_Ad) {
+    k_lora_t<<<(T * D.lora_rank + 7) / 8, 256, 0, s>>>((const uint16_t *)Y.lora_Ad, a, T, D.d_ff, D.top_k,
+                                                        D.lora_rank, lt);
+    NOALLOC_CKL("k_lora_t");
+  }
+  DownArgs W{};
+  W.T = T; W.d = D.d_model; W.I = D.d_ff; W.k = D.top_k; W.r = D.lora_rank; W.c = D.lora_scale;
+  W.src = src; W.shared = (const uint8_t *)Y.shared; W.bl = blob_of(D.d_model, D.d_ff); W.idx = idx; W.gates = gates;
+  W.a = a; W.Bd = (const uint16_t *)Y.lora_Bd; W.lt = lt; W.y = (uint16_t *)y_bf16; W.yf = y_f32;
+  k_down<<<grid_for(T * D.d_model, 4 * nsm), 256, 0, s>>>(W);
+  NOALLOC_CKL("k_down");
+#undef NOALLOC_CKL
+  return E0_OK;
+}
