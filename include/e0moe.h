@@ -171,6 +171,17 @@ int e0_stage_experts(e0_ctx *ctx, int layer, const int32_t *host_idx, int n, voi
 int e0_moe_stack_decode(e0_ctx *ctx, const void *h_in, int B, int step, void *y_out, float *y_f32,
                         int streaming, int chained, void *stream);
 
+/* One prefill chunk of T tokens through all layers ([G] "Temel fikirler", "Sorular":
+ * prediction as routing, one token ahead).  h_in [L, T, d] bf16 (each layer's generated
+ * MoE input), y_out [L, T, d] bf16, y_f32 [L, T, d] or NULL, idx_out [L, T, k] int32 or
+ * NULL (the routing each layer used).  Layer N+1 routes token t by the head of layer N
+ * on token t-1; token 0, and every layer not preceded by a head, use their own router.
+ * From 64 tokens the experts run as tcgen05 grouped GEMMs (fp16 operands from the int4
+ * weights, fp32 accumulation).  Linear heads without one-hot inputs only.
+ * Errors: INVALID_ARG, CUDA. */
+int e0_moe_prefill_stack(e0_ctx *ctx, const void *h_in, int T, void *y_out, float *y_f32, int32_t *idx_out,
+                         void *stream);
+
 /* Routing the last e0_moe_stack_decode used and predicted, copied to host memory:
  * idx [L, B, k] (routing used at that step), pred [L, B, k] (next step's routing; -1 for
  * layers without a head).  Synchronises the context's last stream. */
@@ -222,6 +233,10 @@ int e0_debug_set_slot_tag(e0_ctx *ctx, int pool_set, int slot, int expert);
  * e0_debug_force_general(ctx, on): 1 sends every decode step through the per-layer
  *   kernels instead of the one-launch kernel (for comparisons); 0 restores the default. */
 int e0_debug_decode_stall(e0_ctx *ctx, int cta, unsigned long long timeout_ns);
+/* Expert path of e0_moe_layer_forward: 0 = tensor cores (tcgen05) from 64 tokens per call,
+ * CUDA cores below (default); 1 = CUDA cores always; 2 = tensor cores whenever the context
+ * was created with max_tokens >= 64.  For comparisons between the two paths. */
+int e0_debug_prefill_path(e0_ctx *ctx, int mode);
 /* Profiling: the following one-launch decode steps write %globaltimer stamps (uint64,
  * [grid][L][16], caller-owned device buffer; NULL stops it).  Returns the grid size. */
 int e0_debug_decode_trace(e0_ctx *ctx, unsigned long long *buf);

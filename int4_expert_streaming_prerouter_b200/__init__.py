@@ -69,6 +69,7 @@ _SIGS = {
     "e0_stage_experts": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int32), _I, _P]),
     "e0_moe_stack_decode": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
     "e0_get_routing": (_I, [_P, _I, _P, _P]),
+    "e0_moe_prefill_stack": (_I, [_P, _P, _I, _P, _P, _P, _P]),
     "e0_get_stats": (_I, [_P, ctypes.POINTER(Stats)]),
     "e0_sync_status": (_I, [_P]),
     "e0_last_error": (ctypes.c_char_p, []),
@@ -79,6 +80,7 @@ _SIGS = {
     "e0_debug_decode_stall": (_I, [_P, _I, ctypes.c_ulonglong]),
     "e0_debug_force_general": (_I, [_P, _I]),
     "e0_debug_decode_trace": (_I, [_P, _P]),
+    "e0_debug_prefill_path": (_I, [_P, _I]),
 }
 
 
@@ -226,6 +228,16 @@ class Context:
                                          int(streaming), int(chained), _stream(stream)))
         return y_out
 
+    def prefill_stack(self, h_in, y_out=None, y_f32=None, idx=None, stream=None):
+        """h_in [L, T, d] bf16 -> y_out [L, T, d] bf16 (prediction-as-routing, one token ahead)."""
+        import torch
+        L, T, d = h_in.shape
+        if y_out is None:
+            y_out = torch.empty((L, T, d), dtype=torch.bfloat16, device=h_in.device)
+        _check(lib().e0_moe_prefill_stack(self._h, _ptr(h_in), T, _ptr(y_out), _ptr(y_f32), _ptr(idx),
+                                          _stream(stream)))
+        return y_out
+
     def get_routing(self, B):
         import numpy as np
         k = self.dims.top_k
@@ -255,6 +267,9 @@ class Context:
     def debug_decode_trace(self, buf):
         """buf: int64 CUDA tensor [grid, L, 16] or None; returns the grid size."""
         return lib().e0_debug_decode_trace(self._h, _ptr(buf))
+
+    def debug_prefill_path(self, mode: int):
+        _check(lib().e0_debug_prefill_path(self._h, mode))
 
     def debug_force_general(self, on: bool):
         _check(lib().e0_debug_force_general(self._h, int(on)))

@@ -5,6 +5,7 @@
 #include "e0moe.h"
 #include "e0_kernels.cuh"
 #include "e0_decode.cuh"
+#include "e0_prefill.cuh"
 
 #include <cstdarg>
 #include <cstdio>
@@ -106,6 +107,15 @@ struct e0_ctx {
   cudaStream_t last = nullptr;
   int last_step = -1, last_B = 0;
   bool force_general = false;        // route decode through the general per-layer kernels
+  int prefill_path = 0;              // 0: tensor cores from kTcMinTokens tokens, 1: CUDA cores, 2: tensor cores
+  // tensor-core prefill workspaces
+  __half *x16 = nullptr, *a16 = nullptr;
+  float *yacc = nullptr;
+  TcTile *tiles = nullptr;
+  int *ntiles = nullptr;
+  int tile_cap = 0;
+  int32_t *pf_buf = nullptr;         // prefill: [2][maxT+1][k] head predictions, row 0 = -1
+  int32_t *pf_idx = nullptr;         // prefill: [maxT+1][k] routing scratch, row 0 = -1
   DecodeState dec{};
   StreamPool pool;
   e0_stats stats{};
@@ -135,7 +145,7 @@ extern "C" int e0_destroy(e0_ctx *C) {
   cudaDeviceSynchronize();
   void *bufs[] = {C->xb, C->xf, C->logits, C->hlog, C->lt, C->gates, C->idx, C->a, C->plan_mem,
                   C->yscratch, C->pred_tab, C->hist_tab, C->err, C->h1pre, C->h1, C->pool.mem, C->pool.slot_of,
-                  C->pool.slot_tag};
+                  C->pool.slot_tag, C->x16, C->a16, C->yacc, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
   for (void *b : bufs)
     if (b) cudaFree(b);
   decode_free(C->dec);
@@ -176,6 +186,20 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
                                  (rc = dalloc(&C->h1, T * dims->head_hidden))))) {
     e0_destroy(C);
     return rc;
+  }
+  if ((rc = dalloc(&C->pf_buf, 2 * (T + 1) * k)) || (rc = dalloc(&C->pf_idx, (T + 1) * k))) {
+    e0_destroy(C);
+    return rc;
+  }
+  cudaMemset(C->pf_buf, 0xFF, 2 * (T + 1) * k * sizeof(int32_t));
+  cudaMemset(C->pf_idx, 0xFF, (T + 1) * k * sizeof(int32_t));
+  if (T >= kTcMinTokens) {
+    C->tile_cap = (int)((T * k + kTcN - 1) / kTcN + std::min(E, T * k) + (T + kTcN - 1) / kTcN + 1);
+    if ((rc = dalloc(&C->x16, T * d)) || (rc = dalloc(&C->a16, T * (k + 1) * I)) || (rc = dalloc(&C->yacc, T * d)) ||
+        (rc = dalloc(&C->tiles, (size_t)C->tile_cap)) || (rc = dalloc(&C->ntiles, 1))) {
+      e0_destroy(C);
+      return rc;
+    }
   }
   C->plan.U = C->plan_mem;
   C->plan.uexp = C->plan_mem + 1;
@@ -278,11 +302,54 @@ static int layer_pre(e0_ctx *C, const LayerCall &K, cudaStream_t s) {
   return E0_OK;
 }
 
+// The experts of one layer on the tensor cores (grouped tcgen05 GEMMs); used for prefill.
+static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cudaStream_t s) {
+  const e0_dims &D = C->dims;
+  const e0_layer &Y = C->layers[K.l];
+  const size_t nx = (size_t)K.T * D.d_model;
+  k_bf16_to_f16<<<(unsigned)((nx + 255) / 256), 256, 0, s>>>(C->xb, C->x16, nx);
+  CKL("k_bf16_to_f16");
+  k_tc_tiles<<<1, 32, 0, s>>>(C->plan, K.T, C->tiles, C->ntiles, C->tile_cap);
+  CKL("k_tc_tiles");
+  TcArgs A{};
+  A.mode = 0; A.T = K.T; A.d = D.d_model; A.I = D.d_ff; A.k = D.top_k; A.r = D.lora_rank; A.c = D.lora_scale;
+  A.src = src; A.shared = (const uint8_t *)Y.shared; A.bl = C->bl; A.P = C->plan; A.tiles = C->tiles;
+  A.ntiles = C->ntiles; A.x16 = C->x16; A.a16 = C->a16; A.a16_out = C->a16;
+  A.Bg = (const uint16_t *)Y.lora_Bg; A.Bu = (const uint16_t *)Y.lora_Bu; A.lt = C->lt; A.gates = K.gates;
+  A.yacc = C->yacc; A.err = C->err; A.timeout_ns = 2000000000ull;
+  const int tc_smem_bytes = (int)sizeof(TcSmem) + 1024;
+  static bool attr_done = false;
+  if (!attr_done) {
+    CK(cudaFuncSetAttribute(k_moe_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem_bytes));
+    attr_done = true;
+  }
+  const int tmax = std::min(C->tile_cap, (K.T * D.top_k + kTcN - 1) / kTcN + std::min(D.n_experts, K.T * D.top_k) +
+                                              (K.T + kTcN - 1) / kTcN);
+  k_moe_gemm_tc<<<tmax * (D.d_ff / 64), kTcThreads, tc_smem_bytes, s>>>(A);
+  CKL("k_moe_gemm_tc(gate/up)");
+  if (Y.lora_Ad) {
+    k_lora_t16<<<(K.T * D.lora_rank + 7) / 8, 256, 0, s>>>((const uint16_t *)Y.lora_Ad, C->a16, K.T, D.d_ff,
+                                                            D.top_k, D.lora_rank, C->lt);
+    CKL("k_lora_t16");
+  }
+  CK(cudaMemsetAsync(C->yacc, 0, nx * sizeof(float), s));
+  A.mode = 1;
+  k_moe_gemm_tc<<<tmax * (D.d_model / 128), kTcThreads, tc_smem_bytes, s>>>(A);
+  CKL("k_moe_gemm_tc(down)");
+  k_tc_finish<<<(unsigned)((nx + 255) / 256), 256, 0, s>>>(C->yacc, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
+                                                           D.d_model, D.lora_rank, D.lora_scale, K.y, K.yf);
+  CKL("k_tc_finish");
+  return E0_OK;
+}
+
 static int layer_post(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cudaStream_t s) {
   const e0_dims &D = C->dims;
   const e0_layer &Y = C->layers[K.l];
   k_plan<<<1, 1024, 0, s>>>(K.idx, K.T * D.top_k, D.n_experts, C->plan);
   CKL("k_plan");
+  const bool tc = C->x16 && src.pool == nullptr && D.d_model % 128 == 0 && D.d_ff % 64 == 0 &&
+                  (C->prefill_path == 2 || (C->prefill_path == 0 && K.T >= kTcMinTokens));
+  if (tc) return layer_post_tc(C, K, src, s);
   GateUpArgs G{};
   G.xf = C->xf; G.T = K.T; G.d = D.d_model; G.I = D.d_ff; G.k = D.top_k; G.r = D.lora_rank; G.c = D.lora_scale;
   G.src = src; G.shared = (const uint8_t *)Y.shared; G.bl = C->bl; G.P = C->plan;
@@ -783,6 +850,46 @@ extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step,
   return E0_OK;
 }
 
+// One prefill chunk through every layer.  Layer N+1's routing of token t is the head of
+// layer N on token t-1 (prediction as routing, one token ahead); token 0, and layers after
+// a layer without a head, route with their own router.  Linear heads without one-hot
+// inputs (the workloads' form).
+extern "C" int e0_moe_prefill_stack(e0_ctx *C, const void *h_in, int T, void *y_out, float *y_f32, int32_t *idx_out,
+                                    void *stream) {
+  if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
+  if (!h_in || !y_out || T < 1 || T > C->maxT)
+    return fail(E0_ERR_INVALID_ARG, "e0_moe_prefill_stack: bad arguments (T=%d, max %d)", T, C->maxT);
+  if (C->dims.head_hidden > 0 || C->dims.head_onehot)
+    return fail(E0_ERR_INVALID_ARG, "prefill stack supports the linear head without one-hot inputs");
+  for (int l = 0; l < C->L; l++)
+    if (!C->layers[l].experts) return fail(E0_ERR_INVALID_ARG, "layer %d has no resident experts", l);
+  cudaStream_t s = (cudaStream_t)stream;
+  C->last = s;
+  const e0_dims &D = C->dims;
+  const int k = D.top_k;
+  const size_t ld = (size_t)T * D.d_model;
+  for (int l = 0; l < C->L; l++) {
+    const bool predicted = l > 0 && C->heads[l - 1].w_lin != nullptr;
+    int32_t *pin = C->pf_buf + (size_t)((l + 1) & 1) * (C->maxT + 1) * k;   // written by layer l-1's head
+    int32_t *pout = C->pf_buf + (size_t)(l & 1) * (C->maxT + 1) * k;
+    LayerCall K{};
+    K.l = l; K.T = T; K.h = (const uint16_t *)h_in + l * ld;
+    K.route = predicted ? pin : nullptr;          // row t = prediction made on token t-1
+    K.full_mode = predicted ? 2 : 1;              // row 0 is -1: token 0 uses its own router
+    K.idx = idx_out ? idx_out + (size_t)l * T * k : C->pf_idx + k;
+    K.gates = C->gates;
+    K.head = C->heads[l].w_lin != nullptr;
+    K.prev = nullptr;
+    K.pred = pout + k;                             // prediction of token t -> row t+1
+    K.y = (uint16_t *)y_out + l * ld;
+    K.yf = y_f32 ? y_f32 + l * ld : nullptr;
+    int rc = layer_pre(C, K, s);
+    if (rc) return rc;
+    if ((rc = layer_post(C, K, resident_src(C, l), s))) return rc;
+  }
+  return E0_OK;
+}
+
 extern "C" int e0_get_routing(e0_ctx *C, int B, int32_t *idx_host, int32_t *pred_host) {
   if (!C || C->last_step < 0 || B != C->last_B) return fail(E0_ERR_INVALID_ARG, "no decode step with this B");
   CK(cudaStreamSynchronize(C->last));
@@ -838,6 +945,14 @@ extern "C" int e0_debug_decode_trace(e0_ctx *C, unsigned long long *buf) {
   if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
   C->dec.trace = buf;
   return C->nsm;
+}
+
+// Select the expert path of e0_moe_layer_forward: 0 = tensor cores from kTcMinTokens
+// tokens (default), 1 = CUDA-core kernels, 2 = tensor cores whenever the context has them.
+extern "C" int e0_debug_prefill_path(e0_ctx *C, int mode) {
+  if (!C || mode < 0 || mode > 2) return fail(E0_ERR_INVALID_ARG, "bad prefill path");
+  C->prefill_path = mode;
+  return E0_OK;
 }
 
 // Select the decode implementation: 1 = general per-layer kernels only (comparisons).

@@ -71,7 +71,7 @@ def compare_steps(dims, gpu, ref, chained=False):
     for t in range(S):
         for n in range(L):
             check_y(y32[t, n], ref["y"][t, n], f"step {t} layer {n}")
-            check_bf16(yb[t, n], ref["y"][t, n], f"step {t} layer {n}")
+            check_bf16(yb[t, n], ref["y"][t, n], f"step {t} layer {n}", y32[t, n])
 
 
 @pytest.mark.parametrize("B", [1, 5])

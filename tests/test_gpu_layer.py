@@ -72,7 +72,7 @@ def compare(dims, out_gpu, ref, what):
     for t in range(idx.shape[0]):
         assert idx_ok(idx[t], ref["logits"][t], ref["idx"][t], dims.k), (what, t, idx[t], ref["idx"][t])
     check_y(y32, ref["y"], what)
-    check_bf16(yb, ref["y"], what)
+    check_bf16(yb, ref["y"], what, y32)
     assert np.allclose(gates, ref["gates"], rtol=1e-5, atol=1e-6), what
 
 
@@ -228,3 +228,70 @@ def test_out_of_range_and_duplicate_routes_are_flagged(cfg1):
     assert ei.value.status == "DEVICE"
     cfg1.moe_layer_forward(0, h)
     cfg1.sync_status()          # the error word was cleared
+
+
+# ---------------------------------------------------------------------------------------
+# prefill: the experts on the tensor cores (tcgen05 grouped GEMMs)
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("T", [64, 300])
+def test_prefill_tensor_core_path_small(cuda_ok, T):
+    """Many tokens per expert (E=16): tiles of 128 tokens, ragged tails, shared expert over
+    all T tokens; checked against the oracle and against the CUDA-core path."""
+    ctx, _, _ = make_ctx(CFG1, 200 + T, 512)
+    h = synth.hidden(200 + T, 0, 1, T, CFG1.d)[0]
+    ctx.debug_prefill_path(2)
+    out = run_layer(ctx, CFG1, 200 + T, 0, h)
+    ref = oracle_layer(CFG1, 200 + T, 0, h, gpu_idx=out[2])
+    compare(CFG1, out, ref, f"tc T={T}")
+    ctx.debug_prefill_path(1)
+    out_cc = run_layer(ctx, CFG1, 200 + T, 0, h)
+    assert np.array_equal(out[2], out_cc[2])
+    check_y(out[1], out_cc[1], "tc vs cuda cores")
+    ctx.close()
+
+
+def test_prefill_tensor_core_path_full_width_predicted_routing(cuda_ok):
+    """d=2048, E=256, I=512, r=16, T=512 with prediction-as-routing shifted by one token
+    (token 0 routes with its own router); sampled tokens checked against the oracle."""
+    dims = Dims(d=2048, E=256, I=512, k=4, r=16, L=1, head_layers=(0,))
+    ctx, _, _ = make_ctx(dims, 210, 512)
+    T = 512
+    h = synth.hidden(210, 0, 1, T, dims.d)[0]
+    rng = np.random.default_rng(210)
+    route = np.stack([rng.permutation(dims.E)[:dims.k] for _ in range(T)]).astype(np.int32)
+    route[0] = -1
+    ctx.debug_prefill_path(2)
+    out = run_layer(ctx, dims, 210, 0, h, route=route)
+    sample = [0, 1, 2, 255, 256, 511]
+    ref = oracle_layer(dims, 210, 0, h[sample], route=route[sample],
+                       gpu_idx=out[2][sample])
+    yb, y32, idx, gates = out
+    compare(dims, (yb[sample], y32[sample], idx[sample], gates[sample]), ref, "tc full width")
+    ctx.close()
+
+
+def test_prefill_stack_prediction_as_routing_shifted_one_token(cuda_ok):
+    """Three layers, T=160: layer N+1 routes token t with the head of layer N on token t-1,
+    token 0 and layer 0 with their own router; checked against the oracle layer by layer."""
+    dims = Dims(d=256, E=16, I=128, k=4, r=8, L=3, head_layers=(0, 1))
+    ctx, _, _ = make_ctx(dims, 220, 256)
+    T = 160
+    hs = np.stack([synth.hidden(220 + n, 0, 1, T, dims.d)[0] for n in range(dims.L)])
+    y32 = torch.empty((dims.L, T, dims.d), dtype=torch.float32, device="cuda")
+    idx = torch.empty((dims.L, T, dims.k), dtype=torch.int32, device="cuda")
+    yb = ctx.prefill_stack(bf16_tensor(hs, "cuda"), y_f32=y32, idx=idx)
+    ctx.sync_status()
+    idx = idx.cpu().numpy()
+    yb = bf16_bits_to_np(yb)
+    y32 = y32.cpu().numpy().astype(np.float64)
+    route = None
+    for n in range(dims.L):
+        dense = synth.layer_dense(220, n, dims)
+        ref = oracle_layer(dims, 220, n, hs[n], route=route, gpu_idx=idx[n])
+        compare(dims, (yb[n], y32[n], idx[n], np.zeros((T, dims.k))), dict(ref, gates=np.zeros((T, dims.k))), f"layer {n}")
+        if n in dims.head_layers:
+            preds = np.stack([O.prerouter_head(ref["x"][t], dense, dims)[1] for t in range(T)])
+            route = np.concatenate([np.full((1, dims.k), -1, np.int32), preds[:-1]])
+        else:
+            route = None
+    ctx.close()
