@@ -36,6 +36,23 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
+
+# DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, valid only
+# while the kernel source is the one captured (sha256 prefix of the file); see profiles/.
+KERNEL_TRAFFIC = {
+    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "7e50bdc194a50ca3", 427.0e6,
+                      "4-layer capture (42.64 MB for 40.6 MB algorithmic) scaled by algorithmic bytes"),
+}
+
+
+def kernel_traffic(workload):
+    import hashlib
+    ent = KERNEL_TRAFFIC.get(workload)
+    if not ent:
+        return None, None
+    path, digest, nbytes, how = ent
+    h = hashlib.sha256(open(os.path.join(ROOT, path), "rb").read()).hexdigest()
+    return (nbytes, how) if h.startswith(digest) else (None, "kernel changed since the capture")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
@@ -327,9 +344,12 @@ def run_decode(args, dims, seed, B, ws, rank, local):
                 "expert_GBps": achieved, "all_GBps": all_b / (step_ms / 1e3) / 1e9,
                 "frac_of_measured": achieved / pk["hbm_gbs"], "frac_of_8TBps": achieved / 8000.0},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                     "kernel": "whole decode step (all kernels of one token), expert bytes only",
-                     "peak_source": pk["source"]},
+                     "frac": achieved / pk["hbm_gbs"], "traffic": kernel_traffic(args.workload)[0],
+                     "traffic_note": kernel_traffic(args.workload)[1],
+                     "kernel": ("k_decode (one launch = one decode step, CUDA events on its stream); "
+                                "achieved counts int4 expert bytes only" if B == 1 else
+                                "per-layer kernels of one decode step; achieved counts int4 expert bytes"),
+                     "peak_source": pk["source"] + " copy bandwidth (burst)"},
         "clocks": clk.summary(),
         "setup_s": setup_s,
     }
@@ -407,11 +427,95 @@ def run_prefill(args, dims, seed, ws, rank, local):
     return out, ctx
 
 
+def h2d_probe_gbs(dev, nbytes=1 << 28):
+    """Pinned host -> device copy bandwidth (GB/s), measured once in this run."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        dst.copy_(src, non_blocking=True)
+    torch.cuda.synchronize()
+    e0_, e1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0_.record()
+    for _ in range(4):
+        dst.copy_(src, non_blocking=True)
+    e1_.record()
+    torch.cuda.synchronize()
+    return 4 * nbytes / (e0_.elapsed_time(e1_) / 1e3) / 1e9
+
+
+def run_stream(args, dims, seed, ws, rank, local):
+    """Streaming tier: experts in pinned host memory, staged into a 2 x k slot pool."""
+    import torch
+    import int4_expert_streaming_prerouter_b200 as e0
+    from synth.device import layer_tensors, bf16_tensor, pinned_expert_store
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    t0 = time.time()
+    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, 1)
+    lys, hds = zip(*[layer_tensors(seed, n, dims, dev, resident=False) for n in range(dims.L)])
+    ctx.register_model(list(lys), list(hds))
+    store = pinned_expert_store(seed, dims)
+    ctx.stream_register(store, pool_layers=2, slots_per_layer=dims.k)
+    setup_s = time.time() - t0
+    total = args.warmup + args.steps
+    h_all = torch.stack([bf16_tensor(synth.hidden(seed, t, dims.L, 1, dims.d), dev) for t in range(total)])
+    y = torch.empty((dims.L, 1, dims.d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for t in range(args.warmup):
+        ctx.stack_decode(h_all[t], t, y_out=y, streaming=True)
+    ctx.sync_status()
+    s0 = ctx.stats()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for t in range(args.warmup, total):
+            ctx.stack_decode(h_all[t], t, y_out=y, streaming=True)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ctx.sync_status()
+    s1 = ctx.stats()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), ws)
+    tokens = sum_over_ranks(args.steps, ws)
+    d = {k: s1[k] - s0[k] for k in s1}
+    link = h2d_probe_gbs(dev)
+    bytes_per_token = d["staged_bytes"] / args.steps
+    wall_s = ms / 1e3
+    out = {
+        "metric": "MoE-stack streaming decode tokens/s on 1 B200 (experts in pinned host memory)",
+        "value": tokens / wall_s, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4 weights, fp32 accumulate", "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "layers": dims.L, "batch": 1, "pool": f"2 layers x {dims.k} slots",
+                   "host_store_GB": round(store.numel() / 1e9, 2), "parallelism": f"replicas x{ws}"},
+        "gpu_launches": int(d["kernel_launches"]),
+        "streaming": {"host_link_bytes_per_token": bytes_per_token, "h2d_probe_GBps": link,
+                      "link_GBps": bytes_per_token * tokens / wall_s / 1e9,
+                      "link_frac": bytes_per_token * tokens / wall_s / 1e9 / link,
+                      "stage_ms_per_token": d["stage_ms"] / args.steps,
+                      "exposed_wait_ms_per_token": d["exposed_wait_ms"] / args.steps,
+                      "hidden_frac_of_staging": 1.0 - d["exposed_wait_ms"] / max(d["stage_ms"], 1e-9),
+                      "link_busy_frac_of_wall": d["stage_ms"] / max(ms, 1e-9),
+                      "prefetched_experts": int(d["prefetched_experts"]),
+                      "ondemand_experts": int(d["ondemand_experts"]), "dropped": int(d["dropped"]),
+                      "hbm_pool_MB": 2 * dims.k * synth.blob_bytes(dims.d, dims.I) / 1e6},
+        "roofline": {"bound": "host link", "achieved": bytes_per_token * tokens / wall_s / 1e9, "peak": link,
+                     "unit": "GB/s", "frac": bytes_per_token * tokens / wall_s / 1e9 / link, "traffic": None,
+                     "kernel": "staging copies (copy engine)", "peak_source": "pinned H2D probe in this run"},
+        "clocks": clk.summary(), "setup_s": setup_s,
+    }
+    return out, ctx
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64)
-    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--steps", type=int, default=1024)
+    ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--workload", default="decode_b1_l40")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -423,6 +527,12 @@ def main():
                                                                 int(os.environ.get("RANK", "0")), 0)
     if args.impl == "reference":
         run_reference(args, dims, seed, ws, rank)
+        return
+    if args.workload.startswith("stream"):
+        out, ctx = run_stream(args, dims, seed, ws, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        ctx.close()
         return
     if "tokens" in wl:
         out, ctx = run_prefill(args, dims, seed, ws, rank, local)

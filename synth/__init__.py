@@ -209,6 +209,9 @@ WORKLOADS = {
     "decode_multistream_l40": dict(dims=_full(), seed=2, batch=(8, 32, 64), steps=128),
     "prefill_t4096_l40": dict(dims=_full(), seed=3, tokens=4096),
     "stream_b1_l40": dict(dims=_full(), seed=4, batch=1, steps=256),
+    # the same geometry on a few layers: small cases for profiler captures
+    "decode_b1_l4": dict(dims=_full(L=4, head_layers=(0, 1, 2)), seed=1, batch=1, steps=16),
+    "prefill_t4096_l2": dict(dims=_full(L=2, head_layers=(0,)), seed=3, tokens=4096),
 }
 
 
