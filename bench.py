@@ -276,6 +276,7 @@ def run_decode(args, dims, seed, B, ws, rank, local):
         lys.append(ly)
         hds.append(hd)
     ctx.register_model(lys, hds)
+    ctx.debug_decode_mode(args.decode_mode)
     setup_s = time.time() - t0
     steps, warm = args.steps, args.warmup
     total = steps + warm
@@ -520,6 +521,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-mode", type=int, default=0, help="0 default, 1 one-launch, 2 graph, 3 eager")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     dims, seed = wl["dims"], wl["seed"]

@@ -237,6 +237,10 @@ int e0_debug_decode_stall(e0_ctx *ctx, int cta, unsigned long long timeout_ns);
  * CUDA cores below (default); 1 = CUDA cores always; 2 = tensor cores whenever the context
  * was created with max_tokens >= 64.  For comparisons between the two paths. */
 int e0_debug_prefill_path(e0_ctx *ctx, int mode);
+/* Decode implementation of e0_moe_stack_decode (resident experts): 0 = default (the
+ * one-launch kernel at B = 1, per-layer kernels otherwise),
+ * 1 = one-launch kernel, 2 = graph replay, 3 = per-layer kernels launched one by one. */
+int e0_debug_decode_mode(e0_ctx *ctx, int mode);
 /* Profiling: the following one-launch decode steps write %globaltimer stamps (uint64,
  * [grid][L][16], caller-owned device buffer; NULL stops it).  Returns the grid size. */
 int e0_debug_decode_trace(e0_ctx *ctx, unsigned long long *buf);

@@ -81,6 +81,7 @@ _SIGS = {
     "e0_debug_force_general": (_I, [_P, _I]),
     "e0_debug_decode_trace": (_I, [_P, _P]),
     "e0_debug_prefill_path": (_I, [_P, _I]),
+    "e0_debug_decode_mode": (_I, [_P, _I]),
 }
 
 
@@ -267,6 +268,9 @@ class Context:
     def debug_decode_trace(self, buf):
         """buf: int64 CUDA tensor [grid, L, 16] or None; returns the grid size."""
         return lib().e0_debug_decode_trace(self._h, _ptr(buf))
+
+    def debug_decode_mode(self, mode: int):
+        _check(lib().e0_debug_decode_mode(self._h, mode))
 
     def debug_prefill_path(self, mode: int):
         _check(lib().e0_debug_prefill_path(self._h, mode))

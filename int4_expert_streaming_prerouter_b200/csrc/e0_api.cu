@@ -84,6 +84,13 @@ static void decode_free(DecodeState &S) {
   S = DecodeState{};
 }
 
+// One captured decode step (the per-layer kernel sequence of every layer) and its key.
+struct DecodeGraph {
+  cudaGraphExec_t exec = nullptr;
+  int B = 0, parity = -1, step0 = -1, chained = -1, has_f32 = -1;
+  unsigned long long launches = 0;
+};
+
 struct e0_ctx {
   e0_dims dims{};
   int L = 0, maxT = 0, dev = 0, nsm = 0;
@@ -108,6 +115,12 @@ struct e0_ctx {
   int last_step = -1, last_B = 0;
   bool force_general = false;        // route decode through the general per-layer kernels
   int prefill_path = 0;              // 0: tensor cores from kTcMinTokens tokens, 1: CUDA cores, 2: tensor cores
+  int decode_mode = 0;               // 0 auto, 1 one-launch kernel, 2 graph of per-layer kernels, 3 eager
+  DecodeGraph graphs[6];
+  int graph_next = 0;
+  cudaStream_t cap = nullptr;        // private stream the decode graphs are captured on
+  uint16_t *g_h = nullptr, *g_y = nullptr;   // [L][maxT][d] graph input / output
+  float *g_yf = nullptr;                     // [L][maxT][d]
   // tensor-core prefill workspaces
   __half *x16 = nullptr, *a16 = nullptr;
   float *yacc = nullptr;
@@ -149,6 +162,11 @@ extern "C" int e0_destroy(e0_ctx *C) {
   for (void *b : bufs)
     if (b) cudaFree(b);
   decode_free(C->dec);
+  for (auto &g : C->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (C->cap) cudaStreamDestroy(C->cap);
+  for (void *b : {(void *)C->g_h, (void *)C->g_y, (void *)C->g_yf})
+    if (b) cudaFree(b);
   if (C->host_idx) cudaFreeHost(C->host_idx);
   for (auto *v : {&C->pool.ready, &C->pool.freed})
     for (auto e : *v) cudaEventDestroy(e);
@@ -246,6 +264,10 @@ extern "C" int e0_register_model(e0_ctx *C, const e0_layer *layers, const e0_hea
   if (heads) C->heads.assign(heads, heads + C->L);
   C->registered = true;
   C->dec.ready = false;
+  for (auto &g : C->graphs) {   // captured pointers belong to the previous registration
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    g = DecodeGraph{};
+  }
   return E0_OK;
 }
 
@@ -822,6 +844,56 @@ extern "C" int e0_debug_decode_stall(e0_ctx *C, int cta, unsigned long long time
   return E0_OK;
 }
 
+// The decode step as a replay of a captured CUDA graph of the per-layer kernels: the
+// caller's inputs are copied into fixed buffers, the graph runs on the caller's stream and
+// the outputs are copied back.  One graph per (B, step parity, first step, chained, fp32
+// output) is captured on first use.
+static int decode_graph(e0_ctx *C, const uint16_t *h_in, int B, int step, uint16_t *y_out, float *y_f32, int chained,
+                        cudaStream_t s) {
+  const e0_dims &D = C->dims;
+  const size_t full = (size_t)C->L * C->maxT * D.d_model;
+  if (!C->g_h) {
+    int rc;
+    if ((rc = dalloc(&C->g_h, full)) || (rc = dalloc(&C->g_y, full)) || (rc = dalloc(&C->g_yf, full))) return rc;
+    CK(cudaStreamCreateWithFlags(&C->cap, cudaStreamNonBlocking));
+  }
+  const int parity = step & 1, step0 = step == 0, has_f32 = y_f32 != nullptr;
+  DecodeGraph *G = nullptr;
+  for (auto &g : C->graphs)
+    if (g.exec && g.B == B && g.parity == parity && g.step0 == step0 && g.chained == chained && g.has_f32 == has_f32)
+      G = &g;
+  if (!G) {
+    G = &C->graphs[C->graph_next];
+    C->graph_next = (C->graph_next + 1) % (int)(sizeof(C->graphs) / sizeof(C->graphs[0]));
+    if (G->exec) cudaGraphExecDestroy(G->exec);
+    *G = DecodeGraph{};
+    const unsigned long long l0 = C->stats.kernel_launches;
+    CK(cudaStreamBeginCapture(C->cap, cudaStreamCaptureModeThreadLocal));
+    int rc = stack_decode_general(C, C->g_h, B, step, C->g_y, has_f32 ? C->g_yf : nullptr, 0, chained, C->cap);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(C->cap, &graph);
+    if (rc || e != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      C->stats.kernel_launches = l0;
+      return rc ? rc : fail(E0_ERR_CUDA, "decode graph capture: %s", cudaGetErrorString(e));
+    }
+    e = cudaGraphInstantiate(&G->exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) return fail(E0_ERR_CUDA, "decode graph instantiate: %s", cudaGetErrorString(e));
+    G->B = B; G->parity = parity; G->step0 = step0; G->chained = chained; G->has_f32 = has_f32;
+    G->launches = C->stats.kernel_launches - l0;
+    C->stats.kernel_launches = l0;
+  }
+  // the graph reads and writes packed [L][B][d] buffers of its own
+  const size_t n = (size_t)C->L * B * D.d_model;
+  CK(cudaMemcpyAsync(C->g_h, h_in, n * 2, cudaMemcpyDeviceToDevice, s));
+  CK(cudaGraphLaunch(G->exec, s));
+  C->stats.kernel_launches += G->launches;
+  CK(cudaMemcpyAsync(y_out, C->g_y, n * 2, cudaMemcpyDeviceToDevice, s));
+  if (y_f32) CK(cudaMemcpyAsync(y_f32, C->g_yf, n * 4, cudaMemcpyDeviceToDevice, s));
+  return E0_OK;
+}
+
 extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step, void *y_out, float *y_f32,
                                    int streaming, int chained, void *stream) {
   if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
@@ -839,8 +911,15 @@ extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step,
   cudaStream_t s = (cudaStream_t)stream;
   C->last = s;
   int rc;
-  if (!streaming && !C->force_general && decode_supported(C, B))
+  const bool one_launch = decode_supported(C, B);
+  int mode = C->force_general ? 3 : C->decode_mode;
+  if (mode == 0) mode = one_launch ? 1 : 3;   // default: measured fastest per batch
+  if (mode == 1 && !one_launch) mode = 2;
+  if (streaming) mode = 3;                                  // host decisions between layers
+  if (mode == 1)
     rc = decode_persistent(C, (const uint16_t *)h_in, step, (uint16_t *)y_out, y_f32, chained, s);
+  else if (mode == 2)
+    rc = decode_graph(C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, chained, s);
   else
     rc = stack_decode_general(C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, streaming, chained, s);
   if (rc) return rc;
@@ -952,6 +1031,14 @@ extern "C" int e0_debug_decode_trace(e0_ctx *C, unsigned long long *buf) {
 extern "C" int e0_debug_prefill_path(e0_ctx *C, int mode) {
   if (!C || mode < 0 || mode > 2) return fail(E0_ERR_INVALID_ARG, "bad prefill path");
   C->prefill_path = mode;
+  return E0_OK;
+}
+
+// Decode implementation: 0 = default, 1 = one-launch kernel (B = 1), 2 = CUDA-graph replay
+// of the per-layer kernels, 3 = per-layer kernels launched one by one.
+extern "C" int e0_debug_decode_mode(e0_ctx *C, int mode) {
+  if (!C || mode < 0 || mode > 3) return fail(E0_ERR_INVALID_ARG, "bad decode mode");
+  C->decode_mode = mode;
   return E0_OK;
 }
 

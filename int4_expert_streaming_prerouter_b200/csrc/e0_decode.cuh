@@ -78,7 +78,7 @@ struct DecodeParams {
 enum : int {
   TR_LAYER = 0, TR_NORM = 1, TR_ROUTE = 2, TR_GU_FULL = 3, TR_GU_DONE = 4, TR_A_POLL = 5,
   TR_TD_POLL = 6, TR_DN_FULL = 7, TR_DN_DONE = 8, TR_P_GU = 9, TR_P_DN = 10, TR_P_R = 11,
-  TR_P_GU_START = 12, TR_P_DN_START = 13
+  TR_P_GU_START = 12, TR_P_DN_START = 13, TR_GU_ROWS = 14, TR_DN_DOTS = 15
 };
 
 // ---------------------------------------------------------------------------------------
@@ -576,23 +576,6 @@ struct Ctl {
 };
 
 
-// Slow path of a poll: spin on one word until its tag matches (bounded).  Returns the
-// word, or 0 (never a valid word: tags start at 64) on timeout or abort.
-__device__ __noinline__ unsigned long long spin_tag(const unsigned long long *p, uint32_t tag, const Ctl &C) {
-  unsigned long long t0 = 0;
-  do {
-    __nanosleep(16);
-    const unsigned long long v = ld_tag(p);
-    if ((uint32_t)v == tag) return v;
-    if (*C.abort) return 0ull;
-    if (timed_out(t0, C.timeout)) {
-      atomicOr(C.err, DERR_TIMEOUT);
-      *C.abort = 1;
-      return 0ull;
-    }
-  } while (true);
-}
-
 // A source range of tagged words and where its 32-bit payloads go (shared memory).
 struct Range {
   const unsigned long long *src;
@@ -607,13 +590,13 @@ struct Range {
 __device__ __noinline__ bool poll_ranges(const Range *rg, int nr, uint32_t tag, int tid, const Ctl &C) {
   constexpr int W = 8;
   int total = 0;
-  #pragma unroll 1
+#pragma unroll 1
   for (int q = 0; q < nr; q++) total += rg[q].n;
-  #pragma unroll 1
+#pragma unroll 1
   for (int base = 0; base < total; base += W * kDecConsumers) {
-    unsigned long long v[W];
     const unsigned long long *ad[W];
     uint32_t *dd[W];
+    unsigned pending = 0;
 #pragma unroll
     for (int m = 0; m < W; m++) {
       int i = base + tid + m * kDecConsumers;
@@ -624,17 +607,30 @@ __device__ __noinline__ bool poll_ranges(const Range *rg, int nr, uint32_t tag, 
         while (i >= rg[q].n) i -= rg[q++].n;
         ad[m] = rg[q].src + i;
         dd[m] = rg[q].dst + i;
+        pending |= 1u << m;
       }
-      v[m] = ad[m] ? ld_tag(ad[m]) : 0ull;
     }
+    // every still-stale word of the batch is re-read together, so each wave of arrivals
+    // costs one L2 round trip
+    unsigned long long t0 = 0;
+    while (pending) {
+      unsigned long long v[W];
 #pragma unroll
-    for (int m = 0; m < W; m++) {
-      if (!ad[m]) continue;
-      if ((uint32_t)v[m] != tag) {
-        v[m] = spin_tag(ad[m], tag, C);
-        if ((uint32_t)v[m] != tag) return false;
+      for (int m = 0; m < W; m++) v[m] = ((pending >> m) & 1u) ? ld_tag(ad[m]) : 0ull;
+#pragma unroll
+      for (int m = 0; m < W; m++)
+        if (((pending >> m) & 1u) && (uint32_t)v[m] == tag) {
+          *dd[m] = (uint32_t)(v[m] >> 32);
+          pending &= ~(1u << m);
+        }
+      if (!pending) break;
+      if (*C.abort) return false;
+      if (timed_out(t0, C.timeout)) {
+        atomicOr(C.err, DERR_TIMEOUT);
+        *C.abort = 1;
+        return false;
       }
-      *dd[m] = (uint32_t)(v[m] >> 32);
+      __nanosleep(20);
     }
   }
   return true;
@@ -906,6 +902,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         roff += R;
       }
       cbar();
+      if (ct == 0) stamp(P, l, TR_GU_ROWS);
       // publish: routed rows as a = bf16(silu(g) u); shared rows as raw (g, u)
       roff = 0;
       #pragma unroll 1
@@ -1060,6 +1057,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           if (valid && sl == 0) yd[row * (k + 1) + j] = acc;
         }
       }
+      if (ct == 0) stamp(P, l, TR_DN_DOTS);
       // head rows (this layer's prerouter head on x)
       if (Y.head) {
         int ha, hb;

@@ -210,3 +210,15 @@ def test_one_launch_decode_bounded_wait_reports_timeout(cuda_ok):
     ref = oracle_steps(SMALL, 94, 1, 2, gpu[2], gpu[3])
     compare_steps(SMALL, gpu, ref)
     ctx.close()
+
+
+@pytest.mark.parametrize("B", [1, 5])
+def test_graph_replay_decode_matches_oracle(cuda_ok, B):
+    """The decode step replayed as a captured CUDA graph of the per-layer kernels."""
+    ctx, _, _ = build(SMALL, 95 + B, 8)
+    ctx.debug_decode_mode(2)
+    S = 3
+    gpu = run_steps(ctx, SMALL, 95 + B, B, S)
+    ref = oracle_steps(SMALL, 95 + B, B, S, gpu[2], gpu[3])
+    compare_steps(SMALL, gpu, ref)
+    ctx.close()
