@@ -6,11 +6,12 @@
 //             the shared expert adds c * B (A x) to g and u first;
 //   down:     Y_e = Dq(W_d) A_e^T, y[t] += w_{t,j} Y_e[:, t]  (w = 1 for the shared expert).
 //
-// B200 design.  One CTA = one 128-row weight tile of one expert x up to 128 tokens.  Four
-// warps produce each 64-wide K block: they dequantise the int4 weight tile to fp16
-// (w = s q + m, one group of 64 per row per K block) and gather the token rows (fp16),
-// writing both into shared memory in the 128-byte-swizzled K-major layout the tensor core
-// reads.  One thread issues four tcgen05.mma (M=128, N=tokens, K=16 each) per K block
+// B200 design.  One CTA = one 128-row weight tile of one expert x up to 128 tokens.  Eight
+// warps produce each 64-wide K block: two threads per weight row dequantise the int4 tile
+// to fp16 (w = s q + m, one group of 64 per row per K block) and the token rows (fp16) are
+// gathered beside it, both written into shared memory in the 128-byte-swizzled K-major
+// layout the tensor core reads; each thread's global loads for the next K block are
+// issued before it works on the current one.  One thread issues four tcgen05.mma (M=128, N=tokens, K=16 each) per K block
 // into a TMEM accumulator and commits to an mbarrier that frees the stage; four stages are
 // in flight.  The epilogue reads TMEM with tcgen05.ld and applies SwiGLU (gate rows 0..63
 // and up rows 64..127 of the tile are the same intermediate units) or the gate-weighted
@@ -26,7 +27,7 @@
 
 namespace e0 {
 
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 256;
 constexpr int kTcMinTokens = 64;    // contexts with at least this many tokens get the tensor-core path
 constexpr int kTcN = 128;           // tokens per tile (TMEM columns)
 constexpr int kTcStages = 4;
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_gemm_tc(TcArgs A) {
   extern __shared__ __align__(1024) uint8_t tc_raw[];
   // the swizzled tiles need 1024-byte alignment
   TcSmem &S = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(tc_raw) + 1023) & ~(uintptr_t)1023);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int mtiles = A.mode == 0 ? A.I / 64 : A.d / 128;
   const int tile = blockIdx.x / mtiles, mt = blockIdx.x % mtiles;
   if (tile >= *A.ntiles) return;
@@ -233,80 +234,96 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_gemm_tc(TcArgs A) {
   const uint32_t idesc = tc_idesc(128, N);
   bool ok = true;
 
-  // weight rows of this tile: mode 0 -> gate rows i0..i0+63 then up rows i0..i0+63
-  // (i0 = 64 mt); mode 1 -> down rows 128 mt .. 128 mt + 127
-  const int row = tid;
+  // A producer role: two threads per weight row, each 32 of the 64 K elements of a block.
+  // mode 0 -> gate rows i0..i0+63 then up rows i0..i0+63 (i0 = 64 mt); mode 1 -> down
+  // rows 128 mt .. 128 mt + 127
+  const int row = tid >> 1, half = tid & 1;
   const uint8_t *codes;
   const uint16_t *scl, *mnv;
-  int kdim;
   if (A.mode == 0) {
     const int i = mt * 64 + (row & 63);
     const bool up = row >= 64;
     codes = base + (up ? A.bl.uc : A.bl.gc) + (size_t)i * (A.d / 2);
     scl = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.us : A.bl.gs)) + (size_t)i * (A.d / 64);
     mnv = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.um : A.bl.gm)) + (size_t)i * (A.d / 64);
-    kdim = A.d;
   } else {
     const int n = mt * 128 + row;
     codes = base + A.bl.dc + (size_t)n * (A.I / 2);
     scl = reinterpret_cast<const uint16_t *>(base + A.bl.ds) + (size_t)n * (A.I / 64);
     mnv = reinterpret_cast<const uint16_t *>(base + A.bl.dm) + (size_t)n * (A.I / 64);
-    kdim = A.I;
   }
-  (void)kdim;
+  // B producer role: (column, chunk) pairs e = tid + m * kTcThreads, m < kBPer
+  constexpr int kBPer = kTcN * 8 / kTcThreads;
+  const __half *bsrc[kBPer];
+#pragma unroll
+  for (int m = 0; m < kBPer; m++) {
+    const int e = tid + m * kTcThreads, c = e >> 3, ch = e & 7;
+    const int tok = c < N ? S.tok[c] : -1;
+    bsrc[m] = nullptr;
+    if (tok >= 0)
+      bsrc[m] = (A.mode == 0 ? A.x16 + (size_t)tok * A.d
+                             : A.a16 + (size_t)(tok * (A.k + 1) + (shared ? A.k : S.dst[c] % A.k)) * A.I) + ch * 8;
+  }
+  // loads of one K block into registers (issued one block ahead of their use)
+  uint4 qa, qb[kBPer];
+  float sc = 0.f, mn = 0.f;
+  auto load_block = [&](int kb) {
+    qa = __ldg(reinterpret_cast<const uint4 *>(codes + kb * 32 + half * 16));
+    sc = bf(__ldg(scl + kb));
+    mn = bf(__ldg(mnv + kb));
+#pragma unroll
+    for (int m = 0; m < kBPer; m++)
+      qb[m] = bsrc[m] ? __ldg(reinterpret_cast<const uint4 *>(bsrc[m] + kb * 64)) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  load_block(0);
 
   int issued = 0;   // K blocks whose MMAs were issued (uniform across the block)
+#pragma unroll 1
   for (int kb = 0; kb < nkb && ok; kb++) {
     const int s = kb % kTcStages;
+    // this block's data, then start the next block's loads
+    const uint4 ca = qa;
+    const float csc = sc, cmn = mn;
+    uint4 cb[kBPer];
+#pragma unroll
+    for (int m = 0; m < kBPer; m++) cb[m] = qb[m];
+    if (kb + 1 < nkb) load_block(kb + 1);
     if (kb >= kTcStages) ok = tc_wait(&S.done[s], (uint32_t)(((kb / kTcStages) - 1) & 1), A);
     if (__syncthreads_or(!ok)) {
       ok = false;
       break;
     }
-    // A: this thread's weight row, one group of 64 -> fp16, swizzled
+    // A: 32 weights -> fp16 hi + lo (about 22 significant bits together), swizzled
     {
-      const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(codes + kb * 32));
-      const uint4 q1 = __ldg(reinterpret_cast<const uint4 *>(codes + kb * 32 + 16));
-      const float sc = bf(scl[kb]), mn = bf(mnv[kb]);
-      const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const uint32_t w[4] = {ca.x, ca.y, ca.z, ca.w};
       uint8_t *dstA = S.a[s], *dstL = S.alo[s];
 #pragma unroll
-      for (int ch = 0; ch < 8; ch++) {
-        // chunk ch holds K elements 8ch..8ch+7 = code word ch; each weight is split into
-        // fp16 hi + fp16 lo so that the pair carries ~22 significant bits
-        const uint32_t wd = w[ch];
+      for (int j = 0; j < 4; j++) {
+        // code word j of this half = K elements 8 (4 half + j) .. + 7 = chunk 4 half + j
+        const uint32_t wd = w[j];
         __half2 h[4], l[4];
 #pragma unroll
         for (int p = 0; p < 4; p++) {
-          const float w0 = fmaf(sc, (float)((wd >> (8 * p)) & 0xFu), mn);
-          const float w1 = fmaf(sc, (float)((wd >> (8 * p + 4)) & 0xFu), mn);
+          const float w0 = fmaf(csc, (float)((wd >> (8 * p)) & 0xFu), cmn);
+          const float w1 = fmaf(csc, (float)((wd >> (8 * p + 4)) & 0xFu), cmn);
           h[p] = __floats2half2_rn(w0, w1);
           const float2 hf = __half22float2(h[p]);
           l[p] = __floats2half2_rn(w0 - hf.x, w1 - hf.y);
         }
-        *reinterpret_cast<uint4 *>(dstA + sw128(row, ch)) =
+        const uint32_t off = sw128(row, half * 4 + j);
+        *reinterpret_cast<uint4 *>(dstA + off) =
             make_uint4(*reinterpret_cast<uint32_t *>(&h[0]), *reinterpret_cast<uint32_t *>(&h[1]),
                        *reinterpret_cast<uint32_t *>(&h[2]), *reinterpret_cast<uint32_t *>(&h[3]));
-        *reinterpret_cast<uint4 *>(dstL + sw128(row, ch)) =
+        *reinterpret_cast<uint4 *>(dstL + off) =
             make_uint4(*reinterpret_cast<uint32_t *>(&l[0]), *reinterpret_cast<uint32_t *>(&l[1]),
                        *reinterpret_cast<uint32_t *>(&l[2]), *reinterpret_cast<uint32_t *>(&l[3]));
       }
     }
     // B: token rows of this K block (zero for padding columns), swizzled
-    {
-      uint8_t *dstB = S.b[s];
-      // 8 chunks per token row; threads walk (column, chunk) pairs
-      for (int e = tid; e < N * 8; e += kTcThreads) {
-        const int c = e >> 3, ch = e & 7;
-        const int tok = S.tok[c];
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (tok >= 0) {
-          const __half *srcrow = A.mode == 0 ? A.x16 + (size_t)tok * A.d
-                                             : A.a16 + (size_t)(tok * (A.k + 1) + (shared ? A.k : S.dst[c] % A.k)) * A.I;
-          v = __ldg(reinterpret_cast<const uint4 *>(srcrow + kb * 64 + ch * 8));
-        }
-        *reinterpret_cast<uint4 *>(dstB + sw128(c, ch)) = v;
-      }
+#pragma unroll
+    for (int m = 0; m < kBPer; m++) {
+      const int e = tid + m * kTcThreads, c = e >> 3, ch = e & 7;
+      if (c < N) *reinterpret_cast<uint4 *>(S.b[s] + sw128(c, ch)) = cb[m];
     }
     // generic-proxy smem writes -> visible to the tensor core (async proxy)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -339,20 +356,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_gemm_tc(TcArgs A) {
   }
 
   // ------------------------------- epilogue ------------------------------------------
-  // this thread owns TMEM lane `row` (warp w reads lanes 32w..32w+31)
+  // warp w reads TMEM lanes 32 (w % 4) .. + 31 (tile row = that lane); warps 0-3 take the
+  // first half of the columns, warps 4-7 the second
+  const int erow = 32 * (warp & 3) + (tid & 31);
+  const int cbeg = (warp >> 2) * (kTcN / 2);
+  const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
   float *ex = reinterpret_cast<float *>(S.b[0]);   // 64 x kTcN floats: the up values (mode 0)
-  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
   if (A.mode == 0) {
-    const int i = mt * 64 + (row & 63);
-    const bool up = row >= 64;
+    const int i = mt * 64 + (erow & 63);
+    const bool up = erow >= 64;
     float lb[kMaxR];
     const bool lora = shared && A.Bg != nullptr;
     if (lora)
       for (int q = 0; q < A.r; q++) lb[q] = bf((up ? A.Bu : A.Bg)[(size_t)i * A.r + q]);
-    for (int c0 = 0; c0 < N; c0 += 32) {
+#pragma unroll 1
+    for (int c0 = cbeg; c0 < cbeg + kTcN / 2; c0 += 32) {
       float v[32];
-      tc_ld32(lane_addr + c0, v);
-      if (lora)
+      const bool live = c0 < N;
+      if (live) tc_ld32(lane_addr + c0, v);
+      if (live && lora)
         for (int cc = 0; cc < 32; cc++) {
           const int tok = S.tok[c0 + cc];
           if (tok < 0) continue;
@@ -361,22 +383,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_gemm_tc(TcArgs A) {
           for (int q = 0; q < A.r; q++) acc = fmaf(lb[q], t[q], acc);
           v[cc] = fmaf(A.c, acc, v[cc]);
         }
-      if (up)
-        for (int cc = 0; cc < 32; cc++) ex[(row - 64) * kTcN + c0 + cc] = v[cc];
+      if (live && up)
+        for (int cc = 0; cc < 32; cc++) ex[(erow - 64) * kTcN + c0 + cc] = v[cc];
       __syncthreads();
-      if (!up)
+      if (live && !up)
         for (int cc = 0; cc < 32; cc++) {
           const int dst = S.dst[c0 + cc];
           if (dst < 0) continue;
-          const float g = v[cc], u = ex[row * kTcN + c0 + cc];
+          const float g = v[cc], u = ex[erow * kTcN + c0 + cc];
           const float act = bf(f2bf(g / (1.0f + expf(-g)) * u));   // bf16 rounding point of a
           A.a16_out[(size_t)dst * A.I + i] = __float2half_rn(act);
         }
       __syncthreads();
     }
   } else {
-    const int n = mt * 128 + row;
-    for (int c0 = 0; c0 < N; c0 += 32) {
+    const int n = mt * 128 + erow;
+#pragma unroll 1
+    for (int c0 = cbeg; c0 < cbeg + kTcN / 2 && c0 < N; c0 += 32) {
       float v[32];
       tc_ld32(lane_addr + c0, v);
       for (int cc = 0; cc < 32; cc++) {
