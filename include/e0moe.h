@@ -245,6 +245,13 @@ int e0_debug_decode_mode(e0_ctx *ctx, int mode);
  * [grid][L][16], caller-owned device buffer; NULL stops it).  Returns the grid size. */
 int e0_debug_decode_trace(e0_ctx *ctx, unsigned long long *buf);
 int e0_debug_force_general(e0_ctx *ctx, int on);
+/* Stage overlap of the one-launch decode kernel on unchained steps (every layer's input
+ * given, none read from another layer's output): the down stage of a layer runs `lag`
+ * layers behind its gate/up stage, so that the exchange of the intermediate activations
+ * between the CTAs overlaps other layers' work.  0 = layers strictly in order; default 2;
+ * chained steps always run in order.  Results do not depend on it (each layer's
+ * arithmetic is the same).  E0_ERR_INVALID_ARG outside 0..8. */
+int e0_debug_decode_lag(e0_ctx *ctx, int lag);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *e0_last_error(void);

@@ -74,6 +74,7 @@ struct DecodeState {
   int G = 0;
   size_t smem = 0;
   int stall_cta = -1;
+  int lag = 2;                           // unchained steps: down stage this many layers behind
   unsigned long long timeout_ns = 2000000000ull;
   unsigned long long *trace = nullptr;   // profiling timeline (caller-owned), or nullptr
 };
@@ -813,6 +814,7 @@ static int decode_persistent(e0_ctx *C, const uint16_t *h, int step, uint16_t *y
   P.onehot = D.head_onehot; P.G = S.G;
   P.eps = D.rms_eps; P.c = D.lora_scale;
   P.h = h; P.y = y; P.yf = yf; P.chained = chained;
+  P.lag = chained ? 0 : S.lag;
   P.epoch = ++S.epoch;
   P.step0 = step == 0;
   P.pred_in = step > 0 ? pred_at(C, prv, 0) : nullptr;
@@ -1039,6 +1041,14 @@ extern "C" int e0_debug_prefill_path(e0_ctx *C, int mode) {
 extern "C" int e0_debug_decode_mode(e0_ctx *C, int mode) {
   if (!C || mode < 0 || mode > 3) return fail(E0_ERR_INVALID_ARG, "bad decode mode");
   C->decode_mode = mode;
+  return E0_OK;
+}
+
+// Stage overlap of the one-launch decode kernel on unchained steps: the down stage of a
+// layer runs `lag` layers behind its gate/up stage (0 = layers strictly in order).
+extern "C" int e0_debug_decode_lag(e0_ctx *C, int lag) {
+  if (!C || lag < 0 || lag > 8) return fail(E0_ERR_INVALID_ARG, "bad decode lag");
+  C->dec.lag = lag;
   return E0_OK;
 }
 

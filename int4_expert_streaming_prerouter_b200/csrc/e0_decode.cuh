@@ -55,6 +55,10 @@ struct DecodeParams {
   uint16_t *y;              // [L][D]
   float *yf;                // [L][D] or nullptr
   int chained;
+  // 0: layers run in order, each layer's first stage waiting for the previous layer's
+  // output; > 0 (unchained inputs only): the stages of different layers overlap, the down
+  // stage of a layer running `lag` layers behind its gate/up stage
+  int lag;
   uint32_t epoch;
   int step0;                // 1: every layer routes with its own router
   const int32_t *pred_in;   // [L+1][maxT][k]: routing predicted for layer l (previous step)
@@ -250,6 +254,13 @@ struct TaskBuf {
 
 enum : int { TK_ROUTER = 0, TK_GU = 1, TK_DN = 2 };
 
+// Items of a launch's schedule, the same sequence for the producer and the consumers:
+//   IT_R   router rows of a reactive layer (producer task),
+//   IT_TK  top-k of a reactive layer over every CTA's router logits (consumers only),
+//   IT_GU  gate/up stage (producer task), IT_DN  down + combine stage (producer task).
+enum : int { IT_R = 0, IT_TK = 1, IT_GU = 2, IT_DN = 3 };
+constexpr int kMaxSched = 4 * 64;
+
 // GU range of a CTA split into per-slot pieces.
 struct GuPiece {
   int slot, i0, i1;
@@ -270,13 +281,14 @@ __device__ __forceinline__ int gu_pieces(int k, int G, int c, GuPiece *out) {
 
 // Segment indices of each task kind (a segment may be empty):
 //   router task: [0] gamma, [1] h, [2] this CTA's router rows
-//   gate/up task: [0] gamma, [1] h (predicted layers; empty otherwise), [2] A_g rows,
-//     [3] A_u rows, [4, 4+kMaxK) selected router rows, then per piece p (up to kMaxPieces)
-//     6 segments: gate codes, gate scale, gate min, up codes, up scale, up min
-//   down task: [3j .. 3j+2] down codes/scale/min of slot j (j = 0..k), then B_d rows, head
-//     rows, B_g, B_u, A_d (LoRA matrices of the shared expert, whole)
+//   gate/up task: [0] gamma, [1] h, [2] A_g rows, [3] A_u rows, [4, 4+kMaxK) selected
+//     router rows, [4+kMaxK] head rows, then per piece p (up to kMaxPieces) 6 segments:
+//     gate codes, gate scale, gate min, up codes, up scale, up min
+//   down task: [3j .. 3j+2] down codes/scale/min of slot j (j = 0..k), then B_d rows, B_g,
+//     B_u, A_d (LoRA matrices of the shared expert, whole)
 constexpr int kMaxPieces = 4;
-constexpr int kGuPiece0 = 4 + kMaxK;
+constexpr int kGuHead = 4 + kMaxK;
+constexpr int kGuPiece0 = 5 + kMaxK;
 __device__ __forceinline__ int dn_bd(int k) { return 3 * (k + 1); }
 
 // Build the segment list of task (kind, layer) for CTA c.  `sel` are the layer's routed
@@ -294,8 +306,8 @@ __device__ __noinline__ void build_task(const DecodeParams &P, const DecLayer &Y
     split_range(P.E, P.G, c, a, b);
     T.add(Y.router + (size_t)a * D, (size_t)(b - a) * D * 2);
   } else if (kind == TK_GU) {
-    T.add(Y.gamma, predicted ? D * 2 : 0);
-    T.add(P.h + (size_t)l * D, predicted ? D * 2 : 0);
+    T.add(Y.gamma, D * 2);
+    T.add(P.h + (size_t)l * D, D * 2);
     int a = 0, b = 0;
     if (Y.Ag) split_range(2 * P.r, P.G, c, a, b);
     const int ga = min(a, P.r), gb = min(b, P.r), ua = max(a, P.r) - P.r, ub = max(b, P.r) - P.r;
@@ -308,6 +320,9 @@ __device__ __noinline__ void build_task(const DecodeParams &P, const DecLayer &Y
       const bool on = a + q < b;
       T.add(Y.router + (size_t)(on ? sel[a + q] : 0) * D, on ? D * 2 : 0);
     }
+    int ha = 0, hb = 0;
+    if (Y.head) split_range(P.E, P.G, c, ha, hb);
+    T.add(Y.head + (size_t)ha * P.ldh, (size_t)(hb - ha) * P.ldh * 2);
     GuPiece pc[kMaxPieces];
     const int np = gu_pieces<D, I>(P.k, P.G, c, pc);
     #pragma unroll 1
@@ -333,9 +348,6 @@ __device__ __noinline__ void build_task(const DecodeParams &P, const DecLayer &Y
       T.add(base + bl.dm + (size_t)a * (I / 64) * 2, (size_t)R * (I / 64) * 2);
     }
     T.add(Y.Bd + (size_t)a * P.r, Y.Bd ? (size_t)R * P.r * 2 : 0);
-    int ha = 0, hb = 0;
-    if (Y.head) split_range(P.E, P.G, c, ha, hb);
-    T.add(Y.head + (size_t)ha * P.ldh, (size_t)(hb - ha) * P.ldh * 2);
     const size_t lb = Y.Bg ? (size_t)I * P.r * 2 : 0;
     T.add(Y.Bg, lb);
     T.add(Y.Bu, lb);
@@ -362,14 +374,16 @@ struct DecSmem {
   float tl[2 * kMaxR];               // t_g, t_u
   float td[kMaxR];                   // t_d
   float rl[kMaxE];                   // router logits (reactive) / selected logits / head logits
-  int sel[kMaxK];
-  int sel_all[64][kMaxK];            // routing of every layer this step (head one-hot)
+  int sel_all[64][kMaxK];            // routing of every layer this step
+  float rlsel[64][kMaxK];            // a reactive layer's router logits of its chosen experts
+  volatile int sel_ok[64];           // 1 once a reactive layer's top-k is in sel_all
+  uint16_t sched[kMaxSched];         // this launch's items: kind << 8 | layer
+  int nsched;
   DecLayer lay[64];                  // the layer table
   TaskBuf tb;                        // the producer's task being issued
   int tb_off[kMaxSeg];
   uint32_t seg_off[kNSlot][kMaxSeg]; // ring byte offset of each segment's first wanted byte
   uint64_t full[kNSlot], empty[kNSlot];
-  volatile int sel_ready;            // layer whose own-router top-k the consumers published
   volatile int abort;
 };
 
@@ -392,6 +406,52 @@ __device__ __forceinline__ bool timed_out(unsigned long long &t0, unsigned long 
 }
 
 // ---------------------------------------------------------------------------------------
+// The launch's schedule (one thread).  In order (lag 0): per layer [R, TK] GU DN.  With a
+// lag (unchained inputs: no layer reads another layer's output within the step): the
+// layers are taken predicted first, then reactive; the router rows of every reactive
+// layer come first, a reactive layer's top-k two layers before its gate/up stage (so the
+// producer can fetch its experts early), and each down stage `lag` layers after its
+// gate/up stage, so that the exchange between the two stages overlaps other layers' work.
+// ---------------------------------------------------------------------------------------
+template <int D, int I>
+__device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I> &S) {
+  int n = 0;
+  if (P.lag == 0) {
+    #pragma unroll 1
+    for (int l = 0; l < P.L; l++) {
+      if (!is_predicted(P, S, l)) {
+        S.sched[n++] = (uint16_t)((IT_R << 8) | l);
+        S.sched[n++] = (uint16_t)((IT_TK << 8) | l);
+      }
+      S.sched[n++] = (uint16_t)((IT_GU << 8) | l);
+      S.sched[n++] = (uint16_t)((IT_DN << 8) | l);
+    }
+  } else {
+    constexpr int PF = 2;
+    uint8_t ord[64];
+    int no = 0;
+    #pragma unroll 1
+    for (int pass = 0; pass < 2; pass++)
+      #pragma unroll 1
+      for (int l = 0; l < P.L; l++)
+        if (is_predicted(P, S, l) == (pass == 0)) ord[no++] = (uint8_t)l;
+    #pragma unroll 1
+    for (int j = 0; j < no; j++)
+      if (!is_predicted(P, S, ord[j])) S.sched[n++] = (uint16_t)((IT_R << 8) | ord[j]);
+    #pragma unroll 1
+    for (int j = 0; j < PF && j < no; j++)
+      if (!is_predicted(P, S, ord[j])) S.sched[n++] = (uint16_t)((IT_TK << 8) | ord[j]);
+    #pragma unroll 1
+    for (int j = 0; j < no + P.lag; j++) {
+      if (j + PF < no && !is_predicted(P, S, ord[j + PF])) S.sched[n++] = (uint16_t)((IT_TK << 8) | ord[j + PF]);
+      if (j < no) S.sched[n++] = (uint16_t)((IT_GU << 8) | ord[j]);
+      if (j >= P.lag && j - P.lag < no) S.sched[n++] = (uint16_t)((IT_DN << 8) | ord[j - P.lag]);
+    }
+  }
+  S.nsched = n;
+}
+
+// ---------------------------------------------------------------------------------------
 // Producer (warp 0): walk this CTA's task list and stream it through the ring.  Lane 0
 // builds each task's segment list in shared memory and owns the ring bookkeeping; all 32
 // lanes issue the bulk copies.
@@ -405,18 +465,17 @@ __device__ void producer(const DecodeParams &P, DecSmem<D, I> &S) {
   bool ok = true;
 
   #pragma unroll 1
-  for (int l = 0; l < P.L && ok; l++) {
+  for (int it = 0; it < S.nsched && ok; it++) {
+    const int item = S.sched[it] >> 8, l = S.sched[it] & 255;
+    if (item == IT_TK) continue;
     const bool pred = is_predicted(P, S, l);
-    #pragma unroll 1
-    for (int kind = pred ? TK_GU : TK_ROUTER; kind <= TK_DN && ok; kind++) {
-      if (kind == TK_GU) {
-        if (pred) {
-          #pragma unroll 1
-          for (int j = 0; j < P.k; j++) sel[j] = S.sel_all[l & 63][j];
-        } else {
-          // the consumers publish the layer's own top-k once its router has run
+    const int kind = item == IT_R ? TK_ROUTER : item == IT_GU ? TK_GU : TK_DN;
+    {
+      if (kind != TK_ROUTER) {
+        if (!pred) {
+          // the consumers publish a reactive layer's own top-k (its TK item) first
           unsigned long long t0 = 0;
-          while (S.sel_ready != l) {
+          while (S.sel_ok[l & 63] == 0) {
             if (S.abort) { ok = false; break; }
             if (timed_out(t0, P.timeout_ns)) {
               if (lane == 0) atomicOr(P.err, DERR_TIMEOUT);
@@ -427,15 +486,15 @@ __device__ void producer(const DecodeParams &P, DecSmem<D, I> &S) {
             __nanosleep(32);
           }
           if (!ok) break;
-          #pragma unroll 1
-          for (int j = 0; j < P.k; j++) sel[j] = S.sel[j];
         }
         #pragma unroll 1
-        for (int j = 0; j < P.k; j++)
+        for (int j = 0; j < P.k; j++) {
+          sel[j] = S.sel_all[l & 63][j];
           if (sel[j] < 0 || sel[j] >= P.E) {
-            if (lane == 0) atomicOr(P.err, DERR_INDEX);
+            if (lane == 0 && kind == TK_GU) atomicOr(P.err, DERR_INDEX);
             sel[j] = 0;
           }
+        }
       }
       if (kind == TK_GU) stamp(P, l, TR_P_GU_START);
       if (kind == TK_DN) stamp(P, l, TR_P_DN_START);
@@ -709,14 +768,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     #pragma unroll 1
     for (int i = tid; i < P.L * P.k; i += kDecThreads)
       S.sel_all[(i / P.k) & 63][i % P.k] = P.pred_in[((size_t)(i / P.k) * P.maxT) * P.k + i % P.k];
+  if (tid < 64) S.sel_ok[tid] = 0;
+  __syncthreads();
   if (tid == 0) {
     #pragma unroll 1
     for (int s = 0; s < kNSlot; s++) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], kDecCW);
     }
-    S.sel_ready = -1;
     S.abort = 0;
+    build_schedule<D, I>(P, S);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -739,24 +800,47 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
   }
 
   #pragma unroll 1
-  for (int l = 0; l < P.L; l++) {
+  for (int it = 0; it < S.nsched; it++) {
+    const int kind = S.sched[it] >> 8, l = S.sched[it] & 255;
     const DecLayer &Y = S.lay[l];
     const bool pred = is_predicted(P, S, l);
     const bool lora = Y.Bg != nullptr;
     const uint32_t tag = dtag(P, l);
-    // ---- wait for the previous layer's output (data in chained mode, order otherwise)
-    if (l > 0) {
+    if (kind == IT_TK) {
+      // ---- a reactive layer's top-k over every CTA's router logits
+      ab |= !poll_to(P.t_rlog + (size_t)l * P.E, reinterpret_cast<uint32_t *>(S.rl), P.E, tag, ct, C);
+      if (cbar_or(ab)) break;
+      if (warp == 0) {
+        int s8[kMaxK];
+        warp_topk_ool(S.rl, P.E, k, lane, s8);
+        if (lane == 0) {
+          #pragma unroll 1
+          for (int j = 0; j < k; j++) {
+            S.sel_all[l & 63][j] = s8[j];
+            S.rlsel[l & 63][j] = (s8[j] >= 0 && s8[j] < P.E) ? S.rl[s8[j]] : 0.f;
+          }
+          __threadfence_block();
+          S.sel_ok[l & 63] = 1;
+        }
+      }
+      cbar();
+      if (ct == 0) stamp(P, l, TR_ROUTE);
+      continue;
+    }
+    // ---- in order: a layer's first item waits for the previous layer's output (its data
+    // in chained mode)
+    if (P.lag == 0 && l > 0 && (kind == IT_R || (kind == IT_GU && pred))) {
       ab |= !poll_to(P.t_y + (size_t)(l - 1) * D, reinterpret_cast<uint32_t *>(S.yprev), D, dtag(P, l - 1), ct, C);
     }
     if (cbar_or(ab)) break;
-    if (ct == 0) stamp(P, l, TR_LAYER);
+    if (ct == 0 && kind != IT_DN) stamp(P, l, TR_LAYER);
 
-    int slot = q % kNSlot;
-    uint32_t par = (uint32_t)((q / kNSlot) & 1);
-    // ---- the norm: gamma and h are the first two segments of the layer's first task
+    const int slot = q % kNSlot;
+    const uint32_t par = (uint32_t)((q / kNSlot) & 1);
     ab |= !wait_full(&S.full[slot], par, C);
     if (cbar_or(ab)) break;
-    {
+    if (kind != IT_DN) {
+      // ---- the norm: gamma and h are the first two segments of router and gate/up tasks
       const uint16_t *gam = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][0]);
       const uint16_t *hin = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][1]);
       const bool chain = P.chained && l > 0;
@@ -792,9 +876,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       }
       cbar();
     }
-    if (ct == 0) stamp(P, l, TR_NORM);
-    // ---- reactive layer: own router rows, then everyone's logits, then top-k
-    if (!pred) {
+    if (ct == 0 && kind != IT_DN) stamp(P, l, TR_NORM);
+    if (kind == IT_R) {
+      // ---- a reactive layer's router rows of this CTA
       int a, b;
       split_range(P.E, G, c, a, b);
       const uint16_t *rw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][2]);
@@ -803,33 +887,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         const float v = bf16_row_x<D>(rw + (size_t)(row - a) * D, S.x, lane);
         if (lane == 0) st_tag(P.t_rlog + (size_t)l * P.E + row, tag, __float_as_uint(v));
       }
-      cbar();
-      if (lane == 0) mbar_arrive(&S.empty[slot]);
-      q++;
-      ab |= !poll_to(P.t_rlog + (size_t)l * P.E, reinterpret_cast<uint32_t *>(S.rl), P.E, tag, ct, C);
-      if (cbar_or(ab)) break;
-      if (warp == 0) {
-        int s8[kMaxK];
-        warp_topk_ool(S.rl, P.E, k, lane, s8);
-        if (lane == 0) {
-          #pragma unroll 1
-          for (int j = 0; j < k; j++) S.sel_all[l & 63][j] = s8[j];
-          #pragma unroll 1
-          for (int j = 0; j < k; j++) S.sel[j] = s8[j];
-          __threadfence_block();
-          S.sel_ready = l;
-        }
-      }
-      cbar();
-      if (ct == 0) stamp(P, l, TR_ROUTE);
-      slot = q % kNSlot;
-      par = (uint32_t)((q / kNSlot) & 1);
-      ab |= !wait_full(&S.full[slot], par, C);
-      if (cbar_or(ab)) break;
-    }
-    // ---- gate/up phase --------------------------------------------------------------
-    if (ct == 0) stamp(P, l, TR_GU_FULL);
-    {
+    } else if (kind == IT_GU) {
+      // ---- gate/up stage ------------------------------------------------------------
+      if (ct == 0) stamp(P, l, TR_GU_FULL);
       // LoRA A rows of the shared expert (t_g, t_u), published for the down phase
       int a = 0, b = 0;
       if (lora) split_range(2 * r, G, c, a, b);
@@ -851,6 +911,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (warp == kDecCW - 1 - (qq - a) % kDecCW) {
           const float v = bf16_row_x<D>(reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][4 + qq - a]), S.x, lane);
           if (lane == 0) st_tag(P.t_blk + (size_t)l * P.blk + (k + 2) * I + 2 * r + qq, tag, __float_as_uint(v));
+        }
+      }
+      // this CTA's rows of the layer's prerouter head on x
+      if (Y.head) {
+        int ha, hb;
+        split_range(P.E, G, c, ha, hb);
+        const uint16_t *hw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kGuHead]);
+        #pragma unroll 1
+        for (int row = ha; row < hb; row++) {
+          if (warp == (4 + row - ha) % kDecCW) {
+            const float v = bf16_row_x<D>(hw + (size_t)(row - ha) * P.ldh, S.x, lane);
+            if (lane == 0) st_tag(P.t_hlog + (size_t)l * P.E + row, tag, __float_as_uint(v));
+          }
         }
       }
       // this lane's activation chunks stay in registers for every row of the phase
@@ -923,15 +996,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         }
         roff += R;
       }
-      cbar();
-      if (lane == 0) mbar_arrive(&S.empty[slot]);
-      q++;
+      // routing used by this layer (one CTA records it for the host)
+      if (c == 0 && ct < k) P.hist_out[((size_t)l * P.maxT) * k + ct] = S.sel_all[l & 63][ct];
       if (ct == 0) stamp(P, l, TR_GU_DONE);
-    }
-    // ---- down + combine phase ----------------------------------------------------------
-    slot = q % kNSlot;
-    par = (uint32_t)((q / kNSlot) & 1);
-    {
+    } else {
+      // ---- down + combine stage -----------------------------------------------------
       // one batched poll over the layer's block: a of the routed slots, the shared
       // expert's raw g/u, t_g/t_u (with LoRA) and the selected router logits (predicted)
       float *at = S.at, *gus = S.gus;
@@ -953,13 +1022,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         at[j * I + xt_index(e, NCI)] = bf(S.stg[i] & 0xFFFFu) * nib_scale(e & 7);
       }
       if (ct == 0) stamp(P, l, TR_A_POLL);
-      ab |= !wait_full(&S.full[slot], par, C);
-      if (cbar_or(ab)) break;
       if (ct == 0) stamp(P, l, TR_DN_FULL);
       const int sbd = dn_bd(k);
-      const uint16_t *bgm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 2]);
-      const uint16_t *bum = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 3]);
-      const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 4]);
+      const uint16_t *bgm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 1]);
+      const uint16_t *bum = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 2]);
+      const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 3]);
       // the shared expert's activation with its LoRA up branch (every CTA, same order)
       #pragma unroll 1
       for (int i = ct; i < I; i += kDecConsumers) {
@@ -990,7 +1057,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         float lg[kMaxK], mx = -INFINITY, sum = 0.f;
         #pragma unroll 1
         for (int j = 0; j < k; j++) {
-          lg[j] = pred ? S.rl[j] : S.rl[S.sel[j]];
+          lg[j] = pred ? S.rl[j] : S.rlsel[l & 63][j];
           mx = fmaxf(mx, lg[j]);
         }
         #pragma unroll 1
@@ -1058,17 +1125,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         }
       }
       if (ct == 0) stamp(P, l, TR_DN_DOTS);
-      // head rows (this layer's prerouter head on x)
-      if (Y.head) {
-        int ha, hb;
-        split_range(P.E, G, c, ha, hb);
-        const uint16_t *hw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 1]);
-        #pragma unroll 1
-        for (int row = ha + warp; row < hb; row += kDecCW) {
-          const float v = bf16_row_x<D>(hw + (size_t)(row - ha) * P.ldh, S.x, lane);
-          if (lane == 0) st_tag(P.t_hlog + (size_t)l * P.E + row, tag, __float_as_uint(v));
-        }
-      }
       cbar();
       const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd]);
       #pragma unroll 1
@@ -1088,16 +1144,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         P.y[(size_t)l * D + n] = f2bf(y);
         if (P.yf) P.yf[(size_t)l * D + n] = y;
       }
-      cbar();
-      if (lane == 0) mbar_arrive(&S.empty[slot]);
-      q++;
       if (ct == 0) stamp(P, l, TR_DN_DONE);
     }
-    // routing used by this layer (one CTA records it for the host)
-    if (ct < k) {
-      if (!pred) S.sel_all[l & 63][ct] = S.sel[ct];
-      if (c == 0) P.hist_out[((size_t)l * P.maxT) * k + ct] = S.sel_all[l & 63][ct];
-    }
+    // release the item's ring space
+    cbar();
+    if (lane == 0) mbar_arrive(&S.empty[slot]);
+    q++;
   }
   if (ab) return;
   // ---- head top-k: CTA c handles layer c's head; its logits are complete by now ------

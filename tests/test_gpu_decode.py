@@ -177,6 +177,48 @@ def test_one_launch_decode_equals_general_path_small(cuda_ok):
     ref.close()
 
 
+def _decode_bits(ctx, dims, seed, S, lag):
+    ctx.debug_decode_lag(lag)
+    out = []
+    for t in range(S):
+        h = bf16_tensor(synth.hidden(seed, t, dims.L, 1, dims.d), "cuda")
+        y32 = torch.empty((dims.L, 1, dims.d), dtype=torch.float32, device="cuda")
+        y = ctx.stack_decode(h, t, y_f32=y32)
+        ctx.sync_status()
+        idx, pred = ctx.get_routing(1)
+        out.append((y.view(torch.int16).cpu().numpy().copy(), y32.cpu().numpy().copy(), idx, pred))
+    return out
+
+
+@pytest.mark.parametrize("heads", [(0, 1, 2), (0, 2)])
+def test_one_launch_decode_lag_is_bitwise_invariant(cuda_ok, heads):
+    """Overlapping the stages of unchained layers (down stage `lag` layers behind gate/up,
+    reactive layers' routers first) changes the order of the work, not its arithmetic: the
+    outputs, routing and predictions are bit-identical to in-order execution, for a stack of
+    mostly predicted layers and one with reactive layers in between."""
+    dims = Dims(d=256, E=16, I=128, k=4, r=8, L=6, head_layers=heads)
+    ctx, _, _ = build(dims, 95, 4)
+    base = _decode_bits(ctx, dims, 96, 4, 0)
+    for lag in (1, 2, 3, 8):
+        got = _decode_bits(ctx, dims, 96, 4, lag)
+        for t, (a, b) in enumerate(zip(base, got)):
+            for u, v in zip(a, b):
+                assert np.array_equal(u, v), f"lag {lag} step {t}"
+    ctx.close()
+
+
+def test_full_size_decode_lag_is_bitwise_invariant(full_model):
+    """The bench's configuration (40 layers, lag 2) against in-order execution, two steps."""
+    try:
+        base = _decode_bits(full_model, FULL, 7, 2, 0)
+        got = _decode_bits(full_model, FULL, 7, 2, 2)
+    finally:
+        full_model.debug_decode_lag(2)
+    for t, (a, b) in enumerate(zip(base, got)):
+        for u, v in zip(a, b):
+            assert np.array_equal(u, v), f"step {t}"
+
+
 def test_one_launch_decode_chained_b1(cuda_ok):
     ctx, _, _ = build(SMALL, 92, 4)
     gpu = run_steps(ctx, SMALL, 92, 1, 3, chained=True)
