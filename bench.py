@@ -277,8 +277,8 @@ def run_decode(args, dims, seed, B, ws, rank, local):
         hds.append(hd)
     ctx.register_model(lys, hds)
     ctx.debug_decode_mode(args.decode_mode)
-    if args.decode_lag is not None:
-        ctx.debug_decode_lag(args.decode_lag)
+    if args.decode_flat is not None:
+        ctx.debug_decode_flat(args.decode_flat)
     setup_s = time.time() - t0
     steps, warm = args.steps, args.warmup
     total = steps + warm
@@ -524,8 +524,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-mode", type=int, default=0, help="0 default, 1 one-launch, 2 graph, 3 eager")
-    ap.add_argument("--decode-lag", type=int, default=None,
-                    help="one-launch kernel: down stage this many layers behind gate/up (0 = in order)")
+    ap.add_argument("--decode-flat", type=int, default=None,
+                    help="one-launch kernel on unchained steps: 1 flat schedule (default), 0 layers in order")
     args = ap.parse_args()
     wl = synth.WORKLOADS[args.workload]
     dims, seed = wl["dims"], wl["seed"]

@@ -245,13 +245,14 @@ int e0_debug_decode_mode(e0_ctx *ctx, int mode);
  * [grid][L][16], caller-owned device buffer; NULL stops it).  Returns the grid size. */
 int e0_debug_decode_trace(e0_ctx *ctx, unsigned long long *buf);
 int e0_debug_force_general(e0_ctx *ctx, int on);
-/* Stage overlap of the one-launch decode kernel on unchained steps (every layer's input
- * given, none read from another layer's output): the down stage of a layer runs `lag`
- * layers behind its gate/up stage, so that the exchange of the intermediate activations
- * between the CTAs overlaps other layers' work.  0 = layers strictly in order; default 2;
- * chained steps always run in order.  Results do not depend on it (each layer's
- * arithmetic is the same).  E0_ERR_INVALID_ARG outside 0..8. */
-int e0_debug_decode_lag(e0_ctx *ctx, int lag);
+/* Schedule of the one-launch decode kernel on unchained steps (every layer's input
+ * given, none read from another layer's output): 1 (default) = flat — each phase's work
+ * (reactive routers, x rows, gate/up, down) over all layers is one list split evenly and
+ * contiguously across the CTAs, so that a CTA streams long runs of one or two layers and
+ * waits on other CTAs only between phases; 0 = layers in order, every CTA on a share of
+ * each layer.  Chained steps always run in order.  Results are bit-identical under both.
+ * E0_ERR_INVALID_ARG unless 0 or 1. */
+int e0_debug_decode_flat(e0_ctx *ctx, int on);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *e0_last_error(void);

@@ -82,7 +82,7 @@ _SIGS = {
     "e0_debug_decode_trace": (_I, [_P, _P]),
     "e0_debug_prefill_path": (_I, [_P, _I]),
     "e0_debug_decode_mode": (_I, [_P, _I]),
-    "e0_debug_decode_lag": (_I, [_P, _I]),
+    "e0_debug_decode_flat": (_I, [_P, _I]),
 }
 
 
@@ -273,8 +273,8 @@ class Context:
     def debug_decode_mode(self, mode: int):
         _check(lib().e0_debug_decode_mode(self._h, mode))
 
-    def debug_decode_lag(self, lag: int):
-        _check(lib().e0_debug_decode_lag(self._h, lag))
+    def debug_decode_flat(self, on: bool):
+        _check(lib().e0_debug_decode_flat(self._h, int(on)))
 
     def debug_prefill_path(self, mode: int):
         _check(lib().e0_debug_prefill_path(self._h, mode))

@@ -74,7 +74,7 @@ struct DecodeState {
   int G = 0;
   size_t smem = 0;
   int stall_cta = -1;
-  int lag = 2;                           // unchained steps: down stage this many layers behind
+  int flat = 1;                          // unchained steps: the flat schedule
   unsigned long long timeout_ns = 2000000000ull;
   unsigned long long *trace = nullptr;   // profiling timeline (caller-owned), or nullptr
 };
@@ -122,8 +122,9 @@ struct e0_ctx {
   cudaStream_t cap = nullptr;        // private stream the decode graphs are captured on
   uint16_t *g_h = nullptr, *g_y = nullptr;   // [L][maxT][d] graph input / output
   float *g_yf = nullptr;                     // [L][maxT][d]
-  // tensor-core prefill workspaces
-  __half *x16 = nullptr, *a16 = nullptr;
+  // tensor-core prefill workspaces: K-permuted bf16 operands and their group-of-64 sums
+  uint16_t *xp = nullptr, *ap = nullptr;
+  float *xsum = nullptr, *asum = nullptr;
   float *yacc = nullptr;
   TcTile *tiles = nullptr;
   int *ntiles = nullptr;
@@ -159,7 +160,7 @@ extern "C" int e0_destroy(e0_ctx *C) {
   cudaDeviceSynchronize();
   void *bufs[] = {C->xb, C->xf, C->logits, C->hlog, C->lt, C->gates, C->idx, C->a, C->plan_mem,
                   C->yscratch, C->pred_tab, C->hist_tab, C->err, C->h1pre, C->h1, C->pool.mem, C->pool.slot_of,
-                  C->pool.slot_tag, C->x16, C->a16, C->yacc, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
+                  C->pool.slot_tag, C->xp, C->ap, C->xsum, C->asum, C->yacc, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
   for (void *b : bufs)
     if (b) cudaFree(b);
   decode_free(C->dec);
@@ -214,7 +215,9 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
   cudaMemset(C->pf_idx, 0xFF, (T + 1) * k * sizeof(int32_t));
   if (T >= kTcMinTokens) {
     C->tile_cap = (int)((T * k + kTcN - 1) / kTcN + std::min(E, T * k) + (T + kTcN - 1) / kTcN + 1);
-    if ((rc = dalloc(&C->x16, T * d)) || (rc = dalloc(&C->a16, T * (k + 1) * I)) || (rc = dalloc(&C->yacc, T * d)) ||
+    if ((rc = dalloc(&C->xp, T * d)) || (rc = dalloc(&C->ap, T * (k + 1) * I)) ||
+        (rc = dalloc(&C->xsum, T * (d / 64 + 1))) || (rc = dalloc(&C->asum, T * (k + 1) * (I / 64 + 1))) ||
+        (rc = dalloc(&C->yacc, T * d)) ||
         (rc = dalloc(&C->tiles, (size_t)C->tile_cap)) || (rc = dalloc(&C->ntiles, 1))) {
       e0_destroy(C);
       return rc;
@@ -297,6 +300,14 @@ static inline int grid_for(int warps_needed, int cap) {
   return b < 1 ? 1 : (b > cap ? cap : b);
 }
 
+// The tensor-core kernels serve calls of at least kTcMinTokens tokens (or any size when
+// selected), in contexts created with the workspaces for them.
+static bool use_tc(e0_ctx *C, int T) {
+  const e0_dims &D = C->dims;
+  return C->xp && D.d_model % 128 == 0 && D.d_model <= 64 * kTcMaxGroups && D.d_ff % 64 == 0 &&
+         D.d_ff <= 64 * kTcMaxGroups && (C->prefill_path == 2 || (C->prefill_path == 0 && T >= kTcMinTokens));
+}
+
 static int layer_pre(e0_ctx *C, const LayerCall &K, cudaStream_t s) {
   const e0_dims &D = C->dims;
   const e0_layer &Y = C->layers[K.l];
@@ -311,10 +322,31 @@ static int layer_pre(e0_ctx *C, const LayerCall &K, cudaStream_t s) {
   R.hlog = C->hlog;
   R.Ag = (const uint16_t *)Y.lora_Ag; R.Au = (const uint16_t *)Y.lora_Au; R.r = D.lora_rank; R.lt = C->lt;
   R.err = C->err;
-  const int nTT = (K.T + kRowTile - 1) / kRowTile;
-  const int J = D.n_experts * nTT + K.T * D.top_k + (R.Wh ? D.n_experts * nTT : 0) + (R.Ag ? 2 * D.lora_rank * nTT : 0);
-  k_rows<<<grid_for(J, 8 * C->nsm), 256, 0, s>>>(R);
-  CKL("k_rows");
+  if (use_tc(C, K.T)) {
+    // every row on the tensor cores: full router logits for every token, head, LoRA A
+    TcRowsArgs W{};
+    W.x = C->xb; W.T = K.T; W.d = D.d_model; W.err = C->err; W.timeout_ns = 2000000000ull;
+    W.seg[W.nseg++] = RowSeg{R.Wr, D.n_experts, D.d_model, C->logits, D.n_experts, 0};
+    if (R.Wh) W.seg[W.nseg++] = RowSeg{R.Wh, D.n_experts, R.ldh, C->hlog, D.n_experts, 0};
+    if (R.Ag) {
+      W.seg[W.nseg++] = RowSeg{R.Ag, D.lora_rank, D.d_model, C->lt, 3 * D.lora_rank, 0};
+      W.seg[W.nseg++] = RowSeg{R.Au, D.lora_rank, D.d_model, C->lt, 3 * D.lora_rank, D.lora_rank};
+    }
+    for (int q = 0; q < W.nseg; q++) W.total += W.seg[q].rows;
+    const int smem = (int)sizeof(TcRowsSmem) + 1024;
+    static bool attr_rows = false;
+    if (!attr_rows) {
+      CK(cudaFuncSetAttribute(k_tc_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+      attr_rows = true;
+    }
+    k_tc_rows<<<dim3((W.total + 127) / 128, (K.T + kTcN - 1) / kTcN), kTcThreads, smem, s>>>(W);
+    CKL("k_tc_rows");
+  } else {
+    const int nTT = (K.T + kRowTile - 1) / kRowTile;
+    const int J = D.n_experts * nTT + K.T * D.top_k + (R.Wh ? D.n_experts * nTT : 0) + (R.Ag ? 2 * D.lora_rank * nTT : 0);
+    k_rows<<<grid_for(J, 8 * C->nsm), 256, 0, s>>>(R);
+    CKL("k_rows");
+  }
   RouteArgs A{};
   A.logits = C->logits; A.T = K.T; A.E = D.n_experts; A.k = D.top_k; A.route = K.route; A.full_mode = K.full_mode;
   A.idx = K.idx; A.gates = K.gates; A.hist = K.hist;
@@ -330,14 +362,15 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   const e0_dims &D = C->dims;
   const e0_layer &Y = C->layers[K.l];
   const size_t nx = (size_t)K.T * D.d_model;
-  k_bf16_to_f16<<<(unsigned)((nx + 255) / 256), 256, 0, s>>>(C->xb, C->x16, nx);
-  CKL("k_bf16_to_f16");
+  const long long xg = (long long)K.T * (D.d_model / 64);
+  k_perm_sums<<<(unsigned)((xg + 255) / 256), 256, 0, s>>>(C->xb, K.T, D.d_model, C->xp, C->xsum);
+  CKL("k_perm_sums(x)");
   k_tc_tiles<<<1, 32, 0, s>>>(C->plan, K.T, C->tiles, C->ntiles, C->tile_cap);
   CKL("k_tc_tiles");
   TcArgs A{};
   A.mode = 0; A.T = K.T; A.d = D.d_model; A.I = D.d_ff; A.k = D.top_k; A.r = D.lora_rank; A.c = D.lora_scale;
   A.src = src; A.shared = (const uint8_t *)Y.shared; A.bl = C->bl; A.P = C->plan; A.tiles = C->tiles;
-  A.ntiles = C->ntiles; A.x16 = C->x16; A.a16 = C->a16; A.a16_out = C->a16;
+  A.ntiles = C->ntiles; A.xp = C->xp; A.xsum = C->xsum; A.ap = C->ap; A.asum = C->asum; A.ap_out = C->ap;
   A.Bg = (const uint16_t *)Y.lora_Bg; A.Bu = (const uint16_t *)Y.lora_Bu; A.lt = C->lt; A.gates = K.gates;
   A.yacc = C->yacc; A.err = C->err; A.timeout_ns = 2000000000ull;
   const int tc_smem_bytes = (int)sizeof(TcSmem) + 1024;
@@ -350,10 +383,14 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
                                               (K.T + kTcN - 1) / kTcN);
   k_moe_gemm_tc<<<tmax * (D.d_ff / 64), kTcThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(gate/up)");
+  const long long ag = (long long)K.T * (D.top_k + 1) * (D.d_ff / 64);
+  k_perm_sums<<<(unsigned)((ag + 255) / 256), 256, 0, s>>>(C->ap, (long long)K.T * (D.top_k + 1), D.d_ff, nullptr,
+                                                          C->asum);
+  CKL("k_perm_sums(a)");
   if (Y.lora_Ad) {
-    k_lora_t16<<<(K.T * D.lora_rank + 7) / 8, 256, 0, s>>>((const uint16_t *)Y.lora_Ad, C->a16, K.T, D.d_ff,
-                                                            D.top_k, D.lora_rank, C->lt);
-    CKL("k_lora_t16");
+    k_lora_td<<<(K.T * D.lora_rank + 7) / 8, 256, 0, s>>>((const uint16_t *)Y.lora_Ad, C->ap, K.T, D.d_ff,
+                                                           D.top_k, D.lora_rank, C->lt);
+    CKL("k_lora_td");
   }
   CK(cudaMemsetAsync(C->yacc, 0, nx * sizeof(float), s));
   A.mode = 1;
@@ -370,8 +407,7 @@ static int layer_post(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cudaS
   const e0_layer &Y = C->layers[K.l];
   k_plan<<<1, 1024, 0, s>>>(K.idx, K.T * D.top_k, D.n_experts, C->plan);
   CKL("k_plan");
-  const bool tc = C->x16 && src.pool == nullptr && D.d_model % 128 == 0 && D.d_ff % 64 == 0 &&
-                  (C->prefill_path == 2 || (C->prefill_path == 0 && K.T >= kTcMinTokens));
+  const bool tc = src.pool == nullptr && use_tc(C, K.T);
   if (tc) return layer_post_tc(C, K, src, s);
   GateUpArgs G{};
   G.xf = C->xf; G.T = K.T; G.d = D.d_model; G.I = D.d_ff; G.k = D.top_k; G.r = D.lora_rank; G.c = D.lora_scale;
@@ -814,7 +850,7 @@ static int decode_persistent(e0_ctx *C, const uint16_t *h, int step, uint16_t *y
   P.onehot = D.head_onehot; P.G = S.G;
   P.eps = D.rms_eps; P.c = D.lora_scale;
   P.h = h; P.y = y; P.yf = yf; P.chained = chained;
-  P.lag = chained ? 0 : S.lag;
+  P.flat = chained ? 0 : S.flat;
   P.epoch = ++S.epoch;
   P.step0 = step == 0;
   P.pred_in = step > 0 ? pred_at(C, prv, 0) : nullptr;
@@ -1044,11 +1080,11 @@ extern "C" int e0_debug_decode_mode(e0_ctx *C, int mode) {
   return E0_OK;
 }
 
-// Stage overlap of the one-launch decode kernel on unchained steps: the down stage of a
-// layer runs `lag` layers behind its gate/up stage (0 = layers strictly in order).
-extern "C" int e0_debug_decode_lag(e0_ctx *C, int lag) {
-  if (!C || lag < 0 || lag > 8) return fail(E0_ERR_INVALID_ARG, "bad decode lag");
-  C->dec.lag = lag;
+// Schedule of the one-launch decode kernel on unchained steps: 1 = flat (default), 0 =
+// layers in order.
+extern "C" int e0_debug_decode_flat(e0_ctx *C, int on) {
+  if (!C || on < 0 || on > 1) return fail(E0_ERR_INVALID_ARG, "bad decode schedule");
+  C->dec.flat = on;
   return E0_OK;
 }
 

@@ -33,7 +33,7 @@ namespace e0 {
 constexpr int kDecThreads = 416;          // 1 producer warp + 12 consumer warps
 constexpr int kDecConsumers = 384;
 constexpr int kDecCW = 12;
-constexpr int kRingBytes = 142 * 1024;
+constexpr int kRingBytes = 156 * 1024;
 constexpr int kDecMaxK = 4;               // routed experts per token on this path
 constexpr int kNSlot = 8;                 // tasks in flight
 constexpr int kMaxSeg = 96;               // bulk-copy segments per task
@@ -55,10 +55,10 @@ struct DecodeParams {
   uint16_t *y;              // [L][D]
   float *yf;                // [L][D] or nullptr
   int chained;
-  // 0: layers run in order, each layer's first stage waiting for the previous layer's
-  // output; > 0 (unchained inputs only): the stages of different layers overlap, the down
-  // stage of a layer running `lag` layers behind its gate/up stage
-  int lag;
+  // 0: layers in order (each layer's first x item waits for the previous layer's output);
+  // 1 (unchained inputs only): the flat schedule, every phase's work over all layers
+  // split evenly across the CTAs
+  int flat;
   uint32_t epoch;
   int step0;                // 1: every layer routes with its own router
   const int32_t *pred_in;   // [L+1][maxT][k]: routing predicted for layer l (previous step)
@@ -149,24 +149,6 @@ __device__ __forceinline__ bool cbar_or(bool pred) {
 __device__ __forceinline__ void cbar() {
   asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumers) : "memory");
 }
-__device__ __forceinline__ unsigned long long pk2(float a, float b) {
-  return ((unsigned long long)__float_as_uint(b) << 32) | __float_as_uint(a);
-}
-__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b,
-                                                    unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float f2sum(unsigned long long v) {
-  return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
-}
-
 // Balanced contiguous split of N items over G parts (N * G < 2^31 here).
 __host__ __device__ __forceinline__ void split_range(int N, int G, int c, int &a, int &b) {
   a = (int)((unsigned)(N * c) / (unsigned)G);
@@ -252,79 +234,109 @@ struct TaskBuf {
   }
 };
 
-enum : int { TK_ROUTER = 0, TK_GU = 1, TK_DN = 2 };
+// ---------------------------------------------------------------------------------------
+// Work items.  A launch runs a list of items, the same sequence for the producer (which
+// streams each item's bytes into the ring) and the consumers (which compute it).  An item
+// is one kind of work on a contiguous range [a, a + n) of one layer's units:
+//   IT_R   router rows of a reactive layer                         (units: the E experts)
+//   IT_TK  top-k of a reactive layer over all its router logits   (consumers only)
+//   IT_XR  the other rows dotted with x: the layer's head rows (E, if it has a head),
+//          then the shared expert's A_g rows and A_u rows (r each, with LoRA), then the
+//          router rows of the predicted experts (k, predicted layers)
+//   IT_GU  expert gate/up: unit u = slot u / I (k routed, then the shared expert) and
+//          intermediate index u % I, i.e. one gate row and one up row
+//   IT_DN  output rows of the down projection and the weighted combine
+// The flag bit: on R, XR and GU items, compute the layer's RMSNorm first (the
+// previous x item had another layer); on DN items, this is the CTA's first down item of
+// the layer, which assembles the shared expert's a_s (with the LoRA up branch) and
+// t_d = A_d a_s from the whole LoRA matrices that its task carries, kept for the layer's
+// later down items.  The flags are decided when the list is built, so that producer and
+// consumers agree on what each task holds.
+// ---------------------------------------------------------------------------------------
+enum : int { IT_R = 0, IT_TK = 1, IT_XR = 2, IT_GU = 3, IT_DN = 4 };
+constexpr int kMaxItems = 320;
 
-// Items of a launch's schedule, the same sequence for the producer and the consumers:
-//   IT_R   router rows of a reactive layer (producer task),
-//   IT_TK  top-k of a reactive layer over every CTA's router logits (consumers only),
-//   IT_GU  gate/up stage (producer task), IT_DN  down + combine stage (producer task).
-enum : int { IT_R = 0, IT_TK = 1, IT_GU = 2, IT_DN = 3 };
-constexpr int kMaxSched = 4 * 64;
+struct Item {
+  int kind, l, a, n;
+  bool first;
+};
+__device__ __forceinline__ unsigned long long pack_item(int kind, int l, int a, int n, bool first) {
+  return (unsigned long long)kind | ((unsigned long long)first << 4) | ((unsigned long long)l << 8) |
+         ((unsigned long long)a << 16) | ((unsigned long long)n << 40);
+}
+__device__ __forceinline__ Item unpack_item(unsigned long long v) {
+  return Item{(int)(v & 15ull), (int)((v >> 8) & 255ull), (int)((v >> 16) & 0xFFFFFFull), (int)(v >> 40),
+              ((v >> 4) & 1ull) != 0};
+}
 
-// GU range of a CTA split into per-slot pieces.
+// A range of gate/up units split into per-slot pieces.
 struct GuPiece {
   int slot, i0, i1;
 };
-
-template <int D, int I>
-__device__ __forceinline__ int gu_pieces(int k, int G, int c, GuPiece *out) {
-  int a, b;
-  split_range((k + 1) * I, G, c, a, b);
-  int n = 0;
-  while (a < b) {
+constexpr int kMaxPieces = 4;
+__device__ __forceinline__ int pieces_of(int a, int n, int I, GuPiece *out) {
+  const int b = a + n;
+  int np = 0;
+  while (a < b && np < kMaxPieces) {
     const int slot = a / I, end = min(b, (slot + 1) * I);
-    out[n++] = GuPiece{slot, a - slot * I, end - slot * I};
+    out[np++] = GuPiece{slot, a - slot * I, end - slot * I};
     a = end;
   }
-  return n;
+  return np;
 }
 
-// Segment indices of each task kind (a segment may be empty):
-//   router task: [0] gamma, [1] h, [2] this CTA's router rows
-//   gate/up task: [0] gamma, [1] h, [2] A_g rows, [3] A_u rows, [4, 4+kMaxK) selected
-//     router rows, [4+kMaxK] head rows, then per piece p (up to kMaxPieces) 6 segments:
-//     gate codes, gate scale, gate min, up codes, up scale, up min
-//   down task: [3j .. 3j+2] down codes/scale/min of slot j (j = 0..k), then B_d rows, B_g,
-//     B_u, A_d (LoRA matrices of the shared expert, whole)
-constexpr int kMaxPieces = 4;
-constexpr int kGuHead = 4 + kMaxK;
-constexpr int kGuPiece0 = 5 + kMaxK;
+// [s0, s1) = the part of [a, a + n) inside [lo, hi), relative to lo (empty: s0 = s1 = 0)
+__device__ __forceinline__ void sub_range(int a, int n, int lo, int hi, int &s0, int &s1) {
+  s0 = max(a, lo) - lo;
+  s1 = min(a + n, hi) - lo;
+  if (s1 <= s0) s0 = s1 = 0;
+}
+
+// Segment indices of each task (a segment may be empty):
+//   R:  [0] gamma, [1] h (when the item computes the norm), [2] router rows
+//   XR: [0] gamma, [1] h, [2] head rows, [3] A_g rows, [4] A_u rows, [5, 5 + kMaxK) the
+//       selected router rows
+//   GU: [0] gamma, [1] h, then per piece p (up to kMaxPieces) 6 segments from 2 + 6 p:
+//       gate codes, gate scale, gate min, up codes, up scale, up min
+//   DN: [3j .. 3j+2] down codes/scale/min of slot j (j = 0..k), then B_d rows, and on a
+//       layer's first down item B_g, B_u, A_d (the shared expert's LoRA matrices, whole)
+constexpr int kXrHead = 2, kXrAg = 3, kXrAu = 4, kXrSel = 5;
+constexpr int kGuPiece0 = 2;
 __device__ __forceinline__ int dn_bd(int k) { return 3 * (k + 1); }
 
-// Build the segment list of task (kind, layer) for CTA c.  `sel` are the layer's routed
+// Build the segment list of item `it` (rows of layer Y).  `sel` are the layer's routed
 // experts.  The consumer code reads the segments back by the indices above.
 template <int D, int I>
-__device__ __noinline__ void build_task(const DecodeParams &P, const DecLayer &Y, int kind, int l, int c, bool predicted,
-                           const int *sel, TaskBuf &T) {
+__device__ __noinline__ void build_task(const DecodeParams &P, const DecLayer &Y, const Item &it, bool predicted,
+                                        const int *sel, TaskBuf &T) {
   const Blob bl = blob_of(D, I);
   T.n = 0;
   T.overflow = 0;
-  if (kind == TK_ROUTER) {
-    T.add(Y.gamma, D * 2);
-    T.add(P.h + (size_t)l * D, D * 2);
-    int a, b;
-    split_range(P.E, P.G, c, a, b);
-    T.add(Y.router + (size_t)a * D, (size_t)(b - a) * D * 2);
-  } else if (kind == TK_GU) {
-    T.add(Y.gamma, D * 2);
-    T.add(P.h + (size_t)l * D, D * 2);
-    int a = 0, b = 0;
-    if (Y.Ag) split_range(2 * P.r, P.G, c, a, b);
-    const int ga = min(a, P.r), gb = min(b, P.r), ua = max(a, P.r) - P.r, ub = max(b, P.r) - P.r;
-    T.add(Y.Ag + (size_t)ga * D, (size_t)(gb - ga) * D * 2);
-    T.add(Y.Au + (size_t)ua * D, (size_t)(ub - ua) * D * 2);
-    a = b = 0;
-    if (predicted) split_range(P.k, P.G, (c + P.G - min(2 * P.r, P.G - 1)) % P.G, a, b);
+  const int l = it.l, a = it.a, n = it.n;
+  if (it.kind != IT_DN) {
+    T.add(Y.gamma, it.first ? D * 2 : 0);
+    T.add(P.h + (size_t)l * D, it.first ? D * 2 : 0);
+  }
+  if (it.kind == IT_R) {
+    T.add(Y.router + (size_t)a * D, (size_t)n * D * 2);
+  } else if (it.kind == IT_XR) {
+    const int nh = Y.head ? P.E : 0, nl = Y.Ag ? P.r : 0, ns = predicted ? P.k : 0;
+    int s0, s1;
+    sub_range(a, n, 0, nh, s0, s1);
+    T.add(Y.head + (size_t)s0 * P.ldh, (size_t)(s1 - s0) * P.ldh * 2);
+    sub_range(a, n, nh, nh + nl, s0, s1);
+    T.add(Y.Ag + (size_t)s0 * D, (size_t)(s1 - s0) * D * 2);
+    sub_range(a, n, nh + nl, nh + 2 * nl, s0, s1);
+    T.add(Y.Au + (size_t)s0 * D, (size_t)(s1 - s0) * D * 2);
+    sub_range(a, n, nh + 2 * nl, nh + 2 * nl + ns, s0, s1);
     #pragma unroll 1
     for (int q = 0; q < kMaxK; q++) {
-      const bool on = a + q < b;
-      T.add(Y.router + (size_t)(on ? sel[a + q] : 0) * D, on ? D * 2 : 0);
+      const bool on = s0 + q < s1;
+      T.add(Y.router + (size_t)(on ? sel[s0 + q] : 0) * D, on ? D * 2 : 0);
     }
-    int ha = 0, hb = 0;
-    if (Y.head) split_range(P.E, P.G, c, ha, hb);
-    T.add(Y.head + (size_t)ha * P.ldh, (size_t)(hb - ha) * P.ldh * 2);
+  } else if (it.kind == IT_GU) {
     GuPiece pc[kMaxPieces];
-    const int np = gu_pieces<D, I>(P.k, P.G, c, pc);
+    const int np = pieces_of(a, n, I, pc);
     #pragma unroll 1
     for (int p = 0; p < np; p++) {
       const uint8_t *base = pc[p].slot < P.k ? Y.experts + (size_t)sel[pc[p].slot] * bl.bytes : Y.shared;
@@ -336,19 +348,16 @@ __device__ __noinline__ void build_task(const DecodeParams &P, const DecLayer &Y
       T.add(base + bl.us + (size_t)i0 * (D / 64) * 2, (size_t)R * (D / 64) * 2);
       T.add(base + bl.um + (size_t)i0 * (D / 64) * 2, (size_t)R * (D / 64) * 2);
     }
-  } else {
-    int a, b;
-    split_range(D, P.G, c, a, b);
-    const int R = b - a;
+  } else if (it.kind == IT_DN) {
     #pragma unroll 1
     for (int j = 0; j <= P.k; j++) {
       const uint8_t *base = j < P.k ? Y.experts + (size_t)sel[j] * bl.bytes : Y.shared;
-      T.add(base + bl.dc + (size_t)a * (I / 2), (size_t)R * (I / 2));
-      T.add(base + bl.ds + (size_t)a * (I / 64) * 2, (size_t)R * (I / 64) * 2);
-      T.add(base + bl.dm + (size_t)a * (I / 64) * 2, (size_t)R * (I / 64) * 2);
+      T.add(base + bl.dc + (size_t)a * (I / 2), (size_t)n * (I / 2));
+      T.add(base + bl.ds + (size_t)a * (I / 64) * 2, (size_t)n * (I / 64) * 2);
+      T.add(base + bl.dm + (size_t)a * (I / 64) * 2, (size_t)n * (I / 64) * 2);
     }
-    T.add(Y.Bd + (size_t)a * P.r, Y.Bd ? (size_t)R * P.r * 2 : 0);
-    const size_t lb = Y.Bg ? (size_t)I * P.r * 2 : 0;
+    T.add(Y.Bd + (size_t)a * P.r, Y.Bd ? (size_t)n * P.r * 2 : 0);
+    const size_t lb = (Y.Bg && it.first) ? (size_t)I * P.r * 2 : 0;
     T.add(Y.Bg, lb);
     T.add(Y.Bu, lb);
     T.add(Y.Ad, lb);
@@ -377,8 +386,8 @@ struct DecSmem {
   int sel_all[64][kMaxK];            // routing of every layer this step
   float rlsel[64][kMaxK];            // a reactive layer's router logits of its chosen experts
   volatile int sel_ok[64];           // 1 once a reactive layer's top-k is in sel_all
-  uint16_t sched[kMaxSched];         // this launch's items: kind << 8 | layer
-  int nsched;
+  unsigned long long items[kMaxItems];   // this CTA's item list (pack_item)
+  int nitems;
   DecLayer lay[64];                  // the layer table
   TaskBuf tb;                        // the producer's task being issued
   int tb_off[kMaxSeg];
@@ -406,49 +415,122 @@ __device__ __forceinline__ bool timed_out(unsigned long long &t0, unsigned long 
 }
 
 // ---------------------------------------------------------------------------------------
-// The launch's schedule (one thread).  In order (lag 0): per layer [R, TK] GU DN.  With a
-// lag (unchained inputs: no layer reads another layer's output within the step): the
-// layers are taken predicted first, then reactive; the router rows of every reactive
-// layer come first, a reactive layer's top-k two layers before its gate/up stage (so the
-// producer can fetch its experts early), and each down stage `lag` layers after its
-// gate/up stage, so that the exchange between the two stages overlaps other layers' work.
+// The launch's item list of this CTA (one thread).
+//
+// In order (chained inputs, or for comparison): per layer [R, TK] XR GU DN, each x item
+// and the down item over this CTA's balanced share of the layer's units.
+//
+// Flat (unchained inputs: no layer reads another layer's output within the step, so the
+// layers are independent apart from the predictions that cross to the next token): each
+// phase's units over all layers form one list, split evenly and contiguously across the
+// CTAs, so that a CTA streams long runs of rows of one or two layers instead of a sliver
+// of every layer.  Phases: R (reactive layers' routers), XR, TK (the reactive layers this
+// CTA needs), GU, DN.  Items are cut to at most about 36 KB of weight bytes.  A CTA then
+// computes a handful of norms per step, polls other CTAs' results a handful of times, and
+// waits on other CTAs only where a phase needs the previous one (R -> TK, GU -> DN).
 // ---------------------------------------------------------------------------------------
 template <int D, int I>
+__device__ __forceinline__ int xrows_of(const DecodeParams &P, const DecSmem<D, I> &S, int l) {
+  const DecLayer &Y = S.lay[l];
+  return (Y.head ? P.E : 0) + (Y.Ag ? 2 * P.r : 0) + (is_predicted(P, S, l) ? P.k : 0);
+}
+
+template <int D, int I>
 __device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I> &S) {
+  const int G = P.G, c = blockIdx.x, L = P.L, k = P.k;
   int n = 0;
-  if (P.lag == 0) {
+  auto put = [&](int kind, int l, int a, int cnt) {
+    if (n < kMaxItems) S.items[n++] = pack_item(kind, l, a, cnt, false);
+    else atomicOr(P.err, DERR_TIMEOUT);   // cannot happen for the supported sizes
+  };
+  if (!P.flat) {
     #pragma unroll 1
-    for (int l = 0; l < P.L; l++) {
+    for (int l = 0; l < L; l++) {
+      int a, b;
       if (!is_predicted(P, S, l)) {
-        S.sched[n++] = (uint16_t)((IT_R << 8) | l);
-        S.sched[n++] = (uint16_t)((IT_TK << 8) | l);
+        split_range(P.E, G, c, a, b);
+        if (b > a) put(IT_R, l, a, b - a);
+        put(IT_TK, l, 0, 0);
       }
-      S.sched[n++] = (uint16_t)((IT_GU << 8) | l);
-      S.sched[n++] = (uint16_t)((IT_DN << 8) | l);
+      split_range(xrows_of(P, S, l), G, c, a, b);
+      if (b > a) put(IT_XR, l, a, b - a);
+      split_range((k + 1) * I, G, c, a, b);
+      if (b > a) put(IT_GU, l, a, b - a);
+      split_range(D, G, c, a, b);
+      if (b > a) put(IT_DN, l, a, b - a);
     }
   } else {
-    constexpr int PF = 2;
-    uint8_t ord[64];
-    int no = 0;
-    #pragma unroll 1
-    for (int pass = 0; pass < 2; pass++)
+    constexpr int kItemBytes = 36 * 1024;
+    const int gu_chunk = min(kItemBytes / (2 * (D / 2 + D / 16)), 288);
+    const int dn_chunk = min(kItemBytes / ((k + 1) * (I / 2 + I / 16) + 2 * P.r), 64);
+    const int xr_chunk = max(kItemBytes / (2 * P.ldh), 1);
+    // one phase: units(l) per layer over every layer with units, this CTA's share
+    auto phase = [&](int kind, int chunk, int which) {
+      long long tot = 0;
       #pragma unroll 1
-      for (int l = 0; l < P.L; l++)
-        if (is_predicted(P, S, l) == (pass == 0)) ord[no++] = (uint8_t)l;
+      for (int l = 0; l < L; l++) {
+        const int u = which == 0 ? (is_predicted(P, S, l) ? 0 : P.E)
+                    : which == 1 ? xrows_of(P, S, l) : which == 2 ? (k + 1) * I : D;
+        tot += u;
+      }
+      const long long lo = tot * c / G, hi = tot * (c + 1) / G;
+      long long base = 0;
+      #pragma unroll 1
+      for (int l = 0; l < L; l++) {
+        const int u = which == 0 ? (is_predicted(P, S, l) ? 0 : P.E)
+                    : which == 1 ? xrows_of(P, S, l) : which == 2 ? (k + 1) * I : D;
+        const long long s0 = max(lo, base), s1 = min(hi, base + u);
+        for (long long a = s0; a < s1; a += chunk) put(kind, l, (int)(a - base), (int)min((long long)chunk, s1 - a));
+        base += u;
+      }
+    };
+    phase(IT_R, 9, 0);
+    phase(IT_XR, xr_chunk, 1);
+    const int n_before_tk = n;
+    // placeholder for the top-k items: the reactive layers that this CTA's gate/up or
+    // down items touch
+    phase(IT_GU, gu_chunk, 2);
+    phase(IT_DN, dn_chunk, 3);
+    bool need[64];
     #pragma unroll 1
-    for (int j = 0; j < no; j++)
-      if (!is_predicted(P, S, ord[j])) S.sched[n++] = (uint16_t)((IT_R << 8) | ord[j]);
+    for (int l = 0; l < L; l++) need[l] = false;
     #pragma unroll 1
-    for (int j = 0; j < PF && j < no; j++)
-      if (!is_predicted(P, S, ord[j])) S.sched[n++] = (uint16_t)((IT_TK << 8) | ord[j]);
-    #pragma unroll 1
-    for (int j = 0; j < no + P.lag; j++) {
-      if (j + PF < no && !is_predicted(P, S, ord[j + PF])) S.sched[n++] = (uint16_t)((IT_TK << 8) | ord[j + PF]);
-      if (j < no) S.sched[n++] = (uint16_t)((IT_GU << 8) | ord[j]);
-      if (j >= P.lag && j - P.lag < no) S.sched[n++] = (uint16_t)((IT_DN << 8) | ord[j - P.lag]);
+    for (int q = n_before_tk; q < n; q++) {
+      const Item it = unpack_item(S.items[q]);
+      if (!is_predicted(P, S, it.l)) need[it.l] = true;
     }
+    int ntk = 0;
+    #pragma unroll 1
+    for (int l = 0; l < L; l++) ntk += need[l];
+    if (n + ntk > kMaxItems) {
+      atomicOr(P.err, DERR_TIMEOUT);
+      ntk = 0;
+    }
+    #pragma unroll 1
+    for (int q = n - 1; q >= n_before_tk; q--) S.items[q + ntk] = S.items[q];
+    int w = n_before_tk;
+    #pragma unroll 1
+    for (int l = 0; l < L && ntk; l++)
+      if (need[l]) S.items[w++] = pack_item(IT_TK, l, 0, 0, false);
+    n += ntk;
   }
-  S.nsched = n;
+  // flags: x items compute the norm when the previous x item had another layer; the
+  // first down item of each layer assembles the layer's shared-expert inputs
+  int lastx = -1, lastd = -1;
+  #pragma unroll 1
+  for (int q = 0; q < n; q++) {
+    Item it = unpack_item(S.items[q]);
+    bool f = false;
+    if (it.kind == IT_R || it.kind == IT_XR || it.kind == IT_GU) {
+      f = it.l != lastx;
+      lastx = it.l;
+    } else if (it.kind == IT_DN) {
+      f = it.l != lastd;
+      lastd = it.l;
+    }
+    S.items[q] = pack_item(it.kind, it.l, it.a, it.n, f);
+  }
+  S.nitems = n;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -465,15 +547,15 @@ __device__ void producer(const DecodeParams &P, DecSmem<D, I> &S) {
   bool ok = true;
 
   #pragma unroll 1
-  for (int it = 0; it < S.nsched && ok; it++) {
-    const int item = S.sched[it] >> 8, l = S.sched[it] & 255;
-    if (item == IT_TK) continue;
+  for (int q_it = 0; q_it < S.nitems && ok; q_it++) {
+    const Item it = unpack_item(S.items[q_it]);
+    if (it.kind == IT_TK) continue;
+    const int l = it.l;
     const bool pred = is_predicted(P, S, l);
-    const int kind = item == IT_R ? TK_ROUTER : item == IT_GU ? TK_GU : TK_DN;
     {
-      if (kind != TK_ROUTER) {
-        if (!pred) {
-          // the consumers publish a reactive layer's own top-k (its TK item) first
+      if (it.kind == IT_GU || it.kind == IT_DN || it.kind == IT_XR) {
+        if (!pred && it.kind != IT_XR) {
+          // a reactive layer's experts are known once the consumers ran its TK item
           unsigned long long t0 = 0;
           while (S.sel_ok[l & 63] == 0) {
             if (S.abort) { ok = false; break; }
@@ -491,14 +573,14 @@ __device__ void producer(const DecodeParams &P, DecSmem<D, I> &S) {
         for (int j = 0; j < P.k; j++) {
           sel[j] = S.sel_all[l & 63][j];
           if (sel[j] < 0 || sel[j] >= P.E) {
-            if (lane == 0 && kind == TK_GU) atomicOr(P.err, DERR_INDEX);
+            if (lane == 0 && (pred || it.kind != IT_XR)) atomicOr(P.err, DERR_INDEX);
             sel[j] = 0;
           }
         }
       }
-      if (kind == TK_GU) stamp(P, l, TR_P_GU_START);
-      if (kind == TK_DN) stamp(P, l, TR_P_DN_START);
-      if (lane == 0) build_task<D, I>(P, S.lay[l], kind, l, c, pred, sel, S.tb);   // out of line
+      if (it.kind == IT_GU) stamp(P, l, TR_P_GU_START);
+      if (it.kind == IT_DN) stamp(P, l, TR_P_DN_START);
+      if (lane == 0) build_task<D, I>(P, S.lay[l], it, pred, sel, S.tb);   // out of line
       __syncwarp();
       const int n = S.tb.n;
       if (S.tb.overflow) {
@@ -604,7 +686,7 @@ __device__ void producer(const DecodeParams &P, DecSmem<D, I> &S) {
         head = start + need;
       }
       q++;
-      if (lane == 0) stamp(P, l, kind == TK_GU ? TR_P_GU : kind == TK_DN ? TR_P_DN : TR_P_R);
+      if (lane == 0) stamp(P, l, it.kind == IT_GU ? TR_P_GU : it.kind == IT_DN ? TR_P_DN : TR_P_R);
     }
   }
   // drain: every issued copy must have landed before the CTA exits
@@ -800,13 +882,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
   }
 
   #pragma unroll 1
-  for (int it = 0; it < S.nsched; it++) {
-    const int kind = S.sched[it] >> 8, l = S.sched[it] & 255;
+  for (int q_it = 0; q_it < S.nitems; q_it++) {
+    const Item it = unpack_item(S.items[q_it]);
+    const int l = it.l, ia = it.a, in = it.n;
     const DecLayer &Y = S.lay[l];
     const bool pred = is_predicted(P, S, l);
     const bool lora = Y.Bg != nullptr;
     const uint32_t tag = dtag(P, l);
-    if (kind == IT_TK) {
+    if (it.kind == IT_TK) {
       // ---- a reactive layer's top-k over every CTA's router logits
       ab |= !poll_to(P.t_rlog + (size_t)l * P.E, reinterpret_cast<uint32_t *>(S.rl), P.E, tag, ct, C);
       if (cbar_or(ab)) break;
@@ -827,20 +910,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       if (ct == 0) stamp(P, l, TR_ROUTE);
       continue;
     }
-    // ---- in order: a layer's first item waits for the previous layer's output (its data
-    // in chained mode)
-    if (P.lag == 0 && l > 0 && (kind == IT_R || (kind == IT_GU && pred))) {
+    const bool xitem = it.kind != IT_DN;
+    // ---- in order: a layer's norm waits for the previous layer's output (its data in
+    // chained mode)
+    if (!P.flat && xitem && it.first && l > 0) {
       ab |= !poll_to(P.t_y + (size_t)(l - 1) * D, reinterpret_cast<uint32_t *>(S.yprev), D, dtag(P, l - 1), ct, C);
     }
     if (cbar_or(ab)) break;
-    if (ct == 0 && kind != IT_DN) stamp(P, l, TR_LAYER);
+    if (ct == 0 && xitem && it.first) stamp(P, l, TR_LAYER);
 
     const int slot = q % kNSlot;
     const uint32_t par = (uint32_t)((q / kNSlot) & 1);
     ab |= !wait_full(&S.full[slot], par, C);
     if (cbar_or(ab)) break;
-    if (kind != IT_DN) {
-      // ---- the norm: gamma and h are the first two segments of router and gate/up tasks
+    if (xitem && it.first) {
+      // ---- the norm: gamma and h are the first two segments of the task
       const uint16_t *gam = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][0]);
       const uint16_t *hin = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][1]);
       const bool chain = P.chained && l > 0;
@@ -875,58 +959,46 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         }
       }
       cbar();
+      if (ct == 0) stamp(P, l, TR_NORM);
     }
-    if (ct == 0 && kind != IT_DN) stamp(P, l, TR_NORM);
-    if (kind == IT_R) {
-      // ---- a reactive layer's router rows of this CTA
-      int a, b;
-      split_range(P.E, G, c, a, b);
+    if (it.kind == IT_R) {
+      // ---- router rows of a reactive layer
       const uint16_t *rw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][2]);
       #pragma unroll 1
-      for (int row = a + warp; row < b; row += kDecCW) {
-        const float v = bf16_row_x<D>(rw + (size_t)(row - a) * D, S.x, lane);
-        if (lane == 0) st_tag(P.t_rlog + (size_t)l * P.E + row, tag, __float_as_uint(v));
+      for (int q2 = warp; q2 < in; q2 += kDecCW) {
+        const float v = bf16_row_x<D>(rw + (size_t)q2 * D, S.x, lane);
+        if (lane == 0) st_tag(P.t_rlog + (size_t)l * P.E + ia + q2, tag, __float_as_uint(v));
       }
-    } else if (kind == IT_GU) {
-      // ---- gate/up stage ------------------------------------------------------------
+    } else if (it.kind == IT_XR) {
+      // ---- head rows, LoRA A rows and the predicted experts' router rows on x
+      const int nh = Y.head ? P.E : 0, nl = lora ? r : 0;
+      unsigned long long *blk = P.t_blk + (size_t)l * P.blk;
+      #pragma unroll 1
+      for (int q2 = warp; q2 < in; q2 += kDecCW) {
+        const int u = ia + q2;
+        const uint16_t *row;
+        unsigned long long *dst;
+        if (u < nh) {
+          row = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kXrHead]) + (size_t)(u - ia) * P.ldh;
+          dst = P.t_hlog + (size_t)l * P.E + u;
+        } else if (u < nh + nl) {
+          row = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kXrAg]) + (size_t)(u - max(ia, nh)) * D;
+          dst = blk + (k + 2) * I + (u - nh);
+        } else if (u < nh + 2 * nl) {
+          row = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kXrAu]) +
+                (size_t)(u - max(ia, nh + nl)) * D;
+          dst = blk + (k + 2) * I + r + (u - nh - nl);
+        } else {
+          row = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kXrSel + u - max(ia, nh + 2 * nl)]);
+          dst = blk + (k + 2) * I + 2 * r + (u - nh - 2 * nl);
+        }
+        const float v = bf16_row_x<D>(row, S.x, lane);
+        if (lane == 0) st_tag(dst, tag, __float_as_uint(v));
+      }
+    } else if (it.kind == IT_GU) {
+      // ---- gate/up rows of this item's units
       if (ct == 0) stamp(P, l, TR_GU_FULL);
-      // LoRA A rows of the shared expert (t_g, t_u), published for the down phase
-      int a = 0, b = 0;
-      if (lora) split_range(2 * r, G, c, a, b);
-      #pragma unroll 1
-      for (int qq = a; qq < b; qq++) {
-        if (warp == (qq - a) % kDecCW) {
-          const uint16_t *row = qq < r ? reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][2]) + (size_t)(qq - a) * D
-                                       : reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3]) +
-                                             (size_t)(qq - max(a, r)) * D;
-          const float v = bf16_row_x<D>(row, S.x, lane);
-          if (lane == 0) st_tag(P.t_blk + (size_t)l * P.blk + (k + 2) * I + qq, tag, __float_as_uint(v));
-        }
-      }
-      // router logits of the predicted experts (their gate weights)
-      a = b = 0;
-      if (pred) split_range(k, G, (c + G - min(2 * r, G - 1)) % G, a, b);
-      #pragma unroll 1
-      for (int qq = a; qq < b; qq++) {
-        if (warp == kDecCW - 1 - (qq - a) % kDecCW) {
-          const float v = bf16_row_x<D>(reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][4 + qq - a]), S.x, lane);
-          if (lane == 0) st_tag(P.t_blk + (size_t)l * P.blk + (k + 2) * I + 2 * r + qq, tag, __float_as_uint(v));
-        }
-      }
-      // this CTA's rows of the layer's prerouter head on x
-      if (Y.head) {
-        int ha, hb;
-        split_range(P.E, G, c, ha, hb);
-        const uint16_t *hw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kGuHead]);
-        #pragma unroll 1
-        for (int row = ha; row < hb; row++) {
-          if (warp == (4 + row - ha) % kDecCW) {
-            const float v = bf16_row_x<D>(hw + (size_t)(row - ha) * P.ldh, S.x, lane);
-            if (lane == 0) st_tag(P.t_hlog + (size_t)l * P.E + row, tag, __float_as_uint(v));
-          }
-        }
-      }
-      // this lane's activation chunks stay in registers for every row of the phase
+      // this lane's activation chunks stay in registers for every row of the item
       constexpr int LPR = NCH < 32 ? NCH : 32;    // lanes per row
       constexpr int RPW = 32 / LPR;               // rows per warp pass
       constexpr int CPL = NCH / LPR;              // chunks per lane
@@ -939,8 +1011,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         xsr[cc] = chunk_raw_sum(xr[cc]);
       }
       GuPiece pc[kMaxPieces];
-      const int np = gu_pieces<D, I>(k, G, c, pc);
-      float *gu_g = S.ydot;            // raw g and u of every row of this CTA's pieces
+      const int np = pieces_of(ia, in, I, pc);
+      float *gu_g = S.ydot;            // raw g and u of every row of this item
       int roff = 0;
       #pragma unroll 1
       for (int p = 0; p < np; p++) {
@@ -996,95 +1068,92 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         }
         roff += R;
       }
-      // routing used by this layer (one CTA records it for the host)
-      if (c == 0 && ct < k) P.hist_out[((size_t)l * P.maxT) * k + ct] = S.sel_all[l & 63][ct];
       if (ct == 0) stamp(P, l, TR_GU_DONE);
     } else {
-      // ---- down + combine stage -----------------------------------------------------
-      // one batched poll over the layer's block: a of the routed slots, the shared
-      // expert's raw g/u, t_g/t_u (with LoRA) and the selected router logits (predicted)
+      // ---- down + combine ---------------------------------------------------------------
       float *at = S.at, *gus = S.gus;
-      {
-        const unsigned long long *blk = P.t_blk + (size_t)l * P.blk;
-        Range rg[4];
-        int nr = 0;
-        rg[nr++] = Range{blk, S.stg, k * I};
-        rg[nr++] = Range{blk + k * I, reinterpret_cast<uint32_t *>(S.gus), 2 * I};
-        if (lora) rg[nr++] = Range{blk + (k + 2) * I, reinterpret_cast<uint32_t *>(S.tl), 2 * r};
-        if (pred) rg[nr++] = Range{blk + (k + 2) * I + 2 * r, reinterpret_cast<uint32_t *>(S.rl), k};
-        ab |= !poll_ranges(rg, nr, tag, ct, C);
-      }
-      if (cbar_or(ab)) break;
-      // routed a values: bf16 payloads -> pre-scaled, chunk-transposed fp32
+      if (it.first) {
+        // one batched poll over the layer's block: a of the routed slots, the shared
+        // expert's raw g/u, t_g/t_u (with LoRA) and the selected router logits (predicted)
+        {
+          const unsigned long long *blk = P.t_blk + (size_t)l * P.blk;
+          Range rg[4];
+          int nr = 0;
+          rg[nr++] = Range{blk, S.stg, k * I};
+          rg[nr++] = Range{blk + k * I, reinterpret_cast<uint32_t *>(S.gus), 2 * I};
+          if (lora) rg[nr++] = Range{blk + (k + 2) * I, reinterpret_cast<uint32_t *>(S.tl), 2 * r};
+          if (pred) rg[nr++] = Range{blk + (k + 2) * I + 2 * r, reinterpret_cast<uint32_t *>(S.rl), k};
+          ab |= !poll_ranges(rg, nr, tag, ct, C);
+        }
+        if (cbar_or(ab)) break;
+        // routed a values: bf16 payloads -> pre-scaled, chunk-transposed fp32
 #pragma unroll 1
-      for (int i = ct; i < k * I; i += kDecConsumers) {
-        const int j = i / I, e = i - j * I;
-        at[j * I + xt_index(e, NCI)] = bf(S.stg[i] & 0xFFFFu) * nib_scale(e & 7);
-      }
-      if (ct == 0) stamp(P, l, TR_A_POLL);
-      if (ct == 0) stamp(P, l, TR_DN_FULL);
-      const int sbd = dn_bd(k);
-      const uint16_t *bgm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 1]);
-      const uint16_t *bum = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 2]);
-      const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 3]);
-      // the shared expert's activation with its LoRA up branch (every CTA, same order)
-      #pragma unroll 1
-      for (int i = ct; i < I; i += kDecConsumers) {
-        float g = gus[2 * i], u = gus[2 * i + 1];
-        if (lora) {
-          float lg = 0.f, lu = 0.f;
-          #pragma unroll 1
-          for (int j = 0; j < r; j += 8) {
-            const uint4 wg = *reinterpret_cast<const uint4 *>(bgm + i * r + j);
-            const uint4 wu = *reinterpret_cast<const uint4 *>(bum + i * r + j);
-            const uint32_t gw[4] = {wg.x, wg.y, wg.z, wg.w}, uw[4] = {wu.x, wu.y, wu.z, wu.w};
+        for (int i = ct; i < k * I; i += kDecConsumers) {
+          const int j = i / I, e = i - j * I;
+          at[j * I + xt_index(e, NCI)] = bf(S.stg[i] & 0xFFFFu) * nib_scale(e & 7);
+        }
+        if (ct == 0) stamp(P, l, TR_A_POLL);
+        const int sbd = dn_bd(k);
+        const uint16_t *bgm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 1]);
+        const uint16_t *bum = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 2]);
+        const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 3]);
+        // the shared expert's activation with its LoRA up branch (every CTA, same order)
+        #pragma unroll 1
+        for (int i = ct; i < I; i += kDecConsumers) {
+          float g = gus[2 * i], u = gus[2 * i + 1];
+          if (lora) {
+            float lg = 0.f, lu = 0.f;
+            #pragma unroll 1
+            for (int j = 0; j < r; j += 8) {
+              const uint4 wg = *reinterpret_cast<const uint4 *>(bgm + i * r + j);
+              const uint4 wu = *reinterpret_cast<const uint4 *>(bum + i * r + j);
+              const uint32_t gw[4] = {wg.x, wg.y, wg.z, wg.w}, uw[4] = {wu.x, wu.y, wu.z, wu.w};
 #pragma unroll
-            for (int q = 0; q < 4; q++) {
-              lg = fmaf(bf(gw[q] & 0xFFFFu), S.tl[j + 2 * q], lg);
-              lg = fmaf(bf(gw[q] >> 16), S.tl[j + 2 * q + 1], lg);
-              lu = fmaf(bf(uw[q] & 0xFFFFu), S.tl[r + j + 2 * q], lu);
-              lu = fmaf(bf(uw[q] >> 16), S.tl[r + j + 2 * q + 1], lu);
+              for (int q2 = 0; q2 < 4; q2++) {
+                lg = fmaf(bf(gw[q2] & 0xFFFFu), S.tl[j + 2 * q2], lg);
+                lg = fmaf(bf(gw[q2] >> 16), S.tl[j + 2 * q2 + 1], lg);
+                lu = fmaf(bf(uw[q2] & 0xFFFFu), S.tl[r + j + 2 * q2], lu);
+                lu = fmaf(bf(uw[q2] >> 16), S.tl[r + j + 2 * q2 + 1], lu);
+              }
             }
+            g = fmaf(P.c, lg, g);
+            u = fmaf(P.c, lu, u);
           }
-          g = fmaf(P.c, lg, g);
-          u = fmaf(P.c, lu, u);
+          const float av = bf(f2bf(g / (1.0f + expf(-g)) * u));
+          S.asraw[i] = av;
+          at[k * I + xt_index(i, NCI)] = av * nib_scale(i & 7);
         }
-        const float av = bf(f2bf(g / (1.0f + expf(-g)) * u));
-        S.asraw[i] = av;
-        at[k * I + xt_index(i, NCI)] = av * nib_scale(i & 7);
-      }
-      if (ct == 0) {
-        float lg[kMaxK], mx = -INFINITY, sum = 0.f;
-        #pragma unroll 1
-        for (int j = 0; j < k; j++) {
-          lg[j] = pred ? S.rl[j] : S.rlsel[l & 63][j];
-          mx = fmaxf(mx, lg[j]);
-        }
-        #pragma unroll 1
-        for (int j = 0; j < k; j++) {
-          lg[j] = expf(lg[j] - mx);
-          sum += lg[j];
-        }
-        #pragma unroll 1
-        for (int j = 0; j < k; j++) S.gates[j] = lg[j] / sum;
-      }
-      cbar();
-      // t_d = Ad a_s (LoRA down branch)
-      if (lora) {
-        #pragma unroll 1
-        for (int j = warp; j < r; j += kDecCW) {
-          float acc = 0.f;
+        if (ct == 0) {
+          float lg[kMaxK], mx = -INFINITY, sum = 0.f;
           #pragma unroll 1
-          for (int i = lane; i < I; i += 32) acc = fmaf(bf(adm[j * I + i]), S.asraw[i], acc);
-          acc = warp_sum(acc);
-          if (lane == 0) S.td[j] = acc;
+          for (int j = 0; j < k; j++) {
+            lg[j] = pred ? S.rl[j] : S.rlsel[l & 63][j];
+            mx = fmaxf(mx, lg[j]);
+          }
+          #pragma unroll 1
+          for (int j = 0; j < k; j++) {
+            lg[j] = expf(lg[j] - mx);
+            sum += lg[j];
+          }
+          #pragma unroll 1
+          for (int j = 0; j < k; j++) S.gates[j] = lg[j] / sum;
         }
         cbar();
+        // t_d = Ad a_s (LoRA down branch)
+        if (lora) {
+          #pragma unroll 1
+          for (int j = warp; j < r; j += kDecCW) {
+            float acc = 0.f;
+            #pragma unroll 1
+            for (int i = lane; i < I; i += 32) acc = fmaf(bf(adm[j * I + i]), S.asraw[i], acc);
+            acc = warp_sum(acc);
+            if (lane == 0) S.td[j] = acc;
+          }
+        }
+        cbar();
+        if (ct == 0) stamp(P, l, TR_TD_POLL);
       }
-      if (ct == 0) stamp(P, l, TR_TD_POLL);
-      int a, b;
-      split_range(D, G, c, a, b);
-      const int R = b - a;
+      const int R = in;
       constexpr int LPR = NCI < 32 ? NCI : 32;
       constexpr int RPW = 32 / LPR;
       constexpr int CPL = NCI / LPR;
@@ -1126,7 +1195,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       }
       if (ct == 0) stamp(P, l, TR_DN_DOTS);
       cbar();
-      const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd]);
+      const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]);
       #pragma unroll 1
       for (int row = ct; row < R; row += kDecConsumers) {
         float y = 0.f;
@@ -1139,7 +1208,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           for (int j = 0; j < r; j++) lo = fmaf(bf(bd[row * r + j]), S.td[j], lo);
           y = fmaf(P.c, lo, y);
         }
-        const int n = a + row;
+        const int n = ia + row;
         st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(y));
         P.y[(size_t)l * D + n] = f2bf(y);
         if (P.yf) P.yf[(size_t)l * D + n] = y;
@@ -1152,12 +1221,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     q++;
   }
   if (ab) return;
-  // ---- head top-k: CTA c handles layer c's head; its logits are complete by now ------
+  // ---- end of step: CTA c records layer c's routing and runs layer c's head top-k; every
+  // logit is complete by now --------------------------------------------------------------
   #pragma unroll 1
   for (int l = c; l < P.L; l += G) {
     const DecLayer &Y = S.lay[l];
-    if (!Y.head) continue;
     const uint32_t tag = dtag(P, l);
+    if (!is_predicted(P, S, l) && S.sel_ok[l & 63] == 0) {
+      // this CTA did not need the layer's own top-k during the step: take it now
+      bool bad = !poll_to(P.t_rlog + (size_t)l * P.E, reinterpret_cast<uint32_t *>(S.rl), P.E, tag, ct, C);
+      if (cbar_or(bad)) return;
+      if (warp == 0) {
+        int s8[kMaxK];
+        warp_topk_ool(S.rl, P.E, k, lane, s8);
+        if (lane == 0) {
+          #pragma unroll 1
+          for (int j = 0; j < k; j++) S.sel_all[l & 63][j] = s8[j];
+        }
+      }
+      cbar();
+    }
+    if (ct < k) P.hist_out[((size_t)l * P.maxT) * k + ct] = S.sel_all[l & 63][ct];
+    if (!Y.head) continue;
     bool bad = !poll_to(P.t_hlog + (size_t)l * P.E, reinterpret_cast<uint32_t *>(S.rl), P.E, tag, ct, C);
     if (cbar_or(bad)) return;
     if (P.onehot) {

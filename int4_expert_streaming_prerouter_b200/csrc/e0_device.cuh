@@ -105,4 +105,23 @@ __device__ __forceinline__ float chunk_dot_bf16x(const uint4 w, const uint32_t *
   return chunk_dot(w, x, s, m);
 }
 
+// Packed pairs of fp32 (low word = first element) and the f32x2 arithmetic on them.
+__device__ __forceinline__ unsigned long long pk2(float a, float b) {
+  return ((unsigned long long)__float_as_uint(b) << 32) | __float_as_uint(a);
+}
+__device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float f2sum(unsigned long long v) {
+  return __uint_as_float((uint32_t)v) + __uint_as_float((uint32_t)(v >> 32));
+}
+
 }  // namespace e0

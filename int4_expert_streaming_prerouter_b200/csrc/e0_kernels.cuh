@@ -334,41 +334,78 @@ struct Plan {
   int32_t *assign;  // [T * k]  entries t * k + j
 };
 
-__global__ void k_plan(const int32_t *__restrict__ idx, int n, int E, Plan P) {
-  __shared__ int cnt[kMaxE], start[kMaxE + 1];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+// Counting sort by expert, stable in (token, slot) order: each of the 32 warps owns a
+// contiguous chunk of the assignments; per-warp histograms give every (warp, expert) its
+// output offset, and inside a batch of 32 the lanes holding the same expert rank
+// themselves with a match mask.  One block of 1024 threads.
+__global__ void __launch_bounds__(1024) k_plan(const int32_t *__restrict__ idx, int n, int E, Plan P) {
+  __shared__ int cnt[32][kMaxE];      // per-warp counts, then per-warp output offsets
+  __shared__ int tot[kMaxE];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 32 * kMaxE; i += blockDim.x) (&cnt[0][0])[i] = 0;
   __syncthreads();
-  for (int a = threadIdx.x; a < n; a += blockDim.x) {
+  const int chunk = (n + 31) / 32, a0 = warp * chunk, a1 = min(n, a0 + chunk);
+  for (int a = a0 + lane; a < a1; a += 32) {
     const int e = idx[a];
-    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    if (e >= 0 && e < E) atomicAdd(&cnt[warp][e], 1);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int u = 0, off = 0;
-    for (int e = 0; e < E; e++) {
-      start[e] = off;
-      if (cnt[e]) {
-        P.uexp[u] = e;
-        P.ustart[u] = off;
-        u++;
+  // expert totals, then the exclusive scan over experts (one warp)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int t = 0;
+    for (int w = 0; w < 32; w++) t += cnt[w][e];
+    tot[e] = t;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int run = 0, u = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = e < E ? tot[e] : 0;
+      int incl = c;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
       }
-      off += cnt[e];
+      const unsigned nz = __ballot_sync(0xffffffffu, c > 0);
+      if (c > 0) {
+        const int ui = u + __popc(nz & ((1u << lane) - 1u));
+        P.uexp[ui] = e;
+        P.ustart[ui] = run + incl - c;
+      }
+      if (e < E) tot[e] = run + incl - c;    // expert start
+      run += __shfl_sync(0xffffffffu, incl, 31);
+      u += __popc(nz);
     }
-    P.ustart[u] = off;
-    P.U[0] = u;
+    if (lane == 0) {
+      P.ustart[u] = run;
+      P.U[0] = u;
+    }
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nw) {
-    if (cnt[e] == 0) continue;
-    int run = start[e];
-    for (int base = 0; base < n; base += 32) {
-      const int a = base + lane;
-      const bool hit = a < n && idx[a] == e;
-      const unsigned m = __ballot_sync(0xffffffffu, hit);
-      if (hit) P.assign[run + __popc(m & ((1u << lane) - 1u))] = a;
-      run += __popc(m);
+  // per-(warp, expert) offsets: expert start + the counts of the earlier warps
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int off = tot[e];
+    for (int w = 0; w < 32; w++) {
+      const int c = cnt[w][e];
+      cnt[w][e] = off;
+      off += c;
     }
+  }
+  __syncthreads();
+  for (int base = a0; base < a1; base += 32) {
+    const int a = base + lane;
+    const int e = a < a1 ? idx[a] : -1;
+    const bool ok = e >= 0 && e < E;
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+    if (ok) {
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      P.assign[cnt[warp][e] + rank] = a;
+    }
+    __syncwarp();
+    // the lowest lane of each peer group advances its expert's offset
+    if (ok && (peers & ((1u << lane) - 1u)) == 0) cnt[warp][e] += __popc(peers);
+    __syncwarp();
   }
 }
 

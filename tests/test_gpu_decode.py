@@ -177,8 +177,8 @@ def test_one_launch_decode_equals_general_path_small(cuda_ok):
     ref.close()
 
 
-def _decode_bits(ctx, dims, seed, S, lag):
-    ctx.debug_decode_lag(lag)
+def _decode_bits(ctx, dims, seed, S, flat):
+    ctx.debug_decode_flat(flat)
     out = []
     for t in range(S):
         h = bf16_tensor(synth.hidden(seed, t, dims.L, 1, dims.d), "cuda")
@@ -190,33 +190,33 @@ def _decode_bits(ctx, dims, seed, S, lag):
     return out
 
 
-@pytest.mark.parametrize("heads", [(0, 1, 2), (0, 2)])
-def test_one_launch_decode_lag_is_bitwise_invariant(cuda_ok, heads):
-    """Overlapping the stages of unchained layers (down stage `lag` layers behind gate/up,
-    reactive layers' routers first) changes the order of the work, not its arithmetic: the
-    outputs, routing and predictions are bit-identical to in-order execution, for a stack of
-    mostly predicted layers and one with reactive layers in between."""
+def _same(base, got, what):
+    for t, (a, b) in enumerate(zip(base, got)):
+        for u, v in zip(a, b):
+            assert np.array_equal(u, v), f"{what} step {t}"
+
+
+@pytest.mark.parametrize("heads", [(0, 1, 2), (0, 2), ()])
+def test_one_launch_decode_flat_schedule_is_bitwise_in_order(cuda_ok, heads):
+    """The flat schedule (each phase's units over all layers split across the CTAs)
+    changes who computes what and in which order, not the arithmetic: outputs, routing and
+    predictions are bit-identical to in-order execution, for stacks of mostly predicted
+    layers, reactive layers in between, and no heads at all (every layer reactive)."""
     dims = Dims(d=256, E=16, I=128, k=4, r=8, L=6, head_layers=heads)
     ctx, _, _ = build(dims, 95, 4)
     base = _decode_bits(ctx, dims, 96, 4, 0)
-    for lag in (1, 2, 3, 8):
-        got = _decode_bits(ctx, dims, 96, 4, lag)
-        for t, (a, b) in enumerate(zip(base, got)):
-            for u, v in zip(a, b):
-                assert np.array_equal(u, v), f"lag {lag} step {t}"
+    _same(base, _decode_bits(ctx, dims, 96, 4, 1), "flat")
     ctx.close()
 
 
-def test_full_size_decode_lag_is_bitwise_invariant(full_model):
-    """The bench's configuration (40 layers, lag 2) against in-order execution, two steps."""
+def test_full_size_decode_flat_schedule_is_bitwise_in_order(full_model):
+    """The bench's configuration (40 layers, flat schedule) against in-order execution."""
     try:
         base = _decode_bits(full_model, FULL, 7, 2, 0)
-        got = _decode_bits(full_model, FULL, 7, 2, 2)
+        got = _decode_bits(full_model, FULL, 7, 2, 1)
     finally:
-        full_model.debug_decode_lag(2)
-    for t, (a, b) in enumerate(zip(base, got)):
-        for u, v in zip(a, b):
-            assert np.array_equal(u, v), f"step {t}"
+        full_model.debug_decode_flat(1)
+    _same(base, got, "flat")
 
 
 def test_one_launch_decode_chained_b1(cuda_ok):
