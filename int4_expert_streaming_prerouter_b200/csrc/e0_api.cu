@@ -148,9 +148,11 @@ static bool supported(const e0_dims &D) {
 
 template <typename T>
 static int dalloc(T **p, size_t n) {
-  if (cudaMalloc((void **)p, n * sizeof(T) + 16) != cudaSuccess) {
+  const cudaError_t e = cudaMalloc((void **)p, n * sizeof(T) + 16);
+  if (e != cudaSuccess) {
     cudaGetLastError();
-    return fail(E0_ERR_OOM, "cudaMalloc of %zu bytes failed", n * sizeof(T));
+    return fail(e == cudaErrorMemoryAllocation ? E0_ERR_OOM : E0_ERR_CUDA, "cudaMalloc of %zu bytes failed: %s",
+                n * sizeof(T), cudaGetErrorString(e));
   }
   return E0_OK;
 }
@@ -784,11 +786,12 @@ static bool decode_supported(e0_ctx *C, int B) {
     return false;
   for (int l = 0; l < C->L; l++)
     if (!C->layers[l].experts) return false;
-  // a CTA's gate/up rows and down rows must fit its scratch and the task segment table
+  // in order, a CTA's share of a layer's gate/up units must fit the task's pieces and its
+  // share of the down rows the per-warp accumulators
   const int G = C->nsm;
-  const int gu_rows = ((D.top_k + 1) * D.d_ff + G - 1) / G, dn_rows = (D.d_model + G - 1) / G;
-  return 2 * gu_rows <= 64 * (kMaxK + 1) && dn_rows * (D.top_k + 1) <= 64 * (kMaxK + 1) &&
-         kGuPiece0 + 6 * kMaxPieces <= kMaxSeg && gu_rows * kMaxPieces >= 1;
+  const int gu_units = ((D.top_k + 1) * D.d_ff + G - 1) / G, dn_rows = (D.d_model + G - 1) / G;
+  return dn_rows <= kDnMaxRows && gu_units <= 2 * D.d_ff && kGuPiece0 + 6 * kMaxPieces <= kMaxItemSegs &&
+         3 * (D.top_k + 1) + 4 <= kMaxItemSegs;
 }
 
 static int decode_prepare(e0_ctx *C) {

@@ -36,7 +36,6 @@ constexpr int kDecCW = 12;
 constexpr int kRingBytes = 156 * 1024;
 constexpr int kDecMaxK = 4;               // routed experts per token on this path
 constexpr int kNSlot = 8;                 // tasks in flight
-constexpr int kMaxSeg = 96;               // bulk-copy segments per task
 
 struct DecLayer {
   const uint8_t *experts;
@@ -217,24 +216,6 @@ __device__ __forceinline__ uint16_t d2bf_bits(double v) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Task layout shared by the producer (which copies) and the consumers (which read).
-// ---------------------------------------------------------------------------------------
-struct Seg {
-  const uint8_t *src;
-  uint32_t bytes;
-};
-
-struct TaskBuf {
-  int n;
-  int overflow;
-  Seg s[kMaxSeg];
-  __device__ __forceinline__ void add(const void *p, size_t bytes) {
-    if (n < kMaxSeg) s[n++] = Seg{(const uint8_t *)p, (uint32_t)bytes};
-    else overflow = 1;
-  }
-};
-
-// ---------------------------------------------------------------------------------------
 // Work items.  A launch runs a list of items, the same sequence for the producer (which
 // streams each item's bytes into the ring) and the consumers (which compute it).  An item
 // is one kind of work on a contiguous range [a, a + n) of one layer's units:
@@ -269,21 +250,9 @@ __device__ __forceinline__ Item unpack_item(unsigned long long v) {
               ((v >> 4) & 1ull) != 0};
 }
 
-// A range of gate/up units split into per-slot pieces.
-struct GuPiece {
-  int slot, i0, i1;
-};
+// A range of gate/up units touches consecutive slots ("pieces"): at most kMaxPieces.
 constexpr int kMaxPieces = 4;
-__device__ __forceinline__ int pieces_of(int a, int n, int I, GuPiece *out) {
-  const int b = a + n;
-  int np = 0;
-  while (a < b && np < kMaxPieces) {
-    const int slot = a / I, end = min(b, (slot + 1) * I);
-    out[np++] = GuPiece{slot, a - slot * I, end - slot * I};
-    a = end;
-  }
-  return np;
-}
+constexpr int kDnMaxRows = 64;   // down rows per item (register accumulators per warp)
 
 // [s0, s1) = the part of [a, a + n) inside [lo, hi), relative to lo (empty: s0 = s1 = 0)
 __device__ __forceinline__ void sub_range(int a, int n, int lo, int hi, int &s0, int &s1) {
@@ -304,63 +273,85 @@ constexpr int kXrHead = 2, kXrAg = 3, kXrAu = 4, kXrSel = 5;
 constexpr int kGuPiece0 = 2;
 __device__ __forceinline__ int dn_bd(int k) { return 3 * (k + 1); }
 
-// Build the segment list of item `it` (rows of layer Y).  `sel` are the layer's routed
-// experts.  The consumer code reads the segments back by the indices above.
+// Segment i (one per producer lane) of item `it` on the rows of layer Y: its source and
+// byte count (0 = empty).  `sel` are the layer's routed experts.  The consumer code reads
+// the segments back by the indices above.
+constexpr int kMaxItemSegs = 32;
 template <int D, int I>
-__device__ __noinline__ void build_task(const DecodeParams &P, const DecLayer &Y, const Item &it, bool predicted,
-                                        const int *sel, TaskBuf &T) {
+__device__ __forceinline__ void item_seg(const DecodeParams &P, const DecLayer &Y, const Item &it, bool predicted,
+                                         const int (&sel)[kMaxK], int i, const uint8_t *&src, uint32_t &bytes) {
   const Blob bl = blob_of(D, I);
-  T.n = 0;
-  T.overflow = 0;
   const int l = it.l, a = it.a, n = it.n;
-  if (it.kind != IT_DN) {
-    T.add(Y.gamma, it.first ? D * 2 : 0);
-    T.add(P.h + (size_t)l * D, it.first ? D * 2 : 0);
+  src = nullptr;
+  bytes = 0;
+  auto pick = [&](const void *p, size_t b) {
+    src = (const uint8_t *)p;
+    bytes = (uint32_t)b;
+  };
+  if (it.kind != IT_DN && i < 2) {
+    if (it.first) pick(i == 0 ? (const void *)Y.gamma : (const void *)(P.h + (size_t)l * D), D * 2);
+    return;
   }
   if (it.kind == IT_R) {
-    T.add(Y.router + (size_t)a * D, (size_t)n * D * 2);
+    if (i == 2) pick(Y.router + (size_t)a * D, (size_t)n * D * 2);
   } else if (it.kind == IT_XR) {
     const int nh = Y.head ? P.E : 0, nl = Y.Ag ? P.r : 0, ns = predicted ? P.k : 0;
     int s0, s1;
-    sub_range(a, n, 0, nh, s0, s1);
-    T.add(Y.head + (size_t)s0 * P.ldh, (size_t)(s1 - s0) * P.ldh * 2);
-    sub_range(a, n, nh, nh + nl, s0, s1);
-    T.add(Y.Ag + (size_t)s0 * D, (size_t)(s1 - s0) * D * 2);
-    sub_range(a, n, nh + nl, nh + 2 * nl, s0, s1);
-    T.add(Y.Au + (size_t)s0 * D, (size_t)(s1 - s0) * D * 2);
-    sub_range(a, n, nh + 2 * nl, nh + 2 * nl + ns, s0, s1);
-    #pragma unroll 1
-    for (int q = 0; q < kMaxK; q++) {
-      const bool on = s0 + q < s1;
-      T.add(Y.router + (size_t)(on ? sel[s0 + q] : 0) * D, on ? D * 2 : 0);
+    if (i == kXrHead) {
+      sub_range(a, n, 0, nh, s0, s1);
+      pick(Y.head + (size_t)s0 * P.ldh, (size_t)(s1 - s0) * P.ldh * 2);
+    } else if (i == kXrAg) {
+      sub_range(a, n, nh, nh + nl, s0, s1);
+      pick(Y.Ag + (size_t)s0 * D, (size_t)(s1 - s0) * D * 2);
+    } else if (i == kXrAu) {
+      sub_range(a, n, nh + nl, nh + 2 * nl, s0, s1);
+      pick(Y.Au + (size_t)s0 * D, (size_t)(s1 - s0) * D * 2);
+    } else if (i < kXrSel + kMaxK) {
+      sub_range(a, n, nh + 2 * nl, nh + 2 * nl + ns, s0, s1);
+      const int q = i - kXrSel;
+      if (s0 + q < s1) {
+        int e = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxK; j++)
+          if (j == s0 + q) e = sel[j];
+        pick(Y.router + (size_t)e * D, D * 2);
+      }
     }
   } else if (it.kind == IT_GU) {
-    GuPiece pc[kMaxPieces];
-    const int np = pieces_of(a, n, I, pc);
-    #pragma unroll 1
-    for (int p = 0; p < np; p++) {
-      const uint8_t *base = pc[p].slot < P.k ? Y.experts + (size_t)sel[pc[p].slot] * bl.bytes : Y.shared;
-      const int R = pc[p].i1 - pc[p].i0, i0 = pc[p].i0;
-      T.add(base + bl.gc + (size_t)i0 * (D / 2), (size_t)R * (D / 2));
-      T.add(base + bl.gs + (size_t)i0 * (D / 64) * 2, (size_t)R * (D / 64) * 2);
-      T.add(base + bl.gm + (size_t)i0 * (D / 64) * 2, (size_t)R * (D / 64) * 2);
-      T.add(base + bl.uc + (size_t)i0 * (D / 2), (size_t)R * (D / 2));
-      T.add(base + bl.us + (size_t)i0 * (D / 64) * 2, (size_t)R * (D / 64) * 2);
-      T.add(base + bl.um + (size_t)i0 * (D / 64) * 2, (size_t)R * (D / 64) * 2);
+    // piece p = the p-th slot touched by units [a, a + n): slot a / I + p
+    const int p = (i - kGuPiece0) / 6, f = (i - kGuPiece0) % 6;
+    const int slot = a / I + p;
+    const int i0 = p == 0 ? a % I : 0, i1 = min(a + n - slot * I, I);
+    if (i >= kGuPiece0 && i1 > i0) {
+      int e = 0;
+#pragma unroll
+      for (int j = 0; j < kMaxK; j++)
+        if (j == slot) e = sel[j];
+      const uint8_t *base = slot < P.k ? Y.experts + (size_t)e * bl.bytes : Y.shared;
+      const bool codes = f == 0 || f == 3;
+      const size_t off = f == 0 ? bl.gc : f == 1 ? bl.gs : f == 2 ? bl.gm : f == 3 ? bl.uc : f == 4 ? bl.us : bl.um;
+      const size_t rb = codes ? D / 2 : (D / 64) * 2;
+      pick(base + off + (size_t)i0 * rb, (size_t)(i1 - i0) * rb);
     }
   } else if (it.kind == IT_DN) {
-    #pragma unroll 1
-    for (int j = 0; j <= P.k; j++) {
-      const uint8_t *base = j < P.k ? Y.experts + (size_t)sel[j] * bl.bytes : Y.shared;
-      T.add(base + bl.dc + (size_t)a * (I / 2), (size_t)n * (I / 2));
-      T.add(base + bl.ds + (size_t)a * (I / 64) * 2, (size_t)n * (I / 64) * 2);
-      T.add(base + bl.dm + (size_t)a * (I / 64) * 2, (size_t)n * (I / 64) * 2);
+    const int nd = 3 * (P.k + 1);
+    if (i < nd) {
+      const int j = i / 3, f = i % 3;
+      int e = 0;
+#pragma unroll
+      for (int q = 0; q < kMaxK; q++)
+        if (q == j) e = sel[q];
+      const uint8_t *base = j < P.k ? Y.experts + (size_t)e * bl.bytes : Y.shared;
+      const size_t off = f == 0 ? bl.dc : f == 1 ? bl.ds : bl.dm;
+      const size_t rb = f == 0 ? I / 2 : (I / 64) * 2;
+      pick(base + off + (size_t)a * rb, (size_t)n * rb);
+    } else if (i == nd) {
+      if (Y.Bd) pick(Y.Bd + (size_t)a * P.r, (size_t)n * P.r * 2);
+    } else if (i <= nd + 3) {
+      if (Y.Bg && it.first)
+        pick(i == nd + 1 ? (const void *)Y.Bg : i == nd + 2 ? (const void *)Y.Bu : (const void *)Y.Ad,
+             (size_t)I * P.r * 2);
     }
-    T.add(Y.Bd + (size_t)a * P.r, Y.Bd ? (size_t)n * P.r * 2 : 0);
-    const size_t lb = (Y.Bg && it.first) ? (size_t)I * P.r * 2 : 0;
-    T.add(Y.Bg, lb);
-    T.add(Y.Bu, lb);
-    T.add(Y.Ad, lb);
   }
 }
 
@@ -389,9 +380,8 @@ struct DecSmem {
   unsigned long long items[kMaxItems];   // this CTA's item list (pack_item)
   int nitems;
   DecLayer lay[64];                  // the layer table
-  TaskBuf tb;                        // the producer's task being issued
-  int tb_off[kMaxSeg];
-  uint32_t seg_off[kNSlot][kMaxSeg]; // ring byte offset of each segment's first wanted byte
+  int ring_start[kNSlot];            // the producer's ring offset of each slot's task
+  uint32_t seg_off[kNSlot][kMaxItemSegs]; // ring byte offset of each segment's first wanted byte
   uint64_t full[kNSlot], empty[kNSlot];
   volatile int abort;
 };
@@ -462,7 +452,7 @@ __device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I>
   } else {
     constexpr int kItemBytes = 36 * 1024;
     const int gu_chunk = min(kItemBytes / (2 * (D / 2 + D / 16)), 288);
-    const int dn_chunk = min(kItemBytes / ((k + 1) * (I / 2 + I / 16) + 2 * P.r), 64);
+    const int dn_chunk = min(kItemBytes / ((k + 1) * (I / 2 + I / 16) + 2 * P.r), kDnMaxRows);
     const int xr_chunk = max(kItemBytes / (2 * P.ldh), 1);
     // one phase: units(l) per layer over every layer with units, this CTA's share
     auto phase = [&](int kind, int chunk, int which) {
@@ -540,10 +530,11 @@ __device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I>
 // ---------------------------------------------------------------------------------------
 template <int D, int I>
 __device__ void producer(const DecodeParams &P, DecSmem<D, I> &S) {
-  const int c = blockIdx.x, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
   int q = 0, head = 0, oldest = 0;
-  int qs[kNSlot];
   int sel[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; j++) sel[j] = 0;
   bool ok = true;
 
   #pragma unroll 1
@@ -552,142 +543,108 @@ __device__ void producer(const DecodeParams &P, DecSmem<D, I> &S) {
     if (it.kind == IT_TK) continue;
     const int l = it.l;
     const bool pred = is_predicted(P, S, l);
-    {
-      if (it.kind == IT_GU || it.kind == IT_DN || it.kind == IT_XR) {
-        if (!pred && it.kind != IT_XR) {
-          // a reactive layer's experts are known once the consumers ran its TK item
-          unsigned long long t0 = 0;
-          while (S.sel_ok[l & 63] == 0) {
-            if (S.abort) { ok = false; break; }
-            if (timed_out(t0, P.timeout_ns)) {
-              if (lane == 0) atomicOr(P.err, DERR_TIMEOUT);
-              S.abort = 1;
-              ok = false;
-              break;
-            }
-            __nanosleep(32);
+    if (it.kind == IT_GU || it.kind == IT_DN || (it.kind == IT_XR && pred)) {
+      if (!pred) {
+        // a reactive layer's experts are known once the consumers ran its TK item
+        unsigned long long t0 = 0;
+        while (S.sel_ok[l & 63] == 0) {
+          if (S.abort) { ok = false; break; }
+          if (timed_out(t0, P.timeout_ns)) {
+            if (lane == 0) atomicOr(P.err, DERR_TIMEOUT);
+            S.abort = 1;
+            ok = false;
+            break;
           }
-          if (!ok) break;
+          __nanosleep(32);
         }
-        #pragma unroll 1
-        for (int j = 0; j < P.k; j++) {
-          sel[j] = S.sel_all[l & 63][j];
-          if (sel[j] < 0 || sel[j] >= P.E) {
-            if (lane == 0 && (pred || it.kind != IT_XR)) atomicOr(P.err, DERR_INDEX);
-            sel[j] = 0;
-          }
-        }
+        if (!ok) break;
       }
-      if (it.kind == IT_GU) stamp(P, l, TR_P_GU_START);
-      if (it.kind == IT_DN) stamp(P, l, TR_P_DN_START);
-      if (lane == 0) build_task<D, I>(P, S.lay[l], it, pred, sel, S.tb);   // out of line
-      __syncwarp();
-      const int n = S.tb.n;
-      if (S.tb.overflow) {
-        if (lane == 0) atomicOr(P.err, DERR_TIMEOUT);
-        S.abort = 1;
-        ok = false;
-        break;
-      }
-      // each lane sizes its segments (rounded out to 16 bytes); warp prefix sum -> offsets
-      int mine[3] = {0, 0, 0}, my_sum = 0;
 #pragma unroll
-      for (int m = 0; m < 3; m++) {
-        const int i = lane * 3 + m;
-        if (i < n) {
-          const uintptr_t lo = (uintptr_t)S.tb.s[i].src & ~(uintptr_t)15;
-          const uintptr_t hi = ((uintptr_t)S.tb.s[i].src + S.tb.s[i].bytes + 15) & ~(uintptr_t)15;
-          mine[m] = (int)(hi - lo);
-          my_sum += mine[m];
+      for (int j = 0; j < kMaxK; j++) {
+        int e = j < P.k ? S.sel_all[l & 63][j] : 0;
+        if (e < 0 || e >= P.E) {
+          if (lane == 0 && it.kind == IT_GU) atomicOr(P.err, DERR_INDEX);
+          e = 0;
         }
+        sel[j] = e;
       }
-      int incl = my_sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int need = __shfl_sync(0xffffffffu, incl, 31);
-      const int excl = incl - my_sum;
-      if (need > kRingBytes) {
-        if (lane == 0) atomicOr(P.err, DERR_TIMEOUT);
-        S.abort = 1;
-        ok = false;
-        break;
-      }
-      // lane 0: allocate [start, start+need), releasing the oldest tasks as required.  The
-      // in-flight bytes are [tail, head) or wrapped [tail, end) + [0, head); a gap of at
-      // least one byte keeps head == tail meaning "empty".
-      int start = -1;
-      if (lane == 0) {
-        while (ok) {
-          if (q - oldest < kNSlot) {
-            if (q == oldest) {
-              head = 0;
-              start = 0;
-              break;
-            }
-            const int tail = qs[oldest % kNSlot];
-            if (head > tail) {
-              if (head + need <= kRingBytes) { start = head; break; }
-              if (need < tail) { start = 0; break; }
-            } else if (head < tail && head + need < tail) {
-              start = head;
-              break;
-            }
-          }
-          // wait until the consumers have released task `oldest`
-          const int slot = oldest % kNSlot;
-          const uint32_t par = (uint32_t)((oldest / kNSlot) & 1);
-          unsigned long long t0 = 0;
-          while (!mbar_test(&S.empty[slot], par)) {
-            if (S.abort) { ok = false; break; }
-            if (timed_out(t0, P.timeout_ns)) {
-              atomicOr(P.err, DERR_TIMEOUT);
-              S.abort = 1;
-              ok = false;
-              break;
-            }
-          }
-          if (ok) oldest++;
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
-      if (!ok) break;
-      start = __shfl_sync(0xffffffffu, start, 0);
-      const int slot = q % kNSlot;
-      {
-        int off = start + excl;
-#pragma unroll
-        for (int m = 0; m < 3; m++) {
-          const int i = lane * 3 + m;
-          if (i < n) {
-            const uintptr_t lo = (uintptr_t)S.tb.s[i].src & ~(uintptr_t)15;
-            S.seg_off[slot][i] = (uint32_t)(off + ((uintptr_t)S.tb.s[i].src - lo));
-            S.tb_off[i] = off;
-            off += mine[m];
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_expect_tx(&S.full[slot], (uint32_t)need);
-      __syncwarp();
-#pragma unroll
-      for (int m = 0; m < 3; m++) {
-        const int i = lane * 3 + m;
-        if (i < n && mine[m] > 0) {
-          const uintptr_t lo = (uintptr_t)S.tb.s[i].src & ~(uintptr_t)15;
-          bulk_g2s(S.ring + S.tb_off[i], (const void *)lo, (uint32_t)mine[m], &S.full[slot]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        qs[slot] = start;
-        head = start + need;
-      }
-      q++;
-      if (lane == 0) stamp(P, l, it.kind == IT_GU ? TR_P_GU : it.kind == IT_DN ? TR_P_DN : TR_P_R);
     }
+    if (it.kind == IT_GU) stamp(P, l, TR_P_GU_START);
+    if (it.kind == IT_DN) stamp(P, l, TR_P_DN_START);
+    // each lane builds its own segment (rounded out to 16 bytes); warp prefix sum -> offsets
+    const uint8_t *src;
+    uint32_t bytes;
+    item_seg<D, I>(P, S.lay[l], it, pred, sel, lane, src, bytes);
+    const uintptr_t lo = (uintptr_t)src & ~(uintptr_t)15;
+    const int mine = bytes ? (int)((((uintptr_t)src + bytes + 15) & ~(uintptr_t)15) - lo) : 0;
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int need = __shfl_sync(0xffffffffu, incl, 31);
+    const int excl = incl - mine;
+    if (need > kRingBytes) {
+      if (lane == 0) atomicOr(P.err, DERR_TIMEOUT);
+      S.abort = 1;
+      ok = false;
+      break;
+    }
+    // lane 0: allocate [start, start+need), releasing the oldest tasks as required.  The
+    // in-flight bytes are [tail, head) or wrapped [tail, end) + [0, head); a gap of at
+    // least one byte keeps head == tail meaning "empty".
+    int start = -1;
+    if (lane == 0) {
+      while (ok) {
+        if (q - oldest < kNSlot) {
+          if (q == oldest) {
+            head = 0;
+            start = 0;
+            break;
+          }
+          const int tail = S.ring_start[oldest % kNSlot];
+          if (head > tail) {
+            if (head + need <= kRingBytes) { start = head; break; }
+            if (need < tail) { start = 0; break; }
+          } else if (head < tail && head + need < tail) {
+            start = head;
+            break;
+          }
+        }
+        // wait until the consumers have released task `oldest`
+        const int slot = oldest % kNSlot;
+        const uint32_t par = (uint32_t)((oldest / kNSlot) & 1);
+        unsigned long long t0 = 0;
+        while (!mbar_test(&S.empty[slot], par)) {
+          if (S.abort) { ok = false; break; }
+          if (timed_out(t0, P.timeout_ns)) {
+            atomicOr(P.err, DERR_TIMEOUT);
+            S.abort = 1;
+            ok = false;
+            break;
+          }
+        }
+        if (ok) oldest++;
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+    if (!ok) break;
+    start = __shfl_sync(0xffffffffu, start, 0);
+    const int slot = q % kNSlot;
+    const int off = start + excl;
+    S.seg_off[slot][lane] = (uint32_t)(off + ((uintptr_t)src - lo));
+    __syncwarp();
+    if (lane == 0) mbar_expect_tx(&S.full[slot], (uint32_t)need);
+    __syncwarp();
+    if (mine > 0) bulk_g2s(S.ring + off, (const void *)lo, (uint32_t)mine, &S.full[slot]);
+    __syncwarp();
+    if (lane == 0) {
+      S.ring_start[slot] = start;
+      head = start + need;
+    }
+    q++;
+    if (lane == 0) stamp(P, l, it.kind == IT_GU ? TR_P_GU : it.kind == IT_DN ? TR_P_DN : TR_P_R);
   }
   // drain: every issued copy must have landed before the CTA exits
   if (lane == 0) {
@@ -881,6 +838,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     ab |= !poll_to(P.t_y, reinterpret_cast<uint32_t *>(S.yprev), 1, 0xFFFFFFFFu, ct, C);
   }
 
+  // Items run without a consumer-wide barrier: every warp waits for the item's bytes on
+  // its mbarrier, processes its own rows, publishes them and releases its claim on the
+  // ring slot; warps that finish early go on to the next item.  Only items that replace
+  // shared state (a layer's norm, a layer's first down item, a top-k) start with a
+  // barrier.  After a failed wait a warp keeps walking the list without doing work, so
+  // that every consumer thread passes the same barriers.
   #pragma unroll 1
   for (int q_it = 0; q_it < S.nitems; q_it++) {
     const Item it = unpack_item(S.items[q_it]);
@@ -889,11 +852,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     const bool pred = is_predicted(P, S, l);
     const bool lora = Y.Bg != nullptr;
     const uint32_t tag = dtag(P, l);
+    unsigned long long *blk = P.t_blk + (size_t)l * P.blk;
     if (it.kind == IT_TK) {
       // ---- a reactive layer's top-k over every CTA's router logits
-      ab |= !poll_to(P.t_rlog + (size_t)l * P.E, reinterpret_cast<uint32_t *>(S.rl), P.E, tag, ct, C);
-      if (cbar_or(ab)) break;
-      if (warp == 0) {
+      ab = cbar_or(ab);
+      if (!ab) ab |= !poll_to(P.t_rlog + (size_t)l * P.E, reinterpret_cast<uint32_t *>(S.rl), P.E, tag, ct, C);
+      ab = cbar_or(ab);
+      if (!ab && warp == 0) {
         int s8[kMaxK];
         warp_topk_ool(S.rl, P.E, k, lane, s8);
         if (lane == 0) {
@@ -911,19 +876,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       continue;
     }
     const bool xitem = it.kind != IT_DN;
-    // ---- in order: a layer's norm waits for the previous layer's output (its data in
-    // chained mode)
-    if (!P.flat && xitem && it.first && l > 0) {
-      ab |= !poll_to(P.t_y + (size_t)(l - 1) * D, reinterpret_cast<uint32_t *>(S.yprev), D, dtag(P, l - 1), ct, C);
-    }
-    if (cbar_or(ab)) break;
-    if (ct == 0 && xitem && it.first) stamp(P, l, TR_LAYER);
-
+    const bool shared_state = it.first;        // norm (x items) or down inputs (down items)
     const int slot = q % kNSlot;
     const uint32_t par = (uint32_t)((q / kNSlot) & 1);
-    ab |= !wait_full(&S.full[slot], par, C);
-    if (cbar_or(ab)) break;
-    if (xitem && it.first) {
+    q++;
+    if (shared_state) {
+      ab = cbar_or(ab);
+      // in order: a layer's norm waits for the previous layer's output (its data when
+      // chained)
+      if (!ab && !P.flat && xitem && l > 0)
+        ab |= !poll_to(P.t_y + (size_t)(l - 1) * D, reinterpret_cast<uint32_t *>(S.yprev), D, dtag(P, l - 1), ct, C);
+      if (ct == 0 && xitem) stamp(P, l, TR_LAYER);
+      if (!ab) ab |= !wait_full(&S.full[slot], par, C);
+      ab = cbar_or(ab);
+    } else {
+      if (!ab) ab |= !wait_full(&S.full[slot], par, C);
+      ab = __any_sync(0xffffffffu, ab);
+    }
+    if (xitem && shared_state) {
       // ---- the norm: gamma and h are the first two segments of the task
       const uint16_t *gam = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][0]);
       const uint16_t *hin = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][1]);
@@ -935,7 +905,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       for (int m = 0; m < PER; m++) {
         const int i = ct + m * kDecConsumers;
         double v = 0.0;
-        if (i < D) {
+        if (i < D && !ab) {
           v = (double)bf(hin[i]);
           if (chain) v = (double)bf(d2bf_bits(v + (double)S.yprev[i]));
         }
@@ -952,7 +922,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
 #pragma unroll
       for (int m = 0; m < PER; m++) {
         const int i = ct + m * kDecConsumers;
-        if (i < D) {
+        if (i < D && !ab) {
           const float xv = bf(d2bf_bits(hv[m] * (double)bf(gam[i]) * rinv));
           S.x[i] = xv;
           S.xt[xt_index(i, NCH)] = xv * nib_scale(i & 7);
@@ -961,8 +931,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       cbar();
       if (ct == 0) stamp(P, l, TR_NORM);
     }
-    if (it.kind == IT_R) {
-      // ---- router rows of a reactive layer
+    if (ab) {
+      // nothing more for this item (the barriers above are the same for every thread)
+    } else if (it.kind == IT_R) {
+      // ---- router rows of a reactive layer, one warp per row
       const uint16_t *rw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][2]);
       #pragma unroll 1
       for (int q2 = warp; q2 < in; q2 += kDecCW) {
@@ -972,7 +944,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     } else if (it.kind == IT_XR) {
       // ---- head rows, LoRA A rows and the predicted experts' router rows on x
       const int nh = Y.head ? P.E : 0, nl = lora ? r : 0;
-      unsigned long long *blk = P.t_blk + (size_t)l * P.blk;
       #pragma unroll 1
       for (int q2 = warp; q2 < in; q2 += kDecCW) {
         const int u = ia + q2;
@@ -996,87 +967,73 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (lane == 0) st_tag(dst, tag, __float_as_uint(v));
       }
     } else if (it.kind == IT_GU) {
-      // ---- gate/up rows of this item's units
+      // ---- gate/up: a warp takes whole units (the gate row and the up row of one
+      // intermediate index, two independent dot products), applies the SwiGLU and
+      // publishes; RPW units per warp pass when a row needs fewer than 32 lanes
       if (ct == 0) stamp(P, l, TR_GU_FULL);
-      // this lane's activation chunks stay in registers for every row of the item
       constexpr int LPR = NCH < 32 ? NCH : 32;    // lanes per row
-      constexpr int RPW = 32 / LPR;               // rows per warp pass
+      constexpr int RPW = 32 / LPR;               // units per warp pass
       constexpr int CPL = NCH / LPR;              // chunks per lane
       const int sub = lane / LPR, sl = lane % LPR;
-      float xr[CPL][32];
-      float xsr[CPL];
+      const int slot0 = ia / I;
+      if (warp * RPW < in) {
+        float xr[CPL][32];
+        float xsr[CPL];
 #pragma unroll
-      for (int cc = 0; cc < CPL; cc++) {
-        load_chunk(S.xt, NCH, sl + cc * LPR, xr[cc]);
-        xsr[cc] = chunk_raw_sum(xr[cc]);
-      }
-      GuPiece pc[kMaxPieces];
-      const int np = pieces_of(ia, in, I, pc);
-      float *gu_g = S.ydot;            // raw g and u of every row of this item
-      int roff = 0;
-      #pragma unroll 1
-      for (int p = 0; p < np; p++) {
-        const int R = pc[p].i1 - pc[p].i0, sg = kGuPiece0 + 6 * p;
-        const uint8_t *gc = S.ring + S.seg_off[slot][sg + 0];
-        const uint16_t *gs = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 1]);
-        const uint16_t *gm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 2]);
-        const uint8_t *uc = S.ring + S.seg_off[slot][sg + 3];
-        const uint16_t *us = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 4]);
-        const uint16_t *um = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 5]);
+        for (int cc = 0; cc < CPL; cc++) {
+          load_chunk(S.xt, NCH, sl + cc * LPR, xr[cc]);
+          xsr[cc] = chunk_raw_sum(xr[cc]);
+        }
         #pragma unroll 1
-        for (int base = warp * RPW; base < 2 * R; base += kDecCW * RPW) {
-          const int item = base + sub;
-          const bool valid = item < 2 * R;
-          float acc = 0.f;
+        for (int base = warp * RPW; base < in; base += kDecCW * RPW) {
+          const int u = base + sub;
+          const bool valid = u < in;
+          // unit u = global unit ia + u: slot (ia + u) / I, index (ia + u) % I; its piece p
+          // is the slot's order among the item's slots, its row the index minus the
+          // piece's first index
+          const int gidx = ia + u, es = gidx / I, p = es - slot0;   // es: expert slot of the unit
+          const int i = gidx - es * I, row = i - (p == 0 ? ia - slot0 * I : 0), sg = kGuPiece0 + 6 * p;
+          float ag = 0.f, au = 0.f;
           if (valid) {
-            const int row = item >> 1, up = item & 1;
-            const uint8_t *cw = (up ? uc : gc) + (size_t)row * (D / 2);
-            const uint16_t *sc = (up ? us : gs) + (size_t)row * (D / 64);
-            const uint16_t *mn = (up ? um : gm) + (size_t)row * (D / 64);
+            const uint8_t *gcw = S.ring + S.seg_off[slot][sg + 0] + (size_t)row * (D / 2);
+            const uint16_t *gsc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 1]) + (size_t)row * (D / 64);
+            const uint16_t *gmn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 2]) + (size_t)row * (D / 64);
+            const uint8_t *ucw = S.ring + S.seg_off[slot][sg + 3] + (size_t)row * (D / 2);
+            const uint16_t *usc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 4]) + (size_t)row * (D / 64);
+            const uint16_t *umn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 5]) + (size_t)row * (D / 64);
 #pragma unroll
             for (int cc = 0; cc < CPL; cc++) {
               const int ch = sl + cc * LPR;
-              const uint4 w = *reinterpret_cast<const uint4 *>(cw + ch * 16);
-              const float qd = chunk_qdot(w, xr[cc]);
-              acc = fmaf(bf(sc[ch >> 1]), qd, fmaf(bf(mn[ch >> 1]), xsr[cc], acc));
+              const uint4 wg = *reinterpret_cast<const uint4 *>(gcw + ch * 16);
+              const uint4 wu = *reinterpret_cast<const uint4 *>(ucw + ch * 16);
+              const float qg = chunk_qdot(wg, xr[cc]);
+              const float qu = chunk_qdot(wu, xr[cc]);
+              ag = fmaf(bf(gsc[ch >> 1]), qg, fmaf(bf(gmn[ch >> 1]), xsr[cc], ag));
+              au = fmaf(bf(usc[ch >> 1]), qu, fmaf(bf(umn[ch >> 1]), xsr[cc], au));
             }
           }
-          acc = group_sum(acc, LPR);
-          if (valid && sl == 0) gu_g[2 * roff + item] = acc;
-        }
-        roff += R;
-      }
-      cbar();
-      if (ct == 0) stamp(P, l, TR_GU_ROWS);
-      // publish: routed rows as a = bf16(silu(g) u); shared rows as raw (g, u)
-      roff = 0;
-      #pragma unroll 1
-      for (int p = 0; p < np; p++) {
-        const int R = pc[p].i1 - pc[p].i0;
-        const bool shared = pc[p].slot == k;
-        #pragma unroll 1
-        for (int row = ct; row < R; row += kDecConsumers) {
-          const float g = gu_g[2 * (roff + row)], u = gu_g[2 * (roff + row) + 1];
-          const int i = pc[p].i0 + row;
-          unsigned long long *blk = P.t_blk + (size_t)l * P.blk;
-          if (shared) {
-            st_tag(blk + k * I + 2 * i, tag, __float_as_uint(g));
-            st_tag(blk + k * I + 2 * i + 1, tag, __float_as_uint(u));
-          } else {
-            st_tag(blk + pc[p].slot * I + i, tag, f2bf(g / (1.0f + expf(-g)) * u));
+          ag = group_sum(ag, LPR);
+          au = group_sum(au, LPR);
+          if (valid && sl == 0) {
+            if (es == k) {
+              st_tag(blk + k * I + 2 * i, tag, __float_as_uint(ag));
+              st_tag(blk + k * I + 2 * i + 1, tag, __float_as_uint(au));
+            } else {
+              st_tag(blk + es * I + i, tag, f2bf(ag / (1.0f + expf(-ag)) * au));
+            }
           }
         }
-        roff += R;
       }
       if (ct == 0) stamp(P, l, TR_GU_DONE);
     } else {
       // ---- down + combine ---------------------------------------------------------------
       float *at = S.at, *gus = S.gus;
-      if (it.first) {
-        // one batched poll over the layer's block: a of the routed slots, the shared
-        // expert's raw g/u, t_g/t_u (with LoRA) and the selected router logits (predicted)
+      if (shared_state) {
+        // the layer's first down item here: one batched poll over the layer's block (a of
+        // the routed slots, the shared expert's raw g/u, t_g/t_u with LoRA, the selected
+        // router logits of a predicted layer), then a_s, the gates and t_d, kept for the
+        // layer's later down items
         {
-          const unsigned long long *blk = P.t_blk + (size_t)l * P.blk;
           Range rg[4];
           int nr = 0;
           rg[nr++] = Range{blk, S.stg, k * I};
@@ -1085,62 +1042,64 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           if (pred) rg[nr++] = Range{blk + (k + 2) * I + 2 * r, reinterpret_cast<uint32_t *>(S.rl), k};
           ab |= !poll_ranges(rg, nr, tag, ct, C);
         }
-        if (cbar_or(ab)) break;
-        // routed a values: bf16 payloads -> pre-scaled, chunk-transposed fp32
+        ab = cbar_or(ab);
+        if (!ab) {
+          // routed a values: bf16 payloads -> pre-scaled, chunk-transposed fp32
 #pragma unroll 1
-        for (int i = ct; i < k * I; i += kDecConsumers) {
-          const int j = i / I, e = i - j * I;
-          at[j * I + xt_index(e, NCI)] = bf(S.stg[i] & 0xFFFFu) * nib_scale(e & 7);
-        }
-        if (ct == 0) stamp(P, l, TR_A_POLL);
-        const int sbd = dn_bd(k);
-        const uint16_t *bgm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 1]);
-        const uint16_t *bum = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 2]);
-        const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 3]);
-        // the shared expert's activation with its LoRA up branch (every CTA, same order)
-        #pragma unroll 1
-        for (int i = ct; i < I; i += kDecConsumers) {
-          float g = gus[2 * i], u = gus[2 * i + 1];
-          if (lora) {
-            float lg = 0.f, lu = 0.f;
-            #pragma unroll 1
-            for (int j = 0; j < r; j += 8) {
-              const uint4 wg = *reinterpret_cast<const uint4 *>(bgm + i * r + j);
-              const uint4 wu = *reinterpret_cast<const uint4 *>(bum + i * r + j);
-              const uint32_t gw[4] = {wg.x, wg.y, wg.z, wg.w}, uw[4] = {wu.x, wu.y, wu.z, wu.w};
+          for (int i = ct; i < k * I; i += kDecConsumers) {
+            const int j = i / I, e = i - j * I;
+            at[j * I + xt_index(e, NCI)] = bf(S.stg[i] & 0xFFFFu) * nib_scale(e & 7);
+          }
+          if (ct == 0) stamp(P, l, TR_A_POLL);
+          const int sbd = dn_bd(k);
+          const uint16_t *bgm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 1]);
+          const uint16_t *bum = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sbd + 2]);
+          // the shared expert's activation with its LoRA up branch (every CTA, same order)
+          #pragma unroll 1
+          for (int i = ct; i < I; i += kDecConsumers) {
+            float g = gus[2 * i], u = gus[2 * i + 1];
+            if (lora) {
+              float lg = 0.f, lu = 0.f;
+              #pragma unroll 1
+              for (int j = 0; j < r; j += 8) {
+                const uint4 wg = *reinterpret_cast<const uint4 *>(bgm + i * r + j);
+                const uint4 wu = *reinterpret_cast<const uint4 *>(bum + i * r + j);
+                const uint32_t gw[4] = {wg.x, wg.y, wg.z, wg.w}, uw[4] = {wu.x, wu.y, wu.z, wu.w};
 #pragma unroll
-              for (int q2 = 0; q2 < 4; q2++) {
-                lg = fmaf(bf(gw[q2] & 0xFFFFu), S.tl[j + 2 * q2], lg);
-                lg = fmaf(bf(gw[q2] >> 16), S.tl[j + 2 * q2 + 1], lg);
-                lu = fmaf(bf(uw[q2] & 0xFFFFu), S.tl[r + j + 2 * q2], lu);
-                lu = fmaf(bf(uw[q2] >> 16), S.tl[r + j + 2 * q2 + 1], lu);
+                for (int q2 = 0; q2 < 4; q2++) {
+                  lg = fmaf(bf(gw[q2] & 0xFFFFu), S.tl[j + 2 * q2], lg);
+                  lg = fmaf(bf(gw[q2] >> 16), S.tl[j + 2 * q2 + 1], lg);
+                  lu = fmaf(bf(uw[q2] & 0xFFFFu), S.tl[r + j + 2 * q2], lu);
+                  lu = fmaf(bf(uw[q2] >> 16), S.tl[r + j + 2 * q2 + 1], lu);
+                }
               }
+              g = fmaf(P.c, lg, g);
+              u = fmaf(P.c, lu, u);
             }
-            g = fmaf(P.c, lg, g);
-            u = fmaf(P.c, lu, u);
+            const float av = bf(f2bf(g / (1.0f + expf(-g)) * u));
+            S.asraw[i] = av;
+            at[k * I + xt_index(i, NCI)] = av * nib_scale(i & 7);
           }
-          const float av = bf(f2bf(g / (1.0f + expf(-g)) * u));
-          S.asraw[i] = av;
-          at[k * I + xt_index(i, NCI)] = av * nib_scale(i & 7);
-        }
-        if (ct == 0) {
-          float lg[kMaxK], mx = -INFINITY, sum = 0.f;
-          #pragma unroll 1
-          for (int j = 0; j < k; j++) {
-            lg[j] = pred ? S.rl[j] : S.rlsel[l & 63][j];
-            mx = fmaxf(mx, lg[j]);
+          if (ct == 0) {
+            float lg[kMaxK], mx = -INFINITY, sum = 0.f;
+            #pragma unroll 1
+            for (int j = 0; j < k; j++) {
+              lg[j] = pred ? S.rl[j] : S.rlsel[l & 63][j];
+              mx = fmaxf(mx, lg[j]);
+            }
+            #pragma unroll 1
+            for (int j = 0; j < k; j++) {
+              lg[j] = expf(lg[j] - mx);
+              sum += lg[j];
+            }
+            #pragma unroll 1
+            for (int j = 0; j < k; j++) S.gates[j] = lg[j] / sum;
           }
-          #pragma unroll 1
-          for (int j = 0; j < k; j++) {
-            lg[j] = expf(lg[j] - mx);
-            sum += lg[j];
-          }
-          #pragma unroll 1
-          for (int j = 0; j < k; j++) S.gates[j] = lg[j] / sum;
         }
         cbar();
-        // t_d = Ad a_s (LoRA down branch)
-        if (lora) {
+        if (!ab && lora) {
+          // t_d = Ad a_s (LoRA down branch)
+          const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k) + 3]);
           #pragma unroll 1
           for (int j = warp; j < r; j += kDecCW) {
             float acc = 0.f;
@@ -1153,73 +1112,82 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         cbar();
         if (ct == 0) stamp(P, l, TR_TD_POLL);
       }
-      const int R = in;
-      constexpr int LPR = NCI < 32 ? NCI : 32;
-      constexpr int RPW = 32 / LPR;
-      constexpr int CPL = NCI / LPR;
-      const int sub = lane / LPR, sl = lane % LPR;
-      float *yd = S.ydot;
-      #pragma unroll 1
-      for (int j = 0; j <= k; j++) {
-        // expert j's activation chunks in registers, then its rows
-        float ar[CPL][32];
-        float asr[CPL];
+      if (!ab) {
+        // a warp owns its rows across every expert: y accumulates in registers in the
+        // combine order (routed experts with their gates, then the shared expert)
+        constexpr int LPR = NCI < 32 ? NCI : 32;
+        constexpr int RPW = 32 / LPR;
+        constexpr int CPL = NCI / LPR;
+        constexpr int PM = kDnMaxRows / (kDecCW * RPW) + 1;
+        const int sub = lane / LPR, sl = lane % LPR;
+        float y[PM];
 #pragma unroll
-        for (int cc = 0; cc < CPL; cc++) {
-          load_chunk(S.at + j * I, NCI, sl + cc * LPR, ar[cc]);
-          asr[cc] = chunk_raw_sum(ar[cc]);
-        }
-        const uint8_t *cb = S.ring + S.seg_off[slot][3 * j];
-        const uint16_t *sb = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3 * j + 1]);
-        const uint16_t *mb = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3 * j + 2]);
-        #pragma unroll 1
-        for (int base = warp * RPW; base < R; base += kDecCW * RPW) {
-          const int row = base + sub;
-          const bool valid = row < R;
-          float acc = 0.f;
-          if (valid) {
-            const uint8_t *cw = cb + (size_t)row * (I / 2);
-            const uint16_t *sc = sb + (size_t)row * (I / 64);
-            const uint16_t *mn = mb + (size_t)row * (I / 64);
+        for (int pp = 0; pp < PM; pp++) y[pp] = 0.f;
+        if (warp * RPW < in) {
+          #pragma unroll 1
+          for (int j = 0; j <= k; j++) {
+            float ar[CPL][32];
+            float asr[CPL];
 #pragma unroll
             for (int cc = 0; cc < CPL; cc++) {
-              const int ch = sl + cc * LPR;
-              const uint4 w = *reinterpret_cast<const uint4 *>(cw + ch * 16);
-              const float qd = chunk_qdot(w, ar[cc]);
-              acc = fmaf(bf(sc[ch >> 1]), qd, fmaf(bf(mn[ch >> 1]), asr[cc], acc));
+              load_chunk(S.at + j * I, NCI, sl + cc * LPR, ar[cc]);
+              asr[cc] = chunk_raw_sum(ar[cc]);
+            }
+            const float gj = j < k ? S.gates[j] : 1.f;
+            const uint8_t *cb = S.ring + S.seg_off[slot][3 * j];
+            const uint16_t *sb = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3 * j + 1]);
+            const uint16_t *mb = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3 * j + 2]);
+#pragma unroll
+            for (int pp = 0; pp < PM; pp++) {
+              const int base = pp * kDecCW * RPW + warp * RPW;
+              if (base < in) {
+                const int row = base + sub;
+                const bool valid = row < in;
+                float acc = 0.f;
+                if (valid) {
+                  const uint8_t *cw = cb + (size_t)row * (I / 2);
+                  const uint16_t *sc = sb + (size_t)row * (I / 64);
+                  const uint16_t *mn = mb + (size_t)row * (I / 64);
+#pragma unroll
+                  for (int cc = 0; cc < CPL; cc++) {
+                    const int ch = sl + cc * LPR;
+                    const uint4 w = *reinterpret_cast<const uint4 *>(cw + ch * 16);
+                    const float qd = chunk_qdot(w, ar[cc]);
+                    acc = fmaf(bf(sc[ch >> 1]), qd, fmaf(bf(mn[ch >> 1]), asr[cc], acc));
+                  }
+                }
+                acc = group_sum(acc, LPR);
+                y[pp] = j < k ? fmaf(gj, acc, y[pp]) : y[pp] + acc;
+              }
             }
           }
-          acc = group_sum(acc, LPR);
-          if (valid && sl == 0) yd[row * (k + 1) + j] = acc;
+          const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]);
+#pragma unroll
+          for (int pp = 0; pp < PM; pp++) {
+            const int row = pp * kDecCW * RPW + warp * RPW + sub;
+            if (row < in && sl == 0) {
+              float yv = y[pp];
+              if (lora) {
+                float lo = 0.f;
+                #pragma unroll 1
+                for (int j = 0; j < r; j++) lo = fmaf(bf(bd[row * r + j]), S.td[j], lo);
+                yv = fmaf(P.c, lo, yv);
+              }
+              const int n = ia + row;
+              st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(yv));
+              P.y[(size_t)l * D + n] = f2bf(yv);
+              if (P.yf) P.yf[(size_t)l * D + n] = yv;
+            }
+          }
         }
-      }
-      if (ct == 0) stamp(P, l, TR_DN_DOTS);
-      cbar();
-      const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]);
-      #pragma unroll 1
-      for (int row = ct; row < R; row += kDecConsumers) {
-        float y = 0.f;
-        #pragma unroll 1
-        for (int j = 0; j < k; j++) y = fmaf(S.gates[j], yd[row * (k + 1) + j], y);
-        y += yd[row * (k + 1) + k];
-        if (lora) {
-          float lo = 0.f;
-          #pragma unroll 1
-          for (int j = 0; j < r; j++) lo = fmaf(bf(bd[row * r + j]), S.td[j], lo);
-          y = fmaf(P.c, lo, y);
-        }
-        const int n = ia + row;
-        st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(y));
-        P.y[(size_t)l * D + n] = f2bf(y);
-        if (P.yf) P.yf[(size_t)l * D + n] = y;
       }
       if (ct == 0) stamp(P, l, TR_DN_DONE);
     }
-    // release the item's ring space
-    cbar();
+    // this warp is done with the item's bytes
+    __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty[slot]);
-    q++;
   }
+  ab = cbar_or(ab);
   if (ab) return;
   // ---- end of step: CTA c records layer c's routing and runs layer c's head top-k; every
   // logit is complete by now --------------------------------------------------------------
