@@ -33,7 +33,7 @@ namespace e0 {
 constexpr int kDecThreads = 416;          // 1 producer warp + 12 consumer warps
 constexpr int kDecConsumers = 384;
 constexpr int kDecCW = 12;
-constexpr int kRingBytes = 156 * 1024;
+constexpr int kRingBytes = 174 * 1024;
 constexpr int kDecMaxK = 4;               // routed experts per token on this path
 constexpr int kNSlot = 8;                 // tasks in flight
 
@@ -361,14 +361,14 @@ __device__ __forceinline__ void item_seg(const DecodeParams &P, const DecLayer &
 template <int D, int I>
 struct DecSmem {
   uint8_t ring[kRingBytes];
-  float x[D];                        // x (natural order): router, head and LoRA rows
   float xt[D];                       // x pre-scaled per nibble position, chunk-transposed
-  float yprev[D];                    // previous layer's y (fp32)
+  union {                            // used by different items, never at the same time:
+    float yprev[D];                  //   the previous layer's y (fp32), in order + chained
+    uint32_t stg[kDecMaxK * I];      //   routed a payloads as polled (a layer's first down item)
+  };
   float at[(kDecMaxK + 1) * I];      // a of every slot, pre-scaled, chunk-transposed per slot
-  uint32_t stg[kDecMaxK * I];        // routed a payloads as polled
   float asraw[I];                    // the shared expert's a (natural order, for t_d)
   float gus[2 * I];                  // the shared expert's raw g and u (interleaved per row)
-  float ydot[64 * (kMaxK + 1)];
   double dred[16];
   float gates[kMaxK];
   float tl[2 * kMaxR];               // t_g, t_u
@@ -415,7 +415,7 @@ __device__ __forceinline__ bool timed_out(unsigned long long &t0, unsigned long 
 // phase's units over all layers form one list, split evenly and contiguously across the
 // CTAs, so that a CTA streams long runs of rows of one or two layers instead of a sliver
 // of every layer.  Phases: R (reactive layers' routers), XR, TK (the reactive layers this
-// CTA needs), GU, DN.  Items are cut to at most about 36 KB of weight bytes.  A CTA then
+// CTA needs), GU, DN.  Items are cut to at most about 58 KB of weight bytes (three fit the ring).  A CTA then
 // computes a handful of norms per step, polls other CTAs' results a handful of times, and
 // waits on other CTAs only where a phase needs the previous one (R -> TK, GU -> DN).
 // ---------------------------------------------------------------------------------------
@@ -450,7 +450,7 @@ __device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I>
       if (b > a) put(IT_DN, l, a, b - a);
     }
   } else {
-    constexpr int kItemBytes = 36 * 1024;
+    constexpr int kItemBytes = 58 * 1024;
     const int gu_chunk = min(kItemBytes / (2 * (D / 2 + D / 16)), 288);
     const int dn_chunk = min(kItemBytes / ((k + 1) * (I / 2 + I / 16) + 2 * P.r), kDnMaxRows);
     const int xr_chunk = max(kItemBytes / (2 * P.ldh), 1);
@@ -754,23 +754,26 @@ __device__ __forceinline__ bool wait_full(uint64_t *bar, uint32_t par, const Ctl
   return true;
 }
 
-// bf16 row (D elements in shared memory) dotted with x (fp32, shared memory): one warp.
+// bf16 row (D elements in shared memory) dotted with x, read from its pre-scaled,
+// chunk-transposed copy xt (elements 8c..8c+3 and 8c+4..8c+7 are two float4 there; the
+// per-position scales 2^-p are undone exactly): one warp.
 template <int D>
-__device__ __noinline__ float bf16_row_x(const uint16_t *w, const float *x, int lane) {
+__device__ __noinline__ float bf16_row_x(const uint16_t *w, const float *xt, int lane) {
+  constexpr int NCH = D / 32;
   float acc = 0.f;
 #pragma unroll 2
   for (int ch = lane; ch < D / 8; ch += 32) {
     const uint4 v = *reinterpret_cast<const uint4 *>(w + ch * 8);
-    const float4 a = *reinterpret_cast<const float4 *>(x + ch * 8);
-    const float4 b = *reinterpret_cast<const float4 *>(x + ch * 8 + 4);
-    acc = fmaf(bf(v.x & 0xFFFFu), a.x, acc);
-    acc = fmaf(bf(v.x >> 16), a.y, acc);
-    acc = fmaf(bf(v.y & 0xFFFFu), a.z, acc);
-    acc = fmaf(bf(v.y >> 16), a.w, acc);
-    acc = fmaf(bf(v.z & 0xFFFFu), b.x, acc);
-    acc = fmaf(bf(v.z >> 16), b.y, acc);
-    acc = fmaf(bf(v.w & 0xFFFFu), b.z, acc);
-    acc = fmaf(bf(v.w >> 16), b.w, acc);
+    const float4 a = *reinterpret_cast<const float4 *>(xt + ((2 * (ch & 3)) * NCH + (ch >> 2)) * 4);
+    const float4 b = *reinterpret_cast<const float4 *>(xt + ((2 * (ch & 3) + 1) * NCH + (ch >> 2)) * 4);
+    acc = fmaf(bf(v.x & 0xFFFFu), a.x * (1.0f / nib_scale(0)), acc);
+    acc = fmaf(bf(v.x >> 16), a.y * (1.0f / nib_scale(1)), acc);
+    acc = fmaf(bf(v.y & 0xFFFFu), a.z * (1.0f / nib_scale(2)), acc);
+    acc = fmaf(bf(v.y >> 16), a.w * (1.0f / nib_scale(3)), acc);
+    acc = fmaf(bf(v.z & 0xFFFFu), b.x * (1.0f / nib_scale(4)), acc);
+    acc = fmaf(bf(v.z >> 16), b.y * (1.0f / nib_scale(5)), acc);
+    acc = fmaf(bf(v.w & 0xFFFFu), b.z * (1.0f / nib_scale(6)), acc);
+    acc = fmaf(bf(v.w >> 16), b.w * (1.0f / nib_scale(7)), acc);
   }
   return warp_sum(acc);
 }
@@ -924,7 +927,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         const int i = ct + m * kDecConsumers;
         if (i < D && !ab) {
           const float xv = bf(d2bf_bits(hv[m] * (double)bf(gam[i]) * rinv));
-          S.x[i] = xv;
           S.xt[xt_index(i, NCH)] = xv * nib_scale(i & 7);
         }
       }
@@ -938,7 +940,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       const uint16_t *rw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][2]);
       #pragma unroll 1
       for (int q2 = warp; q2 < in; q2 += kDecCW) {
-        const float v = bf16_row_x<D>(rw + (size_t)q2 * D, S.x, lane);
+        const float v = bf16_row_x<D>(rw + (size_t)q2 * D, S.xt, lane);
         if (lane == 0) st_tag(P.t_rlog + (size_t)l * P.E + ia + q2, tag, __float_as_uint(v));
       }
     } else if (it.kind == IT_XR) {
@@ -963,7 +965,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           row = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kXrSel + u - max(ia, nh + 2 * nl)]);
           dst = blk + (k + 2) * I + 2 * r + (u - nh - 2 * nl);
         }
-        const float v = bf16_row_x<D>(row, S.x, lane);
+        const float v = bf16_row_x<D>(row, S.xt, lane);
         if (lane == 0) st_tag(dst, tag, __float_as_uint(v));
       }
     } else if (it.kind == IT_GU) {
