@@ -7,6 +7,8 @@
 #include "e0_decode.cuh"
 #include "e0_prefill.cuh"
 
+#include <cudaTypedefs.h>
+
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -123,7 +125,7 @@ struct e0_ctx {
   uint16_t *g_h = nullptr, *g_y = nullptr;   // [L][maxT][d] graph input / output
   float *g_yf = nullptr;                     // [L][maxT][d]
   // tensor-core prefill workspaces: K-permuted bf16 operands and their group-of-64 sums
-  uint16_t *xp = nullptr, *ap = nullptr;
+  uint16_t *xp = nullptr, *ap = nullptr, *xg = nullptr;
   float *xsum = nullptr, *asum = nullptr;
   float *yacc = nullptr;
   TcTile *tiles = nullptr;
@@ -162,7 +164,7 @@ extern "C" int e0_destroy(e0_ctx *C) {
   cudaDeviceSynchronize();
   void *bufs[] = {C->xb, C->xf, C->logits, C->hlog, C->lt, C->gates, C->idx, C->a, C->plan_mem,
                   C->yscratch, C->pred_tab, C->hist_tab, C->err, C->h1pre, C->h1, C->pool.mem, C->pool.slot_of,
-                  C->pool.slot_tag, C->xp, C->ap, C->xsum, C->asum, C->yacc, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
+                  C->pool.slot_tag, C->xp, C->ap, C->xg, C->xsum, C->asum, C->yacc, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
   for (void *b : bufs)
     if (b) cudaFree(b);
   decode_free(C->dec);
@@ -217,7 +219,7 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
   cudaMemset(C->pf_idx, 0xFF, (T + 1) * k * sizeof(int32_t));
   if (T >= kTcMinTokens) {
     C->tile_cap = (int)((T * k + kTcN - 1) / kTcN + std::min(E, T * k) + (T + kTcN - 1) / kTcN + 1);
-    if ((rc = dalloc(&C->xp, T * d)) || (rc = dalloc(&C->ap, T * (k + 1) * I)) ||
+    if ((rc = dalloc(&C->xp, T * d)) || (rc = dalloc(&C->ap, T * (k + 1) * I)) || (rc = dalloc(&C->xg, T * k * d)) ||
         (rc = dalloc(&C->xsum, T * (d / 64 + 1))) || (rc = dalloc(&C->asum, T * (k + 1) * (I / 64 + 1))) ||
         (rc = dalloc(&C->yacc, T * d)) ||
         (rc = dalloc(&C->tiles, (size_t)C->tile_cap)) || (rc = dalloc(&C->ntiles, 1))) {
@@ -302,6 +304,32 @@ static inline int grid_for(int warps_needed, int cap) {
   return b < 1 ? 1 : (b > cap ? cap : b);
 }
 
+// TMA descriptor of a row-major bf16 matrix [rows, K] read in boxes of 64 columns x 128
+// rows with the 128-byte swizzle of the tensor-core operand tiles (zeros past the end).
+// The encoder comes from the driver through the runtime's entry-point query.
+static int tmap_bf16_rows(CUtensorMap *m, const void *base, int K, long long rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return fail(E0_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  }
+  if (((uintptr_t)base & 15) || K % 64 || rows < 1)
+    return fail(E0_ERR_INVALID_ARG, "tensor map: base, K or rows not supported");
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(E0_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return E0_OK;
+}
+
 // The tensor-core kernels serve calls of at least kTcMinTokens tokens (or any size when
 // selected), in contexts created with the workspaces for them.
 static bool use_tc(e0_ctx *C, int T) {
@@ -369,13 +397,20 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   CKL("k_perm_sums(x)");
   k_tc_tiles<<<1, 32, 0, s>>>(C->plan, K.T, C->tiles, C->ntiles, C->tile_cap);
   CKL("k_tc_tiles");
+  // the routed tokens' x rows in expert-grouped order (each tile's tokens consecutive)
+  k_group_rows<<<K.T * D.top_k, std::min(256, D.d_model / 8), 0, s>>>(C->xp, C->plan.assign, D.top_k, D.d_model, C->xg);
+  CKL("k_group_rows");
   TcArgs A{};
+  int rc;
+  if ((rc = tmap_bf16_rows(&A.tmB[0], C->xg, D.d_model, (long long)K.T * D.top_k)) ||
+      (rc = tmap_bf16_rows(&A.tmB[1], C->xp, D.d_model, K.T)))
+    return rc;
   A.mode = 0; A.T = K.T; A.d = D.d_model; A.I = D.d_ff; A.k = D.top_k; A.r = D.lora_rank; A.c = D.lora_scale;
   A.src = src; A.shared = (const uint8_t *)Y.shared; A.bl = C->bl; A.P = C->plan; A.tiles = C->tiles;
   A.ntiles = C->ntiles; A.xp = C->xp; A.xsum = C->xsum; A.ap = C->ap; A.asum = C->asum; A.ap_out = C->ap;
   A.Bg = (const uint16_t *)Y.lora_Bg; A.Bu = (const uint16_t *)Y.lora_Bu; A.lt = C->lt; A.gates = K.gates;
   A.yacc = C->yacc; A.err = C->err; A.timeout_ns = 2000000000ull;
-  const int tc_smem_bytes = (int)sizeof(TcSmem) + 1024;
+  const int tc_smem_bytes = (int)sizeof(TwSmem) + 1024;
   static bool attr_done = false;
   if (!attr_done) {
     CK(cudaFuncSetAttribute(k_moe_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem_bytes));
@@ -383,7 +418,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   }
   const int tmax = std::min(C->tile_cap, (K.T * D.top_k + kTcN - 1) / kTcN + std::min(D.n_experts, K.T * D.top_k) +
                                               (K.T + kTcN - 1) / kTcN);
-  k_moe_gemm_tc<<<tmax * (D.d_ff / 64), kTcThreads, tc_smem_bytes, s>>>(A);
+  k_moe_gemm_tc<<<tmax * (D.d_ff / 64), kTwThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(gate/up)");
   const long long ag = (long long)K.T * (D.top_k + 1) * (D.d_ff / 64);
   k_perm_sums<<<(unsigned)((ag + 255) / 256), 256, 0, s>>>(C->ap, (long long)K.T * (D.top_k + 1), D.d_ff, nullptr,
@@ -396,7 +431,9 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   }
   CK(cudaMemsetAsync(C->yacc, 0, nx * sizeof(float), s));
   A.mode = 1;
-  k_moe_gemm_tc<<<tmax * (D.d_model / 128), kTcThreads, tc_smem_bytes, s>>>(A);
+  if ((rc = tmap_bf16_rows(&A.tmB[0], C->ap, D.d_ff, (long long)K.T * (D.top_k + 1)))) return rc;
+  A.tmB[1] = A.tmB[0];
+  k_moe_gemm_tc<<<tmax * (D.d_model / 128), kTwThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(down)");
   k_tc_finish<<<(unsigned)((nx + 255) / 256), 256, 0, s>>>(C->yacc, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
                                                            D.d_model, D.lora_rank, D.lora_scale, K.y, K.yf);

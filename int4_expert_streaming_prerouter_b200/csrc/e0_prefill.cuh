@@ -21,19 +21,16 @@
 // relative error at the tail of a 40k-output layer); x and a are bf16 values, exactly
 // representable in fp16 in their range.
 #pragma once
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include "e0_device.cuh"
 #include "e0_kernels.cuh"
 
 namespace e0 {
 
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 256;     // threads of the dense-rows kernel
 constexpr int kTcMinTokens = 64;    // contexts with at least this many tokens get the tensor-core path
 constexpr int kTcN = 128;           // tokens per tile (TMEM columns per accumulator)
-constexpr int kTcRawStages = 8;     // int4 code tiles of a K group (4 KB each) in the ring
-constexpr int kTcRawAhead = 7;      //   groups loaded ahead of the one being converted
-constexpr int kTcBStages = 4;       // activation tiles (16 KB each)
-constexpr int kTcBAhead = 3;
 constexpr int kTcMaxGroups = 64;    // K / 64 <= 64 (K <= 4096)
 
 struct TcTile {
@@ -42,6 +39,10 @@ struct TcTile {
 };
 
 struct TcArgs {
+  // B operands as TMA tensor maps (bf16, K-permuted rows, box 64 x 128, 128-byte swizzle):
+  // mode 0: [0] x in expert-grouped row order [T k, d], [1] x in token order [T, d];
+  // mode 1: [0] a in grouped order [T k + T, I] (the shared expert's rows last)
+  CUtensorMap tmB[2];
   int mode;                 // 0: gate/up + SwiGLU, 1: down + weighted combine
   int T, d, I, k, r;
   float c;
@@ -53,9 +54,9 @@ struct TcArgs {
   const int *ntiles;
   const uint16_t *xp;       // [T, d] x, bf16, K-permuted within 8-blocks (mode 0)
   const float *xsum;        // [T, d/64] group sums of x (mode 0)
-  const uint16_t *ap;       // [T, k+1, I] a, bf16, K-permuted (mode 1 input)
-  const float *asum;        // [T, k+1, I/64] group sums of a (mode 1)
-  uint16_t *ap_out;         // [T, k+1, I] (mode 0 output)
+  const uint16_t *ap;       // [T k + T, I] a, bf16, K-permuted, grouped rows (mode 1 input)
+  const float *asum;        // [T k + T, I/64] group sums of a (mode 1)
+  uint16_t *ap_out;         // [T k + T, I] (mode 0 output)
   const uint16_t *Bg, *Bu;  // [I, r] shared-expert LoRA up (mode 0), or nullptr
   const float *lt;          // [T, 3, r]
   const float *gates;       // [T, k] (mode 1)
@@ -93,6 +94,23 @@ __device__ __forceinline__ uint32_t tc_idesc(int M, int N) {
 // 16-byte asynchronous global -> shared copy; src_bytes = 0 fills the 16 bytes with zeros.
 __device__ __forceinline__ void tc_cp16(uint32_t dst, const void *src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// L2 policies: the int4 codes stream through once (evict first); the activations are read
+// again by every weight tile of the same expert (evict last)
+__device__ __forceinline__ unsigned long long tc_policy_first() {
+  unsigned long long p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ unsigned long long tc_policy_last() {
+  unsigned long long p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tc_cp16_hint(uint32_t dst, const void *src, uint32_t src_bytes, unsigned long long pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src), "r"(src_bytes),
+               "l"(pol)
+               : "memory");
 }
 __device__ __forceinline__ void tc_cp4(uint32_t dst, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
@@ -214,28 +232,68 @@ __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
 //   acc += s_g * P_g + (m_g - 128 s_g) * X_g      CUDA cores, X_g = sum_{k in g} x_k
 // which is sum_k (s_g q_k + m_g) x_k, the affine dequantisation folded into the
 // accumulation; so the weights need no fp32 dequantisation and one MMA per K = 16.
-// The MMA of group g overlaps the fold of group g - 1 and the conversion of group g + 1.
-// Codes and activations stream into shared memory through cp.async rings whose stages
-// complete on mbarriers, so loads run several groups ahead of their use.
+//
+// Warp-specialised, every hand-off on an mbarrier, so that loads, conversion, MMAs and
+// folds of different groups overlap:
+//   warp  0    loader: one TMA tile load per group brings the tile's 128 activation rows
+//              (stored in expert-grouped order, so a tile's tokens are consecutive rows)
+//              as the 128-byte swizzled B tile; the lanes copy the columns' group sums
+//   warp  1    TMEM owner; one thread issues the four MMAs of each group
+//   warps 2-5  converters: thread t owns weight row t; it streams its own row's codes
+//              kTwRawAhead groups ahead with cp.async (no hand-off needed) and writes
+//              128 + q as bf16 into the A tile ring (kTwAStages stages)
+//   warps 6-13 folders: TMEM lane quadrant warp % 4, half of the columns each; they fold
+//              every group into registers and run the epilogue (SwiGLU, or the weighted
+//              combine into y)
 // ---------------------------------------------------------------------------------------
-struct TcSmem {
-  uint8_t a[2][128 * 128];                 // A tiles (bf16, 128-byte swizzled K-major)
-  uint8_t b[kTcBStages][kTcN * 128];       // B tiles
-  uint8_t raw[kTcRawStages][128 * 32];     // int4 codes of one group, 32 bytes per row
+constexpr int kTwThreads = 448;
+constexpr int kTwLoadWarps = 1, kTwMmaWarp = 1, kTwConv0 = 2, kTwFold0 = 6;
+constexpr int kTwAStages = 3;
+constexpr int kTwBStages = 6;
+constexpr int kTwRawAhead = 3;      // groups of codes in flight per converter thread
+
+struct TwSmem {
+  uint8_t a[kTwAStages][128 * 128];        // A tiles (bf16, 128-byte swizzled K-major)
+  uint8_t b[kTwBStages][kTcN * 128];       // B tiles
+  float xs[kTwBStages][kTcN];              // the B columns' group sums
+  uint8_t raw[kTwRawAhead][128 * 32];      // int4 codes: converter thread t's row t
   uint16_t sc[128 * kTcMaxGroups];         // scale of every row and group [row][g]
   uint16_t mn[128 * kTcMaxGroups];         // min
-  float xs[kTcMaxGroups * kTcN];           // group sums of the B columns [g][column]
-  uint64_t rfull[kTcRawStages], bfull[kTcBStages], pre, mma[2];
+  uint64_t bfull[kTwBStages], bempty[kTwBStages], afull[kTwAStages], aempty[kTwAStages];
+  uint64_t tfull[2], tempty[2], pre;
   uint32_t tmem;
+  volatile int abort;
   int tok[kTcN];       // token of each column
   int dst[kTcN];       // ap row (mode 0) / gate index (mode 1) of each column, -1 = none
+  float gw[kTcN];      // combine weight of each column (mode 1)
 };
 
-__global__ void __launch_bounds__(kTcThreads, 1) k_moe_gemm_tc(TcArgs A) {
+// bounded wait on an mbarrier phase that also gives up once another role has aborted
+__device__ __forceinline__ bool tw_wait(uint64_t *b, uint32_t parity, unsigned long long budget, int *err,
+                                        volatile int *abort) {
+  unsigned long long t0 = 0;
+  while (!tc_mbar_test(b, parity)) {
+    if (*abort) return false;
+    const unsigned long long now = tc_now();
+    if (!t0) t0 = now;
+    else if (now - t0 > budget) {
+      atomicOr(err, DERR_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tc_mbar_arrive(uint64_t *b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc_smem(b)) : "memory");
+}
+
+__global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_constant__ TcArgs A) {
   extern __shared__ __align__(1024) uint8_t tc_raw[];
   // the swizzled tiles need 1024-byte alignment
-  TcSmem &S = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(tc_raw) + 1023) & ~(uintptr_t)1023);
-  const int tid = threadIdx.x, warp = tid >> 5;
+  TwSmem &S = *reinterpret_cast<TwSmem *>((reinterpret_cast<uintptr_t>(tc_raw) + 1023) & ~(uintptr_t)1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mtiles = A.mode == 0 ? A.I / 64 : A.d / 128;
   const int tile = blockIdx.x / mtiles, mt = blockIdx.x % mtiles;
   if (tile >= *A.ntiles) return;
@@ -250,31 +308,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_gemm_tc(TcArgs A) {
   const int G = K / 64;
   const unsigned long long budget = A.timeout_ns;
 
-  // column bookkeeping: token and destination of each column of this tile
-  for (int c = tid; c < kTcN; c += kTcThreads) {
+  // column bookkeeping: token, destination and combine weight of each column of this tile
+  for (int c = tid; c < kTcN; c += kTwThreads) {
     int tok = -1, dst = -1;
+    float w = 0.f;
     if (c < ncol) {
       if (shared) {
         tok = tl.n0 + c;
-        dst = A.mode == 0 ? tok * (A.k + 1) + A.k : -1;
+        dst = A.mode == 0 ? A.T * A.k + tok : -1;             // grouped row of a
+        w = 1.f;
       } else {
         const int asg = A.P.assign[A.P.ustart[tl.unit] + tl.n0 + c];   // t * k + slot
         tok = asg / A.k;
-        dst = A.mode == 0 ? tok * (A.k + 1) + asg % A.k : asg;
+        dst = A.mode == 0 ? A.P.ustart[tl.unit] + tl.n0 + c : asg;   // grouped row of a / gate index
+        if (A.mode == 1) w = A.gates[asg];
       }
     }
     S.tok[c] = tok;
     S.dst[c] = dst;
+    S.gw[c] = w;
   }
   if (tid == 0) {
-    for (int s = 0; s < kTcRawStages; s++) tc_mbar_init(&S.rfull[s], kTcThreads);
-    for (int s = 0; s < kTcBStages; s++) tc_mbar_init(&S.bfull[s], kTcThreads);
-    tc_mbar_init(&S.pre, kTcThreads);
-    tc_mbar_init(&S.mma[0], 1);
-    tc_mbar_init(&S.mma[1], 1);
+    for (int s = 0; s < kTwBStages; s++) {
+      tc_mbar_init(&S.bfull[s], 33);   // the TMA's expect_tx arrival + 32 group-sum lanes
+      tc_mbar_init(&S.bempty[s], 8);
+    }
+    for (int s = 0; s < kTwAStages; s++) {
+      tc_mbar_init(&S.afull[s], 4);
+      tc_mbar_init(&S.aempty[s], 1);
+    }
+    for (int s = 0; s < 2; s++) {
+      tc_mbar_init(&S.tfull[s], 1);
+      tc_mbar_init(&S.tempty[s], 8);
+    }
+    tc_mbar_init(&S.pre, 128);
+    S.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == kTwMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_smem(&S.tmem)),
                  "r"(2 * kTcN)
                  : "memory");
@@ -284,258 +355,251 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_moe_gemm_tc(TcArgs A) {
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = S.tmem;
-  const uint32_t idesc = tc_idesc(128, N);
 
-  // this thread's weight row (code loads and conversion): two threads per row, 16 code
-  // bytes (32 K elements) each.  mode 0 -> gate rows i0..i0+63 then up rows i0..i0+63
-  // (i0 = 64 mt); mode 1 -> down rows 128 mt .. 128 mt + 127
-  const int row = tid >> 1, half = tid & 1;
-  const uint8_t *codes;
-  const uint16_t *scl, *mnv;
-  if (A.mode == 0) {
-    const int i = mt * 64 + (row & 63);
-    const bool up = row >= 64;
-    codes = base + (up ? A.bl.uc : A.bl.gc) + (size_t)i * (A.d / 2);
-    scl = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.us : A.bl.gs)) + (size_t)i * G;
-    mnv = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.um : A.bl.gm)) + (size_t)i * G;
-  } else {
-    const int n = mt * 128 + row;
-    codes = base + A.bl.dc + (size_t)n * (A.I / 2);
-    scl = reinterpret_cast<const uint16_t *>(base + A.bl.ds) + (size_t)n * G;
-    mnv = reinterpret_cast<const uint16_t *>(base + A.bl.dm) + (size_t)n * G;
-  }
-  // B role: (column, 16-byte chunk) pairs e = tid + m * kTcThreads
-  constexpr int kBPer = kTcN * 8 / kTcThreads;
-  const uint16_t *bsrc[kBPer];
-#pragma unroll
-  for (int m = 0; m < kBPer; m++) {
-    const int e = tid + m * kTcThreads, c = e >> 3, ch = e & 7;
-    const int tok = S.tok[c];
-    bsrc[m] = nullptr;
-    if (tok >= 0)
-      bsrc[m] = (A.mode == 0 ? A.xp + (size_t)tok * A.d
-                             : A.ap + (size_t)(tok * (A.k + 1) + (shared ? A.k : S.dst[c] % A.k)) * A.I) + ch * 8;
-  }
-  auto load_raw = [&](int g) {
-    tc_cp16(tc_smem(S.raw[g % kTcRawStages] + row * 32 + half * 16), codes + g * 32 + half * 16, 16);
-    tc_cp_arrive(&S.rfull[g % kTcRawStages]);
-  };
-  auto load_b = [&](int g) {
-    uint8_t *dstb = S.b[g % kTcBStages];
-#pragma unroll
-    for (int m = 0; m < kBPer; m++) {
-      const int e = tid + m * kTcThreads, c = e >> 3, ch = e & 7;
-      if (c < N) tc_cp16(tc_smem(dstb + sw128(c, ch)), bsrc[m] ? (const void *)(bsrc[m] + g * 64) : (const void *)A.xsum,
-                         bsrc[m] ? 16u : 0u);
+  if (warp < kTwLoadWarps) {
+    // ---------------- loader: one TMA tile load per group + the columns' group sums -------
+    // the tile's tokens are consecutive rows of the grouped operand starting at row0; rows
+    // past the tensor's end arrive as zeros (their columns are never used)
+    const CUtensorMap *map = (A.mode == 0 && shared) ? &A.tmB[1] : &A.tmB[0];
+    const int row0 = shared ? (A.mode == 0 ? tl.n0 : A.T * A.k + tl.n0) : A.P.ustart[tl.unit] + tl.n0;
+    #pragma unroll 1
+    for (int g = 0; g < G; g++) {
+      const int bs = g % kTwBStages;
+      if (g >= kTwBStages &&
+          !tw_wait(&S.bempty[bs], (uint32_t)(((g / kTwBStages) - 1) & 1), budget, A.err, &S.abort))
+        break;
+      if (lane == 0) {
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_smem(&S.bfull[bs])),
+                     "r"(kTcN * 128)
+                     : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+                tc_smem(S.b[bs])),
+            "l"(map), "r"(g * 64), "r"(row0), "r"(tc_smem(&S.bfull[bs]))
+            : "memory");
+      }
+      for (int c = lane; c < N; c += 32) {
+        const int tok = S.tok[c];
+        if (tok < 0) continue;    // padding column: its sum is never used
+        const float *src = A.mode == 0 ? A.xsum + (size_t)tok * G : A.asum + (size_t)(row0 + c) * G;
+        tc_cp4(tc_smem(&S.xs[bs][c]), src + g);
+      }
+      tc_cp_arrive(&S.bfull[bs]);
     }
-    tc_cp_arrive(&S.bfull[g % kTcBStages]);
-  };
-
-  // scales, mins and the columns' group sums (staged [column][g] in the A area first);
-  // rows of fewer than 16 bytes (K < 512) go in 4-byte copies
-  {
-    const int rb = G * 2;                       // bytes of a row of scales (or mins)
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == kTwMmaWarp) {
+    // ---------------- one thread issues the MMAs ------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = tc_idesc(128, N);
+      int issued = 0;
+      #pragma unroll 1
+      for (int g = 0; g < G; g++) {
+        const int as = g % kTwAStages, bs = g % kTwBStages, tb = g & 1;
+        if (!tw_wait(&S.afull[as], (uint32_t)((g / kTwAStages) & 1), budget, A.err, &S.abort)) break;
+        if (!tw_wait(&S.bfull[bs], (uint32_t)((g / kTwBStages) & 1), budget, A.err, &S.abort)) break;
+        if (g >= 2 && !tw_wait(&S.tempty[tb], (uint32_t)(((g >> 1) - 1) & 1), budget, A.err, &S.abort)) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t sa = tc_smem(S.a[as]), sb = tc_smem(S.b[bs]);
+        const uint32_t td = tmem + (uint32_t)(tb * kTcN);
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)   // K = 16 per instruction: 32 bytes along the swizzled row
+          tc_mma(td, tc_desc(sa + kk * 32), tc_desc(sb + kk * 32), idesc, kk ? 1u : 0u);
+        tc_commit(&S.tfull[tb]);
+        tc_commit(&S.aempty[as]);
+        issued = g + 1;
+      }
+      // after an abort, the MMAs in flight finish before TMEM is given back
+      if (issued > 0 && issued < G)
+        tc_wait_all(&S.tfull[(issued - 1) & 1], (uint32_t)(((issued - 1) >> 1) & 1), budget, A.err);
+    }
+    __syncwarp();
+  } else if (warp < kTwFold0) {
+    // ---------------- converters: thread r owns weight row r ------------------------------
+    // mode 0 -> gate rows i0..i0+63 then up rows i0..i0+63 (i0 = 64 mt); mode 1 -> down
+    // rows 128 mt .. 128 mt + 127
+    const int r = tid - kTwConv0 * 32;
+    const uint8_t *codes;
+    const uint16_t *scl, *mnv;
+    if (A.mode == 0) {
+      const int i = mt * 64 + (r & 63);
+      const bool up = r >= 64;
+      codes = base + (up ? A.bl.uc : A.bl.gc) + (size_t)i * (A.d / 2);
+      scl = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.us : A.bl.gs)) + (size_t)i * G;
+      mnv = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.um : A.bl.gm)) + (size_t)i * G;
+    } else {
+      const int n = mt * 128 + r;
+      codes = base + A.bl.dc + (size_t)n * (A.I / 2);
+      scl = reinterpret_cast<const uint16_t *>(base + A.bl.ds) + (size_t)n * G;
+      mnv = reinterpret_cast<const uint16_t *>(base + A.bl.dm) + (size_t)n * G;
+    }
+    // the row's scales and mins for the folders (rows of fewer than 16 bytes in 4-byte copies)
+    const int rb = G * 2;
     if (rb % 16 == 0) {
-      for (int q = half; q < rb / 16; q += 2) {
-        tc_cp16(tc_smem(S.sc + row * G + q * 8), scl + q * 8, 16);
-        tc_cp16(tc_smem(S.mn + row * G + q * 8), mnv + q * 8, 16);
+      for (int q = 0; q < rb / 16; q++) {
+        tc_cp16(tc_smem(S.sc + r * G + q * 8), scl + q * 8, 16);
+        tc_cp16(tc_smem(S.mn + r * G + q * 8), mnv + q * 8, 16);
       }
     } else {
-      for (int q = half; q < rb / 4; q += 2) {
-        tc_cp4(tc_smem(S.sc + row * G + q * 2), scl + q * 2);
-        tc_cp4(tc_smem(S.mn + row * G + q * 2), mnv + q * 2);
+      for (int q = 0; q < rb / 4; q++) {
+        tc_cp4(tc_smem(S.sc + r * G + q * 2), scl + q * 2);
+        tc_cp4(tc_smem(S.mn + r * G + q * 2), mnv + q * 2);
       }
-    }
-    const int cb = G * 4;                       // bytes of a column's group sums
-    const int csz = cb % 16 == 0 ? 16 : 4;
-    const int cpc = cb / csz;
-    float *stage = reinterpret_cast<float *>(S.a[0]);
-    for (int e = tid; e < kTcN * cpc; e += kTcThreads) {
-      const int c = e / cpc, q = e % cpc;
-      const int tok = S.tok[c];
-      if (tok < 0) continue;                    // never read: the MMA columns there are zero
-      const float *src = A.mode == 0 ? A.xsum + (size_t)tok * G
-                                     : A.asum + (size_t)(tok * (A.k + 1) + (shared ? A.k : S.dst[c] % A.k)) * G;
-      if (csz == 16) tc_cp16(tc_smem(stage + c * G + q * 4), src + q * 4, 16);
-      else tc_cp4(tc_smem(stage + c * G + q), src + q);
     }
     tc_cp_arrive(&S.pre);
-  }
-  for (int g = 0; g < kTcRawAhead && g < G; g++) load_raw(g);
-  for (int g = 0; g < kTcBAhead && g < G; g++) load_b(g);
-  bool ok = tc_wait_all(&S.pre, 0, budget, A.err);
-  ok = !__syncthreads_or(!ok);
-  {
-    const float *stage = reinterpret_cast<const float *>(S.a[0]);
-    for (int e = tid; e < kTcN * G; e += kTcThreads) {
-      const int g = e / kTcN, c = e % kTcN;
-      S.xs[g * kTcN + c] = stage[c * G + g];
-    }
-  }
-  __syncthreads();
-
-  // fold role: TMEM lane = tile row; warps 0-3 take columns 0..63, warps 4-7 64..127
-  const int erow = 32 * (warp & 3) + (tid & 31);
-  const int cbeg = (warp >> 2) * (kTcN / 2);
-  const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-  unsigned long long acc[kTcN / 4];          // 64 fp32 accumulators as packed pairs
-#pragma unroll
-  for (int i = 0; i < kTcN / 4; i++) acc[i] = 0ull;
-  auto fold = [&](int g) {
-    const float s = bf(S.sc[erow * G + g]), m = fmaf(-128.f, s, bf(S.mn[erow * G + g]));
-    const unsigned long long s2 = pk2(s, s), m2 = pk2(m, m);
-    const float *xg = S.xs + g * kTcN + cbeg;
-    const uint32_t taddr = lane_addr + (uint32_t)((g & 1) * kTcN + cbeg);
-#pragma unroll
-    for (int c0 = 0; c0 < kTcN / 2; c0 += 32) {
-      if (cbeg + c0 < N) {
-        float v[32];
-        tc_ld32(taddr + c0, v);
-#pragma unroll
-        for (int cc = 0; cc < 32; cc += 4) {
-          const float4 x4 = *reinterpret_cast<const float4 *>(xg + c0 + cc);
-          unsigned long long &a0 = acc[(c0 + cc) / 2], &a1 = acc[(c0 + cc) / 2 + 1];
-          a0 = f2fma(m2, pk2(x4.x, x4.y), f2fma(s2, pk2(v[cc], v[cc + 1]), a0));
-          a1 = f2fma(m2, pk2(x4.z, x4.w), f2fma(s2, pk2(v[cc + 2], v[cc + 3]), a1));
-        }
+    // the row's codes, kTwRawAhead groups in flight, one cp.async group per K group
+    const unsigned long long pol = tc_policy_first();
+    for (int g = 0; g < kTwRawAhead; g++) {
+      if (g < G) {
+        tc_cp16_hint(tc_smem(S.raw[g] + r * 32), codes + g * 32, 16, pol);
+        tc_cp16_hint(tc_smem(S.raw[g] + r * 32 + 16), codes + g * 32 + 16, 16, pol);
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
-  };
-
-  int issued = 0;   // groups whose MMAs were issued
-  // `ok` only turns false; the barrier of step (c) makes the exit uniform
-#pragma unroll 1
-  for (int g = 0; g < G; g++) {
-    // (a) this group's codes and activations have landed
-    if (ok) ok = tc_wait_all(&S.rfull[g % kTcRawStages], (uint32_t)((g / kTcRawStages) & 1), budget, A.err);
-    if (ok) ok = tc_wait_all(&S.bfull[g % kTcBStages], (uint32_t)((g / kTcBStages) & 1), budget, A.err);
-    // (b) codes -> A tile: word j of this thread's 16 bytes = K elements 8 (4 half + j) ..
-    // + 7 = chunk 4 half + j, unpacked in the permuted order (0,4,1,5,2,6,3,7)
-    if (ok) {
-      const uint4 w = *reinterpret_cast<const uint4 *>(S.raw[g % kTcRawStages] + row * 32 + half * 16);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-      uint8_t *dstA = S.a[g & 1];
+    #pragma unroll 1
+    for (int g = 0; g < G; g++) {
+      const int as = g % kTwAStages, rs = g % kTwRawAhead;
+      asm volatile("cp.async.wait_group %0;" ::"n"(kTwRawAhead - 1) : "memory");   // own codes of g
+      if (g >= kTwAStages &&
+          !tw_wait(&S.aempty[as], (uint32_t)(((g / kTwAStages) - 1) & 1), budget, A.err, &S.abort))
+        break;
+      // word j of the row's 32 code bytes = K elements 8 j .. 8 j + 7 = chunk j, unpacked in
+      // the permuted order (0,4,1,5,2,6,3,7) as bf16 128 + q
+      const uint4 w0 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32);
+      const uint4 w1 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32 + 16);
+      const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      uint8_t *dstA = S.a[as];
 #pragma unroll
-      for (int j = 0; j < 4; j++) {
+      for (int j = 0; j < 8; j++) {
         const uint32_t wd = ws[j];
         const uint32_t p0 = (wd & 0x000F000Fu) | 0x43004300u;
         const uint32_t p1 = ((wd >> 4) & 0x000F000Fu) | 0x43004300u;
         const uint32_t p2 = ((wd >> 8) & 0x000F000Fu) | 0x43004300u;
         const uint32_t p3 = ((wd >> 12) & 0x000F000Fu) | 0x43004300u;
-        *reinterpret_cast<uint4 *>(dstA + sw128(row, half * 4 + j)) = make_uint4(p0, p1, p2, p3);
+        *reinterpret_cast<uint4 *>(dstA + sw128(r, j)) = make_uint4(p0, p1, p2, p3);
       }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) tc_mbar_arrive(&S.afull[as]);
+      // refill this row's slot (its words are consumed above) with group g + kTwRawAhead
+      if (g + kTwRawAhead < G) {
+        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32), codes + (g + kTwRawAhead) * 32, 16, pol);
+        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32 + 16), codes + (g + kTwRawAhead) * 32 + 16, 16, pol);
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    // (c) generic-proxy shared writes (and the landed cp.async data) -> tensor core
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;
-    }
-    if (tid == 0) {
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sa = tc_smem(S.a[g & 1]), sb = tc_smem(S.b[g % kTcBStages]);
-      const uint32_t td = tmem + (uint32_t)((g & 1) * kTcN);
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++)   // K = 16 per instruction: 32 bytes along the swizzled row
-        tc_mma(td, tc_desc(sa + kk * 32), tc_desc(sb + kk * 32), idesc, kk ? 1u : 0u);
-      tc_commit(&S.mma[g & 1]);
-    }
-    issued = g + 1;
-    // (d) fold the previous group once its MMAs are done
-    if (g >= 1) {
-      ok = tc_wait_all(&S.mma[(g - 1) & 1], (uint32_t)(((g - 1) >> 1) & 1), budget, A.err);
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      if (ok) fold(g - 1);
-      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    }
-    // (e) refill: the code stage of group g + kTcRawAhead was last converted at g - 1;
-    // the activation stage of g + kTcBAhead was last read by MMA(g - 1), complete
-    if (ok) {
-      if (g + kTcRawAhead < G) load_raw(g + kTcRawAhead);
-      if (g + kTcBAhead < G) load_b(g + kTcBAhead);
-    }
-  }
-  if (ok) {
-    ok = tc_wait_all(&S.mma[(G - 1) & 1], (uint32_t)(((G - 1) >> 1) & 1), budget, A.err);
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (ok) fold(G - 1);
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  if (__syncthreads_or(!ok)) {
-    // drain MMAs still in flight and every outstanding copy before giving TMEM back
-    if (issued > 0) tc_wait_all(&S.mma[(issued - 1) & 1], (uint32_t)(((issued - 1) >> 1) & 1), budget, A.err);
     asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
-    if (warp == 0)
-      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kTcN) : "memory");
-    return;
-  }
-
-  // ------------------------------- epilogue ------------------------------------------
-  float *ex = reinterpret_cast<float *>(S.b[0]);   // 64 x kTcN floats: the up values (mode 0)
-  if (A.mode == 0) {
-    const int i = mt * 64 + (erow & 63);
-    const bool up = erow >= 64;
-    const bool lora = shared && A.Bg != nullptr;
-    float lb[kMaxR];
-    if (lora)
-      for (int q = 0; q < A.r; q++) lb[q] = bf((up ? A.Bu : A.Bg)[(size_t)i * A.r + q]);
+  } else {
+    // ---------------- folders: TMEM -> registers, acc += s P + (m - 128 s) X -------------
+    const int fw = warp - kTwFold0;                 // 0..7
+    const int erow = 32 * (warp & 3) + lane;        // tile row = TMEM lane
+    const int cbeg = (fw >> 2) * (kTcN / 2);        // this warp's half of the columns
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    unsigned long long acc[kTcN / 4];               // 64 fp32 accumulators as packed pairs
 #pragma unroll
-    for (int cp = 0; cp < kTcN / 4; cp++) {
-      float v0 = __uint_as_float((uint32_t)acc[cp]), v1 = __uint_as_float((uint32_t)(acc[cp] >> 32));
-      const int c = cbeg + 2 * cp;
-      if (lora && c < ncol) {
-        for (int h2 = 0; h2 < 2; h2++) {
-          const int tok = S.tok[c + h2];
-          if (tok < 0) continue;
-          const float *t = A.lt + (size_t)tok * 3 * A.r + (up ? A.r : 0);
-          float la = 0.f;
-          for (int q = 0; q < A.r; q++) la = fmaf(lb[q], t[q], la);
-          if (h2 == 0) v0 = fmaf(A.c, la, v0);
-          else v1 = fmaf(A.c, la, v1);
+    for (int i = 0; i < kTcN / 4; i++) acc[i] = 0ull;
+    bool ok = tw_wait(&S.pre, 0, budget, A.err, &S.abort);
+    #pragma unroll 1
+    for (int g = 0; g < G && ok; g++) {
+      const int tb = g & 1, bs = g % kTwBStages;
+      ok = tw_wait(&S.tfull[tb], (uint32_t)((g >> 1) & 1), budget, A.err, &S.abort) &&
+           tw_wait(&S.bfull[bs], (uint32_t)((g / kTwBStages) & 1), budget, A.err, &S.abort);
+      if (!ok) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const float s = bf(S.sc[erow * G + g]), m = fmaf(-128.f, s, bf(S.mn[erow * G + g]));
+      const unsigned long long s2 = pk2(s, s), m2 = pk2(m, m);
+      const float *xg = S.xs[bs] + cbeg;
+      const uint32_t taddr = lane_addr + (uint32_t)(tb * kTcN + cbeg);
+#pragma unroll
+      for (int c0 = 0; c0 < kTcN / 2; c0 += 32) {
+        if (cbeg + c0 < N) {
+          float v[32];
+          tc_ld32(taddr + c0, v);
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 4) {
+            const float4 x4 = *reinterpret_cast<const float4 *>(xg + c0 + cc);
+            unsigned long long &a0 = acc[(c0 + cc) / 2], &a1 = acc[(c0 + cc) / 2 + 1];
+            a0 = f2fma(m2, pk2(x4.x, x4.y), f2fma(s2, pk2(v[cc], v[cc + 1]), a0));
+            a1 = f2fma(m2, pk2(x4.z, x4.w), f2fma(s2, pk2(v[cc + 2], v[cc + 3]), a1));
+          }
         }
       }
-      if (up) {
-        ex[(erow - 64) * kTcN + c] = v0;
-        ex[(erow - 64) * kTcN + c + 1] = v1;
-      } else {
-        acc[cp] = pk2(v0, v1);
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        tc_mbar_arrive(&S.tempty[tb]);
+        tc_mbar_arrive(&S.bempty[bs]);
       }
     }
-    __syncthreads();
-    if (!up) {
-      const int ipos = kperm_pos(i);
+    // every folder agrees before the epilogue (named barrier 1: the 8 folder warps)
+    {
+      uint32_t bad;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbarrier.red.or.pred q, 1, %2, p;\n\t"
+          "selp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(bad)
+          : "r"((uint32_t)!ok), "r"(256)
+          : "memory");
+      ok = bad == 0;
+    }
+    if (ok) {
+      if (A.mode == 0) {
+        // gate rows 0..63 and up rows 64..127 (with the shared expert's LoRA up branch)
+        // go to shared memory as ex[row][column]; then all 256 folder threads form
+        // a = bf16(silu(g) u), thread t taking unit t % 64 of four columns per pass
+        float *ex = reinterpret_cast<float *>(S.b[0]);   // 128 x kTcN floats (64 KB)
+        const int i = mt * 64 + (erow & 63);
+        const bool up = erow >= 64;
+        const bool lora = shared && A.Bg != nullptr;
+        float lb[kMaxR];
+        if (lora)
+          for (int q = 0; q < A.r; q++) lb[q] = bf((up ? A.Bu : A.Bg)[(size_t)i * A.r + q]);
 #pragma unroll
-      for (int cp = 0; cp < kTcN / 4; cp++) {
-#pragma unroll
-        for (int h2 = 0; h2 < 2; h2++) {
-          const int c = cbeg + 2 * cp + h2;
-          const int dst = c < ncol ? S.dst[c] : -1;
+        for (int cp = 0; cp < kTcN / 4; cp++) {
+          float v0 = __uint_as_float((uint32_t)acc[cp]), v1 = __uint_as_float((uint32_t)(acc[cp] >> 32));
+          const int c = cbeg + 2 * cp;
+          if (lora && c < ncol) {
+            for (int h2 = 0; h2 < 2; h2++) {
+              const int tok = S.tok[c + h2];
+              if (tok < 0) continue;
+              const float *t = A.lt + (size_t)tok * 3 * A.r + (up ? A.r : 0);
+              float la = 0.f;
+              for (int q = 0; q < A.r; q++) la = fmaf(lb[q], t[q], la);
+              if (h2 == 0) v0 = fmaf(A.c, la, v0);
+              else v1 = fmaf(A.c, la, v1);
+            }
+          }
+          *reinterpret_cast<float2 *>(ex + erow * kTcN + c) = make_float2(v0, v1);
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        const int ft = tid - kTwFold0 * 32, iu = ft & 63;
+        const int ipos = kperm_pos(mt * 64 + iu);
+        #pragma unroll 4
+        for (int c = ft >> 6; c < ncol; c += 4) {
+          const int dst = S.dst[c];
           if (dst < 0) continue;
-          const float g = __uint_as_float(h2 ? (uint32_t)(acc[cp] >> 32) : (uint32_t)acc[cp]);
-          const float u = ex[erow * kTcN + c];
+          const float g = ex[iu * kTcN + c], u = ex[(64 + iu) * kTcN + c];
           A.ap_out[(size_t)dst * A.I + ipos] = f2bf(g / (1.0f + expf(-g)) * u);   // bf16 rounding point of a
         }
-      }
-    }
-  } else {
-    const int n = mt * 128 + erow;
+      } else {
+        const int n = mt * 128 + erow;
 #pragma unroll
-    for (int cp = 0; cp < kTcN / 4; cp++) {
+        for (int cp = 0; cp < kTcN / 4; cp++) {
 #pragma unroll
-      for (int h2 = 0; h2 < 2; h2++) {
-        const int c = cbeg + 2 * cp + h2;
-        const int tok = c < ncol ? S.tok[c] : -1;
-        if (tok < 0) continue;
-        const float v = __uint_as_float(h2 ? (uint32_t)(acc[cp] >> 32) : (uint32_t)acc[cp]);
-        const float w = shared ? 1.0f : A.gates[S.dst[c]];
-        atomicAdd(A.yacc + (size_t)tok * A.d + n, w * v);
+          for (int h2 = 0; h2 < 2; h2++) {
+            const int c = cbeg + 2 * cp + h2;
+            const int tok = c < ncol ? S.tok[c] : -1;
+            if (tok < 0) continue;
+            const float v = __uint_as_float(h2 ? (uint32_t)(acc[cp] >> 32) : (uint32_t)acc[cp]);
+            atomicAdd(A.yacc + (size_t)tok * A.d + n, S.gw[c] * v);
+          }
+        }
       }
     }
   }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0)
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (warp == kTwMmaWarp)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kTcN) : "memory");
 }
 
@@ -731,14 +795,25 @@ __global__ void k_perm_sums(const uint16_t *__restrict__ x, long long rows, int 
   sums[i] = s;
 }
 
-// t_d = Ad a_s from the K-permuted bf16 activations (one warp per token and rank row)
+// x rows in expert-grouped order: row p of xg = the permuted x row of the token of
+// assignment assign[p] (t * k + slot).  One block per row, one 16-byte chunk per thread.
+__global__ void k_group_rows(const uint16_t *__restrict__ xp, const int32_t *__restrict__ assign, int k, int d,
+                             uint16_t *__restrict__ xg) {
+  const int p = blockIdx.x, t = assign[p] / k;
+  const uint4 *src = reinterpret_cast<const uint4 *>(xp + (size_t)t * d);
+  uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)p * d);
+  for (int i = threadIdx.x; i < d / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+// t_d = Ad a_s from the K-permuted bf16 activations (one warp per token and rank row); the
+// shared expert's a rows are rows T k .. T k + T - 1 of the grouped a
 __global__ void k_lora_td(const uint16_t *__restrict__ Ad, const uint16_t *__restrict__ ap, int T, int I, int k,
                           int r, float *__restrict__ lt) {
   const int lane = threadIdx.x & 31;
   const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (w >= T * r) return;
   const int t = w / r, j = w % r;
-  const uint16_t *as = ap + ((size_t)t * (k + 1) + k) * I;
+  const uint16_t *as = ap + ((size_t)T * k + t) * I;
   float acc = 0.f;
   for (int i = lane; i < I; i += 32) acc = fmaf(bf(Ad[(size_t)j * I + i]), bf(as[kperm_pos(i)]), acc);
   acc = warp_sum(acc);
