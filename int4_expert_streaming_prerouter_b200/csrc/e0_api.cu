@@ -435,7 +435,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   A.tmB[1] = A.tmB[0];
   k_moe_gemm_tc<<<tmax * (D.d_model / 128), kTwThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(down)");
-  k_tc_finish<<<(unsigned)((nx + 255) / 256), 256, 0, s>>>(C->yacc, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
+  k_tc_finish<<<K.T, 256, 0, s>>>(C->yacc, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
                                                            D.d_model, D.lora_rank, D.lora_scale, K.y, K.yf);
   CKL("k_tc_finish");
   return E0_OK;

@@ -186,6 +186,18 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 
+// 64 TMEM columns of this warp's 32 lanes into registers (one load, one wait)
+__device__ __forceinline__ void tc_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; i++) v[i] = __uint_as_float(r[i]);
+}
+
 // byte offset of 16-byte chunk `ch` (0..7) of row `row` in a 128-byte-swizzled K-major tile
 __device__ __forceinline__ uint32_t sw128(int row, int ch) {
   return (uint32_t)(row * 128 + ((ch ^ (row & 7)) << 4));
@@ -212,14 +224,28 @@ __device__ __forceinline__ bool tc_wait_all(uint64_t *b, uint32_t parity, unsign
 // tokens) cut into tiles of up to kTcN tokens.  One block.
 // ---------------------------------------------------------------------------------------
 __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
-  if (threadIdx.x != 0) return;
+  // one warp: tiles per unit, an exclusive scan over the units in order, then every lane
+  // writes its units' tiles
+  const int lane = threadIdx.x;
+  if (lane >= 32) return;
   const int U = P.U[0];
-  int n = 0;
-  for (int u = 0; u <= U && n < cap; u++) {
-    const int cnt = u < U ? P.ustart[u + 1] - P.ustart[u] : T;
-    for (int n0 = 0; n0 < cnt && n < cap; n0 += kTcN) tiles[n++] = TcTile{u, n0};
+  int base = 0;
+  for (int u0 = 0; u0 <= U; u0 += 32) {
+    const int u = u0 + lane;
+    const int cnt = u < U ? P.ustart[u + 1] - P.ustart[u] : (u == U ? T : 0);
+    const int nt = (cnt + kTcN - 1) / kTcN;
+    int incl = nt;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    for (int q = 0; q < nt; q++) {
+      const int idx = base + incl - nt + q;
+      if (idx < cap) tiles[idx] = TcTile{u, q * kTcN};
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
   }
-  *ntiles = n;
+  if (lane == 0) *ntiles = min(base, cap);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -239,18 +265,19 @@ __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
 //              (stored in expert-grouped order, so a tile's tokens are consecutive rows)
 //              as the 128-byte swizzled B tile; the lanes copy the columns' group sums
 //   warp  1    TMEM owner; one thread issues the four MMAs of each group
-//   warps 2-5  converters: thread t owns weight row t; it streams its own row's codes
-//              kTwRawAhead groups ahead with cp.async (no hand-off needed) and writes
-//              128 + q as bf16 into the A tile ring (kTwAStages stages)
-//   warps 6-13 folders: TMEM lane quadrant warp % 4, half of the columns each; they fold
+//   warps 2-3  converters: thread t owns weight rows t and t + 64; it streams its own rows'
+//              codes kTwRawAhead groups ahead with cp.async (no hand-off needed) and
+//              writes 128 + q as bf16 into the A tile ring (kTwAStages stages)
+//   warps 4-11 folders: TMEM lane quadrant warp % 4, half of the columns each; they fold
 //              every group into registers and run the epilogue (SwiGLU, or the weighted
 //              combine into y)
 // ---------------------------------------------------------------------------------------
-constexpr int kTwThreads = 448;
-constexpr int kTwLoadWarps = 1, kTwMmaWarp = 1, kTwConv0 = 2, kTwFold0 = 6;
+constexpr int kTwThreads = 384;
+constexpr int kTwLoadWarps = 1, kTwMmaWarp = 1, kTwConv0 = 2, kTwFold0 = 4;
 constexpr int kTwAStages = 3;
 constexpr int kTwBStages = 6;
 constexpr int kTwRawAhead = 3;      // groups of codes in flight per converter thread
+constexpr int kTwTBufs = 4;         // TMEM accumulators (kTcN columns each): MMAs run up to 4 groups ahead of the folds
 
 struct TwSmem {
   uint8_t a[kTwAStages][128 * 128];        // A tiles (bf16, 128-byte swizzled K-major)
@@ -260,7 +287,7 @@ struct TwSmem {
   uint16_t sc[128 * kTcMaxGroups];         // scale of every row and group [row][g]
   uint16_t mn[128 * kTcMaxGroups];         // min
   uint64_t bfull[kTwBStages], bempty[kTwBStages], afull[kTwAStages], aempty[kTwAStages];
-  uint64_t tfull[2], tempty[2], pre;
+  uint64_t tfull[kTwTBufs], tempty[kTwTBufs], pre;
   uint32_t tmem;
   volatile int abort;
   int tok[kTcN];       // token of each column
@@ -334,20 +361,20 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
       tc_mbar_init(&S.bempty[s], 8);
     }
     for (int s = 0; s < kTwAStages; s++) {
-      tc_mbar_init(&S.afull[s], 4);
+      tc_mbar_init(&S.afull[s], 2);
       tc_mbar_init(&S.aempty[s], 1);
     }
-    for (int s = 0; s < 2; s++) {
+    for (int s = 0; s < kTwTBufs; s++) {
       tc_mbar_init(&S.tfull[s], 1);
       tc_mbar_init(&S.tempty[s], 8);
     }
-    tc_mbar_init(&S.pre, 128);
+    tc_mbar_init(&S.pre, 64);
     S.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kTwMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_smem(&S.tmem)),
-                 "r"(2 * kTcN)
+                 "r"(kTwTBufs * kTcN)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -394,10 +421,11 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
       int issued = 0;
       #pragma unroll 1
       for (int g = 0; g < G; g++) {
-        const int as = g % kTwAStages, bs = g % kTwBStages, tb = g & 1;
+        const int as = g % kTwAStages, bs = g % kTwBStages, tb = g % kTwTBufs;
         if (!tw_wait(&S.afull[as], (uint32_t)((g / kTwAStages) & 1), budget, A.err, &S.abort)) break;
         if (!tw_wait(&S.bfull[bs], (uint32_t)((g / kTwBStages) & 1), budget, A.err, &S.abort)) break;
-        if (g >= 2 && !tw_wait(&S.tempty[tb], (uint32_t)(((g >> 1) - 1) & 1), budget, A.err, &S.abort)) break;
+        if (g >= kTwTBufs && !tw_wait(&S.tempty[tb], (uint32_t)(((g / kTwTBufs) - 1) & 1), budget, A.err, &S.abort))
+          break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t sa = tc_smem(S.a[as]), sb = tc_smem(S.b[bs]);
         const uint32_t td = tmem + (uint32_t)(tb * kTcN);
@@ -410,49 +438,58 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
       }
       // after an abort, the MMAs in flight finish before TMEM is given back
       if (issued > 0 && issued < G)
-        tc_wait_all(&S.tfull[(issued - 1) & 1], (uint32_t)(((issued - 1) >> 1) & 1), budget, A.err);
+        tc_wait_all(&S.tfull[(issued - 1) % kTwTBufs], (uint32_t)(((issued - 1) / kTwTBufs) & 1), budget, A.err);
     }
     __syncwarp();
   } else if (warp < kTwFold0) {
-    // ---------------- converters: thread r owns weight row r ------------------------------
+    // ---------------- converters: thread t owns weight rows t and t + 64 ------------------
     // mode 0 -> gate rows i0..i0+63 then up rows i0..i0+63 (i0 = 64 mt); mode 1 -> down
     // rows 128 mt .. 128 mt + 127
-    const int r = tid - kTwConv0 * 32;
-    const uint8_t *codes;
-    const uint16_t *scl, *mnv;
-    if (A.mode == 0) {
-      const int i = mt * 64 + (r & 63);
-      const bool up = r >= 64;
-      codes = base + (up ? A.bl.uc : A.bl.gc) + (size_t)i * (A.d / 2);
-      scl = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.us : A.bl.gs)) + (size_t)i * G;
-      mnv = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.um : A.bl.gm)) + (size_t)i * G;
-    } else {
-      const int n = mt * 128 + r;
-      codes = base + A.bl.dc + (size_t)n * (A.I / 2);
-      scl = reinterpret_cast<const uint16_t *>(base + A.bl.ds) + (size_t)n * G;
-      mnv = reinterpret_cast<const uint16_t *>(base + A.bl.dm) + (size_t)n * G;
-    }
-    // the row's scales and mins for the folders (rows of fewer than 16 bytes in 4-byte copies)
-    const int rb = G * 2;
-    if (rb % 16 == 0) {
-      for (int q = 0; q < rb / 16; q++) {
-        tc_cp16(tc_smem(S.sc + r * G + q * 8), scl + q * 8, 16);
-        tc_cp16(tc_smem(S.mn + r * G + q * 8), mnv + q * 8, 16);
+    const int t = tid - kTwConv0 * 32;     // 0..63
+    const uint8_t *codes[2];
+    const uint16_t *scl[2], *mnv[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      const int r = t + 64 * h;
+      if (A.mode == 0) {
+        const int i = mt * 64 + (r & 63);
+        const bool up = r >= 64;
+        codes[h] = base + (up ? A.bl.uc : A.bl.gc) + (size_t)i * (A.d / 2);
+        scl[h] = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.us : A.bl.gs)) + (size_t)i * G;
+        mnv[h] = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.um : A.bl.gm)) + (size_t)i * G;
+      } else {
+        const int n = mt * 128 + r;
+        codes[h] = base + A.bl.dc + (size_t)n * (A.I / 2);
+        scl[h] = reinterpret_cast<const uint16_t *>(base + A.bl.ds) + (size_t)n * G;
+        mnv[h] = reinterpret_cast<const uint16_t *>(base + A.bl.dm) + (size_t)n * G;
       }
-    } else {
-      for (int q = 0; q < rb / 4; q++) {
-        tc_cp4(tc_smem(S.sc + r * G + q * 2), scl + q * 2);
-        tc_cp4(tc_smem(S.mn + r * G + q * 2), mnv + q * 2);
+      // the row's scales and mins for the folders (rows of fewer than 16 bytes in 4-byte copies)
+      const int rb = G * 2;
+      if (rb % 16 == 0) {
+        for (int q = 0; q < rb / 16; q++) {
+          tc_cp16(tc_smem(S.sc + r * G + q * 8), scl[h] + q * 8, 16);
+          tc_cp16(tc_smem(S.mn + r * G + q * 8), mnv[h] + q * 8, 16);
+        }
+      } else {
+        for (int q = 0; q < rb / 4; q++) {
+          tc_cp4(tc_smem(S.sc + r * G + q * 2), scl[h] + q * 2);
+          tc_cp4(tc_smem(S.mn + r * G + q * 2), mnv[h] + q * 2);
+        }
       }
     }
     tc_cp_arrive(&S.pre);
-    // the row's codes, kTwRawAhead groups in flight, one cp.async group per K group
+    // the rows' codes, kTwRawAhead groups in flight, one cp.async group per K group
     const unsigned long long pol = tc_policy_first();
-    for (int g = 0; g < kTwRawAhead; g++) {
-      if (g < G) {
-        tc_cp16_hint(tc_smem(S.raw[g] + r * 32), codes + g * 32, 16, pol);
-        tc_cp16_hint(tc_smem(S.raw[g] + r * 32 + 16), codes + g * 32 + 16, 16, pol);
+    auto load_codes = [&](int g, int rs) {
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int r = t + 64 * h;
+        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32), codes[h] + g * 32, 16, pol);
+        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32 + 16), codes[h] + g * 32 + 16, 16, pol);
       }
+    };
+    for (int g = 0; g < kTwRawAhead; g++) {
+      if (g < G) load_codes(g, g);
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
     #pragma unroll 1
@@ -462,29 +499,30 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
       if (g >= kTwAStages &&
           !tw_wait(&S.aempty[as], (uint32_t)(((g / kTwAStages) - 1) & 1), budget, A.err, &S.abort))
         break;
-      // word j of the row's 32 code bytes = K elements 8 j .. 8 j + 7 = chunk j, unpacked in
+      // word j of a row's 32 code bytes = K elements 8 j .. 8 j + 7 = chunk j, unpacked in
       // the permuted order (0,4,1,5,2,6,3,7) as bf16 128 + q
-      const uint4 w0 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32);
-      const uint4 w1 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32 + 16);
-      const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
       uint8_t *dstA = S.a[as];
 #pragma unroll
-      for (int j = 0; j < 8; j++) {
-        const uint32_t wd = ws[j];
-        const uint32_t p0 = (wd & 0x000F000Fu) | 0x43004300u;
-        const uint32_t p1 = ((wd >> 4) & 0x000F000Fu) | 0x43004300u;
-        const uint32_t p2 = ((wd >> 8) & 0x000F000Fu) | 0x43004300u;
-        const uint32_t p3 = ((wd >> 12) & 0x000F000Fu) | 0x43004300u;
-        *reinterpret_cast<uint4 *>(dstA + sw128(r, j)) = make_uint4(p0, p1, p2, p3);
+      for (int h = 0; h < 2; h++) {
+        const int r = t + 64 * h;
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32);
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32 + 16);
+        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          const uint32_t wd = ws[j];
+          const uint32_t p0 = (wd & 0x000F000Fu) | 0x43004300u;
+          const uint32_t p1 = ((wd >> 4) & 0x000F000Fu) | 0x43004300u;
+          const uint32_t p2 = ((wd >> 8) & 0x000F000Fu) | 0x43004300u;
+          const uint32_t p3 = ((wd >> 12) & 0x000F000Fu) | 0x43004300u;
+          *reinterpret_cast<uint4 *>(dstA + sw128(r, j)) = make_uint4(p0, p1, p2, p3);
+        }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) tc_mbar_arrive(&S.afull[as]);
-      // refill this row's slot (its words are consumed above) with group g + kTwRawAhead
-      if (g + kTwRawAhead < G) {
-        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32), codes + (g + kTwRawAhead) * 32, 16, pol);
-        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32 + 16), codes + (g + kTwRawAhead) * 32 + 16, 16, pol);
-      }
+      // refill these rows' slots (their words are consumed above) with group g + kTwRawAhead
+      if (g + kTwRawAhead < G) load_codes(g + kTwRawAhead, rs);
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -500,8 +538,8 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
     bool ok = tw_wait(&S.pre, 0, budget, A.err, &S.abort);
     #pragma unroll 1
     for (int g = 0; g < G && ok; g++) {
-      const int tb = g & 1, bs = g % kTwBStages;
-      ok = tw_wait(&S.tfull[tb], (uint32_t)((g >> 1) & 1), budget, A.err, &S.abort) &&
+      const int tb = g % kTwTBufs, bs = g % kTwBStages;
+      ok = tw_wait(&S.tfull[tb], (uint32_t)((g / kTwTBufs) & 1), budget, A.err, &S.abort) &&
            tw_wait(&S.bfull[bs], (uint32_t)((g / kTwBStages) & 1), budget, A.err, &S.abort);
       if (!ok) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -509,18 +547,17 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
       const unsigned long long s2 = pk2(s, s), m2 = pk2(m, m);
       const float *xg = S.xs[bs] + cbeg;
       const uint32_t taddr = lane_addr + (uint32_t)(tb * kTcN + cbeg);
+      if (cbeg < N) {
+        // this warp's 64 columns in one TMEM load (columns past N hold stale values that
+        // only reach accumulators of unused columns)
+        float v[64];
+        tc_ld64(taddr, v);
 #pragma unroll
-      for (int c0 = 0; c0 < kTcN / 2; c0 += 32) {
-        if (cbeg + c0 < N) {
-          float v[32];
-          tc_ld32(taddr + c0, v);
-#pragma unroll
-          for (int cc = 0; cc < 32; cc += 4) {
-            const float4 x4 = *reinterpret_cast<const float4 *>(xg + c0 + cc);
-            unsigned long long &a0 = acc[(c0 + cc) / 2], &a1 = acc[(c0 + cc) / 2 + 1];
-            a0 = f2fma(m2, pk2(x4.x, x4.y), f2fma(s2, pk2(v[cc], v[cc + 1]), a0));
-            a1 = f2fma(m2, pk2(x4.z, x4.w), f2fma(s2, pk2(v[cc + 2], v[cc + 3]), a1));
-          }
+        for (int cc = 0; cc < 64; cc += 4) {
+          const float4 x4 = *reinterpret_cast<const float4 *>(xg + cc);
+          unsigned long long &a0 = acc[cc / 2], &a1 = acc[cc / 2 + 1];
+          a0 = f2fma(m2, pk2(x4.x, x4.y), f2fma(s2, pk2(v[cc], v[cc + 1]), a0));
+          a1 = f2fma(m2, pk2(x4.z, x4.w), f2fma(s2, pk2(v[cc + 2], v[cc + 3]), a1));
         }
       }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -542,11 +579,15 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
       ok = bad == 0;
     }
     if (ok) {
+      // the tile's results go through shared memory as ex[row][column] with a row stride of
+      // kTcN + 1 floats, so that lanes on consecutive rows hit different banks both when
+      // writing (lane = row) and when reading (lane = row again, or four rows per lane)
+      constexpr int XS = kTcN + 1;
+      float *ex = reinterpret_cast<float *>(S.b[0]);   // 128 x XS floats (66 KB of the B ring)
       if (A.mode == 0) {
-        // gate rows 0..63 and up rows 64..127 (with the shared expert's LoRA up branch)
-        // go to shared memory as ex[row][column]; then all 256 folder threads form
-        // a = bf16(silu(g) u), thread t taking unit t % 64 of four columns per pass
-        float *ex = reinterpret_cast<float *>(S.b[0]);   // 128 x kTcN floats (64 KB)
+        // gate rows 0..63 and up rows 64..127 (with the shared expert's LoRA up branch);
+        // then all 256 folder threads form a = bf16(silu(g) u), thread t taking unit t % 64
+        // of four columns per pass
         const int i = mt * 64 + (erow & 63);
         const bool up = erow >= 64;
         const bool lora = shared && A.Bg != nullptr;
@@ -568,7 +609,8 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
               else v1 = fmaf(A.c, la, v1);
             }
           }
-          *reinterpret_cast<float2 *>(ex + erow * kTcN + c) = make_float2(v0, v1);
+          ex[erow * XS + c] = v0;
+          ex[erow * XS + c + 1] = v1;
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");
         const int ft = tid - kTwFold0 * 32, iu = ft & 63;
@@ -577,21 +619,29 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
         for (int c = ft >> 6; c < ncol; c += 4) {
           const int dst = S.dst[c];
           if (dst < 0) continue;
-          const float g = ex[iu * kTcN + c], u = ex[(64 + iu) * kTcN + c];
+          const float g = ex[iu * XS + c], u = ex[(64 + iu) * XS + c];
           A.ap_out[(size_t)dst * A.I + ipos] = f2bf(g / (1.0f + expf(-g)) * u);   // bf16 rounding point of a
         }
       } else {
-        const int n = mt * 128 + erow;
+        // gate-weighted values to shared memory, then four consecutive output rows of one
+        // column per thread, added into y with one vector reduction
 #pragma unroll
         for (int cp = 0; cp < kTcN / 4; cp++) {
-#pragma unroll
-          for (int h2 = 0; h2 < 2; h2++) {
-            const int c = cbeg + 2 * cp + h2;
-            const int tok = c < ncol ? S.tok[c] : -1;
-            if (tok < 0) continue;
-            const float v = __uint_as_float(h2 ? (uint32_t)(acc[cp] >> 32) : (uint32_t)acc[cp]);
-            atomicAdd(A.yacc + (size_t)tok * A.d + n, S.gw[c] * v);
-          }
+          const int c = cbeg + 2 * cp;
+          ex[erow * XS + c] = S.gw[c] * __uint_as_float((uint32_t)acc[cp]);
+          ex[erow * XS + c + 1] = S.gw[c + 1] * __uint_as_float((uint32_t)(acc[cp] >> 32));
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        const int ft = tid - kTwFold0 * 32;
+        for (int it = ft; it < ncol * 32; it += 256) {
+          const int c = it >> 5, n4 = it & 31;
+          const int tok = S.tok[c];
+          if (tok < 0) continue;
+          const float y0 = ex[(4 * n4) * XS + c], y1 = ex[(4 * n4 + 1) * XS + c];
+          const float y2 = ex[(4 * n4 + 2) * XS + c], y3 = ex[(4 * n4 + 3) * XS + c];
+          float *dstp = A.yacc + (size_t)tok * A.d + mt * 128 + 4 * n4;
+          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dstp), "f"(y0), "f"(y1), "f"(y2), "f"(y3)
+                       : "memory");
         }
       }
     }
@@ -600,7 +650,7 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (warp == kTwMmaWarp)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kTcN) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTwTBufs * kTcN) : "memory");
 }
 
 // ---------------------------------------------------------------------------------------
@@ -820,21 +870,38 @@ __global__ void k_lora_td(const uint16_t *__restrict__ Ad, const uint16_t *__res
   if (lane == 0) lt[((size_t)t * 3 + 2) * r + j] = acc;
 }
 
-// y = yacc + c Bd t_d  -> fp32 and bf16 outputs
+// y = yacc + c Bd t_d  -> fp32 and bf16 outputs.  One block per token: t_d in shared
+// memory, each thread a strided set of output rows n with its B_d row in 16-byte loads.
 __global__ void k_tc_finish(const float *__restrict__ yacc, const uint16_t *__restrict__ Bd,
                             const float *__restrict__ lt, int T, int d, int r, float c, uint16_t *__restrict__ y,
                             float *__restrict__ yf) {
-  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (size_t)T * d) return;
-  const int t = (int)(i / d), n = (int)(i % d);
-  float v = yacc[i];
-  if (Bd) {
-    float lo = 0.f;
-    for (int q = 0; q < r; q++) lo = fmaf(bf(Bd[(size_t)n * r + q]), lt[((size_t)t * 3 + 2) * r + q], lo);
-    v = fmaf(c, lo, v);
+  const int t = blockIdx.x;
+  __shared__ float td[kMaxR];
+  if (Bd && threadIdx.x < r) td[threadIdx.x] = lt[((size_t)t * 3 + 2) * r + threadIdx.x];
+  __syncthreads();
+  for (int n = threadIdx.x; n < d; n += blockDim.x) {
+    const size_t i = (size_t)t * d + n;
+    float v = yacc[i];
+    if (Bd) {
+      float lo = 0.f;
+      if (r % 8 == 0 && ((uintptr_t)Bd & 15) == 0) {
+        for (int q0 = 0; q0 < r; q0 += 8) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(Bd + (size_t)n * r + q0);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+            lo = fmaf(bf(ws[j] & 0xFFFFu), td[q0 + 2 * j], lo);
+            lo = fmaf(bf(ws[j] >> 16), td[q0 + 2 * j + 1], lo);
+          }
+        }
+      } else {
+        for (int q = 0; q < r; q++) lo = fmaf(bf(Bd[(size_t)n * r + q]), td[q], lo);
+      }
+      v = fmaf(c, lo, v);
+    }
+    y[i] = f2bf(v);
+    if (yf) yf[i] = v;
   }
-  y[i] = f2bf(v);
-  if (yf) yf[i] = v;
 }
 
 }  // namespace e0
