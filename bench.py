@@ -40,8 +40,12 @@ METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, valid only
 # while the kernel source is the one captured (sha256 prefix of the file); see profiles/.
 KERNEL_TRAFFIC = {
-    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "7e50bdc194a50ca3", 427.0e6,
-                      "4-layer capture (42.64 MB for 40.6 MB algorithmic) scaled by algorithmic bytes"),
+    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "616f850e44047cee", 421.9e6,
+                      "4-layer capture (42.19 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
+                      "bytes to the 40-layer launch"),
+    "prefill_t4096_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh", "12341c74281dd957", 343.6e6,
+                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 465.8 MB, "
+                          "down 221.4 MB, mean of the two"),
 }
 
 
@@ -379,7 +383,8 @@ def run_prefill(args, dims, seed, ws, rank, local):
     for _ in range(args.warmup):
         ctx.prefill_stack(h, y_out=y)
     ctx.sync_status()
-    l0 = ctx.stats()["kernel_launches"]
+    st0 = ctx.stats()
+    ctx.debug_time_gemm(True)   # event pairs around every expert-GEMM launch, on its stream
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(ws)
     torch.cuda.synchronize()
@@ -391,13 +396,21 @@ def run_prefill(args, dims, seed, ws, rank, local):
         torch.cuda.synchronize()
     barrier(ws)
     ctx.sync_status()
+    ctx.debug_time_gemm(False)
     ms = max_over_ranks(ev0.elapsed_time(ev1), ws)
-    launches = ctx.stats()["kernel_launches"] - l0
+    st1 = ctx.stats()
+    launches = st1["kernel_launches"] - st0["kernel_launches"]
+    gemm_n = st1["gemm_timed"] - st0["gemm_timed"]
+    gemm_ms = max_over_ranks(st1["gemm_ms"] - st0["gemm_ms"], ws)
     tokens = sum_over_ranks(T * args.steps, ws)
+    # algorithmic expert FLOPs: every token through k routed + the shared expert, gate and
+    # up (2 d I each) and down (2 I d), per layer
     flops = dims.L * T * (dims.k + 1) * (2 * dims.d * 2 * dims.I + 2 * dims.I * dims.d)
     pk = peaks()
     step_s = ms / args.steps / 1e3
-    achieved = flops / step_s / 1e12
+    # the dominant kernel: the expert GEMMs' FLOPs over their own measured launch time
+    achieved = flops * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else flops / step_s / 1e12
+    traffic, traffic_how = kernel_traffic(args.workload)
     # end to end: the chunk's inputs from pinned host memory, its outputs back
     h_host = h.cpu().pin_memory()
     y_host = torch.empty_like(h_host).pin_memory()
@@ -414,7 +427,8 @@ def run_prefill(args, dims, seed, ws, rank, local):
         "metric": "MoE-stack prefill tokens/s on 1 B200 (4096-token chunk, 40 layers)", "value": tokens / (ms / 1e3),
         "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 weights, fp16 tensor-core operands, fp32 accumulate", "data": "synthetic (seeded)",
+        "dtype": "int4 weights as exact bf16 tensor-core operands (128+q), bf16 activations, fp32 accumulate",
+        "data": "synthetic (seeded)",
         "config": {"workload": args.workload, "layers": dims.L, "tokens": T, "d": dims.d, "experts": dims.E,
                    "d_ff": dims.I, "top_k": dims.k, "parallelism": f"replicas x{ws}",
                    "l2": "inputs larger than L2 (18.1 GB of expert weights)"},
@@ -422,9 +436,11 @@ def run_prefill(args, dims, seed, ws, rank, local):
                 "d2h_bytes_per_step": int(y.numel() * 2)},
         "gpu_launches": int(launches),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_tflops"], "traffic": None,
-                     "kernel": "whole prefill chunk (expert FLOPs only; fp16 = bf16 dense rate)",
-                     "peak_source": pk["source"]},
+                     "frac": achieved / pk["bf16_tflops"], "traffic": traffic,
+                     "kernel": f"k_moe_gemm_tc ({gemm_n} launches timed, {gemm_ms / max(gemm_n, 1):.3f} ms mean; "
+                               f"expert FLOPs of the chunk / their summed time; "
+                               f"{100 * gemm_ms / max(ms, 1e-9):.0f}% of the step)",
+                     "traffic_note": traffic_how, "peak_source": pk["source"]},
         "clocks": clk.summary(), "setup_s": setup_s,
     }
     return out, ctx

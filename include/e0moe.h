@@ -101,6 +101,8 @@ typedef struct {
   double   stage_ms;           /* sum of copy durations (side-stream event pairs) */
   double   exposed_wait_ms;    /* compute-stream time spent waiting on staging */
   uint64_t kernel_launches;    /* kernels this context has launched */
+  uint64_t gemm_timed;         /* expert-GEMM launches timed (see e0_debug_time_gemm) */
+  double   gemm_ms;            /* their summed durations (event pairs on the launch stream) */
 } e0_stats;
 
 /* Create a context on the current CUDA device.  n_layers >= 1; max_tokens bounds T of
@@ -253,6 +255,11 @@ int e0_debug_force_general(e0_ctx *ctx, int on);
  * each layer.  Chained steps always run in order.  Results are bit-identical under both.
  * E0_ERR_INVALID_ARG unless 0 or 1. */
 int e0_debug_decode_flat(e0_ctx *ctx, int on);
+/* Profiling: on = 1 brackets every tensor-core expert-GEMM launch (prefill) with a CUDA
+ * event pair on its stream; e0_get_stats then reports their count and summed duration
+ * (gemm_timed, gemm_ms; it synchronises on the events).  on = 0 stops it.  The pages
+ * have no counterpart; for the benchmark's per-kernel roofline. */
+int e0_debug_time_gemm(e0_ctx *ctx, int on);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *e0_last_error(void);

@@ -51,7 +51,8 @@ class Stats(ctypes.Structure):
                 ("staged_bytes", ctypes.c_uint64), ("prefetched_experts", ctypes.c_uint64),
                 ("ondemand_experts", ctypes.c_uint64), ("dropped", ctypes.c_uint64),
                 ("stage_ms", ctypes.c_double), ("exposed_wait_ms", ctypes.c_double),
-                ("kernel_launches", ctypes.c_uint64)]
+                ("kernel_launches", ctypes.c_uint64), ("gemm_timed", ctypes.c_uint64),
+                ("gemm_ms", ctypes.c_double)]
 
 
 _lib = None
@@ -83,6 +84,7 @@ _SIGS = {
     "e0_debug_prefill_path": (_I, [_P, _I]),
     "e0_debug_decode_mode": (_I, [_P, _I]),
     "e0_debug_decode_flat": (_I, [_P, _I]),
+    "e0_debug_time_gemm": (_I, [_P, _I]),
 }
 
 
@@ -272,6 +274,9 @@ class Context:
 
     def debug_decode_mode(self, mode: int):
         _check(lib().e0_debug_decode_mode(self._h, mode))
+
+    def debug_time_gemm(self, on: bool):
+        _check(lib().e0_debug_time_gemm(self._h, int(on)))
 
     def debug_decode_flat(self, on: bool):
         _check(lib().e0_debug_decode_flat(self._h, int(on)))

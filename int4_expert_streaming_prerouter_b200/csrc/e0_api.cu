@@ -136,6 +136,8 @@ struct e0_ctx {
   DecodeState dec{};
   StreamPool pool;
   e0_stats stats{};
+  bool time_gemm = false;                          // profiling: event pairs around the GEMMs
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> gemm_ev;
 };
 
 extern "C" const char *e0_last_error(void) { return g_err.c_str(); }
@@ -162,6 +164,10 @@ static int dalloc(T **p, size_t n) {
 extern "C" int e0_destroy(e0_ctx *C) {
   if (!C) return E0_OK;
   cudaDeviceSynchronize();
+  for (auto &e : C->gemm_ev) {
+    cudaEventDestroy(e.first);
+    cudaEventDestroy(e.second);
+  }
   void *bufs[] = {C->xb, C->xf, C->logits, C->hlog, C->lt, C->gates, C->idx, C->a, C->plan_mem,
                   C->yscratch, C->pred_tab, C->hist_tab, C->err, C->h1pre, C->h1, C->pool.mem, C->pool.slot_of,
                   C->pool.slot_tag, C->xp, C->ap, C->xg, C->xsum, C->asum, C->yacc, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
@@ -418,8 +424,16 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   }
   const int tmax = std::min(C->tile_cap, (K.T * D.top_k + kTcN - 1) / kTcN + std::min(D.n_experts, K.T * D.top_k) +
                                               (K.T + kTcN - 1) / kTcN);
+  cudaEvent_t g0 = nullptr, g1 = nullptr;
+  if (C->time_gemm && cudaEventCreate(&g0) == cudaSuccess && cudaEventCreate(&g1) == cudaSuccess)
+    cudaEventRecord(g0, s);
   k_moe_gemm_tc<<<tmax * (D.d_ff / 64), kTwThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(gate/up)");
+  if (g1) {
+    cudaEventRecord(g1, s);
+    C->gemm_ev.push_back({g0, g1});
+    g0 = g1 = nullptr;
+  }
   const long long ag = (long long)K.T * (D.top_k + 1) * (D.d_ff / 64);
   k_perm_sums<<<(unsigned)((ag + 255) / 256), 256, 0, s>>>(C->ap, (long long)K.T * (D.top_k + 1), D.d_ff, nullptr,
                                                           C->asum);
@@ -433,8 +447,14 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   A.mode = 1;
   if ((rc = tmap_bf16_rows(&A.tmB[0], C->ap, D.d_ff, (long long)K.T * (D.top_k + 1)))) return rc;
   A.tmB[1] = A.tmB[0];
+  if (C->time_gemm && cudaEventCreate(&g0) == cudaSuccess && cudaEventCreate(&g1) == cudaSuccess)
+    cudaEventRecord(g0, s);
   k_moe_gemm_tc<<<tmax * (D.d_model / 128), kTwThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(down)");
+  if (g1) {
+    cudaEventRecord(g1, s);
+    C->gemm_ev.push_back({g0, g1});
+  }
   k_tc_finish<<<K.T, 256, 0, s>>>(C->yacc, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
                                                            D.d_model, D.lora_rank, D.lora_scale, K.y, K.yf);
   CKL("k_tc_finish");
@@ -1070,7 +1090,24 @@ extern "C" int e0_get_stats(e0_ctx *C, e0_stats *out) {
     if (C->last) cudaStreamSynchronize(C->last);
     for (auto &r : C->pool.ring) account_rec(C, r);
   }
+  for (auto &e : C->gemm_ev) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(e.second) == cudaSuccess && cudaEventElapsedTime(&ms, e.first, e.second) == cudaSuccess) {
+      C->stats.gemm_timed++;
+      C->stats.gemm_ms += ms;
+    }
+    cudaEventDestroy(e.first);
+    cudaEventDestroy(e.second);
+  }
+  C->gemm_ev.clear();
   *out = C->stats;
+  return E0_OK;
+}
+
+// Profiling: time every expert-GEMM launch with an event pair (see e0_get_stats).
+extern "C" int e0_debug_time_gemm(e0_ctx *C, int on) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  C->time_gemm = on != 0;
   return E0_OK;
 }
 
