@@ -102,7 +102,8 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"e0_clocks_rank{gpu_index}.csv")
         self.uuid = None
         try:
             import torch
@@ -340,7 +341,7 @@ def run_decode(args, dims, seed, B, ws, rank, local):
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": steps, "warmup": warm,
         "ms_per_step": ms_max / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 weights, fp32 accumulate", "data": "synthetic (seeded; see DESIGN.md input recipe)",
+        "dtype": "int4 weights, fp32 accumulate", "data": "synthetic (seeded random weights and inputs of the model's shapes)",
         "config": {"workload": args.workload, "layers": dims.L, "batch": B, "d": dims.d, "experts": dims.E,
                    "d_ff": dims.I, "top_k": dims.k, "lora_rank": dims.r, "heads": len(dims.head_layers),
                    "parallelism": f"replicas x{ws}", "l2": "inputs larger than L2 (18.1 GB of expert weights)"},

@@ -18,7 +18,7 @@ Sources (page title and section; no code is printed on any of them):
      plus one shared expert, top-4 routing, int4 affine quantisation in groups of 64,
      33 prerouter heads.
 
-Readings where the pages are silent (each is listed with its reason in the design doc):
+Readings where the pages are silent (each taken as the plainest reading the rest supports):
   * affine int4: w = scale * q + min, q = 0..15 unsigned; groups of 64 run along K;
     element 2i of a row sits in the low nibble of byte i.
   * activation: SwiGLU, a = silu(gate) * up.
