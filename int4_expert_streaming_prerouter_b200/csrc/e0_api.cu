@@ -79,11 +79,17 @@ struct DecodeState {
   int flat = 1;                          // unchained steps: the flat schedule
   unsigned long long timeout_ns = 2000000000ull;
   unsigned long long *trace = nullptr;   // profiling timeline (caller-owned), or nullptr
+  // item lists of the four schedules (flat or in order) x (first step or not):
+  // [4][G][kMaxItems] items and [4][G] counts, schedule index 2 * flat + step0
+  unsigned long long *sched = nullptr;
+  int *sched_n = nullptr;
 };
 
 static void decode_free(DecodeState &S) {
   if (S.d_layers) cudaFree(S.d_layers);
   if (S.tbuf) cudaFree(S.tbuf);
+  if (S.sched) cudaFree(S.sched);
+  if (S.sched_n) cudaFree(S.sched_n);
   S = DecodeState{};
 }
 
@@ -884,6 +890,30 @@ static int decode_prepare(e0_ctx *C) {
     S.t_rlog = p; p += n_r;
     S.t_hlog = p;
   }
+  // the item lists of every schedule, built once for this model
+  {
+    SchedShape Z{};
+    Z.L = L; Z.G = S.G; Z.E = E; Z.k = k; Z.r = D.lora_rank; Z.D = D.d_model; Z.I = D.d_ff;
+    Z.ldh = D.d_model + (D.head_onehot ? 2 * E : 0);
+    for (int l = 0; l < L; l++) {
+      Z.head[l] = C->heads[l].w_lin != nullptr;
+      Z.lora[l] = C->layers[l].lora_Ag != nullptr;
+    }
+    const size_t per = (size_t)S.G * kMaxItems;
+    std::vector<unsigned long long> items(4 * per, 0ull);
+    std::vector<int> counts(4 * (size_t)S.G, 0);
+    for (int v = 0; v < 4; v++)
+      for (int c = 0; c < S.G; c++) {
+        const int n = build_items(Z, (v >> 1) != 0, (v & 1) != 0, c, items.data() + v * per + (size_t)c * kMaxItems);
+        if (n < 0) return fail(E0_ERR_INVALID_ARG, "decode schedule: more than %d items for one CTA", kMaxItems);
+        counts[(size_t)v * S.G + c] = n;
+      }
+    int rc;
+    if (!S.sched && (rc = dalloc(&S.sched, 4 * per))) return rc;
+    if (!S.sched_n && (rc = dalloc(&S.sched_n, 4 * (size_t)S.G))) return rc;
+    CK(cudaMemcpy(S.sched, items.data(), items.size() * sizeof(unsigned long long), cudaMemcpyHostToDevice));
+    CK(cudaMemcpy(S.sched_n, counts.data(), counts.size() * sizeof(int), cudaMemcpyHostToDevice));
+  }
   int which;
   decode_geometry(D, &which);
   const void *fn = which == 0 ? (const void *)k_decode<2048, 512> : (const void *)k_decode<256, 128>;
@@ -923,6 +953,11 @@ static int decode_persistent(e0_ctx *C, const uint16_t *h, int step, uint16_t *y
   P.timeout_ns = S.timeout_ns;
   P.stall_cta = S.stall_cta;
   P.trace = S.trace;
+  {
+    const int v = 2 * (P.flat ? 1 : 0) + (P.step0 ? 1 : 0);
+    P.sched = S.sched + (size_t)v * S.G * kMaxItems;
+    P.sched_n = S.sched_n + (size_t)v * S.G;
+  }
   S.stall_cta = -1;
   int which;
   decode_geometry(D, &which);

@@ -25,14 +25,15 @@
 //   * Work per layer is split into contiguous, balanced ranges per CTA: the (k+1)*I
 //     intermediate rows of the gate/up phase and the d output rows of the down phase.
 #pragma once
+#include <algorithm>
 #include "e0_device.cuh"
 #include "e0_kernels.cuh"
 
 namespace e0 {
 
-constexpr int kDecThreads = 416;          // 1 producer warp + 12 consumer warps
-constexpr int kDecConsumers = 384;
-constexpr int kDecCW = 12;
+constexpr int kDecCW = 12;                // consumer warps
+constexpr int kDecConsumers = 32 * kDecCW;
+constexpr int kDecThreads = 32 + kDecConsumers;   // + 1 producer warp
 constexpr int kRingBytes = 174 * 1024;
 constexpr int kDecMaxK = 4;               // routed experts per token on this path
 constexpr int kNSlot = 8;                 // tasks in flight
@@ -75,6 +76,8 @@ struct DecodeParams {
   unsigned long long timeout_ns;
   int stall_cta;            // test hook: this CTA waits on a tag nobody writes (-1: none)
   unsigned long long *trace;  // optional [G][L][16] %globaltimer stamps (profiling), or nullptr
+  const unsigned long long *sched;  // [G][kMaxItems] item lists (pack_item), built on the host
+  const int *sched_n;               // [G] items per CTA
 };
 
 // Timeline stamps of the optional trace (one row of 16 per CTA and layer).
@@ -241,11 +244,11 @@ struct Item {
   int kind, l, a, n;
   bool first;
 };
-__device__ __forceinline__ unsigned long long pack_item(int kind, int l, int a, int n, bool first) {
+__host__ __device__ __forceinline__ unsigned long long pack_item(int kind, int l, int a, int n, bool first) {
   return (unsigned long long)kind | ((unsigned long long)first << 4) | ((unsigned long long)l << 8) |
          ((unsigned long long)a << 16) | ((unsigned long long)n << 40);
 }
-__device__ __forceinline__ Item unpack_item(unsigned long long v) {
+__host__ __device__ __forceinline__ Item unpack_item(unsigned long long v) {
   return Item{(int)(v & 15ull), (int)((v >> 8) & 255ull), (int)((v >> 16) & 0xFFFFFFull), (int)(v >> 40),
               ((v >> 4) & 1ull) != 0};
 }
@@ -368,6 +371,8 @@ struct DecSmem {
   };
   float at[(kDecMaxK + 1) * I];      // a of every slot, pre-scaled, chunk-transposed per slot
   float asraw[I];                    // the shared expert's a (natural order, for t_d)
+  float xsum[D / 32];                // raw sum of each 32-element chunk of x
+  float asum[(kDecMaxK + 1) * (I / 32)];   // raw sum of each 32-element chunk of each slot's a
   float gus[2 * I];                  // the shared expert's raw g and u (interleaved per row)
   double dred[16];
   float gates[kMaxK];
@@ -405,7 +410,7 @@ __device__ __forceinline__ bool timed_out(unsigned long long &t0, unsigned long 
 }
 
 // ---------------------------------------------------------------------------------------
-// The launch's item list of this CTA (one thread).
+// The item lists, one per CTA, built on the host.
 //
 // In order (chained inputs, or for comparison): per layer [R, TK] XR GU DN, each x item
 // and the down item over this CTA's balanced share of the layer's units.
@@ -415,34 +420,45 @@ __device__ __forceinline__ bool timed_out(unsigned long long &t0, unsigned long 
 // phase's units over all layers form one list, split evenly and contiguously across the
 // CTAs, so that a CTA streams long runs of rows of one or two layers instead of a sliver
 // of every layer.  Phases: R (reactive layers' routers), XR, TK (the reactive layers this
-// CTA needs), GU, DN.  Items are cut to at most about 58 KB of weight bytes (three fit the ring).  A CTA then
-// computes a handful of norms per step, polls other CTAs' results a handful of times, and
-// waits on other CTAs only where a phase needs the previous one (R -> TK, GU -> DN).
+// CTA needs), GU, DN.  Items are cut to at most about 58 KB of weight bytes (three fit the
+// ring).  A CTA then computes a handful of norms per step, polls other CTAs' results a
+// handful of times, and waits on other CTAs only where a phase needs the previous one
+// (R -> TK, GU -> DN).
+//
+// A list depends only on the model's shape, on which layers carry a head or LoRA, on the
+// schedule and on whether the step is a sequence's first (no predictions yet), so the host
+// builds each combination once and a CTA copies its own list at launch.
 // ---------------------------------------------------------------------------------------
-template <int D, int I>
-__device__ __forceinline__ int xrows_of(const DecodeParams &P, const DecSmem<D, I> &S, int l) {
-  const DecLayer &Y = S.lay[l];
-  return (Y.head ? P.E : 0) + (Y.Ag ? 2 * P.r : 0) + (is_predicted(P, S, l) ? P.k : 0);
+struct SchedShape {
+  int L, G, E, k, r, ldh, D, I;
+  bool head[64], lora[64];
+};
+
+inline bool sched_predicted(const SchedShape &Z, bool step0, int l) {
+  return !step0 && l > 0 && Z.head[l - 1];
+}
+inline int sched_xrows(const SchedShape &Z, bool step0, int l) {
+  return (Z.head[l] ? Z.E : 0) + (Z.lora[l] ? 2 * Z.r : 0) + (sched_predicted(Z, step0, l) ? Z.k : 0);
 }
 
-template <int D, int I>
-__device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I> &S) {
-  const int G = P.G, c = blockIdx.x, L = P.L, k = P.k;
+// CTA c's items into out[0, kMaxItems); returns their count, or -1 if they do not fit.
+inline int build_items(const SchedShape &Z, bool flat, bool step0, int c, unsigned long long *out) {
+  const int G = Z.G, L = Z.L, k = Z.k, D = Z.D, I = Z.I;
   int n = 0;
+  bool over = false;
   auto put = [&](int kind, int l, int a, int cnt) {
-    if (n < kMaxItems) S.items[n++] = pack_item(kind, l, a, cnt, false);
-    else atomicOr(P.err, DERR_TIMEOUT);   // cannot happen for the supported sizes
+    if (n < kMaxItems) out[n++] = pack_item(kind, l, a, cnt, false);
+    else over = true;
   };
-  if (!P.flat) {
-    #pragma unroll 1
+  if (!flat) {
     for (int l = 0; l < L; l++) {
       int a, b;
-      if (!is_predicted(P, S, l)) {
-        split_range(P.E, G, c, a, b);
+      if (!sched_predicted(Z, step0, l)) {
+        split_range(Z.E, G, c, a, b);
         if (b > a) put(IT_R, l, a, b - a);
         put(IT_TK, l, 0, 0);
       }
-      split_range(xrows_of(P, S, l), G, c, a, b);
+      split_range(sched_xrows(Z, step0, l), G, c, a, b);
       if (b > a) put(IT_XR, l, a, b - a);
       split_range((k + 1) * I, G, c, a, b);
       if (b > a) put(IT_GU, l, a, b - a);
@@ -451,65 +467,58 @@ __device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I>
     }
   } else {
     constexpr int kItemBytes = 58 * 1024;
-    const int gu_chunk = min(kItemBytes / (2 * (D / 2 + D / 16)), 288);
-    const int dn_chunk = min(kItemBytes / ((k + 1) * (I / 2 + I / 16) + 2 * P.r), kDnMaxRows);
-    const int xr_chunk = max(kItemBytes / (2 * P.ldh), 1);
+    // gate/up items in whole consumer passes where the byte budget allows (a pass covers
+    // two units per row group of each consumer warp); down items take the full budget,
+    // since fewer, longer down items beat whole passes there
+    const int gu_pass = 2 * kDecCW * (32 / (D / 32 < 32 ? D / 32 : 32));
+    int gu_chunk = std::min(kItemBytes / (2 * (D / 2 + D / 16)), 288);
+    const int dn_chunk = std::min(kItemBytes / ((k + 1) * (I / 2 + I / 16) + 2 * Z.r), kDnMaxRows);
+    const int xr_chunk = std::max(kItemBytes / (2 * Z.ldh), 1);
+    if (gu_chunk >= gu_pass) gu_chunk -= gu_chunk % gu_pass;
+    auto units = [&](int which, int l) {
+      return which == 0 ? (sched_predicted(Z, step0, l) ? 0 : Z.E)
+           : which == 1 ? sched_xrows(Z, step0, l) : which == 2 ? (k + 1) * I : D;
+    };
     // one phase: units(l) per layer over every layer with units, this CTA's share
     auto phase = [&](int kind, int chunk, int which) {
       long long tot = 0;
-      #pragma unroll 1
-      for (int l = 0; l < L; l++) {
-        const int u = which == 0 ? (is_predicted(P, S, l) ? 0 : P.E)
-                    : which == 1 ? xrows_of(P, S, l) : which == 2 ? (k + 1) * I : D;
-        tot += u;
-      }
+      for (int l = 0; l < L; l++) tot += units(which, l);
       const long long lo = tot * c / G, hi = tot * (c + 1) / G;
       long long base = 0;
-      #pragma unroll 1
       for (int l = 0; l < L; l++) {
-        const int u = which == 0 ? (is_predicted(P, S, l) ? 0 : P.E)
-                    : which == 1 ? xrows_of(P, S, l) : which == 2 ? (k + 1) * I : D;
-        const long long s0 = max(lo, base), s1 = min(hi, base + u);
-        for (long long a = s0; a < s1; a += chunk) put(kind, l, (int)(a - base), (int)min((long long)chunk, s1 - a));
+        const int u = units(which, l);
+        const long long s0 = std::max(lo, base), s1 = std::min(hi, base + u);
+        for (long long a = s0; a < s1; a += chunk) put(kind, l, (int)(a - base), (int)std::min((long long)chunk, s1 - a));
         base += u;
       }
     };
     phase(IT_R, 9, 0);
     phase(IT_XR, xr_chunk, 1);
     const int n_before_tk = n;
-    // placeholder for the top-k items: the reactive layers that this CTA's gate/up or
-    // down items touch
     phase(IT_GU, gu_chunk, 2);
     phase(IT_DN, dn_chunk, 3);
-    bool need[64];
-    #pragma unroll 1
-    for (int l = 0; l < L; l++) need[l] = false;
-    #pragma unroll 1
+    // the top-k items go before the gate/up phase: the reactive layers that this CTA's
+    // gate/up or down items touch
+    bool need[64] = {};
     for (int q = n_before_tk; q < n; q++) {
-      const Item it = unpack_item(S.items[q]);
-      if (!is_predicted(P, S, it.l)) need[it.l] = true;
+      const Item it = unpack_item(out[q]);
+      if (!sched_predicted(Z, step0, it.l)) need[it.l] = true;
     }
     int ntk = 0;
-    #pragma unroll 1
     for (int l = 0; l < L; l++) ntk += need[l];
-    if (n + ntk > kMaxItems) {
-      atomicOr(P.err, DERR_TIMEOUT);
-      ntk = 0;
-    }
-    #pragma unroll 1
-    for (int q = n - 1; q >= n_before_tk; q--) S.items[q + ntk] = S.items[q];
+    if (n + ntk > kMaxItems) return -1;
+    for (int q = n - 1; q >= n_before_tk; q--) out[q + ntk] = out[q];
     int w = n_before_tk;
-    #pragma unroll 1
-    for (int l = 0; l < L && ntk; l++)
-      if (need[l]) S.items[w++] = pack_item(IT_TK, l, 0, 0, false);
+    for (int l = 0; l < L; l++)
+      if (need[l]) out[w++] = pack_item(IT_TK, l, 0, 0, false);
     n += ntk;
   }
+  if (over) return -1;
   // flags: x items compute the norm when the previous x item had another layer; the
   // first down item of each layer assembles the layer's shared-expert inputs
   int lastx = -1, lastd = -1;
-  #pragma unroll 1
   for (int q = 0; q < n; q++) {
-    Item it = unpack_item(S.items[q]);
+    const Item it = unpack_item(out[q]);
     bool f = false;
     if (it.kind == IT_R || it.kind == IT_XR || it.kind == IT_GU) {
       f = it.l != lastx;
@@ -518,9 +527,9 @@ __device__ __noinline__ void build_schedule(const DecodeParams &P, DecSmem<D, I>
       f = it.l != lastd;
       lastd = it.l;
     }
-    S.items[q] = pack_item(it.kind, it.l, it.a, it.n, f);
+    out[q] = pack_item(it.kind, it.l, it.a, it.n, f);
   }
-  S.nitems = n;
+  return n;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -819,9 +828,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       mbar_init(&S.empty[s], kDecCW);
     }
     S.abort = 0;
-    build_schedule<D, I>(P, S);
+    S.nitems = min(max(P.sched_n[blockIdx.x], 0), kMaxItems);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  #pragma unroll 1
+  for (int i = tid; i < min(max(P.sched_n[blockIdx.x], 0), kMaxItems); i += kDecThreads)
+    S.items[i] = P.sched[(size_t)blockIdx.x * kMaxItems + i];
   __syncthreads();
   if (tid < 32) {
     producer<D, I>(P, S);
@@ -931,6 +943,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         }
       }
       cbar();
+      // the chunk sums that every gate/up row of the layer uses with its minima
+      if (!ab && ct < NCH) {
+        float xr[32];
+        load_chunk(S.xt, NCH, ct, xr);
+        S.xsum[ct] = chunk_raw_sum(xr);
+      }
+      cbar();
       if (ct == 0) stamp(P, l, TR_NORM);
     }
     if (ab) {
@@ -984,45 +1003,55 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
 #pragma unroll
         for (int cc = 0; cc < CPL; cc++) {
           load_chunk(S.xt, NCH, sl + cc * LPR, xr[cc]);
-          xsr[cc] = chunk_raw_sum(xr[cc]);
+          xsr[cc] = S.xsum[sl + cc * LPR];
         }
-        #pragma unroll 1
-        for (int base = warp * RPW; base < in; base += kDecCW * RPW) {
-          const int u = base + sub;
-          const bool valid = u < in;
-          // unit u = global unit ia + u: slot (ia + u) / I, index (ia + u) % I; its piece p
-          // is the slot's order among the item's slots, its row the index minus the
-          // piece's first index
-          const int gidx = ia + u, es = gidx / I, p = es - slot0;   // es: expert slot of the unit
+        // unit u = global unit ia + u: slot es = (ia + u) / I, index i = (ia + u) % I; its
+        // piece p is the slot's order among the item's slots, its row the index minus the
+        // piece's first index.  Two units per warp pass, so that their four dot products
+        // and reductions interleave.
+        auto partial = [&](int u, float &ag, float &au) {
+          const int gidx = ia + u, es = gidx / I, p = es - slot0;
           const int i = gidx - es * I, row = i - (p == 0 ? ia - slot0 * I : 0), sg = kGuPiece0 + 6 * p;
-          float ag = 0.f, au = 0.f;
-          if (valid) {
-            const uint8_t *gcw = S.ring + S.seg_off[slot][sg + 0] + (size_t)row * (D / 2);
-            const uint16_t *gsc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 1]) + (size_t)row * (D / 64);
-            const uint16_t *gmn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 2]) + (size_t)row * (D / 64);
-            const uint8_t *ucw = S.ring + S.seg_off[slot][sg + 3] + (size_t)row * (D / 2);
-            const uint16_t *usc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 4]) + (size_t)row * (D / 64);
-            const uint16_t *umn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 5]) + (size_t)row * (D / 64);
+          const uint8_t *gcw = S.ring + S.seg_off[slot][sg + 0] + (size_t)row * (D / 2);
+          const uint16_t *gsc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 1]) + (size_t)row * (D / 64);
+          const uint16_t *gmn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 2]) + (size_t)row * (D / 64);
+          const uint8_t *ucw = S.ring + S.seg_off[slot][sg + 3] + (size_t)row * (D / 2);
+          const uint16_t *usc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 4]) + (size_t)row * (D / 64);
+          const uint16_t *umn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 5]) + (size_t)row * (D / 64);
 #pragma unroll
-            for (int cc = 0; cc < CPL; cc++) {
-              const int ch = sl + cc * LPR;
-              const uint4 wg = *reinterpret_cast<const uint4 *>(gcw + ch * 16);
-              const uint4 wu = *reinterpret_cast<const uint4 *>(ucw + ch * 16);
-              const float qg = chunk_qdot(wg, xr[cc]);
-              const float qu = chunk_qdot(wu, xr[cc]);
-              ag = fmaf(bf(gsc[ch >> 1]), qg, fmaf(bf(gmn[ch >> 1]), xsr[cc], ag));
-              au = fmaf(bf(usc[ch >> 1]), qu, fmaf(bf(umn[ch >> 1]), xsr[cc], au));
-            }
+          for (int cc = 0; cc < CPL; cc++) {
+            const int ch = sl + cc * LPR;
+            const uint4 wg = *reinterpret_cast<const uint4 *>(gcw + ch * 16);
+            const uint4 wu = *reinterpret_cast<const uint4 *>(ucw + ch * 16);
+            const float qg = chunk_qdot(wg, xr[cc]);
+            const float qu = chunk_qdot(wu, xr[cc]);
+            ag = fmaf(bf(gsc[ch >> 1]), qg, fmaf(bf(gmn[ch >> 1]), xsr[cc], ag));
+            au = fmaf(bf(usc[ch >> 1]), qu, fmaf(bf(umn[ch >> 1]), xsr[cc], au));
           }
-          ag = group_sum(ag, LPR);
-          au = group_sum(au, LPR);
-          if (valid && sl == 0) {
-            if (es == k) {
-              st_tag(blk + k * I + 2 * i, tag, __float_as_uint(ag));
-              st_tag(blk + k * I + 2 * i + 1, tag, __float_as_uint(au));
-            } else {
-              st_tag(blk + es * I + i, tag, f2bf(ag / (1.0f + expf(-ag)) * au));
-            }
+        };
+        auto publish = [&](int u, float ag, float au) {
+          const int gidx = ia + u, es = gidx / I, i = gidx - es * I;
+          if (es == k) {
+            st_tag(blk + k * I + 2 * i, tag, __float_as_uint(ag));
+            st_tag(blk + k * I + 2 * i + 1, tag, __float_as_uint(au));
+          } else {
+            st_tag(blk + es * I + i, tag, f2bf(ag / (1.0f + expf(-ag)) * au));
+          }
+        };
+        #pragma unroll 1
+        for (int base = warp * RPW; base < in; base += 2 * kDecCW * RPW) {
+          const int u0 = base + sub, u1 = base + kDecCW * RPW + sub;
+          const bool v0 = u0 < in, v1 = u1 < in;
+          float ag0 = 0.f, au0 = 0.f, ag1 = 0.f, au1 = 0.f;
+          if (v0) partial(u0, ag0, au0);
+          if (v1) partial(u1, ag1, au1);
+          ag0 = group_sum(ag0, LPR);
+          au0 = group_sum(au0, LPR);
+          ag1 = group_sum(ag1, LPR);
+          au1 = group_sum(au1, LPR);
+          if (sl == 0) {
+            if (v0) publish(u0, ag0, au0);
+            if (v1) publish(u1, ag1, au1);
           }
         }
       }
@@ -1099,6 +1128,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           }
         }
         cbar();
+        // the chunk sums that every down row of the layer uses with its minima
+        if (!ab && ct < (k + 1) * NCI) {
+          float ar[32];
+          load_chunk(S.at + (ct / NCI) * I, NCI, ct % NCI, ar);
+          S.asum[ct] = chunk_raw_sum(ar);
+        }
         if (!ab && lora) {
           // t_d = Ad a_s (LoRA down branch)
           const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k) + 3]);
@@ -1115,8 +1150,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (ct == 0) stamp(P, l, TR_TD_POLL);
       }
       if (!ab) {
-        // a warp owns its rows across every expert: y accumulates in registers in the
-        // combine order (routed experts with their gates, then the shared expert)
+        // a warp owns its rows across every expert: each lane accumulates its chunks'
+        // partial dot products in the combine order (routed experts with their gates, then
+        // the shared expert), and the row's lanes are summed once at the end
         constexpr int LPR = NCI < 32 ? NCI : 32;
         constexpr int RPW = 32 / LPR;
         constexpr int CPL = NCI / LPR;
@@ -1133,7 +1169,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
 #pragma unroll
             for (int cc = 0; cc < CPL; cc++) {
               load_chunk(S.at + j * I, NCI, sl + cc * LPR, ar[cc]);
-              asr[cc] = chunk_raw_sum(ar[cc]);
+              asr[cc] = S.asum[j * NCI + sl + cc * LPR];
             }
             const float gj = j < k ? S.gates[j] : 1.f;
             const uint8_t *cb = S.ring + S.seg_off[slot][3 * j];
@@ -1141,40 +1177,47 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
             const uint16_t *mb = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3 * j + 2]);
 #pragma unroll
             for (int pp = 0; pp < PM; pp++) {
-              const int base = pp * kDecCW * RPW + warp * RPW;
-              if (base < in) {
-                const int row = base + sub;
-                const bool valid = row < in;
+              const int row = pp * kDecCW * RPW + warp * RPW + sub;
+              if (row < in) {
+                const uint8_t *cw = cb + (size_t)row * (I / 2);
+                const uint16_t *sc = sb + (size_t)row * (I / 64);
+                const uint16_t *mn = mb + (size_t)row * (I / 64);
                 float acc = 0.f;
-                if (valid) {
-                  const uint8_t *cw = cb + (size_t)row * (I / 2);
-                  const uint16_t *sc = sb + (size_t)row * (I / 64);
-                  const uint16_t *mn = mb + (size_t)row * (I / 64);
 #pragma unroll
-                  for (int cc = 0; cc < CPL; cc++) {
-                    const int ch = sl + cc * LPR;
-                    const uint4 w = *reinterpret_cast<const uint4 *>(cw + ch * 16);
-                    const float qd = chunk_qdot(w, ar[cc]);
-                    acc = fmaf(bf(sc[ch >> 1]), qd, fmaf(bf(mn[ch >> 1]), asr[cc], acc));
-                  }
+                for (int cc = 0; cc < CPL; cc++) {
+                  const int ch = sl + cc * LPR;
+                  const uint4 w = *reinterpret_cast<const uint4 *>(cw + ch * 16);
+                  const float qd = chunk_qdot(w, ar[cc]);
+                  acc = fmaf(bf(sc[ch >> 1]), qd, fmaf(bf(mn[ch >> 1]), asr[cc], acc));
                 }
-                acc = group_sum(acc, LPR);
                 y[pp] = j < k ? fmaf(gj, acc, y[pp]) : y[pp] + acc;
               }
             }
           }
-          const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]);
+          // the shared expert's LoRA down branch c * (Bd t_d) of the row, its r terms
+          // spread over the row's lanes
+          if (lora) {
+            const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]);
+#pragma unroll
+            for (int pp = 0; pp < PM; pp++) {
+              const int row = pp * kDecCW * RPW + warp * RPW + sub;
+              if (row < in) {
+                float lo = 0.f;
+                #pragma unroll 1
+                for (int j = sl; j < r; j += LPR) lo = fmaf(bf(bd[row * r + j]), S.td[j], lo);
+                y[pp] = fmaf(P.c, lo, y[pp]);
+              }
+            }
+          }
+          // one reduction per row, over the lanes' partial sums
+#pragma unroll
+          for (int pp = 0; pp < PM; pp++)
+            if (pp * kDecCW * RPW + warp * RPW < in) y[pp] = group_sum(y[pp], LPR);   // warp-uniform
 #pragma unroll
           for (int pp = 0; pp < PM; pp++) {
             const int row = pp * kDecCW * RPW + warp * RPW + sub;
             if (row < in && sl == 0) {
-              float yv = y[pp];
-              if (lora) {
-                float lo = 0.f;
-                #pragma unroll 1
-                for (int j = 0; j < r; j++) lo = fmaf(bf(bd[row * r + j]), S.td[j], lo);
-                yv = fmaf(P.c, lo, yv);
-              }
+              const float yv = y[pp];
               const int n = ia + row;
               st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(yv));
               P.y[(size_t)l * D + n] = f2bf(yv);
