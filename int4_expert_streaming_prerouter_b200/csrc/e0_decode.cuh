@@ -157,56 +157,64 @@ __host__ __device__ __forceinline__ void split_range(int N, int G, int c, int &a
   b = (int)((unsigned)(N * (c + 1)) / (unsigned)G);
 }
 
-// nibble i of a 32-bit code word is placed in the mantissa of 2^23 + q * 2^p(i) without
-// shifting (i < 5) or after one shift by 12 (i >= 5); the matching activation is
-// pre-scaled by 2^-p(i) so that the product is exactly q * x.
-__host__ __device__ constexpr float nib_scale(int i) {
-  return i == 0 ? 1.f : i == 1 ? 1.f / 16 : (i == 2 || i == 5) ? 1.f / 256 : (i == 3 || i == 6) ? 1.f / 4096 : 1.f / 65536;
-}
-
-// sum_k q_k x'_k over one 16-byte chunk (32 nibbles) with the 32 pre-scaled activations
-// held in registers.  Exact products (q * 2^p times x * 2^-p), fp32 pairwise accumulation
-// with packed f32x2 instructions.
-__device__ __forceinline__ float chunk_qdot(const uint4 w, const float (&xr)[32]) {
-  const unsigned long long kMagic = pk2(-8388608.f, -8388608.f);
-  unsigned long long acc0 = 0ull, acc1 = 0ull;
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-  for (int t = 0; t < 4; t++) {
-    const uint32_t a = ws[t], b = a >> 12;
-    const uint32_t v0 = (a & 0x0000000Fu) | 0x4B000000u, v1 = (a & 0x000000F0u) | 0x4B000000u;
-    const uint32_t v2 = (a & 0x00000F00u) | 0x4B000000u, v3 = (a & 0x0000F000u) | 0x4B000000u;
-    const uint32_t v4 = (a & 0x000F0000u) | 0x4B000000u, v5 = (b & 0x00000F00u) | 0x4B000000u;
-    const uint32_t v6 = (b & 0x0000F000u) | 0x4B000000u, v7 = (b & 0x000F0000u) | 0x4B000000u;
-    const unsigned long long q01 = f2add(((unsigned long long)v1 << 32) | v0, kMagic);
-    const unsigned long long q23 = f2add(((unsigned long long)v3 << 32) | v2, kMagic);
-    const unsigned long long q45 = f2add(((unsigned long long)v5 << 32) | v4, kMagic);
-    const unsigned long long q67 = f2add(((unsigned long long)v7 << 32) | v6, kMagic);
-    acc0 = f2fma(q01, pk2(xr[8 * t + 0], xr[8 * t + 1]), acc0);
-    acc1 = f2fma(q23, pk2(xr[8 * t + 2], xr[8 * t + 3]), acc1);
-    acc0 = f2fma(q45, pk2(xr[8 * t + 4], xr[8 * t + 5]), acc0);
-    acc1 = f2fma(q67, pk2(xr[8 * t + 6], xr[8 * t + 7]), acc1);
-  }
-  return f2sum(acc0) + f2sum(acc1);
-}
-
-// Activations live in shared memory "chunk-transposed": element e of a row of n16 chunks
-// (32 elements each) sits at float index (((e & 31) >> 2) * n16 + (e >> 5)) * 4 + (e & 3),
-// so the lanes of a warp, each owning one chunk, read their 32 values with eight
-// conflict-free 16-byte loads.
+// x for the bf16 rows lives in shared memory "chunk-transposed": element e of a row of
+// n16 chunks (32 elements each) sits at float index
+// (((e & 31) >> 2) * n16 + (e >> 5)) * 4 + (e & 3), so that the lanes of a warp read their
+// elements with conflict-free 16-byte loads.
 __host__ __device__ __forceinline__ int xt_index(int e, int n16) {
   return ((((e & 31) >> 2) * n16) + (e >> 5)) * 4 + (e & 3);
 }
-__device__ __forceinline__ void load_chunk(const float *xt, int n16, int ch, float (&xr)[32]) {
-#pragma unroll
-  for (int q = 0; q < 8; q++) {
-    const float4 v = *reinterpret_cast<const float4 *>(xt + (q * n16 + ch) * 4);
-    xr[4 * q] = v.x;
-    xr[4 * q + 1] = v.y;
-    xr[4 * q + 2] = v.z;
-    xr[4 * q + 3] = v.w;
-  }
+
+// ---------------------------------------------------------------------------------------
+// Tensor-core dot products of int4 rows with one activation vector (gate/up and down).
+//
+// A warp takes two rows r0, r1 that share the activation vector v and walks their K in
+// steps of 512 (eight groups of 64).  In a step, lane (g, t) (g = lane / 4, t = lane % 4)
+// holds code words 8 g + 2 t and 8 g + 2 t + 1 of the step of both rows (16 codes of
+// group g each).  Word nibbles n0..n7 (elements 8 w .. 8 w + 7) become the bf16 pairs
+// {128 + n_j, 128 + n_(j+4)}, j = 0..3, exact, with one mask and one OR each.  In the
+// m16n8k16 MMA, row g is r0 restricted to group g, row g + 8 is r1 restricted to group g,
+// and column g is v restricted to group g, paired in the same element order, so the
+// diagonal entries D[g][g] and D[g + 8][g] are P = sum (128 + q) v over group g of r0 and
+// of r1 (the other entries are not used).  Four MMAs cover a step.  The lane that holds
+// the diagonal (t = g / 2) folds the group's affine weights w = s q + m into its partial
+// sum as s P + (m - 128 s) V, V = sum v over the group; a warp sum finishes each row.
+//
+// v lives in shared memory as bf16 pairs in the same order: word w of v is the uint4
+// {v0|v4, v1|v5, v2|v6, v3|v7} of elements 8 w .. 8 w + 7 (low half first).
+// ---------------------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int pair_index(int e) {   // uint16 index of element e
+  return (e >> 3) * 8 + (e & 3) * 2 + ((e >> 2) & 1);
 }
+__device__ __forceinline__ uint32_t nib_pair_bf16(uint32_t w, int j) {
+  return ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// one 512-wide step: c0, c1 the two code words of rows r0, r1; va, vb the activation
+// words 8 g + 2 t and 8 g + 2 t + 1 of the step
+__device__ __forceinline__ void pair_step(float (&d)[4], uint2 c0, uint2 c1, uint4 va, uint4 vb) {
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+  mma_bf16_16816(d, nib_pair_bf16(c0.x, 0), nib_pair_bf16(c1.x, 0), nib_pair_bf16(c0.x, 1), nib_pair_bf16(c1.x, 1),
+                 va.x, va.y);
+  mma_bf16_16816(d, nib_pair_bf16(c0.x, 2), nib_pair_bf16(c1.x, 2), nib_pair_bf16(c0.x, 3), nib_pair_bf16(c1.x, 3),
+                 va.z, va.w);
+  mma_bf16_16816(d, nib_pair_bf16(c0.y, 0), nib_pair_bf16(c1.y, 0), nib_pair_bf16(c0.y, 1), nib_pair_bf16(c1.y, 1),
+                 vb.x, vb.y);
+  mma_bf16_16816(d, nib_pair_bf16(c0.y, 2), nib_pair_bf16(c1.y, 2), nib_pair_bf16(c0.y, 3), nib_pair_bf16(c1.y, 3),
+                 vb.z, vb.w);
+}
+// the diagonal lane's affine fold of group G of one row: s P + (m - 128 s) V
+__device__ __forceinline__ float group_fold(float P, const uint16_t *sc, const uint16_t *mn, int G, float V) {
+  const float s = bf(sc[G]);
+  return fmaf(s, P, fmaf(-128.f, s, bf(mn[G])) * V);
+}
+__device__ __forceinline__ uint2 ld_code2(const uint8_t *p) { return *reinterpret_cast<const uint2 *>(p); }
 
 // Round a double to bf16 (nearest, ties to even) on its bit pattern: keep 7 of the 52
 // fraction bits.  Exact for every value in the normal bf16 range; the result is then a
@@ -364,15 +372,16 @@ __device__ __forceinline__ void item_seg(const DecodeParams &P, const DecLayer &
 template <int D, int I>
 struct DecSmem {
   uint8_t ring[kRingBytes];
-  float xt[D];                       // x pre-scaled per nibble position, chunk-transposed
+  float xt[D];                       // x (fp32), chunk-transposed (for the bf16 rows)
   union {                            // used by different items, never at the same time:
     float yprev[D];                  //   the previous layer's y (fp32), in order + chained
     uint32_t stg[kDecMaxK * I];      //   routed a payloads as polled (a layer's first down item)
   };
-  float at[(kDecMaxK + 1) * I];      // a of every slot, pre-scaled, chunk-transposed per slot
+  alignas(16) uint16_t ap[(kDecMaxK + 1) * I];   // a of every slot, bf16 pairs (pair_index order)
+  alignas(16) uint16_t xp[D];        // x as bf16 pairs (pair_index order)
   float asraw[I];                    // the shared expert's a (natural order, for t_d)
-  float xsum[D / 32];                // raw sum of each 32-element chunk of x
-  float asum[(kDecMaxK + 1) * (I / 32)];   // raw sum of each 32-element chunk of each slot's a
+  float xg[D / 64];                  // sum of x over each group of 64
+  float ag[(kDecMaxK + 1) * (I / 64)];     // sum of each slot's a over each group of 64
   float gus[2 * I];                  // the shared expert's raw g and u (interleaved per row)
   double dred[16];
   float gates[kMaxK];
@@ -763,9 +772,8 @@ __device__ __forceinline__ bool wait_full(uint64_t *bar, uint32_t par, const Ctl
   return true;
 }
 
-// bf16 row (D elements in shared memory) dotted with x, read from its pre-scaled,
-// chunk-transposed copy xt (elements 8c..8c+3 and 8c+4..8c+7 are two float4 there; the
-// per-position scales 2^-p are undone exactly): one warp.
+// bf16 row (D elements in shared memory) dotted with x, read from its chunk-transposed
+// fp32 copy xt (elements 8c..8c+3 and 8c+4..8c+7 are two float4 there): one warp.
 template <int D>
 __device__ __noinline__ float bf16_row_x(const uint16_t *w, const float *xt, int lane) {
   constexpr int NCH = D / 32;
@@ -775,14 +783,14 @@ __device__ __noinline__ float bf16_row_x(const uint16_t *w, const float *xt, int
     const uint4 v = *reinterpret_cast<const uint4 *>(w + ch * 8);
     const float4 a = *reinterpret_cast<const float4 *>(xt + ((2 * (ch & 3)) * NCH + (ch >> 2)) * 4);
     const float4 b = *reinterpret_cast<const float4 *>(xt + ((2 * (ch & 3) + 1) * NCH + (ch >> 2)) * 4);
-    acc = fmaf(bf(v.x & 0xFFFFu), a.x * (1.0f / nib_scale(0)), acc);
-    acc = fmaf(bf(v.x >> 16), a.y * (1.0f / nib_scale(1)), acc);
-    acc = fmaf(bf(v.y & 0xFFFFu), a.z * (1.0f / nib_scale(2)), acc);
-    acc = fmaf(bf(v.y >> 16), a.w * (1.0f / nib_scale(3)), acc);
-    acc = fmaf(bf(v.z & 0xFFFFu), b.x * (1.0f / nib_scale(4)), acc);
-    acc = fmaf(bf(v.z >> 16), b.y * (1.0f / nib_scale(5)), acc);
-    acc = fmaf(bf(v.w & 0xFFFFu), b.z * (1.0f / nib_scale(6)), acc);
-    acc = fmaf(bf(v.w >> 16), b.w * (1.0f / nib_scale(7)), acc);
+    acc = fmaf(bf(v.x & 0xFFFFu), a.x, acc);
+    acc = fmaf(bf(v.x >> 16), a.y, acc);
+    acc = fmaf(bf(v.y & 0xFFFFu), a.z, acc);
+    acc = fmaf(bf(v.y >> 16), a.w, acc);
+    acc = fmaf(bf(v.z & 0xFFFFu), b.x, acc);
+    acc = fmaf(bf(v.z >> 16), b.y, acc);
+    acc = fmaf(bf(v.w & 0xFFFFu), b.z, acc);
+    acc = fmaf(bf(v.w >> 16), b.w, acc);
   }
   return warp_sum(acc);
 }
@@ -791,17 +799,6 @@ __device__ __noinline__ void warp_topk_ool(const float *v, int E, int k, int lan
   warp_topk(v, E, k, lane, out);
 }
 
-// sum of the 32 raw values of a chunk whose registers hold them pre-scaled per nibble
-// position (multiplying by 2^p undoes the scaling exactly)
-__device__ __forceinline__ float chunk_raw_sum(const float (&xr)[32]) {
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    s0 = fmaf(xr[i], 1.0f / nib_scale(i & 7), s0);
-    s1 = fmaf(xr[i + 1], 1.0f / nib_scale((i + 1) & 7), s1);
-  }
-  return s0 + s1;
-}
 
 // ---------------------------------------------------------------------------------------
 // The kernel
@@ -841,7 +838,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
   }
   // ------------------------------- consumers -------------------------------------------
   constexpr int NCH = D / 32;                  // 16-byte code chunks per gate/up row
-  constexpr int NCI = I / 32;                  // 16-byte code chunks per down row
   const int ct = tid - 32, warp = ct >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = P.G, k = P.k, r = P.r;
   Ctl C{P.timeout_ns, P.err, &S.abort};
@@ -938,16 +934,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       for (int m = 0; m < PER; m++) {
         const int i = ct + m * kDecConsumers;
         if (i < D && !ab) {
-          const float xv = bf(d2bf_bits(hv[m] * (double)bf(gam[i]) * rinv));
-          S.xt[xt_index(i, NCH)] = xv * nib_scale(i & 7);
+          const uint16_t xb = d2bf_bits(hv[m] * (double)bf(gam[i]) * rinv);
+          S.xt[xt_index(i, NCH)] = bf(xb);
+          S.xp[pair_index(i)] = xb;
         }
       }
       cbar();
-      // the chunk sums that every gate/up row of the layer uses with its minima
-      if (!ab && ct < NCH) {
-        float xr[32];
-        load_chunk(S.xt, NCH, ct, xr);
-        S.xsum[ct] = chunk_raw_sum(xr);
+      // the group sums that every gate/up row of the layer uses with its minima
+      #pragma unroll 1
+      for (int G = warp; G < D / 64 && !ab; G += kDecCW) {
+        const float v = warp_sum(bf(S.xp[pair_index(64 * G + lane)]) + bf(S.xp[pair_index(64 * G + 32 + lane)]));
+        if (lane == 0) S.xg[G] = v;
       }
       cbar();
       if (ct == 0) stamp(P, l, TR_NORM);
@@ -988,77 +985,90 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (lane == 0) st_tag(dst, tag, __float_as_uint(v));
       }
     } else if (it.kind == IT_GU) {
-      // ---- gate/up: a warp takes whole units (the gate row and the up row of one
-      // intermediate index, two independent dot products), applies the SwiGLU and
-      // publishes; RPW units per warp pass when a row needs fewer than 32 lanes
+      // ---- gate/up: a unit is the gate row and the up row of one intermediate index, a
+      // tensor-core row pair (they share x); a warp takes units u and u + kDecCW of each
+      // pass, applies the SwiGLU and publishes
       if (ct == 0) stamp(P, l, TR_GU_FULL);
-      constexpr int LPR = NCH < 32 ? NCH : 32;    // lanes per row
-      constexpr int RPW = 32 / LPR;               // units per warp pass
-      constexpr int CPL = NCH / LPR;              // chunks per lane
-      const int sub = lane / LPR, sl = lane % LPR;
+      constexpr int NG = D / 64, NS = (NG + 7) / 8;   // groups per row, 512-wide steps
+      const int g8 = lane >> 2, t4 = lane & 3;
+      const bool own = t4 == (g8 >> 1);               // this lane holds the diagonal
       const int slot0 = ia / I;
-      if (warp * RPW < in) {
-        float xr[CPL][32];
-        float xsr[CPL];
-#pragma unroll
-        for (int cc = 0; cc < CPL; cc++) {
-          load_chunk(S.xt, NCH, sl + cc * LPR, xr[cc]);
-          xsr[cc] = S.xsum[sl + cc * LPR];
+      // unit u = global unit ia + u: slot es = (ia + u) / I, index i = (ia + u) % I; its
+      // piece p is the slot's order among the item's slots, its row the index minus the
+      // piece's first index
+      struct UnitRows {
+        const uint8_t *gc, *uc;
+        const uint16_t *gs, *gm, *us, *um;
+      };
+      auto unit_rows = [&](int u) {
+        const int gidx = ia + u, es = gidx / I, p = es - slot0;
+        const int i = gidx - es * I, row = i - (p == 0 ? ia - slot0 * I : 0), sg = kGuPiece0 + 6 * p;
+        UnitRows R;
+        R.gc = S.ring + S.seg_off[slot][sg + 0] + (size_t)row * (D / 2);
+        R.gs = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 1]) + (size_t)row * NG;
+        R.gm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 2]) + (size_t)row * NG;
+        R.uc = S.ring + S.seg_off[slot][sg + 3] + (size_t)row * (D / 2);
+        R.us = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 4]) + (size_t)row * NG;
+        R.um = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 5]) + (size_t)row * NG;
+        return R;
+      };
+      auto publish = [&](int u, float ag, float au) {
+        const int gidx = ia + u, es = gidx / I, i = gidx - es * I;
+        if (es == k) {
+          st_tag(blk + k * I + 2 * i, tag, __float_as_uint(ag));
+          st_tag(blk + k * I + 2 * i + 1, tag, __float_as_uint(au));
+        } else {
+          st_tag(blk + es * I + i, tag, f2bf(ag / (1.0f + expf(-ag)) * au));
         }
-        // unit u = global unit ia + u: slot es = (ia + u) / I, index i = (ia + u) % I; its
-        // piece p is the slot's order among the item's slots, its row the index minus the
-        // piece's first index.  Two units per warp pass, so that their four dot products
-        // and reductions interleave.
-        auto partial = [&](int u, float &ag, float &au) {
-          const int gidx = ia + u, es = gidx / I, p = es - slot0;
-          const int i = gidx - es * I, row = i - (p == 0 ? ia - slot0 * I : 0), sg = kGuPiece0 + 6 * p;
-          const uint8_t *gcw = S.ring + S.seg_off[slot][sg + 0] + (size_t)row * (D / 2);
-          const uint16_t *gsc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 1]) + (size_t)row * (D / 64);
-          const uint16_t *gmn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 2]) + (size_t)row * (D / 64);
-          const uint8_t *ucw = S.ring + S.seg_off[slot][sg + 3] + (size_t)row * (D / 2);
-          const uint16_t *usc = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 4]) + (size_t)row * (D / 64);
-          const uint16_t *umn = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][sg + 5]) + (size_t)row * (D / 64);
+      };
+      const uint4 *xw = reinterpret_cast<const uint4 *>(S.xp);
+      #pragma unroll 1
+      for (int u0 = warp; u0 < in; u0 += 2 * kDecCW) {
+        const int u1 = u0 + kDecCW;
+        const bool two = u1 < in;                      // warp-uniform
+        const UnitRows A = unit_rows(u0), B = unit_rows(two ? u1 : u0);
+        float ag0 = 0.f, au0 = 0.f, ag1 = 0.f, au1 = 0.f;
 #pragma unroll
-          for (int cc = 0; cc < CPL; cc++) {
-            const int ch = sl + cc * LPR;
-            const uint4 wg = *reinterpret_cast<const uint4 *>(gcw + ch * 16);
-            const uint4 wu = *reinterpret_cast<const uint4 *>(ucw + ch * 16);
-            const float qg = chunk_qdot(wg, xr[cc]);
-            const float qu = chunk_qdot(wu, xr[cc]);
-            ag = fmaf(bf(gsc[ch >> 1]), qg, fmaf(bf(gmn[ch >> 1]), xsr[cc], ag));
-            au = fmaf(bf(usc[ch >> 1]), qu, fmaf(bf(umn[ch >> 1]), xsr[cc], au));
+        for (int st = 0; st < NS; st++) {
+          // every lane takes part in the MMAs; lanes past the row's last group (rows
+          // shorter than a step) feed zeros and fold nothing
+          const int G = 8 * st + g8;
+          const bool gv = G < NG;
+          const int wi = 64 * st + 8 * g8 + 2 * t4;  // code / activation word of this lane
+          const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+          const uint2 z2 = make_uint2(0u, 0u);
+          const uint4 va = gv ? xw[wi] : z4, vb = gv ? xw[wi + 1] : z4;
+          const float V = gv ? S.xg[G] : 0.f;
+          float d[4];
+          pair_step(d, gv ? ld_code2(A.gc + 4 * wi) : z2, gv ? ld_code2(A.uc + 4 * wi) : z2, va, vb);
+          if (gv) {
+            ag0 += group_fold((g8 & 1) ? d[1] : d[0], A.gs, A.gm, G, V);
+            au0 += group_fold((g8 & 1) ? d[3] : d[2], A.us, A.um, G, V);
           }
-        };
-        auto publish = [&](int u, float ag, float au) {
-          const int gidx = ia + u, es = gidx / I, i = gidx - es * I;
-          if (es == k) {
-            st_tag(blk + k * I + 2 * i, tag, __float_as_uint(ag));
-            st_tag(blk + k * I + 2 * i + 1, tag, __float_as_uint(au));
-          } else {
-            st_tag(blk + es * I + i, tag, f2bf(ag / (1.0f + expf(-ag)) * au));
+          if (two) {
+            pair_step(d, gv ? ld_code2(B.gc + 4 * wi) : z2, gv ? ld_code2(B.uc + 4 * wi) : z2, va, vb);
+            if (gv) {
+              ag1 += group_fold((g8 & 1) ? d[1] : d[0], B.gs, B.gm, G, V);
+              au1 += group_fold((g8 & 1) ? d[3] : d[2], B.us, B.um, G, V);
+            }
           }
-        };
-        #pragma unroll 1
-        for (int base = warp * RPW; base < in; base += 2 * kDecCW * RPW) {
-          const int u0 = base + sub, u1 = base + kDecCW * RPW + sub;
-          const bool v0 = u0 < in, v1 = u1 < in;
-          float ag0 = 0.f, au0 = 0.f, ag1 = 0.f, au1 = 0.f;
-          if (v0) partial(u0, ag0, au0);
-          if (v1) partial(u1, ag1, au1);
-          ag0 = group_sum(ag0, LPR);
-          au0 = group_sum(au0, LPR);
-          ag1 = group_sum(ag1, LPR);
-          au1 = group_sum(au1, LPR);
-          if (sl == 0) {
-            if (v0) publish(u0, ag0, au0);
-            if (v1) publish(u1, ag1, au1);
-          }
+        }
+        ag0 = warp_sum(own ? ag0 : 0.f);
+        au0 = warp_sum(own ? au0 : 0.f);
+        if (two) {
+          ag1 = warp_sum(own ? ag1 : 0.f);
+          au1 = warp_sum(own ? au1 : 0.f);
+        }
+        if (lane == 0) {
+          publish(u0, ag0, au0);
+          if (two) publish(u1, ag1, au1);
         }
       }
       if (ct == 0) stamp(P, l, TR_GU_DONE);
     } else {
       // ---- down + combine ---------------------------------------------------------------
-      float *at = S.at, *gus = S.gus;
+      constexpr int NGI = I / 64, NSI = (NGI + 7) / 8;   // groups per down row, 512-wide steps
+      float *gus = S.gus;
       if (shared_state) {
         // the layer's first down item here: one batched poll over the layer's block (a of
         // the routed slots, the shared expert's raw g/u, t_g/t_u with LoRA, the selected
@@ -1075,11 +1085,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         }
         ab = cbar_or(ab);
         if (!ab) {
-          // routed a values: bf16 payloads -> pre-scaled, chunk-transposed fp32
+          // routed a values: bf16 payloads -> bf16 pairs per slot
 #pragma unroll 1
           for (int i = ct; i < k * I; i += kDecConsumers) {
             const int j = i / I, e = i - j * I;
-            at[j * I + xt_index(e, NCI)] = bf(S.stg[i] & 0xFFFFu) * nib_scale(e & 7);
+            S.ap[j * I + pair_index(e)] = (uint16_t)(S.stg[i] & 0xFFFFu);
           }
           if (ct == 0) stamp(P, l, TR_A_POLL);
           const int sbd = dn_bd(k);
@@ -1107,9 +1117,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
               g = fmaf(P.c, lg, g);
               u = fmaf(P.c, lu, u);
             }
-            const float av = bf(f2bf(g / (1.0f + expf(-g)) * u));
-            S.asraw[i] = av;
-            at[k * I + xt_index(i, NCI)] = av * nib_scale(i & 7);
+            const uint16_t a16 = f2bf(g / (1.0f + expf(-g)) * u);
+            S.asraw[i] = bf(a16);
+            S.ap[k * I + pair_index(i)] = a16;
           }
           if (ct == 0) {
             float lg[kMaxK], mx = -INFINITY, sum = 0.f;
@@ -1128,11 +1138,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           }
         }
         cbar();
-        // the chunk sums that every down row of the layer uses with its minima
-        if (!ab && ct < (k + 1) * NCI) {
-          float ar[32];
-          load_chunk(S.at + (ct / NCI) * I, NCI, ct % NCI, ar);
-          S.asum[ct] = chunk_raw_sum(ar);
+        // the group sums that every down row of the layer uses with its minima
+        #pragma unroll 1
+        for (int G = warp; G < (k + 1) * NGI && !ab; G += kDecCW) {
+          const float v = warp_sum(bf(S.ap[(G / NGI) * I + pair_index((G % NGI) * 64 + lane)]) +
+                                   bf(S.ap[(G / NGI) * I + pair_index((G % NGI) * 64 + 32 + lane)]));
+          if (lane == 0) S.ag[G] = v;
         }
         if (!ab && lora) {
           // t_d = Ad a_s (LoRA down branch)
@@ -1150,78 +1161,72 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (ct == 0) stamp(P, l, TR_TD_POLL);
       }
       if (!ab) {
-        // a warp owns its rows across every expert: each lane accumulates its chunks'
-        // partial dot products in the combine order (routed experts with their gates, then
-        // the shared expert), and the row's lanes are summed once at the end
-        constexpr int LPR = NCI < 32 ? NCI : 32;
-        constexpr int RPW = 32 / LPR;
-        constexpr int CPL = NCI / LPR;
-        constexpr int PM = kDnMaxRows / (kDecCW * RPW) + 1;
-        const int sub = lane / LPR, sl = lane % LPR;
-        float y[PM];
+        // a warp takes rows 4 w .. 4 w + 3 of each pass as two tensor-core row pairs and
+        // owns them across every expert slot: per slot one step per 512 columns, its fold
+        // accumulated per lane in the combine order (routed experts with their gates, then
+        // the shared expert); the rows' lanes are summed once at the end
+        const int g8 = lane >> 2, t4 = lane & 3;
+        const bool own = t4 == (g8 >> 1);
+        const uint4 *aw = reinterpret_cast<const uint4 *>(S.ap);
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        const uint2 z2 = make_uint2(0u, 0u);
+        #pragma unroll 1
+        for (int r0 = 4 * warp; r0 < in; r0 += 4 * kDecCW) {
+          const bool pair2 = r0 + 2 < in;             // warp-uniform
+          bool rv[4];
 #pragma unroll
-        for (int pp = 0; pp < PM; pp++) y[pp] = 0.f;
-        if (warp * RPW < in) {
+          for (int q4 = 0; q4 < 4; q4++) rv[q4] = r0 + q4 < in;
+          float y4[4] = {0.f, 0.f, 0.f, 0.f};
           #pragma unroll 1
           for (int j = 0; j <= k; j++) {
-            float ar[CPL][32];
-            float asr[CPL];
-#pragma unroll
-            for (int cc = 0; cc < CPL; cc++) {
-              load_chunk(S.at + j * I, NCI, sl + cc * LPR, ar[cc]);
-              asr[cc] = S.asum[j * NCI + sl + cc * LPR];
-            }
             const float gj = j < k ? S.gates[j] : 1.f;
             const uint8_t *cb = S.ring + S.seg_off[slot][3 * j];
             const uint16_t *sb = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3 * j + 1]);
             const uint16_t *mb = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][3 * j + 2]);
+            float f4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int pp = 0; pp < PM; pp++) {
-              const int row = pp * kDecCW * RPW + warp * RPW + sub;
-              if (row < in) {
-                const uint8_t *cw = cb + (size_t)row * (I / 2);
-                const uint16_t *sc = sb + (size_t)row * (I / 64);
-                const uint16_t *mn = mb + (size_t)row * (I / 64);
-                float acc = 0.f;
+            for (int st = 0; st < NSI; st++) {
+              // every lane takes part in the MMAs; lanes past the row's last group feed
+              // zeros and fold nothing
+              const int G = 8 * st + g8;
+              const bool gv = G < NGI;
+              const int wi = 64 * st + 8 * g8 + 2 * t4;
+              const uint4 va = gv ? aw[j * (I / 8) + wi] : z4, vb = gv ? aw[j * (I / 8) + wi + 1] : z4;
+              const float V = gv ? S.ag[j * NGI + G] : 0.f;
+              float d[4];
 #pragma unroll
-                for (int cc = 0; cc < CPL; cc++) {
-                  const int ch = sl + cc * LPR;
-                  const uint4 w = *reinterpret_cast<const uint4 *>(cw + ch * 16);
-                  const float qd = chunk_qdot(w, ar[cc]);
-                  acc = fmaf(bf(sc[ch >> 1]), qd, fmaf(bf(mn[ch >> 1]), asr[cc], acc));
-                }
-                y[pp] = j < k ? fmaf(gj, acc, y[pp]) : y[pp] + acc;
+              for (int h = 0; h < 2; h++) {
+                if (h == 1 && !pair2) break;
+                const int ra = r0 + 2 * h, rb = ra + 1;
+                const bool va_ok = gv && rv[2 * h], vb_ok = gv && rv[2 * h + 1];
+                pair_step(d, va_ok ? ld_code2(cb + (size_t)ra * (I / 2) + 4 * wi) : z2,
+                          vb_ok ? ld_code2(cb + (size_t)rb * (I / 2) + 4 * wi) : z2, va, vb);
+                if (va_ok) f4[2 * h] += group_fold((g8 & 1) ? d[1] : d[0], sb + (size_t)ra * NGI, mb + (size_t)ra * NGI, G, V);
+                if (vb_ok) f4[2 * h + 1] += group_fold((g8 & 1) ? d[3] : d[2], sb + (size_t)rb * NGI, mb + (size_t)rb * NGI, G, V);
               }
             }
-          }
-          // the shared expert's LoRA down branch c * (Bd t_d) of the row, its r terms
-          // spread over the row's lanes
-          if (lora) {
-            const uint16_t *bd = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]);
 #pragma unroll
-            for (int pp = 0; pp < PM; pp++) {
-              const int row = pp * kDecCW * RPW + warp * RPW + sub;
-              if (row < in) {
-                float lo = 0.f;
-                #pragma unroll 1
-                for (int j = sl; j < r; j += LPR) lo = fmaf(bf(bd[row * r + j]), S.td[j], lo);
-                y[pp] = fmaf(P.c, lo, y[pp]);
-              }
+            for (int q4 = 0; q4 < 4; q4++) y4[q4] = j < k ? fmaf(gj, f4[q4], y4[q4]) : y4[q4] + f4[q4];
+          }
+          // the shared expert's LoRA down branch c * (Bd t_d) of each row, its r terms
+          // spread over the lanes, then one warp sum per row
+          const uint16_t *bd = lora ? reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]) : nullptr;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; q4++) {
+            if (q4 >= 2 && !pair2) break;
+            float v = own ? y4[q4] : 0.f;
+            if (lora && rv[q4]) {
+              float lo = 0.f;
+              #pragma unroll 1
+              for (int jj = lane; jj < r; jj += 32) lo = fmaf(bf(bd[(r0 + q4) * r + jj]), S.td[jj], lo);
+              v = fmaf(P.c, lo, v);
             }
-          }
-          // one reduction per row, over the lanes' partial sums
-#pragma unroll
-          for (int pp = 0; pp < PM; pp++)
-            if (pp * kDecCW * RPW + warp * RPW < in) y[pp] = group_sum(y[pp], LPR);   // warp-uniform
-#pragma unroll
-          for (int pp = 0; pp < PM; pp++) {
-            const int row = pp * kDecCW * RPW + warp * RPW + sub;
-            if (row < in && sl == 0) {
-              const float yv = y[pp];
-              const int n = ia + row;
-              st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(yv));
-              P.y[(size_t)l * D + n] = f2bf(yv);
-              if (P.yf) P.yf[(size_t)l * D + n] = yv;
+            v = warp_sum(v);
+            if (lane == 0 && rv[q4]) {
+              const int n = ia + r0 + q4;
+              st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(v));
+              P.y[(size_t)l * D + n] = f2bf(v);
+              if (P.yf) P.yf[(size_t)l * D + n] = v;
             }
           }
         }
