@@ -26,6 +26,7 @@
 //     intermediate rows of the gate/up phase and the d output rows of the down phase.
 #pragma once
 #include <algorithm>
+#include <vector>
 #include "e0_device.cuh"
 #include "e0_kernels.cuh"
 
@@ -450,6 +451,54 @@ inline int sched_xrows(const SchedShape &Z, bool step0, int l) {
   return (Z.head[l] ? Z.E : 0) + (Z.lora[l] ? 2 * Z.r : 0) + (sched_predicted(Z, step0, l) ? Z.k : 0);
 }
 
+// Cuts of one phase's unit list (the units of every layer, in layer order) into G
+// contiguous shares of about equal cost: a share costs `per_unit` for each unit plus
+// `per_seg` (and extra[l]) for each layer it touches (a norm, a top-k, the shared-expert
+// inputs of a layer's first down item: work a CTA does once per layer it touches).  The
+// smallest share bound that the greedy cut fits into G shares, found by bisection.
+// cuts[0] = 0, cuts[G] = the phase's unit count.
+inline void balanced_cuts(const int *units, const double *extra, int L, int G, double per_unit, double per_seg,
+                          long long *cuts) {
+  long long tot = 0;
+  for (int l = 0; l < L; l++) tot += units[l];
+  // greedy: each share takes as many units as fit under the bound; true if G shares hold
+  // every unit (when writing, the last share takes whatever is left)
+  auto greedy = [&](double bound, bool write) {
+    long long pos = 0;
+    for (int c = 0; c < G; c++) {
+      if (write) cuts[c] = pos;
+      if (pos >= tot) continue;
+      if (write && c == G - 1) { pos = tot; break; }
+      double rem = bound;
+      long long base = 0;
+      int l = 0;
+      while (l < L && base + units[l] <= pos) base += units[l++];
+      while (l < L && pos < tot) {
+        if (units[l] == 0) { l++; continue; }
+        rem -= per_seg + (extra ? extra[l] : 0.0);
+        if (rem < per_unit) break;
+        const long long left = base + units[l] - pos;
+        const long long take = std::min(left, (long long)(rem / per_unit));
+        pos += take;
+        rem -= take * per_unit;
+        if (take < left) break;
+        base += units[l++];
+      }
+    }
+    if (write) cuts[G] = tot;
+    return pos >= tot;
+  };
+  double lo = 0.0, hi = tot * per_unit + (L + 1) * per_seg + 1.0;
+  if (extra)
+    for (int l = 0; l < L; l++) hi += extra[l];
+  for (int it = 0; it < 60; it++) {
+    const double mid = 0.5 * (lo + hi);
+    if (greedy(mid, false)) hi = mid;
+    else lo = mid;
+  }
+  greedy(hi, true);
+}
+
 // CTA c's items into out[0, kMaxItems); returns their count, or -1 if they do not fit.
 inline int build_items(const SchedShape &Z, bool flat, bool step0, int c, unsigned long long *out) {
   const int G = Z.G, L = Z.L, k = Z.k, D = Z.D, I = Z.I;
@@ -488,11 +537,20 @@ inline int build_items(const SchedShape &Z, bool flat, bool step0, int c, unsign
       return which == 0 ? (sched_predicted(Z, step0, l) ? 0 : Z.E)
            : which == 1 ? sched_xrows(Z, step0, l) : which == 2 ? (k + 1) * I : D;
     };
-    // one phase: units(l) per layer over every layer with units, this CTA's share
-    auto phase = [&](int kind, int chunk, int which) {
-      long long tot = 0;
-      for (int l = 0; l < L; l++) tot += units(which, l);
-      const long long lo = tot * c / G, hi = tot * (c + 1) / G;
+    // one phase: units(l) per layer over every layer with units, this CTA's share of a
+    // cost-balanced cut.  Costs in microseconds on B200: a unit's bytes at the consumers'
+    // rate, and the work done once per layer a share touches (the norm for x phases, the
+    // top-k of a reactive layer before the gate/up phase, the down inputs of a layer)
+    auto phase = [&](int kind, int chunk, int which, double per_unit, double per_seg, bool tk_extra) {
+      int u_l[64];
+      double e_l[64];
+      for (int l = 0; l < L; l++) {
+        u_l[l] = units(which, l);
+        e_l[l] = tk_extra && !sched_predicted(Z, step0, l) ? 2.7 : 0.0;
+      }
+      std::vector<long long> cuts(G + 1);
+      balanced_cuts(u_l, e_l, L, G, per_unit, per_seg, cuts.data());
+      const long long lo = cuts[c], hi = cuts[c + 1];
       long long base = 0;
       for (int l = 0; l < L; l++) {
         const int u = units(which, l);
@@ -501,11 +559,11 @@ inline int build_items(const SchedShape &Z, bool flat, bool step0, int c, unsign
         base += u;
       }
     };
-    phase(IT_R, 9, 0);
-    phase(IT_XR, xr_chunk, 1);
+    phase(IT_R, 9, 0, 0.10, 2.0, false);
+    phase(IT_XR, xr_chunk, 1, 0.15, 2.2, false);
     const int n_before_tk = n;
-    phase(IT_GU, gu_chunk, 2);
-    phase(IT_DN, dn_chunk, 3);
+    phase(IT_GU, gu_chunk, 2, 0.09, 2.6, true);
+    phase(IT_DN, dn_chunk, 3, 0.095, 10.0, false);
     // the top-k items go before the gate/up phase: the reactive layers that this CTA's
     // gate/up or down items touch
     bool need[64] = {};
