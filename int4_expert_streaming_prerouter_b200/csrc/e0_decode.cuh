@@ -455,10 +455,11 @@ inline int sched_xrows(const SchedShape &Z, bool step0, int l) {
 // contiguous shares of about equal cost: a share costs `per_unit` for each unit plus
 // `per_seg` (and extra[l]) for each layer it touches (a norm, a top-k, the shared-expert
 // inputs of a layer's first down item: work a CTA does once per layer it touches).  The
-// smallest share bound that the greedy cut fits into G shares, found by bisection.
+// smallest share bound that the greedy cut fits into G shares, found by bisection; share
+// c also carries start[c], the cost of what its CTA does before this phase (nullptr: 0).
 // cuts[0] = 0, cuts[G] = the phase's unit count.
 inline void balanced_cuts(const int *units, const double *extra, int L, int G, double per_unit, double per_seg,
-                          long long *cuts) {
+                          const double *start, long long *cuts) {
   long long tot = 0;
   for (int l = 0; l < L; l++) tot += units[l];
   // greedy: each share takes as many units as fit under the bound; true if G shares hold
@@ -469,7 +470,7 @@ inline void balanced_cuts(const int *units, const double *extra, int L, int G, d
       if (write) cuts[c] = pos;
       if (pos >= tot) continue;
       if (write && c == G - 1) { pos = tot; break; }
-      double rem = bound;
+      double rem = bound - (start ? start[c] : 0.0);
       long long base = 0;
       int l = 0;
       while (l < L && base + units[l] <= pos) base += units[l++];
@@ -491,12 +492,27 @@ inline void balanced_cuts(const int *units, const double *extra, int L, int G, d
   double lo = 0.0, hi = tot * per_unit + (L + 1) * per_seg + 1.0;
   if (extra)
     for (int l = 0; l < L; l++) hi += extra[l];
+  if (start)
+    for (int c = 0; c < G; c++) hi = std::max(hi, start[c] + tot * per_unit + (L + 1) * per_seg + 1.0);
   for (int it = 0; it < 60; it++) {
     const double mid = 0.5 * (lo + hi);
     if (greedy(mid, false)) hi = mid;
     else lo = mid;
   }
   greedy(hi, true);
+}
+
+// The cost of units [lo, hi) of a phase under the same model.
+inline double share_cost(const int *units, const double *extra, int L, double per_unit, double per_seg, long long lo,
+                         long long hi) {
+  double cost = 0.0;
+  long long base = 0;
+  for (int l = 0; l < L; l++) {
+    const long long s0 = std::max(lo, base), s1 = std::min(hi, base + units[l]);
+    if (s1 > s0) cost += (s1 - s0) * per_unit + per_seg + (extra ? extra[l] : 0.0);
+    base += units[l];
+  }
+  return cost;
 }
 
 // CTA c's items into out[0, kMaxItems); returns their count, or -1 if they do not fit.
@@ -537,33 +553,44 @@ inline int build_items(const SchedShape &Z, bool flat, bool step0, int c, unsign
       return which == 0 ? (sched_predicted(Z, step0, l) ? 0 : Z.E)
            : which == 1 ? sched_xrows(Z, step0, l) : which == 2 ? (k + 1) * I : D;
     };
-    // one phase: units(l) per layer over every layer with units, this CTA's share of a
+    // each phase: units(l) per layer over every layer with units, this CTA's share of a
     // cost-balanced cut.  Costs in microseconds on B200: a unit's bytes at the consumers'
     // rate, and the work done once per layer a share touches (the norm for x phases, the
-    // top-k of a reactive layer before the gate/up phase, the down inputs of a layer)
-    auto phase = [&](int kind, int chunk, int which, double per_unit, double per_seg, bool tk_extra) {
+    // top-k of a reactive layer before the gate/up phase, the down inputs of a layer).
+    // The gate/up cut also balances what each CTA does before it (its router and x-row
+    // shares), so that the CTAs finish the gate/up phase, which the down phase waits
+    // for, together.
+    struct PhaseCost { int kind, chunk, which; double per_unit, per_seg; bool tk; };
+    const PhaseCost ph[4] = {{IT_R, 9, 0, 0.10, 2.0, false},
+                             {IT_XR, xr_chunk, 1, 0.15, 2.2, false},
+                             {IT_GU, gu_chunk, 2, 0.09, 2.6, true},
+                             {IT_DN, dn_chunk, 3, 0.095, 10.0, false}};
+    std::vector<double> before(G, 0.0);
+    std::vector<long long> cuts(G + 1);
+    int n_before_tk = 0;
+    for (int f = 0; f < 4; f++) {
       int u_l[64];
       double e_l[64];
       for (int l = 0; l < L; l++) {
-        u_l[l] = units(which, l);
-        e_l[l] = tk_extra && !sched_predicted(Z, step0, l) ? 2.7 : 0.0;
+        u_l[l] = units(ph[f].which, l);
+        e_l[l] = ph[f].tk && !sched_predicted(Z, step0, l) ? 2.7 : 0.0;
       }
-      std::vector<long long> cuts(G + 1);
-      balanced_cuts(u_l, e_l, L, G, per_unit, per_seg, cuts.data());
+      balanced_cuts(u_l, e_l, L, G, ph[f].per_unit, ph[f].per_seg, ph[f].kind == IT_GU ? before.data() : nullptr,
+                    cuts.data());
+      if (ph[f].kind == IT_R || ph[f].kind == IT_XR)
+        for (int cc = 0; cc < G; cc++)
+          before[cc] += share_cost(u_l, e_l, L, ph[f].per_unit, ph[f].per_seg, cuts[cc], cuts[cc + 1]);
+      if (ph[f].kind == IT_GU) n_before_tk = n;
       const long long lo = cuts[c], hi = cuts[c + 1];
       long long base = 0;
       for (int l = 0; l < L; l++) {
-        const int u = units(which, l);
+        const int u = u_l[l];
         const long long s0 = std::max(lo, base), s1 = std::min(hi, base + u);
-        for (long long a = s0; a < s1; a += chunk) put(kind, l, (int)(a - base), (int)std::min((long long)chunk, s1 - a));
+        for (long long a = s0; a < s1; a += ph[f].chunk)
+          put(ph[f].kind, l, (int)(a - base), (int)std::min((long long)ph[f].chunk, s1 - a));
         base += u;
       }
-    };
-    phase(IT_R, 9, 0, 0.10, 2.0, false);
-    phase(IT_XR, xr_chunk, 1, 0.15, 2.2, false);
-    const int n_before_tk = n;
-    phase(IT_GU, gu_chunk, 2, 0.09, 2.6, true);
-    phase(IT_DN, dn_chunk, 3, 0.095, 10.0, false);
+    }
     // the top-k items go before the gate/up phase: the reactive layers that this CTA's
     // gate/up or down items touch
     bool need[64] = {};
