@@ -32,7 +32,7 @@
 
 namespace e0 {
 
-constexpr int kDecCW = 12;                // consumer warps
+constexpr int kDecCW = 11;                // consumer warps (three warps per SM sub-partition with the producer: 168 registers each)
 constexpr int kDecConsumers = 32 * kDecCW;
 constexpr int kDecThreads = 32 + kDecConsumers;   // + 1 producer warp
 constexpr int kRingBytes = 174 * 1024;
@@ -158,13 +158,6 @@ __host__ __device__ __forceinline__ void split_range(int N, int G, int c, int &a
   b = (int)((unsigned)(N * (c + 1)) / (unsigned)G);
 }
 
-// x for the bf16 rows lives in shared memory "chunk-transposed": element e of a row of
-// n16 chunks (32 elements each) sits at float index
-// (((e & 31) >> 2) * n16 + (e >> 5)) * 4 + (e & 3), so that the lanes of a warp read their
-// elements with conflict-free 16-byte loads.
-__host__ __device__ __forceinline__ int xt_index(int e, int n16) {
-  return ((((e & 31) >> 2) * n16) + (e >> 5)) * 4 + (e & 3);
-}
 
 // ---------------------------------------------------------------------------------------
 // Tensor-core dot products of int4 rows with one activation vector (gate/up and down).
@@ -373,7 +366,7 @@ __device__ __forceinline__ void item_seg(const DecodeParams &P, const DecLayer &
 template <int D, int I>
 struct DecSmem {
   uint8_t ring[kRingBytes];
-  float xt[D];                       // x (fp32), chunk-transposed (for the bf16 rows)
+  alignas(16) uint16_t xn[D];        // x as bf16, natural order (for the bf16 rows)
   union {                            // used by different items, never at the same time:
     float yprev[D];                  //   the previous layer's y (fp32), in order + chained
     uint32_t stg[kDecMaxK * I];      //   routed a payloads as polled (a layer's first down item)
@@ -789,7 +782,7 @@ struct Range {
 // one L2 round trip; a word whose tag is stale is re-polled on the slow path.  Out of line
 // so that one copy of this code serves every call site.
 __device__ __noinline__ bool poll_ranges(const Range *rg, int nr, uint32_t tag, int tid, const Ctl &C) {
-  constexpr int W = 8;
+  constexpr int W = 10;   // a layer's down inputs (about 3,100 words at d = 2048) in one batch
   int total = 0;
 #pragma unroll 1
   for (int q = 0; q < nr; q++) total += rg[q].n;
@@ -857,27 +850,26 @@ __device__ __forceinline__ bool wait_full(uint64_t *bar, uint32_t par, const Ctl
   return true;
 }
 
-// bf16 row (D elements in shared memory) dotted with x, read from its chunk-transposed
-// fp32 copy xt (elements 8c..8c+3 and 8c+4..8c+7 are two float4 there): one warp.
+// Two bf16 rows r0, r1 (D elements each, in shared memory) dotted with x (bf16, natural
+// order), on the tensor cores: one warp.  Per MMA, lane (g, t) holds elements
+// 128 s + 16 g + 4 t .. + 3 of both rows and of x, so that MMA row g (g + 8) is row r0 (r1)
+// restricted to chunk g of the 128 and column g is x restricted to it; the diagonal
+// entries accumulate each row's chunk sums over the steps, and the lanes that hold them
+// (t = g / 2) are summed at the end.  No scale folds: the rows are plain bf16.
 template <int D>
-__device__ __noinline__ float bf16_row_x(const uint16_t *w, const float *xt, int lane) {
-  constexpr int NCH = D / 32;
-  float acc = 0.f;
-#pragma unroll 2
-  for (int ch = lane; ch < D / 8; ch += 32) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(w + ch * 8);
-    const float4 a = *reinterpret_cast<const float4 *>(xt + ((2 * (ch & 3)) * NCH + (ch >> 2)) * 4);
-    const float4 b = *reinterpret_cast<const float4 *>(xt + ((2 * (ch & 3) + 1) * NCH + (ch >> 2)) * 4);
-    acc = fmaf(bf(v.x & 0xFFFFu), a.x, acc);
-    acc = fmaf(bf(v.x >> 16), a.y, acc);
-    acc = fmaf(bf(v.y & 0xFFFFu), a.z, acc);
-    acc = fmaf(bf(v.y >> 16), a.w, acc);
-    acc = fmaf(bf(v.z & 0xFFFFu), b.x, acc);
-    acc = fmaf(bf(v.z >> 16), b.y, acc);
-    acc = fmaf(bf(v.w & 0xFFFFu), b.z, acc);
-    acc = fmaf(bf(v.w >> 16), b.w, acc);
+__device__ __noinline__ float2 bf16_pair_x(const uint16_t *r0, const uint16_t *r1, const uint16_t *xn, int lane) {
+  const int g8 = lane >> 2, t4 = lane & 3;
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int s = 0; s < D / 128; s++) {
+    const int k0 = 128 * s + 16 * g8 + 4 * t4;
+    const uint2 a = *reinterpret_cast<const uint2 *>(r0 + k0);
+    const uint2 b = *reinterpret_cast<const uint2 *>(r1 + k0);
+    const uint2 x = *reinterpret_cast<const uint2 *>(xn + k0);
+    mma_bf16_16816(d, a.x, b.x, a.y, b.y, x.x, x.y);
   }
-  return warp_sum(acc);
+  const bool own = t4 == (g8 >> 1);
+  return make_float2(warp_sum(own ? ((g8 & 1) ? d[1] : d[0]) : 0.f), warp_sum(own ? ((g8 & 1) ? d[3] : d[2]) : 0.f));
 }
 
 __device__ __noinline__ void warp_topk_ool(const float *v, int E, int k, int lane, int *out) {
@@ -922,7 +914,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     return;
   }
   // ------------------------------- consumers -------------------------------------------
-  constexpr int NCH = D / 32;                  // 16-byte code chunks per gate/up row
   const int ct = tid - 32, warp = ct >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = P.G, k = P.k, r = P.r;
   Ctl C{P.timeout_ns, P.err, &S.abort};
@@ -1020,7 +1011,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         const int i = ct + m * kDecConsumers;
         if (i < D && !ab) {
           const uint16_t xb = d2bf_bits(hv[m] * (double)bf(gam[i]) * rinv);
-          S.xt[xt_index(i, NCH)] = bf(xb);
+          S.xn[i] = xb;
           S.xp[pair_index(i)] = xb;
         }
       }
@@ -1037,21 +1028,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     if (ab) {
       // nothing more for this item (the barriers above are the same for every thread)
     } else if (it.kind == IT_R) {
-      // ---- router rows of a reactive layer, one warp per row
+      // ---- router rows of a reactive layer, two rows per warp
       const uint16_t *rw = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][2]);
       #pragma unroll 1
-      for (int q2 = warp; q2 < in; q2 += kDecCW) {
-        const float v = bf16_row_x<D>(rw + (size_t)q2 * D, S.xt, lane);
-        if (lane == 0) st_tag(P.t_rlog + (size_t)l * P.E + ia + q2, tag, __float_as_uint(v));
+      for (int q2 = 2 * warp; q2 < in; q2 += 2 * kDecCW) {
+        const bool two = q2 + 1 < in;                  // warp-uniform
+        const float2 v = bf16_pair_x<D>(rw + (size_t)q2 * D, rw + (size_t)(two ? q2 + 1 : q2) * D, S.xn, lane);
+        if (lane == 0) {
+          st_tag(P.t_rlog + (size_t)l * P.E + ia + q2, tag, __float_as_uint(v.x));
+          if (two) st_tag(P.t_rlog + (size_t)l * P.E + ia + q2 + 1, tag, __float_as_uint(v.y));
+        }
       }
     } else if (it.kind == IT_XR) {
-      // ---- head rows, LoRA A rows and the predicted experts' router rows on x
+      // ---- head rows, LoRA A rows and the predicted experts' router rows on x, two rows
+      // per warp
       const int nh = Y.head ? P.E : 0, nl = lora ? r : 0;
-      #pragma unroll 1
-      for (int q2 = warp; q2 < in; q2 += kDecCW) {
+      auto xr_row = [&](int q2, const uint16_t *&row, unsigned long long *&dst) {
         const int u = ia + q2;
-        const uint16_t *row;
-        unsigned long long *dst;
         if (u < nh) {
           row = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kXrHead]) + (size_t)(u - ia) * P.ldh;
           dst = P.t_hlog + (size_t)l * P.E + u;
@@ -1066,8 +1059,19 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           row = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][kXrSel + u - max(ia, nh + 2 * nl)]);
           dst = blk + (k + 2) * I + 2 * r + (u - nh - 2 * nl);
         }
-        const float v = bf16_row_x<D>(row, S.xt, lane);
-        if (lane == 0) st_tag(dst, tag, __float_as_uint(v));
+      };
+      #pragma unroll 1
+      for (int q2 = 2 * warp; q2 < in; q2 += 2 * kDecCW) {
+        const bool two = q2 + 1 < in;                  // warp-uniform
+        const uint16_t *row0, *row1;
+        unsigned long long *dst0, *dst1;
+        xr_row(q2, row0, dst0);
+        xr_row(two ? q2 + 1 : q2, row1, dst1);
+        const float2 v = bf16_pair_x<D>(row0, row1, S.xn, lane);
+        if (lane == 0) {
+          st_tag(dst0, tag, __float_as_uint(v.x));
+          if (two) st_tag(dst1, tag, __float_as_uint(v.y));
+        }
       }
     } else if (it.kind == IT_GU) {
       // ---- gate/up: a unit is the gate row and the up row of one intermediate index, a
@@ -1233,13 +1237,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (!ab && lora) {
           // t_d = Ad a_s (LoRA down branch)
           const uint16_t *adm = reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k) + 3]);
+          // one half-warp per row (r is a multiple of 8, so a warp's two rows are both in or
+          // both out), four independent partial sums per lane
+          const int hw = ct >> 4, h16 = ct & 15;
           #pragma unroll 1
-          for (int j = warp; j < r; j += kDecCW) {
-            float acc = 0.f;
-            #pragma unroll 1
-            for (int i = lane; i < I; i += 32) acc = fmaf(bf(adm[j * I + i]), S.asraw[i], acc);
-            acc = warp_sum(acc);
-            if (lane == 0) S.td[j] = acc;
+          for (int j = hw; j < r; j += 2 * kDecCW) {
+            float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int i = h16; i < I; i += 16) acc4[(i >> 4) & 3] = fmaf(bf(adm[j * I + i]), S.asraw[i], acc4[(i >> 4) & 3]);
+            const float acc = group_sum((acc4[0] + acc4[1]) + (acc4[2] + acc4[3]), 16);
+            if (h16 == 0) S.td[j] = acc;
           }
         }
         cbar();
