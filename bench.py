@@ -40,8 +40,8 @@ METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, valid only
 # while the kernel source is the one captured (sha256 prefix of the file); see profiles/.
 KERNEL_TRAFFIC = {
-    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "616f850e44047cee", 421.9e6,
-                      "4-layer capture (42.19 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
+    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "bb5f70878b8b2649", 409.9e6,
+                      "4-layer capture (40.99 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
                       "bytes to the 40-layer launch"),
     "prefill_t4096_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh", "12341c74281dd957", 343.6e6,
                           "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 465.8 MB, "
