@@ -249,17 +249,35 @@ int e0_debug_decode_trace(e0_ctx *ctx, unsigned long long *buf);
 int e0_debug_force_general(e0_ctx *ctx, int on);
 /* Schedule of the one-launch decode kernel on unchained steps (every layer's input
  * given, none read from another layer's output): 1 (default) = flat — each phase's work
- * (reactive routers, x rows, gate/up, down) over all layers is one list split evenly and
- * contiguously across the CTAs, so that a CTA streams long runs of one or two layers and
- * waits on other CTAs only between phases; 0 = layers in order, every CTA on a share of
- * each layer.  Chained steps always run in order.  Results are bit-identical under both.
- * E0_ERR_INVALID_ARG unless 0 or 1. */
+ * (reactive routers, x rows, gate/up, down) over all layers is one list cut into
+ * contiguous cost-balanced shares across the CTAs, so that a CTA streams long runs of one
+ * or two layers and waits on other CTAs only between phases; 0 = layers in order, every
+ * CTA on a share of each layer.  Chained steps always run in order.  Results are
+ * bit-identical under both.  E0_ERR_INVALID_ARG unless 0 or 1. */
 int e0_debug_decode_flat(e0_ctx *ctx, int on);
 /* Profiling: on = 1 brackets every tensor-core expert-GEMM launch (prefill) with a CUDA
  * event pair on its stream; e0_get_stats then reports their count and summed duration
  * (gemm_timed, gemm_ms; it synchronises on the events).  on = 0 stops it.  The pages
  * have no counterpart; for the benchmark's per-kernel roofline. */
 int e0_debug_time_gemm(e0_ctx *ctx, int on);
+/* The work-item list of one CTA of the one-launch decode kernel, built by the same host
+ * function the context uses (host only: no context, no device call).  For a model of
+ * n_layers layers of shape `dims` whose layer l carries a prerouter head where
+ * has_head[l] != 0 and the shared expert's LoRA where has_lora[l] != 0, on a grid of
+ * n_ctas CTAs, under the flat (flat = 1) or in-order (0) schedule, for a sequence's first
+ * step (step0 = 1: every layer routes with its own router) or a later one, fills
+ * items_out[0, *n_out) with CTA `cta`'s list in execution order.  Item word: bits 0-3
+ * kind (0 router rows of a reactive layer, 1 its top-k, 2 x rows, 3 gate/up units,
+ * 4 down rows), bit 4 set on the first item of its kind group (x items: R, XR, GU) for its
+ * layer in this list, bits 8-15 layer, bits 16-39 first unit, bits 40-63 unit count.
+ * Units of a layer: router rows 0..E-1; x rows = the head's E rows, then 2r LoRA A rows
+ * (A_g, A_u), then the k router rows of a predicted layer's experts; gate/up = (slot,
+ * index) slot-major over k+1 slots of d_ff; down = d_model output rows.  The caller owns
+ * items_out (cap entries).  E0_ERR_INVALID_ARG on NULL pointers, n_layers outside 1..64,
+ * n_ctas < 1, cta outside [0, n_ctas), dims the kernel cannot take, or a longer list
+ * than cap. */
+int e0_decode_items(const e0_dims *dims, int n_layers, const uint8_t *has_head, const uint8_t *has_lora, int n_ctas,
+                    int flat, int step0, int cta, uint64_t *items_out, int cap, int *n_out);
 
 /* Message of the last failing call on this host thread ("" if none). */
 const char *e0_last_error(void);

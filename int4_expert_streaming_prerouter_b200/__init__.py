@@ -85,6 +85,8 @@ _SIGS = {
     "e0_debug_decode_mode": (_I, [_P, _I]),
     "e0_debug_decode_flat": (_I, [_P, _I]),
     "e0_debug_time_gemm": (_I, [_P, _I]),
+    "e0_decode_items": (_I, [ctypes.POINTER(Dims), _I, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_uint8),
+                             _I, _I, _I, _I, ctypes.POINTER(ctypes.c_uint64), _I, ctypes.POINTER(_I)]),
 }
 
 
@@ -124,6 +126,20 @@ def _stream(stream) -> int:
 
 def make_dims(d, E, I, k, r, head_hidden=0, head_onehot=0, eps=1e-6, lora_scale=1.0) -> Dims:
     return Dims(d, E, I, k, 64, r, head_hidden, head_onehot, eps, lora_scale)
+
+
+def decode_items(dims: Dims, n_layers: int, has_head, has_lora, n_ctas: int, flat: bool, step0: bool, cta: int):
+    """The one-launch decode kernel's work-item list of CTA `cta` (host only; see the C
+    header): a list of (kind, first, layer, first_unit, n_units) with kind 0 router rows,
+    1 top-k, 2 x rows, 3 gate/up units, 4 down rows."""
+    cap = 512
+    out = (ctypes.c_uint64 * cap)()
+    n = ctypes.c_int(0)
+    hh = (ctypes.c_uint8 * n_layers)(*[1 if v else 0 for v in has_head])
+    hl = (ctypes.c_uint8 * n_layers)(*[1 if v else 0 for v in has_lora])
+    _check(lib().e0_decode_items(ctypes.byref(dims), n_layers, hh, hl, n_ctas, int(flat), int(step0), cta, out, cap,
+                                 ctypes.byref(n)))
+    return [(w & 15, (w >> 4) & 1, (w >> 8) & 255, (w >> 16) & 0xFFFFFF, w >> 40) for w in out[:n.value]]
 
 
 def moe_layer_forward_noalloc(dims: Dims, layer: dict, h, route_idx=None, y=None, y_f32=None, idx=None,

@@ -1200,6 +1200,31 @@ extern "C" int e0_debug_decode_flat(e0_ctx *C, int on) {
   return E0_OK;
 }
 
+// The one-launch decode kernel's item list of one CTA, built by the same host function
+// that the context uses (no device call).
+extern "C" int e0_decode_items(const e0_dims *dims, int n_layers, const uint8_t *has_head, const uint8_t *has_lora,
+                               int n_ctas, int flat, int step0, int cta, uint64_t *items_out, int cap, int *n_out) {
+  if (!dims || !has_head || !has_lora || !items_out || !n_out || n_layers < 1 || n_layers > 64 || n_ctas < 1 ||
+      cta < 0 || cta >= n_ctas || cap < 0 || dims->d_model < 64 || dims->d_model % 64 || dims->d_ff < 64 ||
+      dims->d_ff % 64 || dims->n_experts < 1 || dims->top_k < 1 || dims->top_k > kMaxK || dims->lora_rank < 0)
+    return fail(E0_ERR_INVALID_ARG, "e0_decode_items: bad arguments");
+  SchedShape Z{};
+  Z.L = n_layers; Z.G = n_ctas; Z.E = dims->n_experts; Z.k = dims->top_k; Z.r = dims->lora_rank;
+  Z.D = dims->d_model; Z.I = dims->d_ff;
+  Z.ldh = dims->d_model + (dims->head_onehot ? 2 * dims->n_experts : 0);
+  for (int l = 0; l < n_layers; l++) {
+    Z.head[l] = has_head[l] != 0;
+    Z.lora[l] = has_lora[l] != 0;
+  }
+  std::vector<unsigned long long> buf(kMaxItems);
+  const int n = build_items(Z, flat != 0, step0 != 0, cta, buf.data());
+  if (n < 0) return fail(E0_ERR_INVALID_ARG, "e0_decode_items: more than %d items for one CTA", kMaxItems);
+  if (n > cap) return fail(E0_ERR_INVALID_ARG, "e0_decode_items: %d items, capacity %d", n, cap);
+  for (int i = 0; i < n; i++) items_out[i] = buf[i];
+  *n_out = n;
+  return E0_OK;
+}
+
 // Select the decode implementation: 1 = general per-layer kernels only (comparisons).
 extern "C" int e0_debug_force_general(e0_ctx *C, int on) {
   if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
