@@ -173,6 +173,24 @@ int e0_stage_experts(e0_ctx *ctx, int layer, const int32_t *host_idx, int n, voi
 int e0_moe_stack_decode(e0_ctx *ctx, const void *h_in, int B, int step, void *y_out, float *y_f32,
                         int streaming, int chained, void *stream);
 
+/* e0_moe_stack_decode with the step's input and outputs in host memory: h_host [L, B, d]
+ * bf16, y_host [L, B, d] bf16, y_f32_host [L, B, d] fp32 or NULL, all caller-owned and
+ * page-locked for the copies to be asynchronous (pageable memory works, but its copies
+ * block the calling thread).  The library copies them through two alternating device
+ * staging buffers that it owns, on a copy stream of its own, ordered with the step on
+ * `stream` by events, so that the input copy of the next call and the output copy of this
+ * one overlap the steps' kernels.  The outputs are in host memory once the call's copies
+ * have completed: after e0_host_io_wait(ctx, stream) and a synchronisation of `stream`.
+ * The input buffer must not change, and the output buffers must not be read, before then.
+ * Same routing, streaming, step rules and errors as e0_moe_stack_decode; OOM if the
+ * staging buffers (2 x L x max_tokens x d bf16, twice more with fp32 outputs) cannot be
+ * allocated. */
+int e0_moe_stack_decode_host(e0_ctx *ctx, const void *h_host, int B, int step, void *y_host, float *y_f32_host,
+                             int streaming, int chained, void *stream);
+/* Make `stream` wait for every copy issued so far by e0_moe_stack_decode_host (no-op if
+ * there was none).  Errors: INVALID_ARG (NULL context), CUDA. */
+int e0_host_io_wait(e0_ctx *ctx, void *stream);
+
 /* One prefill chunk of T tokens through all layers ([G] "Temel fikirler", "Sorular":
  * prediction as routing, one token ahead).  h_in [L, T, d] bf16 (each layer's generated
  * MoE input), y_out [L, T, d] bf16, y_f32 [L, T, d] or NULL, idx_out [L, T, k] int32 or

@@ -69,6 +69,8 @@ _SIGS = {
     "e0_stream_register": (_I, [_P, _P, ctypes.c_size_t, _I, _I]),
     "e0_stage_experts": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int32), _I, _P]),
     "e0_moe_stack_decode": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
+    "e0_moe_stack_decode_host": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
+    "e0_host_io_wait": (_I, [_P, _P]),
     "e0_get_routing": (_I, [_P, _I, _P, _P]),
     "e0_moe_prefill_stack": (_I, [_P, _P, _I, _P, _P, _P, _P]),
     "e0_get_stats": (_I, [_P, ctypes.POINTER(Stats)]),
@@ -247,6 +249,19 @@ class Context:
         _check(lib().e0_moe_stack_decode(self._h, _ptr(h_in), B, step, _ptr(y_out), _ptr(y_f32),
                                          int(streaming), int(chained), _stream(stream)))
         return y_out
+
+    def stack_decode_host(self, h_host, step, y_host, y_f32_host=None, streaming=False, chained=False, stream=None):
+        """One decode step with host (pinned) tensors; the library overlaps the copies with
+        the kernels.  The outputs are complete after host_io_wait(stream) and a
+        synchronisation of the stream."""
+        L, B, d = h_host.shape
+        assert not h_host.is_cuda and not y_host.is_cuda and (y_f32_host is None or not y_f32_host.is_cuda)
+        _check(lib().e0_moe_stack_decode_host(self._h, _ptr(h_host), B, step, _ptr(y_host), _ptr(y_f32_host),
+                                              int(streaming), int(chained), _stream(stream)))
+        return y_host
+
+    def host_io_wait(self, stream=None):
+        _check(lib().e0_host_io_wait(self._h, _stream(stream)))
 
     def prefill_stack(self, h_in, y_out=None, y_f32=None, idx=None, stream=None):
         """h_in [L, T, d] bf16 -> y_out [L, T, d] bf16 (prediction-as-routing, one token ahead)."""

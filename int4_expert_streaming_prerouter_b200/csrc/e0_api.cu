@@ -144,6 +144,16 @@ struct e0_ctx {
   e0_stats stats{};
   bool time_gemm = false;                          // profiling: event pairs around the GEMMs
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> gemm_ev;
+  // decode steps with host buffers (e0_moe_stack_decode_host): a copy stream and two
+  // alternating device staging buffers, ordered with the steps by events
+  struct HostIO {
+    cudaStream_t cs = nullptr;
+    cudaEvent_t in[2] = {}, out[2] = {}, done[2] = {}, tail = nullptr;
+    uint16_t *h[2] = {}, *y[2] = {};
+    float *yf[2] = {};
+    bool used[2] = {};
+    long long calls = 0;
+  } io;
 };
 
 extern "C" const char *e0_last_error(void) { return g_err.c_str(); }
@@ -191,6 +201,14 @@ extern "C" int e0_destroy(e0_ctx *C) {
   for (auto &r : C->pool.ring)
     for (auto e : {r.c0, r.c1, r.w0, r.w1}) cudaEventDestroy(e);
   if (C->pool.side) cudaStreamDestroy(C->pool.side);
+  for (int b = 0; b < 2; b++) {
+    for (cudaEvent_t e : {C->io.in[b], C->io.out[b], C->io.done[b]})
+      if (e) cudaEventDestroy(e);
+    for (void *m : {(void *)C->io.h[b], (void *)C->io.y[b], (void *)C->io.yf[b]})
+      if (m) cudaFree(m);
+  }
+  if (C->io.tail) cudaEventDestroy(C->io.tail);
+  if (C->io.cs) cudaStreamDestroy(C->io.cs);
   delete C;
   return E0_OK;
 }
@@ -1059,6 +1077,68 @@ extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step,
   C->last_step = step;
   C->last_B = B;
   C->stats.steps++;
+  return E0_OK;
+}
+
+// A decode step with the input and output in (pinned) host memory.  Step n uses staging
+// buffer n % 2: its input copy (copy stream) waits until step n-2's kernels have read the
+// buffer, the step (caller's stream) waits for the input copy and for step n-2's output
+// copy out of the buffer, and its output copy (copy stream) waits for the step.  So the
+// input copy of step n+1 and the output copy of step n run while the kernels of the
+// neighbouring steps do.
+extern "C" int e0_moe_stack_decode_host(e0_ctx *C, const void *h_host, int B, int step, void *y_host,
+                                        float *y_f32_host, int streaming, int chained, void *stream) {
+  if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
+  if (!h_host || !y_host || B < 1 || B > C->maxT || step < 0)
+    return fail(E0_ERR_INVALID_ARG, "e0_moe_stack_decode_host: bad arguments (B=%d, max %d)", B, C->maxT);
+  auto &io = C->io;
+  const size_t n = (size_t)C->L * C->maxT * C->dims.d_model, used = (size_t)C->L * B * C->dims.d_model;
+  if (!io.cs) {
+    CK(cudaStreamCreateWithFlags(&io.cs, cudaStreamNonBlocking));
+    for (int b = 0; b < 2; b++) {
+      CK(cudaEventCreateWithFlags(&io.in[b], cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&io.out[b], cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&io.done[b], cudaEventDisableTiming));
+      int rc;
+      if ((rc = dalloc(&io.h[b], n)) || (rc = dalloc(&io.y[b], n))) return rc;
+    }
+    CK(cudaEventCreateWithFlags(&io.tail, cudaEventDisableTiming));
+  }
+  if (y_f32_host && !io.yf[0]) {
+    int rc;
+    if ((rc = dalloc(&io.yf[0], n)) || (rc = dalloc(&io.yf[1], n))) return rc;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  const int b = (int)(io.calls & 1);
+  if (io.used[b]) {
+    CK(cudaStreamWaitEvent(io.cs, io.out[b], 0));   // step n-2 has read h[b]
+    CK(cudaStreamWaitEvent(s, io.done[b], 0));      // y[b] of step n-2 has been copied out
+  }
+  CK(cudaMemcpyAsync(io.h[b], h_host, used * 2, cudaMemcpyHostToDevice, io.cs));
+  CK(cudaEventRecord(io.in[b], io.cs));
+  CK(cudaStreamWaitEvent(s, io.in[b], 0));
+  const int rc = e0_moe_stack_decode(C, io.h[b], B, step, io.y[b], y_f32_host ? io.yf[b] : nullptr, streaming,
+                                     chained, stream);
+  io.used[b] = true;
+  io.calls++;
+  CK(cudaEventRecord(io.out[b], s));
+  if (rc) {
+    CK(cudaEventRecord(io.done[b], io.cs));
+    return rc;
+  }
+  CK(cudaStreamWaitEvent(io.cs, io.out[b], 0));
+  CK(cudaMemcpyAsync(y_host, io.y[b], used * 2, cudaMemcpyDeviceToHost, io.cs));
+  if (y_f32_host) CK(cudaMemcpyAsync(y_f32_host, io.yf[b], used * 4, cudaMemcpyDeviceToHost, io.cs));
+  CK(cudaEventRecord(io.done[b], io.cs));
+  return E0_OK;
+}
+
+// Make `stream` wait for every copy that the host-buffer decode calls have issued.
+extern "C" int e0_host_io_wait(e0_ctx *C, void *stream) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  if (!C->io.cs) return E0_OK;
+  CK(cudaEventRecord(C->io.tail, C->io.cs));
+  CK(cudaStreamWaitEvent((cudaStream_t)stream, C->io.tail, 0));
   return E0_OK;
 }
 

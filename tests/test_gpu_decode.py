@@ -264,3 +264,28 @@ def test_graph_replay_decode_matches_oracle(cuda_ok, B):
     ref = oracle_steps(SMALL, 95 + B, B, S, gpu[2], gpu[3])
     compare_steps(SMALL, gpu, ref)
     ctx.close()
+
+
+@pytest.mark.parametrize("B", [1, 3])
+def test_host_buffer_decode_matches_device_buffers(cuda_ok, B):
+    """e0_moe_stack_decode_host (pinned host input and outputs, copies overlapped with the
+    kernels through two alternating staging buffers) gives bit-identical outputs and
+    routing to the device-buffer call over a sequence of steps."""
+    seed, S = 71, 5
+    ctx_d, _, _ = build(SMALL, seed, 4)
+    ctx_h, _, _ = build(SMALL, seed, 4)
+    ys, y32s, idxs, preds = run_steps(ctx_d, SMALL, seed, B, S)
+    shape = (SMALL.L, B, SMALL.d)
+    h_host = [bf16_tensor(synth.hidden(seed, t, SMALL.L, B, SMALL.d), "cpu").pin_memory() for t in range(S)]
+    y_host = [torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(S)]
+    f_host = [torch.empty(shape, dtype=torch.float32).pin_memory() for _ in range(S)]
+    for t in range(S):
+        ctx_h.stack_decode_host(h_host[t], t, y_host[t], y_f32_host=f_host[t])
+    ctx_h.host_io_wait()
+    torch.cuda.synchronize()
+    ctx_h.sync_status()
+    idx, pred = ctx_h.get_routing(B)
+    assert np.array_equal(idx, idxs[-1]) and np.array_equal(pred, preds[-1])
+    for t in range(S):
+        assert np.array_equal(bf16_bits_to_np(y_host[t]), ys[t]), f"bf16 outputs differ at step {t}"
+        assert np.array_equal(f_host[t].numpy().astype(np.float64), y32s[t]), f"fp32 outputs differ at step {t}"
