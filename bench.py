@@ -38,24 +38,52 @@ import synth  # noqa: E402
 METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
 
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, valid only
-# while the kernel source is the one captured (sha256 prefix of the file); see profiles/.
+# while the kernel's code is the one captured (sha256 prefix of the source file with its
+# comments removed and white space collapsed, so that comment edits keep the numbers);
+# see profiles/.
 KERNEL_TRAFFIC = {
-    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "bb5f70878b8b2649", 409.9e6,
+    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "02210cdf8e7fbacc", 409.9e6,
                       "4-layer capture (40.99 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
                       "bytes to the 40-layer launch"),
-    "prefill_t4096_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh", "12341c74281dd957", 343.6e6,
+    "prefill_t4096_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh", "861809fb30912006", 343.6e6,
                           "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 465.8 MB, "
                           "down 221.4 MB, mean of the two"),
 }
 
 
-def kernel_traffic(workload):
+def code_digest(path):
+    """sha256 of a C/C++/CUDA source with // and /* */ comments removed (string and
+    character literals kept) and every run of white space collapsed to one blank."""
     import hashlib
+    src = open(path, encoding="utf-8").read()
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return hashlib.sha256(" ".join("".join(out).split()).encode()).hexdigest()
+
+
+def kernel_traffic(workload):
     ent = KERNEL_TRAFFIC.get(workload)
     if not ent:
         return None, None
     path, digest, nbytes, how = ent
-    h = hashlib.sha256(open(os.path.join(ROOT, path), "rb").read()).hexdigest()
+    h = code_digest(os.path.join(ROOT, path))
     return (nbytes, how) if h.startswith(digest) else (None, "kernel changed since the capture")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 

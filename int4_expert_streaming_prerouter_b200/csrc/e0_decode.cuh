@@ -15,15 +15,18 @@
 //     (cp.async.bulk, mbarrier completion).  Because the routing of a predicted layer is
 //     known a whole token ahead, the producer runs ahead of the data dependencies and keeps
 //     HBM busy while the consumers wait for other CTAs.
-//   * Consumers (12 warps) compute warp-per-row int4 dot products with fp32 accumulation
-//     (packed f32x2 FMA), the SwiGLU, the LoRA branch and the weighted combine.
+//   * Consumers (11 warps) compute the int4 dot products on the tensor cores as row pairs
+//     that share one activation vector (mma.sync m16n8k16 bf16 with the codes expanded to
+//     128 + q and the group scale/min folded per group of 64), the SwiGLU, the LoRA branch
+//     and the weighted combine.
 //   * CTAs exchange results (a, y, LoRA intermediates, logits) through global memory as
 //     64-bit words {32-bit tag, payload} written with one relaxed store; a reader polls the
 //     data itself until every tag matches, so there is no separate barrier round trip.
 //     Tags are unique per (launch, layer).  Every wait is bounded by a %globaltimer budget;
 //     on expiry the kernel latches DERR_TIMEOUT, drains its copies and returns.
-//   * Work per layer is split into contiguous, balanced ranges per CTA: the (k+1)*I
-//     intermediate rows of the gate/up phase and the d output rows of the down phase.
+//   * The work is a host-built list of items per CTA: in layer order for chained inputs,
+//     otherwise (flat) each phase's units over all layers cut into contiguous,
+//     cost-balanced shares (router rows, x rows, gate/up units, down rows).
 #pragma once
 #include <algorithm>
 #include <vector>
