@@ -51,3 +51,5 @@ def test_create_rejects_unsupported_dims_without_touching_a_gpu():
     assert L.e0_create(None, 1, 1, ctypes.byref(h)) == -1
     assert L.e0_moe_layer_forward(None, 0, None, 1, None, None, None, None, None, None) == -1
     assert L.e0_sync_status(None) == -1
+    assert L.e0_moe_stack_decode_host(None, None, 1, 0, None, None, 0, 0, None) == -1
+    assert L.e0_host_io_wait(None, None) == -1
