@@ -123,13 +123,26 @@ def step_bytes(dims, idx, B):
 # clocks during the timed region
 # ---------------------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event reasons of one GPU during a timed region.  Two sources run
+    side by side: NVML read every 5 ms from a thread (enough samples for short regions),
+    and `nvidia-smi -lms 100`; the summary uses the NVML samples when there are any.  Only
+    reads; nothing is set.  `nvml` may be a stand-in module (tests)."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, nvml=None, use_smi: bool = True):
         self.gpu = gpu_index
         self.proc = None
+        self.use_smi = use_smi
+        self.nvml = nvml
+        self.samples = []            # NVML: (sm MHz, reason bits)
+        self.max_mhz = None
+        self.thread = None
+        self.stop = None
         import tempfile
         self.path = os.path.join(tempfile.gettempdir(), f"e0_clocks_rank{gpu_index}.csv")
         self.uuid = None
@@ -140,19 +153,50 @@ class ClockSampler:
         except Exception:
             pass
 
+    def _nvml_start(self):
+        import threading
+        nv = self.nvml
+        if nv is None:
+            import pynvml as nv
+        nv.nvmlInit()
+        h = nv.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid else nv.nvmlDeviceGetHandleByIndex(self.gpu)
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        self.stop = threading.Event()
+
+        def loop():
+            while not self.stop.is_set():
+                try:
+                    self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), int(reasons(h))))
+                except Exception:
+                    return
+                self.stop.wait(0.005)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            sel = [f"--id={self.uuid}"] if self.uuid else []
-            self.proc = subprocess.Popen(["nvidia-smi"] + sel + [f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            self._nvml_start()
         except Exception:
-            self.proc = None
+            self.thread = None
+        if self.use_smi:
+            try:
+                os.makedirs(os.path.dirname(self.path), exist_ok=True)
+                self.f = open(self.path, "w")
+                sel = [f"--id={self.uuid}"] if self.uuid else []
+                self.proc = subprocess.Popen(["nvidia-smi"] + sel + [f"--query-gpu={self.Q}",
+                                              "--format=csv,noheader,nounits", "-lms", "100"],
+                                             stdout=self.f, stderr=subprocess.DEVNULL)
+            except Exception:
+                self.proc = None
         return self
 
     def __exit__(self, *a):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -162,6 +206,11 @@ class ClockSampler:
             self.f.close()
 
     def summary(self):
+        if self.samples:
+            sm = [m for m, _ in self.samples]
+            reasons = sorted({name for _, bits in self.samples for name, bit in self.REASONS if bits & bit})
+            return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                    "samples": len(sm), "source": "nvml, 5 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
@@ -179,7 +228,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": sorted(reasons),
-                "samples": len(rows)}
+                "samples": len(rows), "source": "nvidia-smi, 100 ms"}
 
 
 # ---------------------------------------------------------------------------------------
