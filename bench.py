@@ -242,8 +242,11 @@ def dist_init():
         import datetime
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        # NCCL between GPUs; gloo where there is no GPU (the plumbing's CPU tests)
+        dist.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
     return ws, rank, local
 
 
@@ -253,24 +256,27 @@ def barrier(ws):
         dist.barrier()
 
 
+def _reduce(v: float, op):
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
 def max_over_ranks(v: float, ws: int) -> float:
     if ws == 1:
         return v
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return _reduce(v, dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(v: float, ws: int) -> float:
     if ws == 1:
         return v
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(v, dist.ReduceOp.SUM)
 
 
 # ---------------------------------------------------------------------------------------
