@@ -24,7 +24,7 @@ def lists(cfg, flat, step0, G, heads=None, lora=None):
     heads = cfg["heads"] if heads is None else heads
     L = cfg["L"]
     has_head = [l in heads for l in range(L)]
-    has_lora = [True] * L if lora is None else lora
+    has_lora = [cfg["r"] > 0] * L if lora is None else lora
     dims = e0.make_dims(cfg["d"], cfg["E"], cfg["I"], cfg["k"], cfg["r"])
     return [e0.decode_items(dims, L, has_head, has_lora, G, flat, step0, c) for c in range(G)], has_head, has_lora
 
@@ -44,7 +44,8 @@ def units(cfg, has_head, has_lora, step0, kind, l):
     return d
 
 
-CASES = [(FULL, 148), (FULL, 37), (SMALL, 148), (SMALL, 5)]
+TOP2 = dict(d=2048, E=64, I=512, k=2, r=0, L=7, heads=(0, 2, 3, 5))     # no LoRA, sparse heads
+CASES = [(FULL, 148), (FULL, 37), (SMALL, 148), (SMALL, 5), (TOP2, 148), (TOP2, 11)]
 
 
 @pytest.mark.parametrize("cfg,G", CASES)
