@@ -61,7 +61,7 @@ struct DecodeParams {
   int chained;
   // 0: layers in order (each layer's first x item waits for the previous layer's output);
   // 1 (unchained inputs only): the flat schedule, every phase's work over all layers
-  // split evenly across the CTAs
+  // cut into cost-balanced contiguous shares across the CTAs
   int flat;
   uint32_t epoch;
   int step0;                // 1: every layer routes with its own router
@@ -423,8 +423,9 @@ __device__ __forceinline__ bool timed_out(unsigned long long &t0, unsigned long 
 //
 // Flat (unchained inputs: no layer reads another layer's output within the step, so the
 // layers are independent apart from the predictions that cross to the next token): each
-// phase's units over all layers form one list, split evenly and contiguously across the
-// CTAs, so that a CTA streams long runs of rows of one or two layers instead of a sliver
+// phase's units over all layers form one list, cut into contiguous cost-balanced shares
+// across the CTAs (balanced_cuts), so that a CTA streams long runs of rows of one or two
+// layers instead of a sliver
 // of every layer.  Phases: R (reactive layers' routers), XR, TK (the reactive layers this
 // CTA needs), GU, DN.  Items are cut to at most about 58 KB of weight bytes (three fit the
 // ring).  A CTA then computes a handful of norms per step, polls other CTAs' results a
