@@ -38,24 +38,31 @@ import synth  # noqa: E402
 METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
 
 # DRAM bytes (read + write) per launch of the dominant kernel from an ncu capture, valid only
-# while the kernel's code is the one captured (sha256 prefix of the source file with its
-# comments removed and white space collapsed, so that comment edits keep the numbers);
-# see profiles/.
+# while the kernel's code is the one captured: sha256 prefix of its source files (the
+# kernel's file and the headers it includes) with comments removed and white space
+# collapsed, so that comment edits keep the numbers; see profiles/.
 KERNEL_TRAFFIC = {
-    "decode_b1_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh", "02210cdf8e7fbacc", 409.9e6,
+    "decode_b1_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh",
+                       "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
+                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "2e9b3dd381860134", 409.9e6,
                       "4-layer capture (40.99 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
                       "bytes to the 40-layer launch"),
-    "prefill_t4096_l40": ("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh", "861809fb30912006", 343.6e6,
+    "prefill_t4096_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh",
+                           "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
+                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "d088c3d2737d7eff", 343.6e6,
                           "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 465.8 MB, "
                           "down 221.4 MB, mean of the two"),
 }
 
 
-def code_digest(path):
-    """sha256 of a C/C++/CUDA source with // and /* */ comments removed (string and
-    character literals kept) and every run of white space collapsed to one blank."""
+def code_digest(paths):
+    """sha256 of C/C++/CUDA sources (one path or several, in order) with // and /* */
+    comments removed (string and character literals kept) and every run of white space
+    collapsed to one blank."""
     import hashlib
-    src = open(path, encoding="utf-8").read()
+    if isinstance(paths, str):
+        paths = (paths,)
+    src = "\n".join(open(p, encoding="utf-8").read() for p in paths)
     out, i, n = [], 0, len(src)
     while i < n:
         c = src[i]
@@ -82,8 +89,8 @@ def kernel_traffic(workload):
     ent = KERNEL_TRAFFIC.get(workload)
     if not ent:
         return None, None
-    path, digest, nbytes, how = ent
-    h = code_digest(os.path.join(ROOT, path))
+    paths, digest, nbytes, how = ent
+    h = code_digest([os.path.join(ROOT, p) for p in paths])
     return (nbytes, how) if h.startswith(digest) else (None, "kernel changed since the capture")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
