@@ -103,6 +103,8 @@ typedef struct {
   uint64_t kernel_launches;    /* kernels this context has launched */
   uint64_t gemm_timed;         /* expert-GEMM launches timed (see e0_debug_time_gemm) */
   double   gemm_ms;            /* their summed durations (event pairs on the launch stream) */
+  uint64_t hit_experts;        /* staging requests served by an expert already in its slot
+                                  (persistent per-layer sets; no copy) */
 } e0_stats;
 
 /* Create a context on the current CUDA device.  n_layers >= 1; max_tokens bounds T of
@@ -146,10 +148,17 @@ int e0_prerouter_predict(e0_ctx *ctx, int layer, const void *x, int T, const int
 
 /* Streaming tier ([G] "Temel fikirler": weights stay off the GPU, only the working set
  * is resident; "Temel terimler": staged decode with a fixed-slot double buffer and a
- * GPU slot table).  host_blob: pinned host memory [L][E][expert_bytes] (caller-owned,
- * must stay valid).  Allocates the HBM pool of pool_layers x slots_per_layer blobs
- * (pool_layers >= 2, slots_per_layer >= k * max_tokens is not required: slots_per_layer
- * must be >= the number of distinct experts a layer routes to in one step).
+ * GPU slot table, and the incremental sticky-slot stack).  host_blob: pinned host memory
+ * [L][E][expert_bytes] (caller-owned, must stay valid).  Allocates the HBM pool of
+ * pool_layers x slots_per_layer blobs; slots_per_layer must be >= k and >= the number of
+ * distinct experts a layer routes to in one step.
+ *   2 <= pool_layers < n_layers: shared slot sets (layer l uses set l % pool_layers), the
+ *     double buffer of staged decode: every staging rewrites its set.
+ *   pool_layers == n_layers: one persistent set per layer, kept across steps (sticky
+ *     slots): an expert already in the set is not copied again; a missing one replaces
+ *     the least recently needed slot not needed now (empty first, ties to the lower
+ *     slot).  With slots_per_layer = k at one stream this rewrites only the slots whose
+ *     expert changed; with more slots it is a least-recently-used expert cache in HBM.
  * Errors: INVALID_ARG, OOM. */
 int e0_stream_register(e0_ctx *ctx, const void *host_blob, size_t expert_bytes, int pool_layers,
                        int slots_per_layer);
@@ -191,6 +200,15 @@ int e0_moe_stack_decode_host(e0_ctx *ctx, const void *h_host, int B, int step, v
  * there was none).  Errors: INVALID_ARG (NULL context), CUDA. */
 int e0_host_io_wait(e0_ctx *ctx, void *stream);
 
+/* Streaming decode mode ([G] "Sonuçlar": prerouter prefetch against fully reactive
+ * on-demand loading).  reactive = 0 (default): a layer preceded by a head is routed by
+ * that head's prediction made one token earlier and its experts are copied while the
+ * previous layer computes; other layers stage on demand.  reactive = 1: every layer
+ * routes with its own router and its experts are copied only after that router ran; no
+ * head runs (e0_get_routing reports -1 predictions).  Changing the mode starts a new
+ * sequence (the next decode call must be step 0).  Errors: INVALID_ARG. */
+int e0_stream_mode(e0_ctx *ctx, int reactive);
+
 /* One prefill chunk of T tokens through all layers ([G] "Temel fikirler", "Sorular":
  * prediction as routing, one token ahead).  h_in [L, T, d] bf16 (each layer's generated
  * MoE input), y_out [L, T, d] bf16, y_f32 [L, T, d] or NULL, idx_out [L, T, k] int32 or
@@ -227,9 +245,11 @@ int e0_sync_status(e0_ctx *ctx);
  * Scratch: one fixed 4 MiB device array inside the library (every GPU that loads the
  * library holds it until the process exits).  A call whose intermediates do not fit is
  * rejected with E0_ERR_INVALID_ARG and a message naming the bytes needed (at d = 2048,
- * E = 256, I = 512, k = 4, r = 16 the limit is about T = 200 tokens).  The first call on
- * each device looks up the array's device address (cudaGetSymbolAddress); make that first
- * call outside any stream capture.  All calls share the one array and each overwrites it:
+ * E = 256, I = 512, k = 4, r = 16 the limit is about T = 200 tokens).  The array's device
+ * address belongs to the CUDA context the call runs in (a device reset or a second context
+ * on the same device has its own copy): the first call in each context looks it up
+ * (cudaGetSymbolAddress, under a lock, so concurrent first calls from several host threads
+ * are safe); make that first call outside any stream capture.  All calls share the one array and each overwrites it:
  * calls on one device whose work overlaps on the GPU (for example on two streams)
  * race and give wrong results, so serialise them.
  * Errors: INVALID_ARG (arguments, sizes beyond the maximum), CUDA. */
@@ -244,6 +264,14 @@ int e0_moe_layer_forward_noalloc(const e0_dims *dims, const e0_layer *layer, con
  *   `set` tags `slot` with `expert`; the expert kernels must then latch SLOT_MISMATCH. */
 int e0_debug_fail_staging_after(e0_ctx *ctx, int n);
 int e0_debug_set_slot_tag(e0_ctx *ctx, int pool_set, int slot, int expert);
+/* Streaming test hooks:
+ * e0_debug_stream_log(ctx, log): from the next streamed layer on, copy the slot tags of the
+ *   layer's pool set, as its expert kernels read them, into log[layer * slots + s] (int32
+ *   device buffer [L][slots_per_layer], caller-owned; one device-to-device copy on the
+ *   compute stream per layer); NULL stops it.
+ * e0_debug_pool_slot(ctx, set, slot, &ptr): the device address of one pool slot's blob. */
+int e0_debug_stream_log(e0_ctx *ctx, int32_t *log);
+int e0_debug_pool_slot(e0_ctx *ctx, int pool_set, int slot, void **out);
 
 /* Test hooks of the one-launch decode path (B = 1, resident experts, linear heads):
  * e0_debug_decode_stall(ctx, cta, timeout_ns): in the next decode step CTA `cta` waits for

@@ -52,7 +52,7 @@ class Stats(ctypes.Structure):
                 ("ondemand_experts", ctypes.c_uint64), ("dropped", ctypes.c_uint64),
                 ("stage_ms", ctypes.c_double), ("exposed_wait_ms", ctypes.c_double),
                 ("kernel_launches", ctypes.c_uint64), ("gemm_timed", ctypes.c_uint64),
-                ("gemm_ms", ctypes.c_double)]
+                ("gemm_ms", ctypes.c_double), ("hit_experts", ctypes.c_uint64)]
 
 
 _lib = None
@@ -78,6 +78,9 @@ _SIGS = {
     "e0_last_error": (ctypes.c_char_p, []),
     "e0_moe_layer_forward_noalloc": (_I, [ctypes.POINTER(Dims), ctypes.POINTER(Layer), _P, _I, _P, _P, _P, _P,
                                           _P, _P, _P]),
+    "e0_stream_mode": (_I, [_P, _I]),
+    "e0_debug_stream_log": (_I, [_P, _P]),
+    "e0_debug_pool_slot": (_I, [_P, _I, _I, ctypes.POINTER(_P)]),
     "e0_debug_fail_staging_after": (_I, [_P, _I]),
     "e0_debug_set_slot_tag": (_I, [_P, _I, _I, _I]),
     "e0_debug_decode_stall": (_I, [_P, _I, ctypes.c_ulonglong]),
@@ -235,6 +238,21 @@ class Context:
         self._keep.append(host_blob)
         blob = host_blob.shape[-1]
         _check(lib().e0_stream_register(self._h, _ptr(host_blob), blob, pool_layers, slots_per_layer))
+
+    def stream_mode(self, reactive: bool):
+        """False: prerouter prefetch (default); True: every layer routes itself and stages
+        on demand (no prediction).  Starts a new sequence."""
+        _check(lib().e0_stream_mode(self._h, int(reactive)))
+
+    def debug_stream_log(self, log):
+        """log: int32 CUDA tensor [L, slots_per_layer] or None."""
+        self._keep.append(log)
+        _check(lib().e0_debug_stream_log(self._h, _ptr(log)))
+
+    def debug_pool_slot(self, pool_set, slot) -> int:
+        out = _P()
+        _check(lib().e0_debug_pool_slot(self._h, pool_set, slot, ctypes.byref(out)))
+        return int(out.value)
 
     def stage_experts(self, layer, experts, stream=None):
         arr = (ctypes.c_int32 * len(experts))(*[int(e) for e in experts])

@@ -12,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -62,6 +63,15 @@ struct StreamPool {
   std::vector<int> set_rec;                // per pool set: ring entry of its current round
   int fail_after = -1;                     // host-side fault injection for tests
   int corrupt_set = -1, corrupt_slot = 0, corrupt_tag = 0;  // one-shot wrong slot tag
+  // persistent sets (one per layer, kept across steps): the host mirror of every slot's
+  // expert (-1: empty) and the staging round that last needed it, for the sticky-slot /
+  // least-recently-used replacement
+  bool persist = false;
+  std::vector<int> tag_h;
+  std::vector<long long> use_h;
+  long long round = 0;
+  int reactive = 0;                        // 1: every layer routes itself and stages on demand
+  int32_t *log = nullptr;                  // debug: [L][slots] slot tags each layer computed with
 };
 
 // Persistent decode kernel state: device copy of the layer table, tagged exchange buffers
@@ -256,6 +266,17 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
       e0_destroy(C);
       return rc;
     }
+    // the large dynamic shared memory of the tensor-core kernels is an attribute of the
+    // function on the current device: opt in here, for this context's device, so that
+    // contexts on several devices of one process each have it
+    if (cudaFuncSetAttribute(k_tc_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(TcRowsSmem) + 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(k_moe_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(TwSmem) + 1024) != cudaSuccess) {
+      cudaGetLastError();
+      e0_destroy(C);
+      return fail(E0_ERR_CUDA, "e0_create: shared-memory opt-in of the tensor-core kernels failed");
+    }
   }
   C->plan.U = C->plan_mem;
   C->plan.uexp = C->plan_mem + 1;
@@ -393,12 +414,7 @@ static int layer_pre(e0_ctx *C, const LayerCall &K, cudaStream_t s) {
       W.seg[W.nseg++] = RowSeg{R.Au, D.lora_rank, D.d_model, C->lt, 3 * D.lora_rank, D.lora_rank};
     }
     for (int q = 0; q < W.nseg; q++) W.total += W.seg[q].rows;
-    const int smem = (int)sizeof(TcRowsSmem) + 1024;
-    static bool attr_rows = false;
-    if (!attr_rows) {
-      CK(cudaFuncSetAttribute(k_tc_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-      attr_rows = true;
-    }
+    const int smem = (int)sizeof(TcRowsSmem) + 1024;   // opted in at e0_create on this context's device
     k_tc_rows<<<dim3((W.total + 127) / 128, (K.T + kTcN - 1) / kTcN), kTcThreads, smem, s>>>(W);
     CKL("k_tc_rows");
   } else {
@@ -440,12 +456,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   A.ntiles = C->ntiles; A.xp = C->xp; A.xsum = C->xsum; A.ap = C->ap; A.asum = C->asum; A.ap_out = C->ap;
   A.Bg = (const uint16_t *)Y.lora_Bg; A.Bu = (const uint16_t *)Y.lora_Bu; A.lt = C->lt; A.gates = K.gates;
   A.yacc = C->yacc; A.err = C->err; A.timeout_ns = 2000000000ull;
-  const int tc_smem_bytes = (int)sizeof(TwSmem) + 1024;
-  static bool attr_done = false;
-  if (!attr_done) {
-    CK(cudaFuncSetAttribute(k_moe_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem_bytes));
-    attr_done = true;
-  }
+  const int tc_smem_bytes = (int)sizeof(TwSmem) + 1024;   // opted in at e0_create on this context's device
   const int tmax = std::min(C->tile_cap, (K.T * D.top_k + kTcN - 1) / kTcN + std::min(D.n_experts, K.T * D.top_k) +
                                               (K.T + kTcN - 1) / kTcN);
   cudaEvent_t g0 = nullptr, g1 = nullptr;
@@ -623,8 +634,9 @@ extern "C" int e0_stream_register(e0_ctx *C, const void *host_blob, size_t exper
   if (!C || !host_blob) return fail(E0_ERR_INVALID_ARG, "e0_stream_register: NULL argument");
   if (expert_bytes != (size_t)C->bl.bytes)
     return fail(E0_ERR_INVALID_ARG, "expert_bytes %zu != blob size %lld", expert_bytes, C->bl.bytes);
-  if (pool_layers < 2 || slots_per_layer < C->dims.top_k || slots_per_layer > C->dims.n_experts)
-    return fail(E0_ERR_INVALID_ARG, "pool needs >= 2 layer sets and k <= slots <= E");
+  if (pool_layers < 2 || pool_layers > std::max(C->L, 2) || slots_per_layer < C->dims.top_k ||
+      slots_per_layer > C->dims.n_experts)
+    return fail(E0_ERR_INVALID_ARG, "pool needs 2 <= layer sets <= n_layers and k <= slots <= E");
   if ((uintptr_t)host_blob & 15) return fail(E0_ERR_INVALID_ARG, "host store must be 16-byte aligned");
   StreamPool &P = C->pool;
   if (P.mem) return fail(E0_ERR_INVALID_ARG, "a host store is already registered");
@@ -638,6 +650,10 @@ extern "C" int e0_stream_register(e0_ctx *C, const void *host_blob, size_t exper
   P.nsets = pool_layers;
   P.slots = slots_per_layer;
   P.bytes = expert_bytes;
+  P.persist = pool_layers == C->L;
+  P.tag_h.assign((size_t)pool_layers * slots_per_layer, -1);
+  P.use_h.assign((size_t)pool_layers * slots_per_layer, -1);
+  P.round = 0;
   P.host = (const uint8_t *)host_blob;
   CK(cudaStreamCreateWithFlags(&P.side, cudaStreamNonBlocking));
   for (auto *v : {&P.ready, &P.freed}) {
@@ -681,23 +697,83 @@ static void account_rec(e0_ctx *C, StreamPool::Rec &r) {
   r.state = 0;
 }
 
+// Stage the distinct experts of host_idx[0..n) into the slot set of `layer`.
+//   Shared sets (fewer sets than layers: the staged-decode double buffer of [G] "Temel
+//   terimler"): the set is rewritten, slot s receives the s-th distinct expert.
+//   Persistent sets (one per layer, kept across steps: the incremental sticky-slot stack
+//   `incr_stack` of [G] "Temel terimler"): an expert already in the set stays in its slot
+//   and costs nothing; each missing expert, in first-seen order, replaces the least
+//   recently needed slot among those not needed now (empty slots first, then the oldest
+//   staging round, ties to the lower slot).  With as many slots as the step routes to,
+//   that is "only the changed slots are rewritten"; with more, the set is a least-
+//   recently-used expert cache in HBM in front of the host store.
 static int stage_impl(e0_ctx *C, int layer, const int32_t *host_idx, int n, cudaStream_t compute,
                       bool prefetch) {
   StreamPool &P = C->pool;
   if (!P.mem) return fail(E0_ERR_INVALID_ARG, "no host store registered");
   if (layer < 0 || layer >= C->L || n < 1 || !host_idx) return fail(E0_ERR_INVALID_ARG, "stage: bad arguments");
-  SlotList lst{};
+  SlotList need{};
   for (int i = 0; i < n; i++) {
     const int e = host_idx[i];
     if (e < 0 || e >= C->dims.n_experts) return fail(E0_ERR_INVALID_ARG, "stage: expert %d out of range", e);
     bool dup = false;
-    for (int q = 0; q < lst.n; q++) dup |= lst.e[q] == e;
+    for (int q = 0; q < need.n; q++) dup |= need.e[q] == e;
     if (dup) continue;
-    if (lst.n >= P.slots || lst.n >= kMaxSlots)
+    if (need.n >= P.slots || need.n >= kMaxSlots)
       return fail(E0_ERR_INVALID_ARG, "stage: more distinct experts than pool slots (%d)", P.slots);
-    lst.e[lst.n++] = e;
+    need.e[need.n++] = e;
   }
   const int p = layer % P.nsets;
+  // copies[q] = (slot, expert); lst = the set's content after this round (slot -> expert)
+  std::vector<std::pair<int, int>> copies;
+  SlotList lst{};
+  int hits = 0;
+  if (!P.persist) {
+    lst = need;
+    for (int s = 0; s < need.n; s++) copies.push_back({s, need.e[s]});
+  } else {
+    int *tag = P.tag_h.data() + (size_t)p * P.slots;
+    long long *use = P.use_h.data() + (size_t)p * P.slots;
+    const long long rnd = ++P.round;
+    std::vector<char> held(P.slots, 0);
+    std::vector<int> miss;
+    for (int q = 0; q < need.n; q++) {
+      int at = -1;
+      for (int s = 0; s < P.slots; s++)
+        if (tag[s] == need.e[q]) at = s;
+      if (at >= 0) {
+        held[at] = 1;
+        use[at] = rnd;
+        hits++;
+      } else {
+        miss.push_back(need.e[q]);
+      }
+    }
+    std::vector<int> victims;
+    for (int s = 0; s < P.slots; s++)
+      if (!held[s]) victims.push_back(s);
+    std::stable_sort(victims.begin(), victims.end(), [&](int a, int b) { return use[a] < use[b]; });
+    for (size_t q = 0; q < miss.size(); q++) {
+      const int s = victims[q];            // need.n <= slots, so there are enough victims
+      copies.push_back({s, miss[q]});
+      tag[s] = miss[q];
+      use[s] = rnd;
+    }
+    lst.n = P.slots;
+    for (int s = 0; s < P.slots; s++) lst.e[s] = tag[s];
+  }
+  C->stats.hit_experts += hits;
+  int bad_slot = -1, bad_tag = 0;
+  if (P.corrupt_set == p) {
+    bad_slot = P.corrupt_slot;
+    bad_tag = P.corrupt_tag;
+    P.corrupt_set = -1;
+  }
+  if (copies.empty() && bad_slot < 0) {
+    // every expert is already in its slot: nothing to copy, the slot table is unchanged
+    P.set_rec[p] = -1;
+    return E0_OK;
+  }
   StreamPool::Rec &rec = P.ring[P.ring_pos];
   account_rec(C, rec);
   P.set_rec[p] = P.ring_pos;
@@ -706,22 +782,19 @@ static int stage_impl(e0_ctx *C, int layer, const int32_t *host_idx, int n, cuda
   CK(cudaStreamWaitEvent(P.side, P.freed[p], 0));
   CK(cudaEventRecord(rec.c0, P.side));
   uint8_t *dst = P.mem + (size_t)p * P.slots * P.bytes;
-  for (int s = 0; s < lst.n; s++) {
-    const uint8_t *src = P.host + ((size_t)layer * C->dims.n_experts + lst.e[s]) * P.bytes;
+  for (const auto &cp : copies) {
+    const uint8_t *src = P.host + ((size_t)layer * C->dims.n_experts + cp.second) * P.bytes;
     if (P.fail_after == 0) {
       P.fail_after = -1;
-      return fail(E0_ERR_STAGING, "staging copy of layer %d expert %d refused (injected)", layer, lst.e[s]);
+      if (P.persist) P.tag_h[(size_t)p * P.slots + cp.first] = -1;   // the slot's content is now unknown
+      return fail(E0_ERR_STAGING, "staging copy of layer %d expert %d refused (injected)", layer, cp.second);
     }
     if (P.fail_after > 0) P.fail_after--;
-    cudaError_t e = cudaMemcpyAsync(dst + (size_t)s * P.bytes, src, P.bytes, cudaMemcpyHostToDevice, P.side);
-    if (e != cudaSuccess)
-      return fail(E0_ERR_STAGING, "staging copy of layer %d expert %d: %s", layer, lst.e[s], cudaGetErrorString(e));
-  }
-  int bad_slot = -1, bad_tag = 0;
-  if (P.corrupt_set == p) {
-    bad_slot = P.corrupt_slot;
-    bad_tag = P.corrupt_tag;
-    P.corrupt_set = -1;
+    cudaError_t e = cudaMemcpyAsync(dst + (size_t)cp.first * P.bytes, src, P.bytes, cudaMemcpyHostToDevice, P.side);
+    if (e != cudaSuccess) {
+      if (P.persist) P.tag_h[(size_t)p * P.slots + cp.first] = -1;
+      return fail(E0_ERR_STAGING, "staging copy of layer %d expert %d: %s", layer, cp.second, cudaGetErrorString(e));
+    }
   }
   k_set_slots<<<1, 256, 0, P.side>>>(P.slot_of + (size_t)p * C->dims.n_experts, P.slot_tag + (size_t)p * P.slots,
                                      C->dims.n_experts, P.slots, lst, bad_slot, bad_tag);
@@ -729,9 +802,9 @@ static int stage_impl(e0_ctx *C, int layer, const int32_t *host_idx, int n, cuda
   CK(cudaEventRecord(rec.c1, P.side));
   CK(cudaEventRecord(P.ready[p], P.side));
   rec.state = 1;
-  C->stats.staged_experts += lst.n;
-  C->stats.staged_bytes += (uint64_t)lst.n * P.bytes;
-  (prefetch ? C->stats.prefetched_experts : C->stats.ondemand_experts) += lst.n;
+  C->stats.staged_experts += copies.size();
+  C->stats.staged_bytes += (uint64_t)copies.size() * P.bytes;
+  (prefetch ? C->stats.prefetched_experts : C->stats.ondemand_experts) += copies.size();
   (void)compute;
   return E0_OK;
 }
@@ -746,12 +819,22 @@ extern "C" int e0_stage_experts(e0_ctx *C, int layer, const int32_t *host_idx, i
 static int wait_ready(e0_ctx *C, int layer, cudaStream_t s) {
   StreamPool &P = C->pool;
   const int p = layer % P.nsets;
-  if (P.set_rec[p] < 0) return fail(E0_ERR_STAGING, "layer %d was never staged", layer);
-  StreamPool::Rec &rec = P.ring[P.set_rec[p]];
-  CK(cudaEventRecord(rec.w0, s));
-  CK(cudaStreamWaitEvent(s, P.ready[p], 0));
-  CK(cudaEventRecord(rec.w1, s));
-  if (rec.state == 1) rec.state = 2;
+  if (P.set_rec[p] >= 0) {
+    StreamPool::Rec &rec = P.ring[P.set_rec[p]];
+    CK(cudaEventRecord(rec.w0, s));
+    CK(cudaStreamWaitEvent(s, P.ready[p], 0));
+    CK(cudaEventRecord(rec.w1, s));
+    if (rec.state == 1) rec.state = 2;
+  } else if (!P.persist) {
+    return fail(E0_ERR_STAGING, "layer %d was never staged", layer);
+  } else {
+    // a persistent set that needed no copy: its previous round's copies completed before
+    // the previous reader of the set ran; order after them all the same
+    CK(cudaStreamWaitEvent(s, P.ready[p], 0));
+  }
+  if (P.log)
+    CK(cudaMemcpyAsync(P.log + (size_t)layer * P.slots, P.slot_tag + (size_t)p * P.slots, (size_t)P.slots * 4,
+                       cudaMemcpyDeviceToDevice, s));
   return E0_OK;
 }
 
@@ -793,8 +876,14 @@ static int stack_decode_general(e0_ctx *C, const uint16_t *h_in, int B, int step
   const size_t ld = (size_t)B * D.d_model;
   const int cur = step & 1, prv = cur ^ 1;
   std::vector<int32_t> uniq(B * k);
+  // streaming in the reactive mode: no prediction, every layer routes itself and its
+  // experts are staged on demand after its router ran (the comparison point of [G]
+  // "Sonuçlar": prefetch against fully reactive on-demand loading); no head runs
+  const bool reactive = streaming && C->pool.reactive;
+  if (reactive)
+    CK(cudaMemsetAsync(pred_at(C, cur, 0), 0xFF, (size_t)(L + 1) * C->maxT * k * sizeof(int32_t), s));
   for (int l = 0; l < L; l++) {
-    const bool predicted = step > 0 && l > 0 && C->heads[l - 1].w_lin != nullptr;
+    const bool predicted = !reactive && step > 0 && l > 0 && C->heads[l - 1].w_lin != nullptr;
     LayerCall K{};
     K.l = l; K.T = B; K.h = h_in + l * ld;
     float *yf_l = y_f32 ? y_f32 + l * ld : C->yscratch + (size_t)(l & 1) * C->maxT * D.d_model;
@@ -805,7 +894,7 @@ static int stack_decode_general(e0_ctx *C, const uint16_t *h_in, int B, int step
     K.idx = hist_at(C, cur, l);
     K.gates = C->gates;
     K.hist = nullptr;
-    const bool has_head = C->heads[l].w_lin != nullptr;
+    const bool has_head = !reactive && C->heads[l].w_lin != nullptr;
     K.head = has_head && D.head_hidden == 0;   // the linear head is fused into the routing kernel
     K.prev = step > 0 ? hist_at(C, prv, l) : nullptr;
     K.pred = pred_at(C, cur, l + 1);
@@ -838,7 +927,7 @@ static int stack_decode_general(e0_ctx *C, const uint16_t *h_in, int B, int step
       if ((rc = layer_post(C, K, resident_src(C, l), s))) return rc;
     }
   }
-  if (streaming) {
+  if (streaming && !reactive) {
     // next step's predicted routing, for the staging decisions of the next call
     int rc = host_read_idx(C, C->host_idx, pred_at(C, cur, 0), (L + 1) * C->maxT * k, s);
     if (rc) return rc;
@@ -1323,6 +1412,38 @@ extern "C" int e0_debug_set_slot_tag(e0_ctx *C, int pool_set, int slot, int expe
   return E0_OK;
 }
 
+// Streaming mode: 0 = prefetch from the head predictions made one token earlier
+// (prediction as routing; layers without a predictor on demand), 1 = fully reactive:
+// every layer routes with its own router and stages on demand after it ran.
+extern "C" int e0_stream_mode(e0_ctx *C, int reactive) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  if (reactive != 0 && reactive != 1) return fail(E0_ERR_INVALID_ARG, "stream mode must be 0 or 1");
+  if (C->pool.reactive != reactive) C->last_step = -1;      // the routing tables of the two modes differ: a new sequence starts
+  C->pool.reactive = reactive;
+  return E0_OK;
+}
+
+// Debug: record, for every streamed layer, the slot tags of its pool set at the point where
+// its expert kernels read them (one cudaMemcpyAsync on the compute stream after the wait
+// for the staging copies) into log[layer * slots + s]; NULL stops it.
+extern "C" int e0_debug_stream_log(e0_ctx *C, int32_t *log) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  if (!C->pool.mem) return fail(E0_ERR_INVALID_ARG, "no host store registered");
+  C->pool.log = log;
+  return E0_OK;
+}
+
+// Debug: the device address of slot `slot` of pool set `set` (read its blob to check the
+// staged bytes); E0_ERR_INVALID_ARG outside the pool.
+extern "C" int e0_debug_pool_slot(e0_ctx *C, int set, int slot, void **out) {
+  if (!C || !out) return fail(E0_ERR_INVALID_ARG, "NULL argument");
+  const StreamPool &P = C->pool;
+  if (!P.mem || set < 0 || set >= P.nsets || slot < 0 || slot >= P.slots)
+    return fail(E0_ERR_INVALID_ARG, "no such pool slot");
+  *out = P.mem + ((size_t)set * P.slots + slot) * P.bytes;
+  return E0_OK;
+}
+
 // ---------------------------------------------------------------------------------------
 // One MoE block without any allocation.
 //
@@ -1335,11 +1456,68 @@ extern "C" int e0_debug_set_slot_tag(e0_ctx *C, int pool_set, int slot, int expe
 // ---------------------------------------------------------------------------------------
 static constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;   // 4 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-static constexpr int kNoAllocMaxDevices = 64;
-// Device address of g_noalloc_scratch per device (the host-side symbol is not an address a
-// kernel may use), and the SM count, filled by the first call on each device.
-static unsigned char *g_noalloc_dev[kNoAllocMaxDevices];
-static int g_noalloc_nsm[kNoAllocMaxDevices];
+// The device address of g_noalloc_scratch belongs to the library's module as loaded in one
+// CUDA context: the host-side symbol is not an address a kernel may use, and a device
+// reset or another (non-primary) context on the same device loads the module again at
+// another address.  So the address is looked up once per context, keyed by the context's
+// process-unique id (cuCtxGetId; a handle value can be reused after a reset), and kept in
+// a small table that a mutex guards against concurrent first calls from several host
+// threads.
+static constexpr int kNoAllocMaxContexts = 64;
+struct NoAllocEntry {
+  unsigned long long ctx_id;
+  unsigned char *base;
+  int nsm;
+};
+static NoAllocEntry g_noalloc_tab[kNoAllocMaxContexts];
+static int g_noalloc_n = 0;
+static std::mutex g_noalloc_mu;
+
+// The scratch array's address and the SM count for the calling thread's current context.
+static int noalloc_scratch(unsigned char **base, int *nsm) {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!get_cur || !get_id) {
+    void *f1 = nullptr, *f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || !f1 ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+        q2 != cudaDriverEntryPointSuccess || !f2)
+      return fail(E0_ERR_CUDA, "noalloc forward: cuCtxGetCurrent / cuCtxGetId are not available");
+    get_cur = (PFN_cuCtxGetCurrent_v4000)f1;
+    get_id = (PFN_cuCtxGetId_v12000)f2;
+  }
+  int dev = 0;
+  CK(cudaGetDevice(&dev));
+  CUcontext cur = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&cur) != CUDA_SUCCESS || !cur) {
+    // no context current on this thread yet: the symbol lookup below makes the runtime's
+    // primary context current
+    void *p = nullptr;
+    CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    if (get_cur(&cur) != CUDA_SUCCESS || !cur) return fail(E0_ERR_CUDA, "noalloc forward: no current CUDA context");
+  }
+  if (get_id(cur, &id) != CUDA_SUCCESS) return fail(E0_ERR_CUDA, "noalloc forward: cuCtxGetId failed");
+  for (int i = 0; i < g_noalloc_n; i++)
+    if (g_noalloc_tab[i].ctx_id == id) {
+      *base = g_noalloc_tab[i].base;
+      *nsm = g_noalloc_tab[i].nsm;
+      return E0_OK;
+    }
+  // first call in this context: look the address up (must not run inside a stream capture)
+  void *p = nullptr;
+  CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+  int n_sm = 0;
+  CK(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  NoAllocEntry &slot = g_noalloc_tab[g_noalloc_n < kNoAllocMaxContexts ? g_noalloc_n++ : (int)(id % kNoAllocMaxContexts)];
+  slot = NoAllocEntry{id, (unsigned char *)p, n_sm};
+  *base = slot.base;
+  *nsm = slot.nsm;
+  return E0_OK;
+}
 
 static size_t noalloc_align(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -1373,20 +1551,9 @@ extern "C" int e0_moe_layer_forward_noalloc(const e0_dims *dims, const e0_layer 
     return fail(E0_ERR_INVALID_ARG,
                 "noalloc forward: T=%d needs %zu bytes of scratch, the fixed maximum is %zu bytes", T, off,
                 kNoAllocScratchBytes);
-  int dev = 0;
-  CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(E0_ERR_INVALID_ARG, "noalloc forward: device %d", dev);
-  if (!g_noalloc_dev[dev]) {
-    // one-time set-up on this device (must not run inside a stream capture)
-    void *p = nullptr;
-    CK(cudaGetSymbolAddress(&p, g_noalloc_scratch));
-    int nsm = 0;
-    CK(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
-    g_noalloc_nsm[dev] = nsm;
-    g_noalloc_dev[dev] = (unsigned char *)p;
-  }
-  unsigned char *base = g_noalloc_dev[dev];
-  const int nsm = g_noalloc_nsm[dev];
+  unsigned char *base = nullptr;
+  int nsm = 0;
+  if (int rc = noalloc_scratch(&base, &nsm)) return rc;
   cudaStream_t s = (cudaStream_t)stream;
   int *err = dev_status ? dev_status : (int *)(base + o_err);
   if (!dev_status) CK(cudaMemsetAsync(err, 0, sizeof(int), s));

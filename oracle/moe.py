@@ -45,6 +45,7 @@ __all__ = [
     "rmsnorm", "router_logits", "topk", "topk_alternatives", "gates_softmax",
     "silu", "gelu_erf", "routed_expert", "shared_expert", "moe_layer",
     "head_input", "prerouter_head", "predicted_layers", "stack_decode", "staging_plan",
+    "sticky_plan",
 ]
 
 
@@ -328,7 +329,7 @@ def predicted_layers(dims) -> set:
 
 
 def stack_decode(h_steps, dense_of, expert_of, shared_of, dims, chained: bool = False,
-                 choose=None) -> dict:
+                 choose=None, prediction: bool = True) -> dict:
     """Decode ``S`` steps of ``B`` streams through all ``L`` layers.
 
     h_steps    [S, L, B, d] bf16 bit patterns (generated MoE inputs).
@@ -338,6 +339,8 @@ def stack_decode(h_steps, dense_of, expert_of, shared_of, dims, chained: bool = 
     Routing of layer N at step t: the head prediction of layer N-1 made at step t-1 when
     N is a predicted layer and t > 0, else the layer's own router top-k.  The heads of
     every layer run at every step and their top-k become the next step's routing.
+    prediction=False is the fully reactive comparison point of [G] "Sonuçlar" (no
+    prerouter): every layer routes with its own router and no head runs (pred stays -1).
     Returns y [S,L,B,d] (float64), y_bf16, idx [S,L,B,k], gates, pred [S,L,B,k] (-1 where
     a layer has no head) and head logits.
     """
@@ -357,12 +360,12 @@ def stack_decode(h_steps, dense_of, expert_of, shared_of, dims, chained: bool = 
             if chained and n > 0:
                 h = round_bf16(h + y[t, n - 1])
             hb = f64_to_bf16_bits(h)
-            route = pred[t - 1, n - 1] if (t > 0 and n in pl) else None
+            route = pred[t - 1, n - 1] if (prediction and t > 0 and n in pl) else None
             pick = None if choose is None else (lambda b, c, a, t=t, n=n: choose(("route", t, n, b), c, a))
             out = moe_layer(hb, dense, lambda e, n=n: expert_of(n, e), shared_of(n), dims,
                             route_idx=route, choose=pick)
             y[t, n], idx[t, n], gates[t, n] = out["y"], out["idx"], out["gates"]
-            if n in dims.head_layers:
+            if prediction and n in dims.head_layers:
                 for b in range(B):
                     prev = idx[t - 1, n, b] if t > 0 else None
                     z, p = prerouter_head(out["x"][b], dense, dims, idx[t, n, b], prev)
@@ -392,4 +395,54 @@ def staging_plan(idx, dims) -> dict:
                 if int(e) not in seen:
                     seen.append(int(e))
             plan[(t, n)] = {"experts": seen, "prefetched": bool(t > 0 and n in pl)}
+    return plan
+
+
+def sticky_plan(idx, dims, slots: int) -> dict:
+    """Copies made by per-layer persistent expert slot sets (one set of ``slots`` slots
+    per layer, kept across decode steps).
+
+    [G] "Temel terimler" describes the incremental sticky-slot stack (``incr_stack``):
+    persistent stacked expert tensors in which only the expert slots that changed are
+    rewritten, in place.  Reading taken for which slot a new expert overwrites when the
+    set has more slots than one step needs (then the set acts as an expert cache in front
+    of the host store): the slot least recently needed among those not needed at this
+    step, an empty slot counting as never needed and equal ages going to the lower slot.
+
+    For every (step t, layer n) the step's experts are the distinct entries of idx[t, n]
+    in first-seen order (streams, then rank).  An expert already in the set is a hit; each
+    missing expert, in that order, is copied into the next victim slot.  Returns
+    {(t, n): {"copies": [(slot, expert), ...], "hits": h, "content": [expert or -1 per
+    slot after the step]}}.
+    """
+    idx = np.asarray(idx)
+    S, L = idx.shape[:2]
+    content = {n: [-1] * slots for n in range(L)}
+    last = {n: [-1] * slots for n in range(L)}      # staging round that last needed a slot
+    plan = {}
+    rnd = 0
+    for t in range(S):
+        for n in range(L):
+            rnd += 1
+            need = []
+            for e in idx[t, n].reshape(-1):
+                if int(e) not in need:
+                    need.append(int(e))
+            assert len(need) <= slots, "a step routes to more experts than the set has slots"
+            held, misses, hits = set(), [], 0
+            for e in need:
+                if e in content[n]:
+                    s = content[n].index(e)
+                    held.add(s)
+                    last[n][s] = rnd
+                    hits += 1
+                else:
+                    misses.append(e)
+            victims = sorted((s for s in range(slots) if s not in held), key=lambda s: (last[n][s], s))
+            copies = []
+            for e, s in zip(misses, victims):
+                content[n][s] = e
+                last[n][s] = rnd
+                copies.append((s, e))
+            plan[(t, n)] = {"copies": copies, "hits": hits, "content": list(content[n])}
     return plan

@@ -9,69 +9,11 @@ import synth
 from synth import Dims
 from synth.device import bf16_tensor, layer_tensors
 from parity import bf16_bits_to_np, check_bf16, check_y, choose_following, idx_ok
+from stack_helpers import build, compare_steps, oracle_steps, run_steps
 
 pytestmark = pytest.mark.gpu
 
 SMALL = Dims(d=256, E=16, I=128, k=4, r=8, L=4, head_layers=(0, 1, 2))
-
-
-def build(dims, seed, max_tokens, resident=True):
-    import int4_expert_streaming_prerouter_b200 as e0
-    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, max_tokens,
-                     head_hidden=dims.head_hidden, head_onehot=dims.head_onehot)
-    lys, hds = zip(*[layer_tensors(seed, n, dims, "cuda", resident=resident) for n in range(dims.L)])
-    ctx.register_model(list(lys), list(hds))
-    return ctx, lys, hds
-
-
-def run_steps(ctx, dims, seed, B, S, chained=False, streaming=False):
-    ys, y32s, idxs, preds = [], [], [], []
-    for t in range(S):
-        h = bf16_tensor(synth.hidden(seed, t, dims.L, B, dims.d), "cuda")
-        y32 = torch.empty((dims.L, B, dims.d), dtype=torch.float32, device="cuda")
-        y = ctx.stack_decode(h, t, y_f32=y32, chained=chained, streaming=streaming)
-        ctx.sync_status()
-        idx, pred = ctx.get_routing(B)
-        ys.append(bf16_bits_to_np(y))
-        y32s.append(y32.cpu().numpy().astype(np.float64))
-        idxs.append(idx)
-        preds.append(pred)
-    return np.stack(ys), np.stack(y32s), np.stack(idxs), np.stack(preds)
-
-
-def oracle_steps(dims, seed, B, S, gpu_idx, gpu_pred, chained=False):
-    hs = np.stack([synth.hidden(seed, t, dims.L, B, dims.d) for t in range(S)])
-    dense = {n: synth.layer_dense(seed, n, dims) for n in range(dims.L)}
-    cache = {}
-
-    def expert(n, e):
-        if (n, e) not in cache:
-            cache[(n, e)] = synth.expert_blob(seed, n, e, dims)
-        return cache[(n, e)]
-
-    sets = {}
-    for t in range(S):
-        for n in range(dims.L):
-            for b in range(B):
-                sets[("route", t, n, b)] = gpu_idx[t, n, b]
-                sets[("head", t, n, b)] = gpu_pred[t, n, b]
-    return O.stack_decode(hs, dense.__getitem__, expert, lambda n: synth.shared_blob(seed, n, dims), dims,
-                          chained=chained, choose=choose_following(sets))
-
-
-def compare_steps(dims, gpu, ref, chained=False):
-    yb, y32, idx, pred = gpu
-    S, L, B = idx.shape[:3]
-    assert np.array_equal(idx, ref["idx"]), "routing differs beyond admissible near ties"
-    for n in range(L):
-        if n in dims.head_layers:
-            assert np.array_equal(pred[:, n], ref["pred"][:, n])
-        else:
-            assert np.all(pred[:, n] == -1)
-    for t in range(S):
-        for n in range(L):
-            check_y(y32[t, n], ref["y"][t, n], f"step {t} layer {n}")
-            check_bf16(yb[t, n], ref["y"][t, n], f"step {t} layer {n}", y32[t, n])
 
 
 @pytest.mark.parametrize("B", [1, 5])
@@ -92,7 +34,7 @@ def test_small_stack_chained_matches_oracle(cuda_ok):
     ctx, _, _ = build(SMALL, 70, 8)
     gpu = run_steps(ctx, SMALL, 70, 2, 3, chained=True)
     ref = oracle_steps(SMALL, 70, 2, 3, gpu[2], gpu[3], chained=True)
-    compare_steps(SMALL, gpu, ref, chained=True)
+    compare_steps(SMALL, gpu, ref)
     ctx.close()
 
 
@@ -223,7 +165,7 @@ def test_one_launch_decode_chained_b1(cuda_ok):
     ctx, _, _ = build(SMALL, 92, 4)
     gpu = run_steps(ctx, SMALL, 92, 1, 3, chained=True)
     ref = oracle_steps(SMALL, 92, 1, 3, gpu[2], gpu[3], chained=True)
-    compare_steps(SMALL, gpu, ref, chained=True)
+    compare_steps(SMALL, gpu, ref)
     ctx.close()
 
 
@@ -289,3 +231,99 @@ def test_host_buffer_decode_matches_device_buffers(cuda_ok, B):
     for t in range(S):
         assert np.array_equal(bf16_bits_to_np(y_host[t]), ys[t]), f"bf16 outputs differ at step {t}"
         assert np.array_equal(f_host[t].numpy().astype(np.float64), y32s[t]), f"fp32 outputs differ at step {t}"
+
+
+# ---------------------------------------------------------------------------------------
+# batched decode on the full model (the multi-stream batches 32 and 64)
+# ---------------------------------------------------------------------------------------
+def _oracle_routing(dims, hs_layer, dense):
+    """x, router logits and (for a head layer) head logits of every token of one layer."""
+    x = O.rmsnorm(O.bf16_to_f64(hs_layer), dense["norm_w"], dims.eps)
+    lg = O.router_logits(dense["router_w"], x)
+    hl = O.router_logits(dense["head_w"], x) if dense.get("head_w") is not None else None
+    return x, lg, hl
+
+
+@pytest.mark.parametrize("B", [32, 64])
+def test_full_size_decode_batched_routing_and_sampled_outputs(full_model, B):
+    """Two steps of B streams through the 40-layer model: every layer's routing of every
+    stream (own router at step 0 and on layers without a predictor; the previous step's
+    head prediction elsewhere) and every head prediction against the oracle's logits, and
+    y of sampled streams on sampled layers of both steps against the oracle's MoE block."""
+    dims, wseed, iseed, S = FULL, 1, 3 + B, 2
+    gpu = run_steps(full_model, dims, iseed, B, S)
+    _, y32, idx, pred = gpu
+    pl = O.predicted_layers(dims)
+    streams = sorted({0, 1, B // 2, B - 1} | set(range(3, B, max(1, B // 4))))
+    for t in range(S):
+        hs = synth.hidden(iseed, t, dims.L, B, dims.d)
+        for n in range(dims.L):
+            dense = synth.layer_dense(wseed, n, dims)
+            x, lg, hl = _oracle_routing(dims, hs[n], dense)
+            for b in range(B):
+                if t > 0 and n in pl:
+                    assert np.array_equal(idx[t, n, b], pred[t - 1, n - 1, b]), (t, n, b)
+                else:
+                    assert idx_ok(idx[t, n, b], lg[b], O.topk(lg[b], dims.k), dims.k), (t, n, b)
+                if hl is not None:
+                    assert idx_ok(pred[t, n, b], hl[b], O.topk(hl[b], dims.k), dims.k), ("head", t, n, b)
+            if n in (0, 1, 33, 34, 39):
+                ref = O.moe_layer(hs[n][streams], dense, lambda e: synth.expert_blob(wseed, n, e, dims),
+                                  synth.shared_blob(wseed, n, dims), dims, route_idx=idx[t, n][streams])
+                check_y(y32[t, n][streams], ref["y"], f"B={B} step {t} layer {n}")
+
+
+# ---------------------------------------------------------------------------------------
+# exact ties: equal logits must resolve to the lowest indices, with no alternative admitted
+# ---------------------------------------------------------------------------------------
+def test_exact_ties_take_the_lowest_indices(cuda_ok):
+    """Zero router and head weights make every logit 0: every routing and every prediction
+    must be exactly [0, 1, 2, 3] at E = 256, on the one-launch kernel (B = 1), the per-layer
+    kernels (B = 3), one MoE block, and the tensor-core prefill path (T = 160); the gates
+    are then 1/4 each and y matches the oracle."""
+    import int4_expert_streaming_prerouter_b200 as e0
+    dims = Dims(d=256, E=256, I=128, k=4, r=8, L=3, head_layers=(0, 1))
+    seed = 97
+    lys, hds = [], []
+    denses = []
+    for n in range(dims.L):
+        dense = synth.layer_dense(seed, n, dims)
+        dense["router_w"] = np.zeros_like(dense["router_w"])
+        if dense["head_w"] is not None:
+            dense["head_w"] = np.zeros_like(dense["head_w"])
+        denses.append(dense)
+        ly, hd = layer_tensors(seed, n, dims, "cuda", dense=dense)
+        lys.append(ly)
+        hds.append(hd)
+    want = np.arange(dims.k, dtype=np.int32)
+    for B in (1, 3):
+        ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, 256)
+        ctx.register_model(lys, hds)
+        for t in range(2):
+            h = bf16_tensor(synth.hidden(seed, t, dims.L, B, dims.d), "cuda")
+            y32 = torch.empty((dims.L, B, dims.d), dtype=torch.float32, device="cuda")
+            ctx.stack_decode(h, t, y_f32=y32)
+            ctx.sync_status()
+            idx, pred = ctx.get_routing(B)
+            for n in range(dims.L):
+                for b in range(B):
+                    assert np.array_equal(idx[n, b], want), (B, t, n, b, idx[n, b])
+                    if n in dims.head_layers:
+                        assert np.array_equal(pred[n, b], want), (B, t, n, b, pred[n, b])
+            hs = synth.hidden(seed, t, dims.L, B, dims.d)
+            for n in (0, 2):
+                ref = O.moe_layer(hs[n], denses[n], lambda e, n=n: synth.expert_blob(seed, n, e, dims),
+                                  synth.shared_blob(seed, n, dims), dims)
+                assert np.array_equal(ref["idx"], np.tile(want, (B, 1)))
+                check_y(y32[n].cpu().numpy().astype(np.float64), ref["y"], f"ties B={B} t={t} n={n}")
+        # one block and the tensor-core prefill path
+        for T, path in ((5, 1), (160, 2)):
+            ctx.debug_prefill_path(path)
+            hb = synth.hidden(seed + T, 0, 1, T, dims.d)[0]
+            idx_t = torch.empty((T, dims.k), dtype=torch.int32, device="cuda")
+            gates = torch.empty((T, dims.k), dtype=torch.float32, device="cuda")
+            ctx.moe_layer_forward(0, bf16_tensor(hb, "cuda"), idx=idx_t, gates=gates)
+            ctx.sync_status()
+            assert np.array_equal(idx_t.cpu().numpy(), np.tile(want, (T, 1))), (T, path)
+            assert np.allclose(gates.cpu().numpy(), 0.25, rtol=0, atol=1e-7)
+        ctx.close()

@@ -295,3 +295,30 @@ def test_prefill_stack_prediction_as_routing_shifted_one_token(cuda_ok):
         else:
             route = None
     ctx.close()
+
+
+def test_prefill_tensor_core_path_full_width_t4096(cuda_ok):
+    """The benchmarked prefill chunk size on one full-width layer (d=2048, E=256, I=512,
+    r=16, T=4096, about 64 tokens per routed expert), own-router routing, through the
+    tcgen05 path: every token's routing and gates against the oracle's router, and y on
+    280 sampled tokens (every 16th token, so every expert-tile position is reached, plus
+    the last tokens, which sit in the shared expert's tail tile) against the oracle."""
+    dims = Dims(d=2048, E=256, I=512, k=4, r=16, L=1, head_layers=(0,))
+    seed, T = 230, 4096
+    ctx, _, _ = make_ctx(dims, seed, T)
+    h = synth.prefill_hidden(seed, 0, T, dims.d)
+    ctx.debug_prefill_path(2)
+    yb, y32, idx, gates = run_layer(ctx, dims, seed, 0, h)
+    dense = synth.layer_dense(seed, 0, dims)
+    x = O.rmsnorm(O.bf16_to_f64(h), dense["norm_w"], dims.eps)
+    lg = O.router_logits(dense["router_w"], x)
+    for t in range(T):
+        assert idx_ok(idx[t], lg[t], O.topk(lg[t], dims.k), dims.k), (t, idx[t])
+        assert np.allclose(gates[t], O.gates_softmax(lg[t], idx[t]), rtol=1e-5, atol=1e-6), t
+    counts = np.bincount(idx.reshape(-1), minlength=dims.E)
+    assert counts.max() >= 64 and (counts > 0).sum() == dims.E
+    sample = sorted(set(range(0, T, 16)) | set(range(T - 24, T)))
+    ref = oracle_layer(dims, seed, 0, h[sample], route=idx[sample])
+    check_y(y32[sample], ref["y"], "T=4096 sampled")
+    check_bf16(yb[sample], ref["y"], "T=4096 sampled", y32[sample])
+    ctx.close()

@@ -426,3 +426,61 @@ def test_head_onehot_history_uses_current_and_previous_routing():
         z, p = O.prerouter_head(x, dense[0], dims, out["idx"][t, 0, 0], prev)
         assert np.array_equal(out["head_logits"][t, 0, 0], z)
         assert out["pred"][t, 0, 0].tolist() == p.tolist()
+
+
+# ---------------------------------------------------------------------------------------
+# the fully reactive mode (no prerouter) and the persistent sticky-slot sets
+# ---------------------------------------------------------------------------------------
+def test_reactive_stack_is_each_layer_on_its_own_router():
+    """prediction=False: every layer of every step equals the single-layer oracle with the
+    layer's own router (a brute-force reduction), and no head runs."""
+    S, B = 2, 2
+    hs = np.stack([synth.hidden(13, t, SMALL.L, B, SMALL.d) for t in range(S)])
+    dense = {n: synth.layer_dense(13, n, SMALL) for n in range(SMALL.L)}
+    out = O.stack_decode(hs, dense.__getitem__, lambda n, e: synth.expert_blob(13, n, e, SMALL),
+                         lambda n: synth.shared_blob(13, n, SMALL), SMALL, prediction=False)
+    assert np.all(out["pred"] == -1)
+    for t in range(S):
+        for n in range(SMALL.L):
+            ref = O.moe_layer(hs[t, n], dense[n], lambda e, n=n: synth.expert_blob(13, n, e, SMALL),
+                              synth.shared_blob(13, n, SMALL), SMALL)
+            assert np.array_equal(out["idx"][t, n], ref["idx"])
+            assert np.array_equal(out["y"][t, n], ref["y"])
+
+
+def test_sticky_plan_hand_worked_example():
+    """One layer, one stream, k=2, three slots; worked by hand:
+    t0 [0,1]: copies 0->slot0, 1->slot1 (empty slots, lower first)          -> [0, 1, -]
+    t1 [1,2]: 1 hit; 2 -> slot2 (empty, never needed, before slot0)        -> [0, 1, 2]
+    t2 [3,0]: 0 hit; 3 -> slot1 (slots 1 and 2 both last needed at t1)     -> [0, 3, 2]
+    t3 [1,2]: 2 hit; 1 -> slot0 (slots 0 and 1 both last needed at t2)     -> [1, 3, 2]"""
+    dims = Dims(d=64, E=8, I=64, k=2, r=0, L=1, head_layers=())
+    idx = np.array([[[[0, 1]]], [[[1, 2]]], [[[3, 0]]], [[[1, 2]]]], np.int32)
+    plan = O.sticky_plan(idx, dims, 3)
+    assert plan[(0, 0)]["copies"] == [(0, 0), (1, 1)] and plan[(0, 0)]["hits"] == 0
+    assert plan[(1, 0)]["copies"] == [(2, 2)] and plan[(1, 0)]["hits"] == 1
+    assert plan[(2, 0)]["copies"] == [(1, 3)] and plan[(2, 0)]["hits"] == 1
+    assert plan[(3, 0)]["copies"] == [(0, 1)] and plan[(3, 0)]["hits"] == 1
+    assert plan[(3, 0)]["content"] == [1, 3, 2]
+
+
+def test_sticky_plan_invariants():
+    """k slots at one stream rewrite exactly the experts that changed since the previous
+    token; with a set as large as every expert the layer ever sees, each expert is copied
+    once; every step's experts are resident after its copies (nothing dropped)."""
+    dims = Dims(d=64, E=16, I=64, k=4, r=0, L=3, head_layers=())
+    rng = np.random.default_rng(5)
+    S = 12
+    idx = np.stack([[rng.permutation(16)[:4][None] for _ in range(3)] for _ in range(S)]).astype(np.int32)
+    plan = O.sticky_plan(idx, dims, 4)
+    for t in range(S):
+        for n in range(3):
+            now = set(idx[t, n, 0].tolist())
+            before = set(idx[t - 1, n, 0].tolist()) if t else set()
+            assert len(plan[(t, n)]["copies"]) == len(now - before)
+            assert plan[(t, n)]["hits"] == len(now & before)
+            assert now <= set(plan[(t, n)]["content"])
+    big = O.sticky_plan(idx, dims, 16)
+    for n in range(3):
+        total = sum(len(big[(t, n)]["copies"]) for t in range(S))
+        assert total == len(set(idx[:, n].reshape(-1).tolist()))
