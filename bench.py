@@ -108,22 +108,29 @@ def peaks():
 # ---------------------------------------------------------------------------------------
 # algorithmic bytes of one decode step (what the kernels must read at least once)
 # ---------------------------------------------------------------------------------------
-def step_bytes(dims, idx, B):
-    """idx [L, B, k] routing of the step.  Returns (expert bytes, all bytes)."""
+def step_bytes(dims, idx, B, parts=False):
+    """idx [L, B, k] routing of the step.  Returns (expert bytes, all bytes), or with
+    parts=True a dict: gate/up and down expert bytes, bf16 rows (routers, heads, LoRA A)
+    and the rest."""
     blob = synth.blob_bytes(dims.d, dims.I)
     d, E, I, r = dims.d, dims.E, dims.I, dims.r
-    expert = other = 0
+    gu_bytes = 2 * (I * d // 2 + 2 * I * (d // 64) * 2)          # gate + up of one expert
+    dn_bytes = blob - gu_bytes
+    gu = dn = rows = rest = 0
     heads = set(dims.head_layers)
     for n in range(dims.L):
-        u = len(set(idx[n].reshape(-1).tolist()))
-        expert += (u + 1) * blob                            # routed uniques + shared expert
+        u = len(set(idx[n].reshape(-1).tolist())) + 1             # routed uniques + shared expert
+        gu += u * gu_bytes
+        dn += u * dn_bytes
         predicted = n > 0 and (n - 1) in heads
-        other += (B * dims.k * d * 2) if predicted else E * d * 2   # router rows
-        other += E * d * 2 if n in heads else 0                     # head
-        other += (2 * r * d + 2 * I * r + r * I + d * r) * 2        # LoRA
-        other += d * 2                                               # gamma
-        other += B * d * 2 * 2                                       # h in, y out (bf16)
-    return expert, expert + other
+        rows += min(B * dims.k, E) * d * 2 if predicted else E * d * 2     # router rows
+        rows += E * dims.head_in * 2 if n in heads else 0                   # head
+        rows += 2 * r * d * 2                                                # LoRA A_g, A_u
+        rest += (2 * I * r + r * I + d * r) * 2                              # LoRA B_g, B_u, A_d, B_d
+        rest += d * 2 + B * d * 2 * 2                                        # gamma, h in, y out
+    if parts:
+        return {"gate_up": gu, "down": dn, "rows": rows, "rest": rest}
+    return gu + dn, gu + dn + rows + rest
 
 
 # ---------------------------------------------------------------------------------------
@@ -298,16 +305,30 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
+def _oracle_layer_inputs(dims, seed, n, h_bits):
+    """The weights the oracle needs for one layer on the given tokens, drawn before any
+    timing: the dense weights, the shared expert and the routed experts that the layer's own
+    router selects (a cheap routing pass over the same inputs)."""
+    import oracle as O
+    dense = synth.layer_dense(seed, n, dims)
+    x = O.rmsnorm(O.bf16_to_f64(h_bits), dense["norm_w"], dims.eps)
+    lg = O.router_logits(dense["router_w"], x)
+    used = sorted({int(e) for t in range(lg.shape[0]) for e in O.topk(lg[t], dims.k)})
+    blobs = {e: synth.expert_blob(seed, n, e, dims) for e in used}
+    return dense, blobs, synth.shared_blob(seed, n, dims)
+
+
 def oracle_decode_sample(dims, seed, n_layers: int, step: int = 0):
     """Time the oracle on one token of one stream through the first `n_layers` layers
-    (own-router routing, as at step 0).  Returns seconds."""
+    (own-router routing, as at step 0), the layer's head included.  Weights are drawn
+    before the clock starts.  Returns seconds."""
     import oracle as O
     hs = synth.hidden(seed, step, dims.L, 1, dims.d)
+    pre = [_oracle_layer_inputs(dims, seed, n, hs[n]) for n in range(n_layers)]
     t0 = time.perf_counter()
     for n in range(n_layers):
-        dense = synth.layer_dense(seed, n, dims)
-        out = O.moe_layer(hs[n], dense, lambda e, n=n: synth.expert_blob(seed, n, e, dims),
-                          synth.shared_blob(seed, n, dims), dims)
+        dense, blobs, shared = pre[n]
+        out = O.moe_layer(hs[n], dense, blobs.__getitem__, shared, dims)
         if n in dims.head_layers:
             O.prerouter_head(out["x"][0], dense, dims)
     return time.perf_counter() - t0
@@ -321,8 +342,22 @@ def cpu_baseline(dims, seed, budget_s=20.0):
     t = oracle_decode_sample(dims, seed, n)
     per_token = t * dims.L / n
     return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"1 token (B=1) through {n} of {dims.L} layers, own-router routing; "
-                      f"time scaled x{dims.L / n:.2f} to the full stack (incl. weight generation per layer)"}
+            "sample": f"1 token (B=1) through {n} of {dims.L} layers, own-router routing, heads included; "
+                      f"time scaled x{dims.L / n:.2f} to the full stack; weights drawn before timing"}
+
+
+def cpu_baseline_tokens(dims, seed, hs_layer, layer: int, scale_layers: int, what: str):
+    """The oracle on the given tokens of one layer (own-router routing), weights drawn
+    before timing; tokens/s of the whole stack = tokens / (time x scale_layers)."""
+    import oracle as O
+    dense, blobs, shared = _oracle_layer_inputs(dims, seed, layer, hs_layer)
+    t0 = time.perf_counter()
+    O.moe_layer(hs_layer, dense, blobs.__getitem__, shared, dims)
+    t = time.perf_counter() - t0
+    T = hs_layer.shape[0]
+    return {"value": T / (t * scale_layers), "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{what}: {T} tokens through layer {layer} (own-router routing), time scaled "
+                      f"x{scale_layers} to the {dims.L}-layer stack; weights drawn before timing"}
 
 
 def run_reference(args, dims, seed, ws, rank):
@@ -341,7 +376,7 @@ def run_reference(args, dims, seed, ws, rank):
     per_token = sum(times) / len(times)
     v = 1.0 / per_token
     sample = (f"each step: 1 token (B=1) through {per_step_layers} of {dims.L} layers, "
-              f"time scaled to the full stack")
+              f"time scaled to the full stack; weights drawn before timing")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_token * 1e3, "higher_is_better": True,
@@ -356,21 +391,103 @@ def run_reference(args, dims, seed, ws, rank):
 # ---------------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------------
-def run_decode(args, dims, seed, B, ws, rank, local):
+def _free_gpu():
+    import gc
+    import torch
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _load_model(dims, seed, dev, resident=True):
+    import int4_expert_streaming_prerouter_b200 as e0
+    from synth.device import layer_tensors
+    lys, hds = [], []
+    for n in range(dims.L):
+        ly, hd = layer_tensors(seed, n, dims, dev, resident=resident)
+        lys.append(ly)
+        hds.append(hd)
+    return lys, hds
+
+
+def _context(dims, lys, hds, max_tokens):
+    import int4_expert_streaming_prerouter_b200 as e0
+    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, max_tokens,
+                     head_hidden=dims.head_hidden, head_onehot=dims.head_onehot)
+    ctx.register_model(lys, hds)
+    return ctx
+
+
+def _timed_steps(ctx, h_all, t0, n, y, ws, local, chained=False, streaming=False):
+    """n decode steps t0..t0+n-1 bracketed by CUDA events on the launching stream, barrier
+    and synchronisation on both sides; returns (ms, clocks, kernel launches, routing of the
+    last step)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    ctx.sync_status()
+    l0 = ctx.stats()["kernel_launches"]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for t in range(t0, t0 + n):
+            ctx.stack_decode(h_all[t % len(h_all)], t, y_out=y, chained=chained, streaming=streaming)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    ctx.sync_status()
+    return ev0.elapsed_time(ev1), clk.summary(), ctx.stats()["kernel_launches"] - l0
+
+
+def _hbm_roofline(bytes_per_step, ms_per_step, pk, kernel, traffic=None, note=None):
+    ach = bytes_per_step / (ms_per_step / 1e3) / 1e9
+    out = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": ach / pk["hbm_gbs"],
+           "traffic": traffic, "kernel": kernel, "peak_source": pk["source"] + " copy bandwidth (burst)"}
+    if note:
+        out["traffic_note"] = note
+    return out
+
+
+PHASE_NAMES = ("k_ph_norm", "k_ph_rows", "k_ph_route", "k_ph_gateup", "k_ph_tdsum", "k_ph_down")
+
+
+def phase_breakdown(ctx, h_all, t0, n, y, parts, pk):
+    """Per-kernel CUDA-event times of the phased decode kernels (launched one after another
+    for this pass only) and each streaming kernel's achieved HBM bandwidth on its
+    algorithmic bytes."""
+    ms0, n0 = ctx.debug_phase_times()
+    ctx.debug_phase_timing(True)
+    for t in range(t0, t0 + n):
+        ctx.stack_decode(h_all[t % len(h_all)], t, y_out=y)
+    ctx.debug_phase_timing(False)
+    ms1, n1 = ctx.debug_phase_times()
+    steps = n1 - n0
+    if steps <= 0:
+        return None
+    per = [(b - a) / steps for a, b in zip(ms0, ms1)]
+    nbytes = {"k_ph_rows": parts["rows"], "k_ph_gateup": parts["gate_up"], "k_ph_down": parts["down"]}
+    out = {"ms_per_step_serialised": sum(per), "steps": steps, "kernels": {}}
+    for name, m in zip(PHASE_NAMES, per):
+        ent = {"ms": m}
+        if name in nbytes:
+            ent["algorithmic_bytes"] = nbytes[name]
+            ent["GBps"] = nbytes[name] / (m / 1e3) / 1e9
+            ent["frac"] = ent["GBps"] / pk["hbm_gbs"]
+        out["kernels"][name] = ent
+    return out
+
+
+def run_decode(args, dims, seed, B, ws, rank, local, extras):
     import torch
     import int4_expert_streaming_prerouter_b200 as e0
-    from synth.device import layer_tensors, bf16_tensor
+    from synth.device import bf16_tensor
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     t0 = time.time()
-    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, max(B, 1))
-    lys, hds = [], []
-    for n in range(dims.L):
-        ly, hd = layer_tensors(seed, n, dims, dev)
-        lys.append(ly)
-        hds.append(hd)
-    ctx.register_model(lys, hds)
+    lys, hds = _load_model(dims, seed, dev)
+    ctx = _context(dims, lys, hds, max(B, 1))
     ctx.debug_decode_mode(args.decode_mode)
     if args.decode_flat is not None:
         ctx.debug_decode_flat(args.decode_flat)
@@ -378,38 +495,25 @@ def run_decode(args, dims, seed, B, ws, rank, local):
     steps, warm = args.steps, args.warmup
     total = steps + warm
     # every step has its own generated inputs, resident before the timed region
-    h_all = torch.stack([bf16_tensor(synth.hidden(seed, t, dims.L, B, dims.d), dev) for t in range(total)])
+    h_all = torch.stack([bf16_tensor(synth.hidden(seed, t, dims.L, B, dims.d), dev) for t in range(total + 16)])
     y = torch.empty((dims.L, B, dims.d), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
     for t in range(warm):
         ctx.stack_decode(h_all[t], t, y_out=y)
-    ctx.sync_status()
-    launches0 = ctx.stats()["kernel_launches"]
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    routes = []
-    barrier(ws)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for t in range(warm, total):
-            ctx.stack_decode(h_all[t], t, y_out=y)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    barrier(ws)
-    ctx.sync_status()
-    ms = ev0.elapsed_time(ev1)
-    launches = ctx.stats()["kernel_launches"] - launches0
+    ms, clocks, launches = _timed_steps(ctx, h_all, warm, steps, y, ws, local)
     idx, _ = ctx.get_routing(B)
-    exp_b, all_b = step_bytes(dims, idx, B)
+    parts = step_bytes(dims, idx, B, parts=True)
+    exp_b = parts["gate_up"] + parts["down"]
+    all_b = exp_b + parts["rows"] + parts["rest"]
     ms_max = max_over_ranks(ms, ws)
     tokens = sum_over_ranks(B * steps, ws)
     value = tokens / (ms_max / 1e3)
 
-    # end-to-end through the C ABI with host buffers (e0_moe_stack_decode_host): every
+    # end to end through the C ABI with host buffers (e0_moe_stack_decode_host): every
     # step's input copied in from pinned host memory and its output copied back, the
     # library overlapping those copies with the neighbouring steps' kernels
+    stream = torch.cuda.current_stream(dev)
     h_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
-    h_host.copy_(h_all[warm:].cpu())
+    h_host.copy_(h_all[warm:total].cpu())
     y_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
     torch.cuda.synchronize()
     nxt = total          # continue the same decode sequence
@@ -424,10 +528,18 @@ def run_decode(args, dims, seed, B, ws, rank, local):
     barrier(ws)
     e2e_ms = max_over_ranks(e0_.elapsed_time(e1_), ws)
     e2e_value = tokens / (e2e_ms / 1e3)
+    nxt += steps
 
     pk = peaks()
     step_ms = ms / steps
-    achieved = exp_b / (step_ms / 1e3) / 1e9
+    phased = args.decode_mode in (0, 4) and B <= 8
+    traffic, how = kernel_traffic("decode_b1_l40_phased" if phased else args.workload) if B == 1 else (None, None)
+    kernel = ("decode step = six phased kernels (norm, bf16 rows, routing, gate/up, sums, down) launched "
+              "with programmatic dependent launch; CUDA events around the timed steps on their stream; "
+              "achieved counts int4 expert bytes only" if phased else
+              "k_decode (one launch = one decode step, CUDA events on its stream); achieved counts int4 "
+              "expert bytes only" if B == 1 else
+              "per-layer kernels of one decode step; achieved counts int4 expert bytes")
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": steps, "warmup": warm,
         "ms_per_step": ms_max / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -439,34 +551,51 @@ def run_decode(args, dims, seed, B, ws, rank, local):
                 "d2h_bytes_per_step": int(y_host[0].numel() * 2)},
         "gpu_launches": int(launches),
         "hbm": {"expert_bytes_per_step": exp_b, "all_bytes_per_step": all_b,
-                "expert_GBps": achieved, "all_GBps": all_b / (step_ms / 1e3) / 1e9,
-                "frac_of_measured": achieved / pk["hbm_gbs"], "frac_of_8TBps": achieved / 8000.0},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / pk["hbm_gbs"], "traffic": kernel_traffic(args.workload)[0],
-                     "traffic_note": kernel_traffic(args.workload)[1],
-                     "kernel": ("k_decode (one launch = one decode step, CUDA events on its stream); "
-                                "achieved counts int4 expert bytes only" if B == 1 else
-                                "per-layer kernels of one decode step; achieved counts int4 expert bytes"),
-                     "peak_source": pk["source"] + " copy bandwidth (burst)"},
-        "clocks": clk.summary(),
+                "expert_GBps": exp_b / (step_ms / 1e3) / 1e9, "all_GBps": all_b / (step_ms / 1e3) / 1e9,
+                "frac_of_measured": exp_b / (step_ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                "frac_of_8TBps": exp_b / (step_ms / 1e3) / 1e9 / 8000.0},
+        "roofline": _hbm_roofline(exp_b, step_ms, pk, kernel, traffic, how),
+        "clocks": clocks,
         "setup_s": setup_s,
     }
+    if phased:
+        pb = phase_breakdown(ctx, h_all, nxt, 8, y, parts, pk)
+        nxt += 8
+        if pb:
+            out["phased_kernels"] = pb
+    if extras:
+        # the one-launch persistent kernel on the same unchained steps, and the chained step
+        # (layer N's input is bf16(h_N + y_{N-1}): layers in order, as a real decoder runs)
+        n_x = min(steps, 64)
+        sub = {}
+        for name, mode, chained in (("one_launch_unchained", 1, False), ("chained_in_order", 0, True)):
+            ctx.debug_decode_mode(mode)
+            for t in range(2):
+                ctx.stack_decode(h_all[t], t, y_out=y, chained=chained)
+            ms_x, clk_x, l_x = _timed_steps(ctx, h_all, 2, n_x, y, ws, local, chained=chained)
+            ms_x = max_over_ranks(ms_x, ws)
+            sub[name] = {"value": sum_over_ranks(B * n_x, ws) / (ms_x / 1e3), "unit": "tokens/s",
+                         "ms_per_step": ms_x / n_x, "steps": n_x, "gpu_launches": int(l_x),
+                         "roofline": _hbm_roofline(exp_b, ms_x / n_x, pk,
+                                                   "k_decode (one cooperative launch per step; in layer order "
+                                                   "when chained)"),
+                         "clocks": clk_x}
+        ctx.debug_decode_mode(args.decode_mode)
+        out["decode_variants"] = sub
     return out, ctx
 
 
-def run_prefill(args, dims, seed, ws, rank, local):
+def run_prefill(args, dims, seed, ws, rank, local, T=4096):
     """One step = one prefill chunk of T tokens through all layers."""
     import torch
-    import int4_expert_streaming_prerouter_b200 as e0
-    from synth.device import layer_tensors, bf16_tensor
+    from synth.device import bf16_tensor
 
-    T = synth.WORKLOADS[args.workload]["tokens"]
+    T = synth.WORKLOADS[args.workload].get("tokens", T)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     t0 = time.time()
-    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, T)
-    lys, hds = zip(*[layer_tensors(seed, n, dims, dev) for n in range(dims.L)])
-    ctx.register_model(list(lys), list(hds))
+    lys, hds = _load_model(dims, seed, dev)
+    ctx = _context(dims, lys, hds, T)
     h = torch.stack([bf16_tensor(synth.prefill_hidden(seed, n, T, dims.d), dev) for n in range(dims.L)])
     setup_s = time.time() - t0
     y = torch.empty_like(h)
@@ -501,7 +630,7 @@ def run_prefill(args, dims, seed, ws, rank, local):
     step_s = ms / args.steps / 1e3
     # the dominant kernel: the expert GEMMs' FLOPs over their own measured launch time
     achieved = flops * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else flops / step_s / 1e12
-    traffic, traffic_how = kernel_traffic(args.workload)
+    traffic, traffic_how = kernel_traffic("prefill_t4096_l40")
     # end to end: the chunk's inputs from pinned host memory, its outputs back
     h_host = h.cpu().pin_memory()
     y_host = torch.empty_like(h_host).pin_memory()
@@ -520,7 +649,7 @@ def run_prefill(args, dims, seed, ws, rank, local):
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 weights as exact bf16 tensor-core operands (128+q), bf16 activations, fp32 accumulate",
         "data": "synthetic (seeded)",
-        "config": {"workload": args.workload, "layers": dims.L, "tokens": T, "d": dims.d, "experts": dims.E,
+        "config": {"workload": "prefill_t4096_l40", "layers": dims.L, "tokens": T, "d": dims.d, "experts": dims.E,
                    "d_ff": dims.I, "top_k": dims.k, "parallelism": f"replicas x{ws}",
                    "l2": "inputs larger than L2 (18.1 GB of expert weights)"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h.numel() * 2),
@@ -534,7 +663,7 @@ def run_prefill(args, dims, seed, ws, rank, local):
                      "traffic_note": traffic_how, "peak_source": pk["source"]},
         "clocks": clk.summary(), "setup_s": setup_s,
     }
-    return out, ctx
+    return out, ctx, h
 
 
 def h2d_probe_gbs(dev, nbytes=1 << 28):
@@ -554,83 +683,214 @@ def h2d_probe_gbs(dev, nbytes=1 << 28):
     return 4 * nbytes / (e0_.elapsed_time(e1_) / 1e3) / 1e9
 
 
-def run_stream(args, dims, seed, ws, rank, local):
-    """Streaming tier: experts in pinned host memory, staged into a 2 x k slot pool."""
+def _stream_case(ctx, dims, h_all, warm, steps, ws, local, link, B=1, e2e=False):
+    """Streamed decode steps; tok/s, host-link bytes per token and the staging accounting."""
+    import torch
+    y = torch.empty((dims.L, B, dims.d), dtype=torch.bfloat16, device=h_all.device)
+    for t in range(warm):
+        ctx.stack_decode(h_all[t], t, y_out=y, streaming=True)
+    ctx.sync_status()
+    s0 = ctx.stats()
+    ms, clocks, _ = _timed_steps(ctx, h_all, warm, steps, y, ws, local, streaming=True)
+    s1 = ctx.stats()
+    idx_rec = None
+    d = {k: s1[k] - s0[k] for k in s1}
+    ms = max_over_ranks(ms, ws)
+    tokens = sum_over_ranks(B * steps, ws)
+    wall_s = ms / 1e3
+    bpt = d["staged_bytes"] / (B * steps)
+    link_gbps = d["staged_bytes"] / wall_s / 1e9
+    req = d["staged_experts"] + d["hit_experts"]
+    out = {"value": tokens / wall_s, "unit": "tokens/s", "ms_per_step": ms / steps, "steps": steps, "batch": B,
+           "host_link_bytes_per_token": bpt, "link_GBps": link_gbps, "link_frac": link_gbps / link,
+           "stage_ms_per_step": d["stage_ms"] / steps, "exposed_wait_ms_per_step": d["exposed_wait_ms"] / steps,
+           "hidden_frac_of_staging": 1.0 - d["exposed_wait_ms"] / max(d["stage_ms"], 1e-9),
+           "link_busy_frac_of_wall": d["stage_ms"] / max(ms, 1e-9),
+           "copied_experts": int(d["staged_experts"]), "hit_experts": int(d["hit_experts"]),
+           "hit_rate": d["hit_experts"] / max(req, 1),
+           "prefetched_experts": int(d["prefetched_experts"]), "ondemand_experts": int(d["ondemand_experts"]),
+           "dropped": int(d["dropped"]), "gpu_launches": int(d["kernel_launches"]), "clocks": clocks,
+           "roofline": {"bound": "host link", "achieved": link_gbps, "peak": link, "unit": "GB/s",
+                        "frac": link_gbps / link, "traffic": None, "kernel": "staging copies (copy engine)",
+                        "peak_source": "pinned H2D probe in this run"}}
+    if e2e:
+        # the step's input from pinned host memory and its output back, through the C ABI
+        h_host = h_all[warm:warm + steps].cpu().pin_memory()
+        y_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
+        t_base = warm + steps
+        stream = torch.cuda.current_stream()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for t in range(steps):
+            ctx.stack_decode_host(h_host[t], t_base + t, y_host[t], streaming=True)
+        ctx.host_io_wait()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms_e = max_over_ranks(a.elapsed_time(b), ws)
+        out["e2e"] = {"value": tokens / (ms_e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h_host[0].numel() * 2),
+                      "d2h_bytes_per_step": int(y_host[0].numel() * 2)}
+    return out
+
+
+def run_stream(args, dims, seed, ws, rank, local, variants=True):
+    """Streaming tier: experts in pinned host memory, staged into HBM slot sets.  The
+    workload's configuration (two shared 4-slot sets, prefetch from the predictions) is the
+    headline; with `variants`, the same model also runs the fully reactive mode, persistent
+    sticky sets, and both on inputs shaped to the multi-stream routing statistics (next-token
+    reuse ~0.44), plus a least-recently-used HBM cache at batch 8."""
     import torch
     import int4_expert_streaming_prerouter_b200 as e0
-    from synth.device import layer_tensors, bf16_tensor, pinned_expert_store
+    from synth.device import bf16_tensor, pinned_expert_store
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     t0 = time.time()
-    ctx = e0.Context(dims.d, dims.E, dims.I, dims.k, dims.r, dims.L, 1)
-    lys, hds = zip(*[layer_tensors(seed, n, dims, dev, resident=False) for n in range(dims.L)])
-    ctx.register_model(list(lys), list(hds))
+    lys, hds = _load_model(dims, seed, dev, resident=False)
     store = pinned_expert_store(seed, dims)
-    ctx.stream_register(store, pool_layers=2, slots_per_layer=dims.k)
     setup_s = time.time() - t0
-    total = args.warmup + args.steps
-    h_all = torch.stack([bf16_tensor(synth.hidden(seed, t, dims.L, 1, dims.d), dev) for t in range(total)])
-    y = torch.empty((dims.L, 1, dims.d), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    for t in range(args.warmup):
-        ctx.stack_decode(h_all[t], t, y_out=y, streaming=True)
-    ctx.sync_status()
-    s0 = ctx.stats()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(ws)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        ev0.record(stream)
-        for t in range(args.warmup, total):
-            ctx.stack_decode(h_all[t], t, y_out=y, streaming=True)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    barrier(ws)
-    ctx.sync_status()
-    s1 = ctx.stats()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), ws)
-    tokens = sum_over_ranks(args.steps, ws)
-    d = {k: s1[k] - s0[k] for k in s1}
     link = h2d_probe_gbs(dev)
-    bytes_per_token = d["staged_bytes"] / args.steps
-    wall_s = ms / 1e3
+    warm, steps = args.warmup, args.steps
+    total = warm + 2 * steps + 2
+    h_all = torch.stack([bf16_tensor(synth.hidden(seed, t, dims.L, 1, dims.d), dev) for t in range(total)])
+
+    def case(pool_layers, slots, reactive, h, B=1, e2e=False):
+        ctx = _context(dims, lys, hds, B)
+        ctx.stream_register(store, pool_layers=pool_layers, slots_per_layer=slots)
+        ctx.stream_mode(reactive)
+        r = _stream_case(ctx, dims, h, warm, steps, ws, local, link, B=B, e2e=e2e)
+        idx, _ = ctx.get_routing(B)
+        ctx.close()
+        r["config"] = {"pool_sets": pool_layers, "slots_per_set": slots, "mode": "reactive" if reactive else "prefetch",
+                       "hbm_pool_MB": pool_layers * slots * synth.blob_bytes(dims.d, dims.I) / 1e6}
+        return r
+
+    head = case(2, dims.k, False, h_all, e2e=True)
     out = {
         "metric": "MoE-stack streaming decode tokens/s on 1 B200 (experts in pinned host memory)",
-        "value": tokens / wall_s, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "value": head["value"], "unit": "tokens/s", "n_gpus": ws, "steps": steps, "warmup": warm,
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int4 weights, fp32 accumulate", "data": "synthetic (seeded)",
-        "config": {"workload": args.workload, "layers": dims.L, "batch": 1, "pool": f"2 layers x {dims.k} slots",
+        "config": {"workload": "stream_b1_l40", "layers": dims.L, "batch": 1, "pool": f"2 layers x {dims.k} slots",
                    "host_store_GB": round(store.numel() / 1e9, 2), "parallelism": f"replicas x{ws}"},
-        "gpu_launches": int(d["kernel_launches"]),
-        "streaming": {"host_link_bytes_per_token": bytes_per_token, "h2d_probe_GBps": link,
-                      "link_GBps": bytes_per_token * tokens / wall_s / 1e9,
-                      "link_frac": bytes_per_token * tokens / wall_s / 1e9 / link,
-                      "stage_ms_per_token": d["stage_ms"] / args.steps,
-                      "exposed_wait_ms_per_token": d["exposed_wait_ms"] / args.steps,
-                      "hidden_frac_of_staging": 1.0 - d["exposed_wait_ms"] / max(d["stage_ms"], 1e-9),
-                      "link_busy_frac_of_wall": d["stage_ms"] / max(ms, 1e-9),
-                      "prefetched_experts": int(d["prefetched_experts"]),
-                      "ondemand_experts": int(d["ondemand_experts"]), "dropped": int(d["dropped"]),
-                      "hbm_pool_MB": 2 * dims.k * synth.blob_bytes(dims.d, dims.I) / 1e6},
-        "roofline": {"bound": "host link", "achieved": bytes_per_token * tokens / wall_s / 1e9, "peak": link,
-                     "unit": "GB/s", "frac": bytes_per_token * tokens / wall_s / 1e9 / link, "traffic": None,
-                     "kernel": "staging copies (copy engine)", "peak_source": "pinned H2D probe in this run"},
-        "clocks": clk.summary(), "setup_s": setup_s,
+        "gpu_launches": head["gpu_launches"], "e2e": head["e2e"],
+        "streaming": {k: v for k, v in head.items() if k not in ("roofline", "clocks", "e2e", "gpu_launches")},
+        "roofline": head["roofline"], "clocks": head["clocks"], "setup_s": setup_s,
+        "h2d_probe_GBps": link,
     }
-    return out, ctx
+    if variants:
+        var = {}
+        var["reactive_on_demand"] = case(2, dims.k, True, h_all)
+        var["sticky_per_layer_sets"] = case(dims.L, dims.k, False, h_all)
+        # the same model on inputs shaped to the multi-stream routing statistics
+        n_sh = warm + steps + 1
+        tg = synth.route_targets(seed, dims, 1, n_sh)
+        hs = torch.from_numpy(synth.shaped_hidden(seed, seed, dims, 1, tg).view(np.int16)).to(dev).view(torch.bfloat16)
+        for name, pl, sl, rv in (("shaped_prefetch_shared_sets", 2, dims.k, False),
+                                 ("shaped_sticky_per_layer_sets", dims.L, dims.k, False),
+                                 ("shaped_reactive_on_demand", 2, dims.k, True)):
+            r = case(pl, sl, rv, hs)
+            r["routing"] = synth.routing_stats(tg[warm:warm + steps])
+            var[name] = r
+        # batch 8 with a least-recently-used cache of 32 experts per layer
+        B = 8
+        tg8 = synth.route_targets(seed, dims, B, n_sh)
+        hs8 = torch.from_numpy(synth.shaped_hidden(seed, seed, dims, B, tg8).view(np.int16)).to(dev).view(torch.bfloat16)
+        for name, pl, sl in (("shaped_b8_shared_sets", 2, 32), ("shaped_b8_lru_cache_32", dims.L, 32),
+                             ("shaped_b8_lru_cache_64", dims.L, 64)):
+            r = case(pl, sl, False, hs8, B=B)
+            r["routing"] = synth.routing_stats(tg8[warm:warm + steps])
+            var[name] = r
+        out["variants"] = var
+    return out, store
+
+
+def run_multistream(args, dims, seed, ws, rank, local, batches=(8, 32, 64)):
+    """Batched decode on inputs shaped to the pages' multi-stream routing statistics
+    (next-token reuse ~0.44, Zipf popularity).  Algorithmic bytes come from the realised
+    distinct experts of every layer and step."""
+    import torch
+    from synth.device import bf16_tensor
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lys, hds = _load_model(dims, seed, dev)
+    pk = peaks()
+    res = {}
+    warm, steps = 3, min(args.steps, 24)
+    for B in batches:
+        tg = synth.route_targets(seed, dims, B, warm + steps + 1)
+        hs_np = synth.shaped_hidden(seed, seed, dims, B, tg)
+        h_all = torch.from_numpy(hs_np.view(np.int16)).to(dev).view(torch.bfloat16)
+        ctx = _context(dims, lys, hds, B)
+        y = torch.empty((dims.L, B, dims.d), dtype=torch.bfloat16, device=dev)
+        for t in range(warm):
+            ctx.stack_decode(h_all[t], t, y_out=y)
+        # per-step routing for the realised unique-expert bytes
+        ctx.sync_status()
+        idx_steps, exp_total = [], 0
+        ms_sum = 0.0
+        clocks = None
+        launches = 0
+        for t in range(warm, warm + steps):
+            ms, clocks_t, l_t = _timed_steps(ctx, h_all, t, 1, y, ws, local)
+            ms_sum += ms
+            launches += l_t
+            clocks = clocks_t if clocks is None else clocks
+            idx, _ = ctx.get_routing(B)
+            idx_steps.append(idx)
+            exp_total += step_bytes(dims, idx, B)[0]
+        # one uninterrupted timed region for the tokens/s figure
+        ctx.close()
+        ctx = _context(dims, lys, hds, B)
+        for t in range(warm):
+            ctx.stack_decode(h_all[t], t, y_out=y)
+        ms_run, clk_run, l_run = _timed_steps(ctx, h_all, warm, steps, y, ws, local)
+        ms_run = max_over_ranks(ms_run, ws)
+        # end to end with host buffers
+        h_host = h_all[warm:warm + steps].cpu().pin_memory()
+        y_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
+        stream = torch.cuda.current_stream()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for t in range(steps):
+            ctx.stack_decode_host(h_host[t], warm + steps + t, y_host[t])
+        ctx.host_io_wait()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms_e = max_over_ranks(a.elapsed_time(b), ws)
+        ctx.close()
+        tokens = sum_over_ranks(B * steps, ws)
+        st = synth.routing_stats(np.stack(idx_steps))
+        res[f"b{B}"] = {
+            "value": tokens / (ms_run / 1e3), "unit": "tokens/s", "ms_per_step": ms_run / steps, "steps": steps,
+            "batch": B, "path": "phased kernels" if B <= 8 else "per-layer kernels",
+            "gpu_launches": int(l_run), "clocks": clk_run,
+            "routing": dict(st, matches_targets=bool(np.array_equal(np.sort(np.stack(idx_steps), -1),
+                                                                    np.sort(tg[warm:warm + steps], -1)))),
+            "roofline": _hbm_roofline(exp_total / steps, ms_run / steps, pk,
+                                      "decode step (realised distinct experts of every layer + shared)"),
+            "e2e": {"value": tokens / (ms_e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h_host[0].numel() * 2),
+                    "d2h_bytes_per_step": int(y_host[0].numel() * 2)},
+        }
+        del h_all
+        _free_gpu()
+    return res
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1024)
+    ap.add_argument("--steps", type=int, default=256)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--workload", default="decode_b1_l40")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--decode-mode", type=int, default=0, help="0 default, 1 one-launch, 2 graph, 3 eager")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="only the named workload (default run adds the other workloads as sub-objects)")
+    ap.add_argument("--decode-mode", type=int, default=0,
+                    help="0 default, 1 one-launch, 2 graph, 3 eager per-layer, 4 phased")
     ap.add_argument("--decode-flat", type=int, default=None,
                     help="one-launch kernel on unchained steps: 1 flat schedule (default), 0 layers in order")
     args = ap.parse_args()
@@ -641,25 +901,63 @@ def main():
     if args.impl == "reference":
         run_reference(args, dims, seed, ws, rank)
         return
+    cpu = not args.no_cpu_baseline and rank == 0 and ws == 1
     if args.workload.startswith("stream"):
-        out, ctx = run_stream(args, dims, seed, ws, rank, local)
+        out, _ = run_stream(args, dims, seed, ws, rank, local, variants=not args.no_extras)
         if rank == 0:
             print(json.dumps(out), flush=True)
-        ctx.close()
         return
     if "tokens" in wl:
-        out, ctx = run_prefill(args, dims, seed, ws, rank, local)
+        out, ctx, _ = run_prefill(args, dims, seed, ws, rank, local)
+        if cpu:
+            import torch  # noqa: F401
+            hs = synth.prefill_hidden(seed, 0, wl["tokens"], dims.d)[:256]
+            out["cpu_baseline"] = cpu_baseline_tokens(dims, seed, hs, 0, dims.L, "256 of the chunk's 4096 tokens")
         if rank == 0:
             print(json.dumps(out), flush=True)
         ctx.close()
         return
     B = args.batch or (wl["batch"] if isinstance(wl.get("batch"), int) else 8)
-    out, ctx = run_decode(args, dims, seed, B, ws, rank, local)
-    if rank == 0:
-        if not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline(dims, seed)
-        print(json.dumps(out), flush=True)
+    extras = not args.no_extras and ws == 1 and args.workload == "decode_b1_l40" and B == 1
+    out, ctx = run_decode(args, dims, seed, B, ws, rank, local, extras)
     ctx.close()
+    if cpu:
+        out["cpu_baseline"] = cpu_baseline(dims, seed)
+    if extras:
+        # the other workloads of the same model family, each with its own timing, roofline,
+        # clocks, end-to-end figure and CPU baseline
+        _free_gpu()
+        pargs = argparse.Namespace(**vars(args))
+        pargs.steps, pargs.warmup = 3, 2
+        pwl = synth.WORKLOADS["prefill_t4096_l40"]
+        pre, pctx, _ = run_prefill(pargs, pwl["dims"], pwl["seed"], ws, rank, local)
+        pctx.close()
+        if cpu:
+            hs = synth.prefill_hidden(pwl["seed"], 0, pwl["tokens"], dims.d)[:256]
+            pre["cpu_baseline"] = cpu_baseline_tokens(pwl["dims"], pwl["seed"], hs, 0, dims.L,
+                                                      "256 of the chunk's 4096 tokens")
+        out["prefill_t4096_l40"] = pre
+        _free_gpu()
+        sargs = argparse.Namespace(**vars(args))
+        sargs.steps, sargs.warmup = 16, 3
+        swl = synth.WORKLOADS["stream_b1_l40"]
+        st, store = run_stream(sargs, swl["dims"], swl["seed"], ws, rank, local, variants=True)
+        del store
+        if cpu:
+            st["cpu_baseline"] = dict(out.get("cpu_baseline", {}), sample="the streaming tier computes exactly the "
+                                      "resident decode step; its CPU baseline is the decode oracle's (this run)")
+        out["stream_b1_l40"] = st
+        _free_gpu()
+        mwl = synth.WORKLOADS["decode_multistream_l40"]
+        ms_res = run_multistream(args, mwl["dims"], mwl["seed"], ws, rank, local)
+        if cpu:
+            tg = synth.route_targets(mwl["seed"], mwl["dims"], 8, 1)
+            hs8 = synth.shaped_hidden(mwl["seed"], mwl["seed"], mwl["dims"], 8, tg)
+            ms_res["cpu_baseline"] = cpu_baseline_tokens(mwl["dims"], mwl["seed"], hs8[0, 0], 0, dims.L,
+                                                         "one step of the batch-8 streams")
+        out["decode_multistream_l40"] = ms_res
+    if rank == 0:
+        print(json.dumps(out), flush=True)
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -286,12 +286,23 @@ int e0_debug_decode_stall(e0_ctx *ctx, int cta, unsigned long long timeout_ns);
  * was created with max_tokens >= 64.  For comparisons between the two paths. */
 int e0_debug_prefill_path(e0_ctx *ctx, int mode);
 /* Decode implementation of e0_moe_stack_decode (resident experts): 0 = default (the
- * one-launch kernel at B = 1, per-layer kernels otherwise),
- * 1 = one-launch kernel, 2 = graph replay, 3 = per-layer kernels launched one by one. */
+ * one-launch kernel at B = 1 where it applies, the phased kernels for unchained steps of
+ * up to 8 streams, per-layer kernels otherwise), 1 = one-launch kernel, 2 = graph replay
+ * of the per-layer kernels, 3 = per-layer kernels launched one by one, 4 = phased kernels
+ * (six kernels per step over every layer, programmatic dependent launch; unchained steps,
+ * B <= 8, head_hidden <= 512; other steps fall back to the default). */
 int e0_debug_decode_mode(e0_ctx *ctx, int mode);
 /* Profiling: the following one-launch decode steps write %globaltimer stamps (uint64,
  * [grid][L][16], caller-owned device buffer; NULL stops it).  Returns the grid size. */
 int e0_debug_decode_trace(e0_ctx *ctx, unsigned long long *buf);
+/* Profiling of the phased decode kernels: e0_debug_phase_timing(ctx, 1) makes the
+ * following phased steps launch their six kernels one after another (no programmatic
+ * overlap) with a CUDA event before each and after the last; e0_debug_phase_times adds the
+ * elapsed times up per kernel (ms6[0..5]: norm, bf16 rows, routing, gate/up, sums and t_d,
+ * down), synchronising on the events, and reports how many steps were timed since the
+ * context was created.  Results are unchanged. */
+int e0_debug_phase_timing(e0_ctx *ctx, int on);
+int e0_debug_phase_times(e0_ctx *ctx, double *ms6, unsigned long long *steps);
 int e0_debug_force_general(e0_ctx *ctx, int on);
 /* Schedule of the one-launch decode kernel on unchained steps (every layer's input
  * given, none read from another layer's output): 1 (default) = flat — each phase's work

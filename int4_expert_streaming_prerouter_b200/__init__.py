@@ -90,6 +90,8 @@ _SIGS = {
     "e0_debug_decode_mode": (_I, [_P, _I]),
     "e0_debug_decode_flat": (_I, [_P, _I]),
     "e0_debug_time_gemm": (_I, [_P, _I]),
+    "e0_debug_phase_timing": (_I, [_P, _I]),
+    "e0_debug_phase_times": (_I, [_P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_ulonglong)]),
     "e0_decode_items": (_I, [ctypes.POINTER(Dims), _I, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_uint8),
                              _I, _I, _I, _I, ctypes.POINTER(ctypes.c_uint64), _I, ctypes.POINTER(_I)]),
 }
@@ -323,6 +325,17 @@ class Context:
 
     def debug_decode_mode(self, mode: int):
         _check(lib().e0_debug_decode_mode(self._h, mode))
+
+    def debug_phase_timing(self, on: bool):
+        _check(lib().e0_debug_phase_timing(self._h, int(on)))
+
+    def debug_phase_times(self):
+        """(per-kernel summed ms of the phased decode kernels [norm, rows, route, gate/up,
+        sums+t_d, down], steps timed)."""
+        ms = (ctypes.c_double * 6)()
+        n = ctypes.c_ulonglong(0)
+        _check(lib().e0_debug_phase_times(self._h, ms, ctypes.byref(n)))
+        return list(ms), int(n.value)
 
     def debug_time_gemm(self, on: bool):
         _check(lib().e0_debug_time_gemm(self._h, int(on)))

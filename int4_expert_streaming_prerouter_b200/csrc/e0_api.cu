@@ -5,6 +5,7 @@
 #include "e0moe.h"
 #include "e0_kernels.cuh"
 #include "e0_decode.cuh"
+#include "e0_phased.cuh"
 #include "e0_prefill.cuh"
 
 #include <cudaTypedefs.h>
@@ -103,6 +104,38 @@ static void decode_free(DecodeState &S) {
   S = DecodeState{};
 }
 
+// Phased decode state: the device layer table, the workspace (token stride kPhMaxB) and
+// the bf16-rows work lists, one per (batch, first step or not).
+struct PhState {
+  bool ready = false;
+  PhLayer *d_layers = nullptr;
+  void *mem = nullptr;                   // one allocation for the whole workspace
+  uint16_t *x16 = nullptr, *xp = nullptr, *a = nullptr;
+  float *xs = nullptr, *rlog = nullptr, *rsel = nullptr, *hlog = nullptr, *lt = nullptr, *h1 = nullptr,
+        *gates = nullptr, *asum = nullptr, *gus = nullptr;
+  int *plan = nullptr;                   // [2][L][kPlanInts], by step parity
+  int8_t *slot = nullptr;                // [2][L][kPhMaxU][kPhMaxB]
+  int last_step = -1;                    // the last step that ran the phased kernels
+  PhBlock *blocks[2 * (kPhMaxB + 1)] = {};
+  int nblocks[2 * (kPhMaxB + 1)] = {};
+  // profiling: kernels launched one after another with an event before each and after the
+  // last (7 per step), accounted by e0_debug_phase_times
+  bool timing = false;
+  std::vector<std::vector<cudaEvent_t>> pending;
+  double ms[6] = {};
+  unsigned long long steps_timed = 0;
+};
+
+static void phased_free(PhState &S) {
+  for (auto &v : S.pending)
+    for (auto e : v) cudaEventDestroy(e);
+  if (S.d_layers) cudaFree(S.d_layers);
+  if (S.mem) cudaFree(S.mem);
+  for (auto *b : S.blocks)
+    if (b) cudaFree(b);
+  S = PhState{};
+}
+
 // One captured decode step (the per-layer kernel sequence of every layer) and its key.
 struct DecodeGraph {
   cudaGraphExec_t exec = nullptr;
@@ -150,6 +183,7 @@ struct e0_ctx {
   int32_t *pf_buf = nullptr;         // prefill: [2][maxT+1][k] head predictions, row 0 = -1
   int32_t *pf_idx = nullptr;         // prefill: [maxT+1][k] routing scratch, row 0 = -1
   DecodeState dec{};
+  PhState ph{};
   StreamPool pool;
   e0_stats stats{};
   bool time_gemm = false;                          // profiling: event pairs around the GEMMs
@@ -200,6 +234,7 @@ extern "C" int e0_destroy(e0_ctx *C) {
   for (void *b : bufs)
     if (b) cudaFree(b);
   decode_free(C->dec);
+  phased_free(C->ph);
   for (auto &g : C->graphs)
     if (g.exec) cudaGraphExecDestroy(g.exec);
   if (C->cap) cudaStreamDestroy(C->cap);
@@ -323,6 +358,7 @@ extern "C" int e0_register_model(e0_ctx *C, const e0_layer *layers, const e0_hea
   if (heads) C->heads.assign(heads, heads + C->L);
   C->registered = true;
   C->dec.ready = false;
+  C->ph.ready = false;
   for (auto &g : C->graphs) {   // captured pointers belong to the previous registration
     if (g.exec) cudaGraphExecDestroy(g.exec);
     g = DecodeGraph{};
@@ -1075,6 +1111,200 @@ static int decode_persistent(e0_ctx *C, const uint16_t *h, int step, uint16_t *y
   return E0_OK;
 }
 
+// ---------------------------------------------------------------------------------------
+// Phased decode path (unchained steps of up to kPhMaxB streams, resident experts)
+// ---------------------------------------------------------------------------------------
+static bool phased_geometry(const e0_dims &Dm, int *which) {
+  if (Dm.d_model == 2048 && Dm.d_ff == 512) *which = 0;
+  else if (Dm.d_model == 256 && Dm.d_ff == 128) *which = 1;
+  else return false;
+  return true;
+}
+
+static bool phased_supported(e0_ctx *C, int B) {
+  const e0_dims &D = C->dims;
+  int which;
+  if (B < 1 || B > kPhMaxB || !phased_geometry(D, &which) || C->L > 64 || D.head_hidden > kPhMaxH ||
+      D.head_hidden % 16 != 0)
+    return false;
+  for (int l = 0; l < C->L; l++)
+    if (!C->layers[l].experts) return false;
+  return true;
+}
+
+static int phased_prepare(e0_ctx *C) {
+  PhState &S = C->ph;
+  if (S.ready) return E0_OK;
+  const e0_dims &D = C->dims;
+  const int L = C->L;
+  std::vector<PhLayer> h(L);
+  for (int l = 0; l < L; l++) {
+    const e0_layer &Y = C->layers[l];
+    const e0_head &H = C->heads[l];
+    h[l] = PhLayer{(const uint8_t *)Y.experts, (const uint8_t *)Y.shared, (const uint16_t *)Y.router_w,
+                   (const uint16_t *)Y.norm_w, (const uint16_t *)H.w_lin, (const uint16_t *)H.fc1_w,
+                   (const uint16_t *)H.fc1_b, (const uint16_t *)H.fc2_w, (const uint16_t *)H.fc2_b,
+                   (const uint16_t *)Y.lora_Ag, (const uint16_t *)Y.lora_Bg, (const uint16_t *)Y.lora_Au,
+                   (const uint16_t *)Y.lora_Bu, (const uint16_t *)Y.lora_Ad, (const uint16_t *)Y.lora_Bd};
+  }
+  int rc;
+  if (!S.d_layers && (rc = dalloc(&S.d_layers, L))) return rc;
+  CK(cudaMemcpy(S.d_layers, h.data(), L * sizeof(PhLayer), cudaMemcpyHostToDevice));
+  if (!S.mem) {
+    const size_t T = (size_t)L * kPhMaxB, d = D.d_model, E = D.n_experts, I = D.d_ff, k = D.top_k;
+    const size_t r = std::max(D.lora_rank, 1), H = std::max(D.head_hidden, 1);
+    // sizes in 4-byte words, each region rounded to 16 bytes
+    auto w4 = [](size_t bytes) { return (bytes + 15) / 16 * 4; };
+    const size_t n_x16 = w4(T * d * 2), n_xp = w4(T * d * 2), n_a = w4(T * (k + 1) * I * 2), n_xs = w4(T * (d / 64) * 4),
+                 n_rl = w4(T * E * 4), n_rs = w4(T * k * 4), n_hl = w4(T * E * 4), n_lt = w4(T * 3 * r * 4),
+                 n_h1 = w4(T * H * 4), n_g = w4(T * k * 4), n_as = w4(T * (k + 1) * (I / 64) * 4),
+                 n_pl = w4((size_t)2 * L * kPlanInts * 4), n_sl = w4((size_t)2 * L * kPhMaxU * kPhMaxB),
+                 n_gus = w4(T * 2 * I * 4);
+    const size_t tot = n_x16 + n_xp + n_a + n_xs + n_rl + n_rs + n_hl + n_lt + n_h1 + n_g + n_as + n_pl + n_sl + n_gus;
+    uint32_t *p = nullptr;
+    if ((rc = dalloc(&p, tot))) return rc;
+    CK(cudaMemset(p, 0, tot * 4));
+    S.mem = p;
+    S.x16 = (uint16_t *)p; p += n_x16;
+    S.xp = (uint16_t *)p; p += n_xp;
+    S.a = (uint16_t *)p; p += n_a;
+    S.xs = (float *)p; p += n_xs;
+    S.rlog = (float *)p; p += n_rl;
+    S.rsel = (float *)p; p += n_rs;
+    S.hlog = (float *)p; p += n_hl;
+    S.lt = (float *)p; p += n_lt;
+    S.h1 = (float *)p; p += n_h1;
+    S.gates = (float *)p; p += n_g;
+    S.asum = (float *)p; p += n_as;
+    S.plan = (int *)p; p += n_pl;
+    S.slot = (int8_t *)p; p += n_sl;
+    S.gus = (float *)p;
+  }
+  int which;
+  phased_geometry(D, &which);
+  // the down kernel's dynamic shared memory at the largest batch
+  const size_t dn_max = which == 0 ? ph_dn_smem<2048, 512>(kPhMaxB, D.top_k) : ph_dn_smem<256, 128>(kPhMaxB, D.top_k);
+  const void *dn = which == 0 ? (const void *)k_ph_down<2048, 512> : (const void *)k_ph_down<256, 128>;
+  CK(cudaFuncSetAttribute(dn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn_max));
+  S.ready = true;
+  return E0_OK;
+}
+
+// The bf16-rows work list for batch B, first step or not (built once per shape).
+static int phased_blocks(e0_ctx *C, int B, bool step0, const PhBlock **out, int *n) {
+  PhState &S = C->ph;
+  const int v = 2 * B + (step0 ? 1 : 0);
+  if (!S.blocks[v]) {
+    PhShape Z{};
+    Z.L = C->L; Z.E = C->dims.n_experts; Z.k = C->dims.top_k; Z.r = C->dims.lora_rank; Z.H = C->dims.head_hidden;
+    Z.B = B;
+    for (int l = 0; l < C->L; l++) {
+      Z.head[l] = C->heads[l].w_lin != nullptr;
+      Z.lora[l] = C->layers[l].lora_Ag != nullptr;
+    }
+    const std::vector<PhBlock> bl = ph_blocks(Z, step0);
+    int rc;
+    if ((rc = dalloc(&S.blocks[v], bl.size()))) return rc;
+    CK(cudaMemcpy(S.blocks[v], bl.data(), bl.size() * sizeof(PhBlock), cudaMemcpyHostToDevice));
+    S.nblocks[v] = (int)bl.size();
+  }
+  *out = S.blocks[v];
+  *n = S.nblocks[v];
+  return E0_OK;
+}
+
+// Launch one kernel of the phased step; pdl = it may start while the previous kernel on the
+// stream is still running (it waits with griddepcontrol.wait before reading its outputs).
+template <typename Kern>
+static cudaError_t ph_launch(Kern kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t s, bool pdl,
+                             const PhParams &P) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? at : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, P);
+}
+
+template <int D, int I>
+static int phased_launch(e0_ctx *C, const PhParams &P, cudaStream_t s) {
+  const int L = P.L, B = P.B;
+  const int Umax = std::min(B * P.k, P.E) + 1;
+  PhState &S = C->ph;
+  // profiling: no overlap between the kernels, an event before each and after the last
+  const bool tm = S.timing;
+  std::vector<cudaEvent_t> ev;
+  if (tm) {
+    ev.resize(7);
+    for (auto &e : ev) CK(cudaEventCreate(&e));
+  }
+  int q = 0;
+#define PHL(call, what)                                                                     \
+  do {                                                                                     \
+    if (tm) CK(cudaEventRecord(ev[q++], s));                                               \
+    C->stats.kernel_launches++;                                                            \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess) return fail(E0_ERR_CUDA, "launch %s: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+  const bool pdl = !tm;
+  // the first kernel waits for the previous step in full (stream order): whatever the later
+  // kernels read before their wait (weights, the previous step's predictions) is complete
+  PHL(ph_launch(k_ph_norm<D>, L * B, 256, 0, s, false, P), "k_ph_norm");
+  PHL(ph_launch(k_ph_rows<D>, P.nblocks, 32 * PhRowsCfg<D>::NW, 0, s, pdl, P), "k_ph_rows");
+  PHL(ph_launch(k_ph_route, L, 256, 0, s, pdl, P), "k_ph_route");
+  PHL(ph_launch(k_ph_gateup<D, I>, L * Umax * (I / 8), 32 * (D / 256), 0, s, pdl, P), "k_ph_gateup");
+  PHL(ph_launch(k_ph_tdsum<I>, L * B, 256, 0, s, pdl, P), "k_ph_tdsum");
+  PHL(ph_launch(k_ph_down<D, I>, L * (D / 16), 32 * (I / 64), ph_dn_smem<D, I>(B, P.k), s, pdl, P), "k_ph_down");
+#undef PHL
+  if (tm) {
+    CK(cudaEventRecord(ev[6], s));
+    S.pending.push_back(ev);
+  }
+  return E0_OK;
+}
+
+static int decode_phased(e0_ctx *C, const uint16_t *h, int B, int step, uint16_t *y, float *yf, cudaStream_t s) {
+  int rc = phased_prepare(C);
+  if (rc) return rc;
+  PhState &S = C->ph;
+  const e0_dims &D = C->dims;
+  const int cur = step & 1, prv = cur ^ 1;
+  PhParams P{};
+  P.layers = S.d_layers;
+  P.L = C->L; P.B = B; P.E = D.n_experts; P.k = D.top_k; P.r = D.lora_rank; P.H = D.head_hidden;
+  P.ldh = D.d_model + (D.head_onehot ? 2 * D.n_experts : 0);
+  P.onehot = D.head_onehot; P.step0 = step == 0; P.maxT = C->maxT;
+  P.eps = D.rms_eps; P.c = D.lora_scale;
+  P.h = h; P.y = y; P.yf = yf;
+  P.x16 = S.x16; P.xp = S.xp; P.xs = S.xs; P.rlog = S.rlog; P.rsel = S.rsel; P.hlog = S.hlog; P.lt = S.lt;
+  P.h1 = S.h1; P.gates = S.gates; P.a = S.a; P.asum = S.asum; P.gus = S.gus;
+  P.plan_cur = S.plan + (size_t)cur * C->L * kPlanInts;
+  P.plan_next = S.plan + (size_t)prv * C->L * kPlanInts;
+  P.slot_cur = S.slot + (size_t)cur * C->L * kPhMaxU * kPhMaxB;
+  P.slot_next = S.slot + (size_t)prv * C->L * kPhMaxU * kPhMaxB;
+  P.pred_in = step > 0 ? pred_at(C, prv, 0) : nullptr;
+  P.pred_out = pred_at(C, cur, 0);
+  P.hist_out = hist_at(C, cur, 0);
+  P.hist_prev = step > 0 ? hist_at(C, prv, 0) : nullptr;
+  P.err = C->err;
+  if ((rc = phased_blocks(C, B, step == 0, &P.blocks, &P.nblocks))) return rc;
+  if (step > 0 && S.last_step != step - 1) {
+    // the previous step ran another path: the predicted layers' plans come from its predictions
+    k_ph_plan_pred<<<C->L, 32, 0, s>>>(P);
+    CKL("k_ph_plan_pred");
+  }
+  int which;
+  phased_geometry(D, &which);
+  rc = which == 0 ? phased_launch<2048, 512>(C, P, s) : phased_launch<256, 128>(C, P, s);
+  S.last_step = rc == E0_OK ? step : -1;
+  return rc;
+}
+
 // Test hook: make CTA `cta` of the next persistent decode launch wait on a word nobody
 // writes, with a wait budget of `timeout_ns`; the launch must come back with TIMEOUT.
 extern "C" int e0_debug_decode_stall(e0_ctx *C, int cta, unsigned long long timeout_ns) {
@@ -1152,11 +1382,17 @@ extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step,
   C->last = s;
   int rc;
   const bool one_launch = decode_supported(C, B);
+  const bool phased = !chained && phased_supported(C, B);
   int mode = C->force_general ? 3 : C->decode_mode;
-  if (mode == 0) mode = one_launch ? 1 : 3;   // default: measured fastest per batch
+  // default: the measured fastest per batch: at one stream the one-launch kernel, up to
+  // kPhMaxB streams the phased kernels, beyond that the per-layer kernels
+  if (mode == 0) mode = one_launch ? 1 : phased ? 4 : 3;
+  if (mode == 4 && !phased) mode = one_launch ? 1 : 3;
   if (mode == 1 && !one_launch) mode = 2;
   if (streaming) mode = 3;                                  // host decisions between layers
-  if (mode == 1)
+  if (mode == 4)
+    rc = decode_phased(C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, s);
+  else if (mode == 1)
     rc = decode_persistent(C, (const uint16_t *)h_in, step, (uint16_t *)y_out, y_f32, chained, s);
   else if (mode == 2)
     rc = decode_graph(C, (const uint16_t *)h_in, B, step, (uint16_t *)y_out, y_f32, chained, s);
@@ -1354,10 +1590,38 @@ extern "C" int e0_debug_prefill_path(e0_ctx *C, int mode) {
 }
 
 // Decode implementation: 0 = default, 1 = one-launch kernel (B = 1), 2 = CUDA-graph replay
-// of the per-layer kernels, 3 = per-layer kernels launched one by one.
+// of the per-layer kernels, 3 = per-layer kernels launched one by one, 4 = phased kernels.
 extern "C" int e0_debug_decode_mode(e0_ctx *C, int mode) {
-  if (!C || mode < 0 || mode > 3) return fail(E0_ERR_INVALID_ARG, "bad decode mode");
+  if (!C || mode < 0 || mode > 4) return fail(E0_ERR_INVALID_ARG, "bad decode mode");
   C->decode_mode = mode;
+  return E0_OK;
+}
+
+// Profiling of the phased decode path: on = 1 launches its six kernels one after another
+// (no programmatic overlap) with an event before each; e0_debug_phase_times adds up the
+// kernels' durations over the timed steps.
+extern "C" int e0_debug_phase_timing(e0_ctx *C, int on) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  C->ph.timing = on != 0;
+  return E0_OK;
+}
+
+extern "C" int e0_debug_phase_times(e0_ctx *C, double *ms6, unsigned long long *steps) {
+  if (!C || !ms6 || !steps) return fail(E0_ERR_INVALID_ARG, "NULL argument");
+  PhState &S = C->ph;
+  for (auto &v : S.pending) {
+    CK(cudaEventSynchronize(v[6]));
+    for (int q = 0; q < 6; q++) {
+      float ms = 0.f;
+      CK(cudaEventElapsedTime(&ms, v[q], v[q + 1]));
+      S.ms[q] += ms;
+    }
+    S.steps_timed++;
+    for (auto e : v) cudaEventDestroy(e);
+  }
+  S.pending.clear();
+  for (int q = 0; q < 6; q++) ms6[q] = S.ms[q];
+  *steps = S.steps_timed;
   return E0_OK;
 }
 

@@ -264,3 +264,89 @@ def hidden_for_logits(W: np.ndarray, target: np.ndarray, d: int, rng: np.random.
         noise *= np.sqrt(need / float(noise @ noise))
         x = x + noise
     return x
+
+
+def shaped_hidden(seed: int, wseed: int, dims: Dims, B: int, targets: np.ndarray, margin: float = 1.5) -> np.ndarray:
+    """Decode inputs ``[steps, L, B, d]`` (bf16 bits) shaped so that the routing the stack
+    takes is ``targets [steps, L, B, k]`` (e.g. from :func:`route_targets`).
+
+    The routing of layer n at step t comes from layer n's router on its own input when n
+    routes itself (step 0, layer 0, layers after a layer without a head), and from layer
+    n-1's prerouter head on its input of step t-1 otherwise.  So the input of (t, n) is
+    drawn to meet up to two sets of linear constraints: router rows giving logits whose
+    top-k is targets[t, n] (when n routes itself at t), and head rows giving logits whose
+    top-k is targets[t+1, n+1] (when n carries a head).  Target logits: the chosen experts
+    at 3.0, 2.9, ... in rank order, the others ~ N(0, 0.4^2) clipped below 3.0 - margin.
+    The least-norm solution plus noise orthogonal to the constraint rows, scaled to unit
+    RMS, is rounded to bf16 (RMSNorm then leaves the top-k sets unchanged: it is a
+    positive scale).  Uses the bf16 router/head weights of ``layer_dense(wseed, n)``; linear
+    heads only.  The realised routing is measured by the caller, not assumed.
+    """
+    S, L, Bt, k = targets.shape
+    assert Bt == B and L == dims.L and dims.head_hidden == 0 and not dims.head_onehot
+    d, E = dims.d, dims.E
+    g = _rng(seed, _T_ROUTE, 1, 0)
+    out = np.empty((S, L, B, d), dtype=np.uint16)
+
+    def target_logits(sets):                     # sets [N, k] -> [N, E]
+        z = np.clip(g.standard_normal((sets.shape[0], E)) * 0.4, None, 3.0 - margin)
+        for j in range(k):
+            z[np.arange(sets.shape[0]), sets[:, j]] = 3.0 - 0.1 * j
+        return z
+
+    def bf(bits):
+        return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    for n in range(L):
+        dense = layer_dense(wseed, n, dims)
+        Wr = bf(dense["router_w"])
+        Wh = bf(dense["head_w"]) if dense.get("head_w") is not None else None
+        own_always = n == 0 or (n - 1) not in dims.head_layers
+        for step_set in ((0,), tuple(range(1, S))) if not own_always else (tuple(range(S)),):
+            if not step_set:
+                continue
+            own = own_always or step_set == (0,)
+            rows, zs = [], []
+            ts = np.array(step_set)
+            if own:
+                rows.append(Wr)
+                zs.append(target_logits(targets[ts, n].reshape(-1, k)).reshape(len(ts), B, E))
+            if Wh is not None:
+                nxt = np.minimum(ts + 1, S - 1)
+                zh = target_logits(targets[nxt, min(n + 1, L - 1)].reshape(-1, k)).reshape(len(ts), B, E)
+                rows.append(Wh)
+                zs.append(zh)
+            if not rows:
+                x = g.standard_normal((len(ts) * B, d))
+            else:
+                W = np.concatenate(rows, 0)                          # [m, d]
+                Z = np.concatenate(zs, 2).reshape(len(ts) * B, -1)   # [N, m]
+                q, r = np.linalg.qr(W.T)                            # W.T = q r
+                x = np.linalg.solve(r.T, Z.T).T @ q.T               # least-norm: W x = z
+                noise = g.standard_normal(x.shape)
+                noise -= (noise @ q) @ q.T
+                need = d - np.sum(x * x, axis=1, keepdims=True)
+                scale = np.sqrt(np.maximum(need, 0.0) / np.maximum(np.sum(noise * noise, axis=1, keepdims=True), 1e-30))
+                x = x + noise * scale
+            out[ts, n] = f32_to_bf16_bits(x.astype(np.float32)).reshape(len(ts), B, d)
+    return out
+
+
+def routing_stats(idx: np.ndarray) -> dict:
+    """Realised next-token expert reuse and popularity concentration of a routing record
+    ``[steps, L, B, k]``: reuse = mean over (step > 0, layer, stream) of the fraction of the
+    k experts that the same stream used at the previous step; share95 = mean over layers
+    of the fraction of experts that carry 95 % of that layer's assignments."""
+    S, L, B, k = idx.shape
+    reuse = []
+    for t in range(1, S):
+        for n in range(L):
+            for b in range(B):
+                reuse.append(len(set(idx[t, n, b].tolist()) & set(idx[t - 1, n, b].tolist())) / k)
+    shares = []
+    for n in range(L):
+        c = np.sort(np.bincount(idx[:, n].reshape(-1), minlength=int(idx.max()) + 1))[::-1]
+        cum = np.cumsum(c) / c.sum()
+        E = max(int(idx.max()) + 1, 1)
+        shares.append((int(np.searchsorted(cum, 0.95)) + 1) / E)
+    return {"next_token_reuse": float(np.mean(reuse)) if reuse else None, "experts_for_95pct": float(np.mean(shares))}

@@ -72,11 +72,17 @@ def full_model(cuda_ok):
     ctx.close()
 
 
-def test_full_size_decode_b1_sampled(full_model):
-    """Two steps of the 40-layer stack at B=1 in the bench's launch configuration: every
-    layer's routing and head prediction exactly, and y on every layer of both steps."""
+@pytest.mark.parametrize("mode", [4, 1])
+def test_full_size_decode_b1_sampled(full_model, mode):
+    """Two steps of the 40-layer stack at B=1 (the phased kernels, the default, and the
+    one-launch kernel): every layer's routing and head prediction exactly, and y on every
+    layer of both steps."""
     S = 2
-    gpu = run_steps(full_model, FULL, 1, 1, S)
+    full_model.debug_decode_mode(mode)
+    try:
+        gpu = run_steps(full_model, FULL, 1, 1, S)
+    finally:
+        full_model.debug_decode_mode(0)
     ref = oracle_steps(FULL, 1, 1, S, gpu[2], gpu[3])
     compare_steps(FULL, gpu, ref)
 
@@ -100,6 +106,7 @@ def test_full_size_decode_b8_sampled_layers(full_model):
 # ---------------------------------------------------------------------------------------
 def test_one_launch_decode_equals_general_path_small(cuda_ok):
     ctx, _, _ = build(SMALL, 90, 4)
+    ctx.debug_decode_mode(1)
     ref, _, _ = build(SMALL, 90, 4)
     ref.debug_force_general(True)
     for t in range(5):
@@ -120,6 +127,7 @@ def test_one_launch_decode_equals_general_path_small(cuda_ok):
 
 
 def _decode_bits(ctx, dims, seed, S, flat):
+    ctx.debug_decode_mode(1)
     ctx.debug_decode_flat(flat)
     out = []
     for t in range(S):
@@ -158,11 +166,13 @@ def test_full_size_decode_flat_schedule_is_bitwise_in_order(full_model):
         got = _decode_bits(full_model, FULL, 7, 2, 1)
     finally:
         full_model.debug_decode_flat(1)
+        full_model.debug_decode_mode(0)
     _same(base, got, "flat")
 
 
 def test_one_launch_decode_chained_b1(cuda_ok):
     ctx, _, _ = build(SMALL, 92, 4)
+    ctx.debug_decode_mode(1)
     gpu = run_steps(ctx, SMALL, 92, 1, 3, chained=True)
     ref = oracle_steps(SMALL, 92, 1, 3, gpu[2], gpu[3], chained=True)
     compare_steps(SMALL, gpu, ref)
@@ -172,6 +182,7 @@ def test_one_launch_decode_chained_b1(cuda_ok):
 def test_one_launch_decode_onehot_head_b1(cuda_ok):
     dims = Dims(d=256, E=16, I=128, k=4, r=8, L=3, head_layers=(0, 1), head_onehot=1)
     ctx, _, _ = build(dims, 93, 4)
+    ctx.debug_decode_mode(1)
     gpu = run_steps(ctx, dims, 93, 1, 4)
     ref = oracle_steps(dims, 93, 1, 4, gpu[2], gpu[3])
     compare_steps(dims, gpu, ref)
@@ -183,6 +194,7 @@ def test_one_launch_decode_bounded_wait_reports_timeout(cuda_ok):
     the status is TIMEOUT, and the context decodes correctly afterwards."""
     import int4_expert_streaming_prerouter_b200 as e0
     ctx, _, _ = build(SMALL, 94, 4)
+    ctx.debug_decode_mode(1)
     h = bf16_tensor(synth.hidden(94, 0, SMALL.L, 1, SMALL.d), "cuda")
     ctx.debug_decode_stall(0, 20_000_000)          # 20 ms budget
     ctx.stack_decode(h, 0)
@@ -327,3 +339,35 @@ def test_exact_ties_take_the_lowest_indices(cuda_ok):
             assert np.array_equal(idx_t.cpu().numpy(), np.tile(want, (T, 1))), (T, path)
             assert np.allclose(gates.cpu().numpy(), 0.25, rtol=0, atol=1e-7)
         ctx.close()
+
+
+# ---------------------------------------------------------------------------------------
+# the phased kernels (unchained steps, B <= 8): every head form, routing width and batch
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("heads,onehot,hidden,k,B", [
+    ((0, 1, 2), 0, 0, 4, 1), ((0, 1, 2), 0, 0, 4, 3), ((0, 1, 2), 0, 0, 4, 8), ((0, 2), 0, 0, 4, 2),
+    ((), 0, 0, 4, 1), ((0, 1, 2), 1, 0, 4, 2), ((0, 1, 2), 1, 64, 4, 1), ((0, 1), 0, 32, 4, 5),
+    ((0, 1, 2), 0, 0, 2, 1), ((0, 1, 2), 0, 0, 8, 3)])
+def test_phased_decode_matches_oracle(cuda_ok, heads, onehot, hidden, k, B):
+    dims = Dims(d=256, E=16, I=128, k=k, r=8, L=4, head_layers=heads, head_onehot=onehot, head_hidden=hidden)
+    seed = 120 + 7 * k + B + hidden
+    ctx, _, _ = build(dims, seed, 8)
+    ctx.debug_decode_mode(4)
+    S = 3
+    gpu = run_steps(ctx, dims, seed, B, S)
+    ref = oracle_steps(dims, seed, B, S, gpu[2], gpu[3])
+    compare_steps(dims, gpu, ref)
+    ctx.close()
+
+
+def test_phased_decode_full_head_k8_full_size(cuda_ok):
+    """The full prerouter head (fc1 -> erf-GELU -> fc2 plus the linear path over
+    u = [x; onehot(cur); onehot(prev)], width d + 2E = 2560, hidden 256) with routing width
+    k = 8 on the full-size geometry, 6 layers, two steps at B = 2."""
+    dims = Dims(d=2048, E=256, I=512, k=8, r=16, L=6, head_layers=(0, 1, 2, 3), head_onehot=1, head_hidden=256)
+    ctx, _, _ = build(dims, 130, 8)
+    ctx.debug_decode_mode(4)
+    gpu = run_steps(ctx, dims, 130, 2, 2)
+    ref = oracle_steps(dims, 130, 2, 2, gpu[2], gpu[3])
+    compare_steps(dims, gpu, ref)
+    ctx.close()
