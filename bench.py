@@ -515,8 +515,12 @@ def run_decode(args, dims, seed, B, ws, rank, local, extras):
     h_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
     h_host.copy_(h_all[warm:total].cpu())
     y_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
-    torch.cuda.synchronize()
     nxt = total          # continue the same decode sequence
+    # one untimed call first: the library allocates its host-I/O staging buffers on first use
+    ctx.stack_decode_host(h_host[0], nxt, y_host[0])
+    ctx.host_io_wait()
+    torch.cuda.synchronize()
+    nxt += 1
     barrier(ws)
     e0_, e1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0_.record(stream)
@@ -532,7 +536,7 @@ def run_decode(args, dims, seed, B, ws, rank, local, extras):
 
     pk = peaks()
     step_ms = ms / steps
-    phased = args.decode_mode in (0, 4) and B <= 8
+    phased = args.decode_mode == 4 or (args.decode_mode == 0 and 2 <= B <= 64)
     traffic, how = kernel_traffic("decode_b1_l40_phased" if phased else args.workload) if B == 1 else (None, None)
     kernel = ("decode step = six phased kernels (norm, bf16 rows, routing, gate/up, sums, down) launched "
               "with programmatic dependent launch; CUDA events around the timed steps on their stream; "
@@ -719,6 +723,9 @@ def _stream_case(ctx, dims, h_all, warm, steps, ws, local, link, B=1, e2e=False)
         y_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
         t_base = warm + steps
         stream = torch.cuda.current_stream()
+        ctx.stack_decode_host(h_host[0], t_base, y_host[0], streaming=True)   # untimed: allocates
+        ctx.host_io_wait()
+        t_base += 1
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -850,11 +857,13 @@ def run_multistream(args, dims, seed, ws, rank, local, batches=(8, 32, 64)):
         h_host = h_all[warm:warm + steps].cpu().pin_memory()
         y_host = torch.empty((steps, dims.L, B, dims.d), dtype=torch.bfloat16, pin_memory=True)
         stream = torch.cuda.current_stream()
+        ctx.stack_decode_host(h_host[0], warm + steps, y_host[0])   # untimed: allocates
+        ctx.host_io_wait()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for t in range(steps):
-            ctx.stack_decode_host(h_host[t], warm + steps + t, y_host[t])
+            ctx.stack_decode_host(h_host[t], warm + steps + 1 + t, y_host[t])
         ctx.host_io_wait()
         b.record(stream)
         torch.cuda.synchronize()
@@ -864,7 +873,8 @@ def run_multistream(args, dims, seed, ws, rank, local, batches=(8, 32, 64)):
         st = synth.routing_stats(np.stack(idx_steps))
         res[f"b{B}"] = {
             "value": tokens / (ms_run / 1e3), "unit": "tokens/s", "ms_per_step": ms_run / steps, "steps": steps,
-            "batch": B, "path": "phased kernels" if B <= 8 else "per-layer kernels",
+            "batch": B, "path": ("phased kernels" if B <= 8 else
+                                 f"phased kernels, {(B + 7) // 8} passes of up to 8 streams"),
             "gpu_launches": int(l_run), "clocks": clk_run,
             "routing": dict(st, matches_targets=bool(np.array_equal(np.sort(np.stack(idx_steps), -1),
                                                                     np.sort(tg[warm:warm + steps], -1)))),
@@ -876,6 +886,47 @@ def run_multistream(args, dims, seed, ws, rank, local, batches=(8, 32, 64)):
         del h_all
         _free_gpu()
     return res
+
+
+def run_full_head_sweep(args, seed, ws, rank, local, ks=(2, 4, 8), H=256):
+    """The prerouter head in its full form (fc1 -> erf-GELU -> fc2 plus the linear path, over
+    u = [x; onehot(cur); onehot(prev)], width d + 2E) on the 40-layer model, at routing
+    widths K = 2, 4, 8, one stream: tokens/s and HBM fraction on the expert bytes."""
+    import torch
+    import dataclasses
+    dims0 = dataclasses.replace(synth.WORKLOADS["decode_b1_l40"]["dims"], head_hidden=H, head_onehot=1)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lys, hds = _load_model(dims0, seed, dev)
+    pk = peaks()
+    out = {}
+    steps, warm = min(args.steps, 32), 3
+    for k in ks:
+        dims = dataclasses.replace(dims0, k=k)
+        ctx = _context(dims, lys, hds, 1)
+        h_all = torch.stack([synth_hidden_tensor(seed, t, dims, 1, dev) for t in range(warm + steps)])
+        y = torch.empty((dims.L, 1, dims.d), dtype=torch.bfloat16, device=dev)
+        for t in range(warm):
+            ctx.stack_decode(h_all[t], t, y_out=y)
+        ms, clk, launches = _timed_steps(ctx, h_all, warm, steps, y, ws, local)
+        ms = max_over_ranks(ms, ws)
+        idx, _ = ctx.get_routing(1)
+        exp_b = step_bytes(dims, idx, 1)[0]
+        hb = 33 * (dims.E * dims.head_in + H * dims.head_in + dims.E * H) * 2
+        out[f"k{k}"] = {"value": sum_over_ranks(steps, ws) / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms / steps,
+                        "steps": steps, "top_k": k, "head_hidden": H, "head_input": dims.head_in,
+                        "head_bytes_per_step": hb, "gpu_launches": int(launches), "clocks": clk,
+                        "roofline": _hbm_roofline(exp_b, ms / steps, pk, "phased decode kernels (full heads)")}
+        ctx.close()
+        del h_all
+    del lys, hds
+    _free_gpu()
+    return out
+
+
+def synth_hidden_tensor(seed, t, dims, B, dev):
+    from synth.device import bf16_tensor
+    return bf16_tensor(synth.hidden(seed, t, dims.L, B, dims.d), dev)
 
 
 def main():
@@ -956,6 +1007,8 @@ def main():
             ms_res["cpu_baseline"] = cpu_baseline_tokens(mwl["dims"], mwl["seed"], hs8[0, 0], 0, dims.L,
                                                          "one step of the batch-8 streams")
         out["decode_multistream_l40"] = ms_res
+        _free_gpu()
+        out["decode_b1_l40_full_head_k_sweep"] = run_full_head_sweep(args, seed, ws, rank, local)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if ws > 1:

@@ -113,8 +113,9 @@ struct PhState {
   uint16_t *x16 = nullptr, *xp = nullptr, *a = nullptr;
   float *xs = nullptr, *rlog = nullptr, *rsel = nullptr, *hlog = nullptr, *lt = nullptr, *h1 = nullptr,
         *gates = nullptr, *asum = nullptr, *gus = nullptr;
-  int *plan = nullptr;                   // [2][L][kPlanInts], by step parity
-  int8_t *slot = nullptr;                // [2][L][kPhMaxU][kPhMaxB]
+  // expert plans by (step parity, group of kPhMaxB streams, layer)
+  int *plan = nullptr;                   // [2][kPhGroups][L][kPlanInts]
+  int8_t *slot = nullptr;                // [2][kPhGroups][L][kPhMaxU][kPhMaxB]
   int last_step = -1;                    // the last step that ran the phased kernels
   PhBlock *blocks[2 * (kPhMaxB + 1)] = {};
   int nblocks[2 * (kPhMaxB + 1)] = {};
@@ -1124,7 +1125,7 @@ static bool phased_geometry(const e0_dims &Dm, int *which) {
 static bool phased_supported(e0_ctx *C, int B) {
   const e0_dims &D = C->dims;
   int which;
-  if (B < 1 || B > kPhMaxB || !phased_geometry(D, &which) || C->L > 64 || D.head_hidden > kPhMaxH ||
+  if (B < 1 || B > kPhMaxB * kPhGroups || !phased_geometry(D, &which) || C->L > 64 || D.head_hidden > kPhMaxH ||
       D.head_hidden % 16 != 0)
     return false;
   for (int l = 0; l < C->L; l++)
@@ -1158,7 +1159,8 @@ static int phased_prepare(e0_ctx *C) {
     const size_t n_x16 = w4(T * d * 2), n_xp = w4(T * d * 2), n_a = w4(T * (k + 1) * I * 2), n_xs = w4(T * (d / 64) * 4),
                  n_rl = w4(T * E * 4), n_rs = w4(T * k * 4), n_hl = w4(T * E * 4), n_lt = w4(T * 3 * r * 4),
                  n_h1 = w4(T * H * 4), n_g = w4(T * k * 4), n_as = w4(T * (k + 1) * (I / 64) * 4),
-                 n_pl = w4((size_t)2 * L * kPlanInts * 4), n_sl = w4((size_t)2 * L * kPhMaxU * kPhMaxB),
+                 n_pl = w4((size_t)2 * kPhGroups * L * kPlanInts * 4),
+                 n_sl = w4((size_t)2 * kPhGroups * L * kPhMaxU * kPhMaxB),
                  n_gus = w4(T * 2 * I * 4);
     const size_t tot = n_x16 + n_xp + n_a + n_xs + n_rl + n_rs + n_hl + n_lt + n_h1 + n_g + n_as + n_pl + n_sl + n_gus;
     uint32_t *p = nullptr;
@@ -1268,41 +1270,49 @@ static int phased_launch(e0_ctx *C, const PhParams &P, cudaStream_t s) {
   return E0_OK;
 }
 
+// One phased decode step of B streams: one pass of the six kernels per group of up to
+// kPhMaxB streams (each group with its own routing-table offset and expert plans).
 static int decode_phased(e0_ctx *C, const uint16_t *h, int B, int step, uint16_t *y, float *yf, cudaStream_t s) {
   int rc = phased_prepare(C);
   if (rc) return rc;
   PhState &S = C->ph;
   const e0_dims &D = C->dims;
-  const int cur = step & 1, prv = cur ^ 1;
-  PhParams P{};
-  P.layers = S.d_layers;
-  P.L = C->L; P.B = B; P.E = D.n_experts; P.k = D.top_k; P.r = D.lora_rank; P.H = D.head_hidden;
-  P.ldh = D.d_model + (D.head_onehot ? 2 * D.n_experts : 0);
-  P.onehot = D.head_onehot; P.step0 = step == 0; P.maxT = C->maxT;
-  P.eps = D.rms_eps; P.c = D.lora_scale;
-  P.h = h; P.y = y; P.yf = yf;
-  P.x16 = S.x16; P.xp = S.xp; P.xs = S.xs; P.rlog = S.rlog; P.rsel = S.rsel; P.hlog = S.hlog; P.lt = S.lt;
-  P.h1 = S.h1; P.gates = S.gates; P.a = S.a; P.asum = S.asum; P.gus = S.gus;
-  P.plan_cur = S.plan + (size_t)cur * C->L * kPlanInts;
-  P.plan_next = S.plan + (size_t)prv * C->L * kPlanInts;
-  P.slot_cur = S.slot + (size_t)cur * C->L * kPhMaxU * kPhMaxB;
-  P.slot_next = S.slot + (size_t)prv * C->L * kPhMaxU * kPhMaxB;
-  P.pred_in = step > 0 ? pred_at(C, prv, 0) : nullptr;
-  P.pred_out = pred_at(C, cur, 0);
-  P.hist_out = hist_at(C, cur, 0);
-  P.hist_prev = step > 0 ? hist_at(C, prv, 0) : nullptr;
-  P.err = C->err;
-  if ((rc = phased_blocks(C, B, step == 0, &P.blocks, &P.nblocks))) return rc;
-  if (step > 0 && S.last_step != step - 1) {
-    // the previous step ran another path: the predicted layers' plans come from its predictions
-    k_ph_plan_pred<<<C->L, 32, 0, s>>>(P);
-    CKL("k_ph_plan_pred");
+  const int cur = step & 1, prv = cur ^ 1, k = D.top_k;
+  const bool fix_plans = step > 0 && S.last_step != step - 1;
+  S.last_step = -1;
+  for (int grp = 0; grp * kPhMaxB < B; grp++) {
+    const int tok0 = grp * kPhMaxB, Bg = std::min(kPhMaxB, B - tok0);
+    PhParams P{};
+    P.layers = S.d_layers;
+    P.L = C->L; P.B = Bg; P.E = D.n_experts; P.k = k; P.r = D.lora_rank; P.H = D.head_hidden;
+    P.ldh = D.d_model + (D.head_onehot ? 2 * D.n_experts : 0);
+    P.onehot = D.head_onehot; P.step0 = step == 0; P.maxT = C->maxT;
+    P.eps = D.rms_eps; P.c = D.lora_scale;
+    P.h = h; P.y = y; P.yf = yf; P.hB = B; P.tok0 = tok0;
+    P.x16 = S.x16; P.xp = S.xp; P.xs = S.xs; P.rlog = S.rlog; P.rsel = S.rsel; P.hlog = S.hlog; P.lt = S.lt;
+    P.h1 = S.h1; P.gates = S.gates; P.a = S.a; P.asum = S.asum; P.gus = S.gus;
+    P.plan_cur = S.plan + ((size_t)cur * kPhGroups + grp) * C->L * kPlanInts;
+    P.plan_next = S.plan + ((size_t)prv * kPhGroups + grp) * C->L * kPlanInts;
+    P.slot_cur = S.slot + ((size_t)cur * kPhGroups + grp) * C->L * kPhMaxU * kPhMaxB;
+    P.slot_next = S.slot + ((size_t)prv * kPhGroups + grp) * C->L * kPhMaxU * kPhMaxB;
+    P.pred_in = step > 0 ? pred_at(C, prv, 0) + (size_t)tok0 * k : nullptr;
+    P.pred_out = pred_at(C, cur, 0) + (size_t)tok0 * k;
+    P.hist_out = hist_at(C, cur, 0) + (size_t)tok0 * k;
+    P.hist_prev = step > 0 ? hist_at(C, prv, 0) + (size_t)tok0 * k : nullptr;
+    P.err = C->err;
+    if ((rc = phased_blocks(C, Bg, step == 0, &P.blocks, &P.nblocks))) return rc;
+    if (fix_plans) {
+      // the previous step ran another path: the predicted layers' plans come from its predictions
+      k_ph_plan_pred<<<C->L, 32, 0, s>>>(P);
+      CKL("k_ph_plan_pred");
+    }
+    int which;
+    phased_geometry(D, &which);
+    rc = which == 0 ? phased_launch<2048, 512>(C, P, s) : phased_launch<256, 128>(C, P, s);
+    if (rc) return rc;
   }
-  int which;
-  phased_geometry(D, &which);
-  rc = which == 0 ? phased_launch<2048, 512>(C, P, s) : phased_launch<256, 128>(C, P, s);
-  S.last_step = rc == E0_OK ? step : -1;
-  return rc;
+  S.last_step = step;
+  return E0_OK;
 }
 
 // Test hook: make CTA `cta` of the next persistent decode launch wait on a word nobody
@@ -1385,7 +1395,7 @@ extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step,
   const bool phased = !chained && phased_supported(C, B);
   int mode = C->force_general ? 3 : C->decode_mode;
   // default: the measured fastest per batch: at one stream the one-launch kernel, up to
-  // kPhMaxB streams the phased kernels, beyond that the per-layer kernels
+  // kPhMaxB x kPhGroups streams the phased kernels, beyond that the per-layer kernels
   if (mode == 0) mode = one_launch ? 1 : phased ? 4 : 3;
   if (mode == 4 && !phased) mode = one_launch ? 1 : 3;
   if (mode == 1 && !one_launch) mode = 2;

@@ -42,7 +42,8 @@
 
 namespace e0 {
 
-constexpr int kPhMaxB = 8;                       // tokens per step on this path
+constexpr int kPhMaxB = 8;                       // tokens per pass of the kernels (the MMA's N)
+constexpr int kPhGroups = 8;                     // passes per step: up to 64 streams
 constexpr int kPhMaxU = kPhMaxB * kMaxK + 1;     // distinct routed experts + the shared one
 constexpr int kPhMaxH = 512;                     // full-head hidden width on this path
 constexpr int kPhBatch = 5;                      // experts whose down rows a warp loads at once
@@ -64,9 +65,12 @@ struct PhParams {
   const PhLayer *layers;
   int L, B, E, k, r, H, ldh, onehot, step0, maxT;
   float eps, c;
-  const uint16_t *h;            // [L][B][D]
-  uint16_t *y;                  // [L][B][D]
-  float *yf;                    // [L][B][D] or nullptr
+  // the caller's step input and outputs [L][hB][D]; this launch serves tokens
+  // tok0 .. tok0 + B - 1 of them (the routing tables are offset to the same tokens)
+  const uint16_t *h;
+  uint16_t *y;
+  float *yf;                    // or nullptr
+  int hB, tok0;
   // workspace, token stride kPhMaxB
   uint16_t *x16, *xp;           // [L][8][D] x (natural order) and x in pair order
   float *xs;                    // [L][8][D/64] group sums of x
@@ -176,7 +180,7 @@ template <int D>
 __global__ void __launch_bounds__(256) k_ph_norm(PhParams P) {
   ph_launch_next();
   const int l = blockIdx.x / P.B, n = blockIdx.x % P.B;
-  const uint16_t *hr = P.h + ((size_t)l * P.B + n) * D;
+  const uint16_t *hr = P.h + ((size_t)l * P.hB + P.tok0 + n) * D;
   const uint16_t *gm = P.layers[l].gamma;
   __shared__ double red[8];
   __shared__ uint16_t xs16[D];
@@ -736,7 +740,7 @@ __global__ void __launch_bounds__(32 * (I / 64)) k_ph_down(PhParams P) {
       for (int q2 = 0; q2 < P.r; q2++) lo = fmaf(bf(Y.Bd[(size_t)row * P.r + q2]), td[q2], lo);
       v = fmaf(P.c, lo, v);
     }
-    const size_t oi = ((size_t)l * B + n) * D + row;
+    const size_t oi = ((size_t)l * P.hB + P.tok0 + n) * D + row;
     P.y[oi] = f2bf(v);
     if (P.yf) P.yf[oi] = v;
   }

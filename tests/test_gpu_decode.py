@@ -347,11 +347,11 @@ def test_exact_ties_take_the_lowest_indices(cuda_ok):
 @pytest.mark.parametrize("heads,onehot,hidden,k,B", [
     ((0, 1, 2), 0, 0, 4, 1), ((0, 1, 2), 0, 0, 4, 3), ((0, 1, 2), 0, 0, 4, 8), ((0, 2), 0, 0, 4, 2),
     ((), 0, 0, 4, 1), ((0, 1, 2), 1, 0, 4, 2), ((0, 1, 2), 1, 64, 4, 1), ((0, 1), 0, 32, 4, 5),
-    ((0, 1, 2), 0, 0, 2, 1), ((0, 1, 2), 0, 0, 8, 3)])
+    ((0, 1, 2), 0, 0, 2, 1), ((0, 1, 2), 0, 0, 8, 3), ((0, 1, 2), 0, 0, 4, 20), ((0, 2), 1, 32, 4, 11)])
 def test_phased_decode_matches_oracle(cuda_ok, heads, onehot, hidden, k, B):
     dims = Dims(d=256, E=16, I=128, k=k, r=8, L=4, head_layers=heads, head_onehot=onehot, head_hidden=hidden)
     seed = 120 + 7 * k + B + hidden
-    ctx, _, _ = build(dims, seed, 8)
+    ctx, _, _ = build(dims, seed, max(B, 8))
     ctx.debug_decode_mode(4)
     S = 3
     gpu = run_steps(ctx, dims, seed, B, S)
