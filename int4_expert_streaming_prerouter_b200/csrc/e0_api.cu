@@ -294,7 +294,7 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
   cudaMemset(C->pf_buf, 0xFF, 2 * (T + 1) * k * sizeof(int32_t));
   cudaMemset(C->pf_idx, 0xFF, (T + 1) * k * sizeof(int32_t));
   if (T >= kTcMinTokens) {
-    C->tile_cap = (int)((T * k + kTcN - 1) / kTcN + std::min(E, T * k) + (T + kTcN - 1) / kTcN + 1);
+    C->tile_cap = (int)((T * k + kTmN - 1) / kTmN + std::min(E, T * k) + (T + kTmN - 1) / kTmN + 1);
     if ((rc = dalloc(&C->xp, T * d)) || (rc = dalloc(&C->ap, T * (k + 1) * I)) || (rc = dalloc(&C->xg, T * k * d)) ||
         (rc = dalloc(&C->xsum, T * (d / 64 + 1))) || (rc = dalloc(&C->asum, T * (k + 1) * (I / 64 + 1))) ||
         (rc = dalloc(&C->yacc, T * d)) ||
@@ -308,7 +308,7 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
     if (cudaFuncSetAttribute(k_tc_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sizeof(TcRowsSmem) + 1024) != cudaSuccess ||
         cudaFuncSetAttribute(k_moe_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(TwSmem) + 1024) != cudaSuccess) {
+                             (int)sizeof(TmSmem) + 1024) != cudaSuccess) {
       cudaGetLastError();
       e0_destroy(C);
       return fail(E0_ERR_CUDA, "e0_create: shared-memory opt-in of the tensor-core kernels failed");
@@ -392,10 +392,11 @@ static inline int grid_for(int warps_needed, int cap) {
   return b < 1 ? 1 : (b > cap ? cap : b);
 }
 
-// TMA descriptor of a row-major bf16 matrix [rows, K] read in boxes of 64 columns x 128
-// rows with the 128-byte swizzle of the tensor-core operand tiles (zeros past the end).
+// TMA descriptor of a row-major 16-bit matrix [rows, K] (bf16, or fp16 when f16) read in
+// boxes of 64 columns x kTmN rows with the 128-byte swizzle of the tensor-core operand
+// tiles (zeros past the end).
 // The encoder comes from the driver through the runtime's entry-point query.
-static int tmap_bf16_rows(CUtensorMap *m, const void *base, int K, long long rows) {
+static int tmap_bf16_rows(CUtensorMap *m, const void *base, int K, long long rows, bool f16 = false) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     void *fn = nullptr;
@@ -409,12 +410,40 @@ static int tmap_bf16_rows(CUtensorMap *m, const void *base, int K, long long row
     return fail(E0_ERR_INVALID_ARG, "tensor map: base, K or rows not supported");
   const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kTmN};
   const cuuint32_t es[2] = {1, 1};
-  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+  const CUresult r = encode(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                            const_cast<void *>(base), dims, strides, box, es,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(E0_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return E0_OK;
+}
+
+// TMA descriptor of the int4 codes of one projection of every expert: a 3-D byte tensor
+// [count][rows][row_bytes] whose experts lie `stride` bytes apart, read in boxes of 128
+// bytes x box_rows rows with the 128-byte swizzle (zeros past the end of a row).
+static int tmap_codes(CUtensorMap *m, const void *base, int row_bytes, int rows, int count, long long stride,
+                      int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return fail(E0_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  }
+  if (((uintptr_t)base & 15) || row_bytes % 16 || stride % 16 || rows < box_rows || count < 1)
+    return fail(E0_ERR_INVALID_ARG, "code tensor map: base, row length, stride or rows not supported");
+  const cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)count};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)stride};
+  const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(E0_ERR_CUDA, "cuTensorMapEncodeTiled (codes) failed (%d)", (int)r);
   return E0_OK;
 }
 
@@ -422,8 +451,9 @@ static int tmap_bf16_rows(CUtensorMap *m, const void *base, int K, long long row
 // selected), in contexts created with the workspaces for them.
 static bool use_tc(e0_ctx *C, int T) {
   const e0_dims &D = C->dims;
-  return C->xp && D.d_model % 128 == 0 && D.d_model <= 64 * kTcMaxGroups && D.d_ff % 64 == 0 &&
-         D.d_ff <= 64 * kTcMaxGroups && (C->prefill_path == 2 || (C->prefill_path == 0 && T >= kTcMinTokens));
+  return C->xp && D.d_model % 128 == 0 && D.d_model <= 64 * kTmMaxG && D.d_ff % 128 == 0 &&
+         (D.lora_rank <= kTmMaxR && D.lora_rank % 2 == 0) &&
+         D.d_ff <= 64 * kTmMaxG && (C->prefill_path == 2 || (C->prefill_path == 0 && T >= kTcMinTokens));
 }
 
 static int layer_pre(e0_ctx *C, const LayerCall &K, cudaStream_t s) {
@@ -476,7 +506,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   const e0_layer &Y = C->layers[K.l];
   const size_t nx = (size_t)K.T * D.d_model;
   const long long xg = (long long)K.T * (D.d_model / 64);
-  k_perm_sums<<<(unsigned)((xg + 255) / 256), 256, 0, s>>>(C->xb, K.T, D.d_model, C->xp, C->xsum);
+  k_perm_sums<<<(unsigned)((xg + 255) / 256), 256, 0, s>>>(C->xb, K.T, D.d_model, C->xp, C->xsum, 0);
   CKL("k_perm_sums(x)");
   k_tc_tiles<<<1, 32, 0, s>>>(C->plan, K.T, C->tiles, C->ntiles, C->tile_cap);
   CKL("k_tc_tiles");
@@ -485,21 +515,28 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   CKL("k_group_rows");
   TcArgs A{};
   int rc;
-  if ((rc = tmap_bf16_rows(&A.tmB[0], C->xg, D.d_model, (long long)K.T * D.top_k)) ||
-      (rc = tmap_bf16_rows(&A.tmB[1], C->xp, D.d_model, K.T)))
+  if ((rc = tmap_bf16_rows(&A.tmB[0], C->xg, D.d_model, (long long)K.T * D.top_k, true)) ||
+      (rc = tmap_bf16_rows(&A.tmB[1], C->xp, D.d_model, K.T, true)))
     return rc;
   A.mode = 0; A.T = K.T; A.d = D.d_model; A.I = D.d_ff; A.k = D.top_k; A.r = D.lora_rank; A.c = D.lora_scale;
   A.src = src; A.shared = (const uint8_t *)Y.shared; A.bl = C->bl; A.P = C->plan; A.tiles = C->tiles;
   A.ntiles = C->ntiles; A.xp = C->xp; A.xsum = C->xsum; A.ap = C->ap; A.asum = C->asum; A.ap_out = C->ap;
   A.Bg = (const uint16_t *)Y.lora_Bg; A.Bu = (const uint16_t *)Y.lora_Bu; A.lt = C->lt; A.gates = K.gates;
   A.yacc = C->yacc; A.err = C->err; A.timeout_ns = 2000000000ull;
-  const int tc_smem_bytes = (int)sizeof(TwSmem) + 1024;   // opted in at e0_create on this context's device
-  const int tmax = std::min(C->tile_cap, (K.T * D.top_k + kTcN - 1) / kTcN + std::min(D.n_experts, K.T * D.top_k) +
-                                              (K.T + kTcN - 1) / kTcN);
+  const int tc_smem_bytes = (int)sizeof(TmSmem) + 1024;   // opted in at e0_create on this context's device
+  const int tmax = std::min(C->tile_cap, (K.T * D.top_k + kTmN - 1) / kTmN + std::min(D.n_experts, K.T * D.top_k) +
+                                              (K.T + kTmN - 1) / kTmN);
+  const uint8_t *ex = (const uint8_t *)src.resident, *sh = (const uint8_t *)Y.shared;
+  const long long bb = C->bl.bytes;
+  if ((rc = tmap_codes(&A.tmC[0], ex + C->bl.gc, D.d_model / 2, D.d_ff, D.n_experts, bb, 64)) ||
+      (rc = tmap_codes(&A.tmC[1], ex + C->bl.uc, D.d_model / 2, D.d_ff, D.n_experts, bb, 64)) ||
+      (rc = tmap_codes(&A.tmC[2], sh + C->bl.gc, D.d_model / 2, D.d_ff, 1, bb, 64)) ||
+      (rc = tmap_codes(&A.tmC[3], sh + C->bl.uc, D.d_model / 2, D.d_ff, 1, bb, 64)))
+    return rc;
   cudaEvent_t g0 = nullptr, g1 = nullptr;
   if (C->time_gemm && cudaEventCreate(&g0) == cudaSuccess && cudaEventCreate(&g1) == cudaSuccess)
     cudaEventRecord(g0, s);
-  k_moe_gemm_tc<<<tmax * (D.d_ff / 64), kTwThreads, tc_smem_bytes, s>>>(A);
+  k_moe_gemm_tc<<<std::min(C->nsm, tmax * (D.d_ff / 64)), kTmThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(gate/up)");
   if (g1) {
     cudaEventRecord(g1, s);
@@ -508,7 +545,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   }
   const long long ag = (long long)K.T * (D.top_k + 1) * (D.d_ff / 64);
   k_perm_sums<<<(unsigned)((ag + 255) / 256), 256, 0, s>>>(C->ap, (long long)K.T * (D.top_k + 1), D.d_ff, nullptr,
-                                                          C->asum);
+                                                          C->asum, 1);
   CKL("k_perm_sums(a)");
   if (Y.lora_Ad) {
     k_lora_td<<<(K.T * D.lora_rank + 7) / 8, 256, 0, s>>>((const uint16_t *)Y.lora_Ad, C->ap, K.T, D.d_ff,
@@ -517,11 +554,16 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   }
   CK(cudaMemsetAsync(C->yacc, 0, nx * sizeof(float), s));
   A.mode = 1;
-  if ((rc = tmap_bf16_rows(&A.tmB[0], C->ap, D.d_ff, (long long)K.T * (D.top_k + 1)))) return rc;
+  if ((rc = tmap_bf16_rows(&A.tmB[0], C->ap, D.d_ff, (long long)K.T * (D.top_k + 1), true)) ||
+      (rc = tmap_codes(&A.tmC[0], ex + C->bl.dc, D.d_ff / 2, D.d_model, D.n_experts, bb, 128)) ||
+      (rc = tmap_codes(&A.tmC[2], sh + C->bl.dc, D.d_ff / 2, D.d_model, 1, bb, 128)))
+    return rc;
   A.tmB[1] = A.tmB[0];
+  A.tmC[1] = A.tmC[0];
+  A.tmC[3] = A.tmC[2];
   if (C->time_gemm && cudaEventCreate(&g0) == cudaSuccess && cudaEventCreate(&g1) == cudaSuccess)
     cudaEventRecord(g0, s);
-  k_moe_gemm_tc<<<tmax * (D.d_model / 128), kTwThreads, tc_smem_bytes, s>>>(A);
+  k_moe_gemm_tc<<<std::min(C->nsm, tmax * (D.d_model / 128)), kTmThreads, tc_smem_bytes, s>>>(A);
   CKL("k_moe_gemm_tc(down)");
   if (g1) {
     cudaEventRecord(g1, s);

@@ -6,20 +6,13 @@
 //             the shared expert adds c * B (A x) to g and u first;
 //   down:     Y_e = Dq(W_d) A_e^T, y[t] += w_{t,j} Y_e[:, t]  (w = 1 for the shared expert).
 //
-// B200 design.  One CTA = one 128-row weight tile of one expert x up to 128 tokens.  Eight
-// warps produce each 64-wide K block: two threads per weight row dequantise the int4 tile
-// to fp16 (w = s q + m, one group of 64 per row per K block) and the token rows (fp16) are
-// gathered beside it, both written into shared memory in the 128-byte-swizzled K-major
-// layout the tensor core reads; each thread's global loads for the next K block are
-// issued before it works on the current one.  One thread issues four tcgen05.mma (M=128, N=tokens, K=16 each) per K block
-// into a TMEM accumulator and commits to an mbarrier that frees the stage; four stages are
-// in flight.  The epilogue reads TMEM with tcgen05.ld and applies SwiGLU (gate rows 0..63
-// and up rows 64..127 of the tile are the same intermediate units) or the gate-weighted
-// combine (fp32 atomics into y).  Each dequantised weight is split into two fp16 values
-// (hi = fp16(w), lo = fp16(w - hi)) and both are multiplied into the same accumulator, so
-// the weights keep ~22 significant bits (one fp16 alone keeps 11, which leaves a ~2e-3
-// relative error at the tail of a 40k-output layer); x and a are bf16 values, exactly
-// representable in fp16 in their range.
+// B200 design.  The int4 codes are expanded exactly into bf16 128 + q (one mask and one OR
+// per two weights) and each K group of 64 is one tensor-core accumulation; the affine
+// dequantisation is folded once per group and output on the CUDA cores.  The expanded
+// weights go from registers straight into tensor memory, the A operand of tcgen05.mma, so
+// shared memory carries only raw codes and activation tiles, both by TMA.  Persistent
+// warp-specialised CTAs overlap code/activation loads, conversion, MMAs, folds and the
+// epilogues of consecutive work units (details at k_moe_gemm_tc).
 #pragma once
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -30,7 +23,8 @@ namespace e0 {
 
 constexpr int kTcThreads = 256;     // threads of the dense-rows kernel
 constexpr int kTcMinTokens = 64;    // contexts with at least this many tokens get the tensor-core path
-constexpr int kTcN = 128;           // tokens per tile (TMEM columns per accumulator)
+constexpr int kTcN = 128;           // tokens per tile of the dense-rows kernel (TMEM columns)
+constexpr int kTmN = 80;            // tokens per expert tile of the grouped expert GEMM
 constexpr int kTcMaxGroups = 64;    // K / 64 <= 64 (K <= 4096)
 
 struct TcTile {
@@ -43,6 +37,10 @@ struct TcArgs {
   // mode 0: [0] x in expert-grouped row order [T k, d], [1] x in token order [T, d];
   // mode 1: [0] a in grouped order [T k + T, I] (the shared expert's rows last)
   CUtensorMap tmB[2];
+  // int4 code tiles as 3-D TMA maps over [experts][rows][K/2 bytes] (box 128 bytes x 64 or
+  // 128 rows, 128-byte swizzle): mode 0: [0] gate, [1] up of the routed experts, [2] gate,
+  // [3] up of the shared expert; mode 1: [0] down of the routed experts, [2] of the shared
+  CUtensorMap tmC[4];
   int mode;                 // 0: gate/up + SwiGLU, 1: down + weighted combine
   int T, d, I, k, r;
   float c;
@@ -138,10 +136,12 @@ __device__ __forceinline__ void tc_mbar_init(uint64_t *b, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(tc_smem(b)), "r"(count) : "memory");
 }
 
+// one test of an mbarrier phase; the thread may sleep in it until the phase completes (at
+// most ~1 ms), so waiting warps do not take issue slots from the working ones
 __device__ __forceinline__ bool tc_mbar_test(uint64_t *b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(tc_smem(b)), "r"(parity)
@@ -221,7 +221,7 @@ __device__ __forceinline__ bool tc_wait_all(uint64_t *b, uint32_t parity, unsign
 
 // ---------------------------------------------------------------------------------------
 // Tile list: every unique routed expert (its token list) and the shared expert (all T
-// tokens) cut into tiles of up to kTcN tokens.  One block.
+// tokens) cut into tiles of up to kTmN tokens.  One block.
 // ---------------------------------------------------------------------------------------
 __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
   // one warp: tiles per unit, an exclusive scan over the units in order, then every lane
@@ -233,7 +233,7 @@ __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
   for (int u0 = 0; u0 <= U; u0 += 32) {
     const int u = u0 + lane;
     const int cnt = u < U ? P.ustart[u + 1] - P.ustart[u] : (u == U ? T : 0);
-    const int nt = (cnt + kTcN - 1) / kTcN;
+    const int nt = (cnt + kTmN - 1) / kTmN;
     int incl = nt;
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -241,7 +241,7 @@ __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
     }
     for (int q = 0; q < nt; q++) {
       const int idx = base + incl - nt + q;
-      if (idx < cap) tiles[idx] = TcTile{u, q * kTcN};
+      if (idx < cap) tiles[idx] = TcTile{u, q * kTmN};
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
@@ -249,54 +249,99 @@ __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
 }
 
 // ---------------------------------------------------------------------------------------
-// The grouped expert GEMM.  One CTA = one 128-row weight tile of one expert x up to kTcN
-// tokens; grid = max tiles x M tiles per expert (blocks past the real tile count return).
+// The grouped expert GEMM: persistent CTAs (one per SM) walk the work units (one 128-row
+// weight tile of one expert x one tile of up to kTmN of its tokens) in a fixed order,
+// unit u = tile * M tiles + M tile, CTA b taking u = b, b + grid, ...
 //
-// Per K group g of 64 (the quantisation group), with A = the int4 codes as bf16 (128 + q,
-// exact) and B = the tokens' activations (bf16, exact):
-//   P_g = sum_{k in g} (128 + q_k) x_k           tcgen05.mma into TMEM buffer g % 2
-//   acc += s_g * P_g + (m_g - 128 s_g) * X_g      CUDA cores, X_g = sum_{k in g} x_k
-// which is sum_k (s_g q_k + m_g) x_k, the affine dequantisation folded into the
-// accumulation; so the weights need no fp32 dequantisation and one MMA per K = 16.
+// Exact affine int4 product without a per-group fold.  With w = s q + m (s, m the bf16
+// scale and min of the row's group g, q in 0..15) and q = (q & 14) + (q & 1):
+//   sum_k w_k x_k = sum_k s (q_k & 14) x_k + sum_k s (q_k & 1) x_k + sum_g m_g X_g,
+// X_g = sum_{k in g} x_k.  s (q & 14) = 2 s (q >> 1) has at most 8 + 3 significant bits and
+// s (q & 1) is 0 or s, so both are exact fp16 values (for 2^-15 <= |s| < 64; the pages'
+// scales are ~1e-2), and x (bf16) is an exact fp16 value in its range, so the tensor core
+// forms every product exactly and accumulates in fp32.  The min term is one more K = 64
+// block per unit: A = the row's mins (exact in fp16) twice, B = each column's group sums
+// split as X = hi + lo in fp16 (hi = fp16(X), lo = fp16(X - hi), ~22 significant bits
+// together).  The shared expert's unmerged LoRA up branch c B (A x) is one more block on
+// gate/up: A = the row's B_g (gate rows) or B_u (up rows) twice, B = c t_g, c t_u (t = A x)
+// split hi/lo the same way, so every term of g and u leaves the tensor core in fp32.
 //
-// Warp-specialised, every hand-off on an mbarrier, so that loads, conversion, MMAs and
-// folds of different groups overlap:
-//   warp  0    loader: one TMA tile load per group brings the tile's 128 activation rows
-//              (stored in expert-grouped order, so a tile's tokens are consecutive rows)
-//              as the 128-byte swizzled B tile; the lanes copy the columns' group sums
-//   warp  1    TMEM owner; one thread issues the four MMAs of each group
-//   warps 2-3  converters: thread t owns weight rows t and t + 64; it streams its own rows'
-//              codes kTwRawAhead groups ahead with cp.async (no hand-off needed) and
-//              writes 128 + q as bf16 into the A tile ring (kTwAStages stages)
-//   warps 4-11 folders: TMEM lane quadrant warp % 4, half of the columns each; they fold
-//              every group into registers and run the epilogue (SwiGLU, or the weighted
-//              combine into y)
+// A tcgen05.mma blocks its issuing thread ~120 cycles whatever N is (N <= 128), so at the
+// ~64 tokens a routed expert receives one issuing thread would leave the tensor core
+// idle most of the time.  Two threads issue, one the extra blocks and the even K groups,
+// the other the odd K groups, each into its own accumulator (the epilogue adds the two);
+// each accumulator is double-buffered across units (4 x kTmN TMEM columns).
+//
+// The expanded operands go from registers straight into tensor memory (A in TMEM), so
+// shared memory carries only raw codes and activations (TMA).  Warp roles, every hand-off
+// on an mbarrier:
+//   warp 0      producer: per 4 K groups one TMA load of the unit's codes (128 rows x 128
+//               bytes, 128-byte swizzle; 3-D map over the expert array), per K group one
+//               TMA load of the activation tile (expert-grouped rows: a tile's tokens are
+//               consecutive rows)
+//   warps 1, 2  the two MMA issuers
+//   warp 3      unit warp, two units ahead: column bookkeeping (token, destination,
+//               combine weight) and the extra blocks' B tiles
+//   warps 4-7   epilogue, TMEM lane quadrant warp % 4: SwiGLU (gate/up), or the
+//               gate-weighted combine into y (down); then, two units ahead, each thread
+//               its weight row's scales and mins as fp16 in [group][row] order
+//   warps 8-15  converters, quadrant warp % 4 (weight row 32 (warp % 4) + lane), half
+//               h = (warp - 8) / 4 of each 64-wide K block: per unit the extra blocks' A,
+//               then per K group both exact fp16 parts, into a 64-column TMEM stage
 // ---------------------------------------------------------------------------------------
-constexpr int kTwThreads = 384;
-constexpr int kTwLoadWarps = 1, kTwMmaWarp = 1, kTwConv0 = 2, kTwFold0 = 4;
-constexpr int kTwAStages = 3;
-constexpr int kTwBStages = 6;
-constexpr int kTwRawAhead = 3;      // groups of codes in flight per converter thread
-constexpr int kTwTBufs = 4;         // TMEM accumulators (kTcN columns each): MMAs run up to 4 groups ahead of the folds
+constexpr int kTmThreads = 512;
+constexpr int kTmProdWarp = 0, kTmMma0 = 1, kTmMma1 = 2, kTmUnitWarp = 3, kTmEpi0 = 4, kTmConv0 = 8;
+constexpr int kTmEpiThreads = 128, kTmConvWarps = 8;
+constexpr int kTmBStages = 6;      // activation tiles in flight (one K group each; even: stage parity = owner)
+static_assert(kTmBStages % 2 == 0, "B stage owners");
+constexpr int kTmCStages = 3;      // code tiles in flight (four K groups each)
+constexpr int kTmAStages = 3;      // A operand stages in TMEM (64 columns: both fp16 parts of one K block): 2 + 1 per issuer
+constexpr int kTmMaxG = 32;        // K <= 2048
+constexpr int kTmMaxR = 16;        // LoRA rank of the extra block (4 r <= 64)
+constexpr int kTmXRow = 65;        // epilogue exchange row stride in floats (conflict-free scalar access)
+constexpr uint32_t kTmACol = 4 * kTmN, kTmCols = 512;
+static_assert(kTmACol + kTmAStages * 64 <= kTmCols, "TMEM budget");
+static_assert((kTmN * 128) % 1024 == 0 && kTmN % 16 == 0, "tile rows");
 
-struct TwSmem {
-  uint8_t a[kTwAStages][128 * 128];        // A tiles (bf16, 128-byte swizzled K-major)
-  uint8_t b[kTwBStages][kTcN * 128];       // B tiles
-  float xs[kTwBStages][kTcN];              // the B columns' group sums
-  uint8_t raw[kTwRawAhead][128 * 32];      // int4 codes: converter thread t's row t
-  uint16_t sc[128 * kTcMaxGroups];         // scale of every row and group [row][g]
-  uint16_t mn[128 * kTcMaxGroups];         // min
-  uint64_t bfull[kTwBStages], bempty[kTwBStages], afull[kTwAStages], aempty[kTwAStages];
-  uint64_t tfull[kTwTBufs], tempty[kTwTBufs], pre;
+struct TmSmem {
+  uint8_t b[kTmBStages][kTmN * 128];   // activation tiles (fp16, 128-byte swizzled K-major)
+  uint8_t c[kTmCStages][128 * 128];    // int4 code tiles: 128 rows x 4 groups (128-byte swizzle)
+  uint8_t bm[2][kTmN * 128];           // min block B tiles: group sums hi | lo | 0, per unit slot
+  uint8_t bl[2][kTmN * 128];           // LoRA block B tiles: c t_g hi | lo | c t_u hi | lo
+  uint16_t sc[2][kTmMaxG][128];        // fp16 scales [group][row], per unit slot
+  uint16_t mn[2][kTmMaxG][128];        // fp16 mins
+  float xch[2][64 * kTmXRow];          // epilogue exchange: gate and up values of 64 columns
+  int tok[2][kTmN];                    // token of each column (-1: padding)
+  int dst[2][kTmN];                    // a row (gate/up) or gate index (down) of each column
+  float gw[2][kTmN];                   // combine weight of each column (down)
+  uint64_t bfull[kTmBStages], bempty[kTmBStages], cfull[kTmCStages], cempty[kTmCStages];
+  uint64_t afull[kTmAStages], aempty[kTmAStages];
+  uint64_t accfull[2], accempty[2], ufull[2], uempty[2], drain[2];
   uint32_t tmem;
   volatile int abort;
-  int tok[kTcN];       // token of each column
-  int dst[kTcN];       // ap row (mode 0) / gate index (mode 1) of each column, -1 = none
-  float gw[kTcN];      // combine weight of each column (mode 1)
 };
 
+struct TmUnit {
+  int tile, mt, unit, n0, ncol, N;
+  bool shared;
+};
+
+__device__ __forceinline__ TmUnit tm_unit(const TcArgs &A, int u, int mtiles) {
+  TmUnit U;
+  U.tile = u / mtiles;
+  U.mt = u % mtiles;
+  const TcTile tl = A.tiles[U.tile];
+  U.unit = tl.unit;
+  U.n0 = tl.n0;
+  U.shared = tl.unit == A.P.U[0];
+  const int cnt = U.shared ? A.T : A.P.ustart[tl.unit + 1] - A.P.ustart[tl.unit];
+  U.ncol = min(kTmN, cnt - tl.n0);
+  U.N = (U.ncol + 15) & ~15;   // MMA N: a multiple of 16
+  return U;
+}
+
 // bounded wait on an mbarrier phase that also gives up once another role has aborted
-__device__ __forceinline__ bool tw_wait(uint64_t *b, uint32_t parity, unsigned long long budget, int *err,
+__device__ __forceinline__ bool tm_wait(uint64_t *b, uint32_t parity, unsigned long long budget, int *err,
                                         volatile int *abort) {
   unsigned long long t0 = 0;
   while (!tc_mbar_test(b, parity)) {
@@ -312,69 +357,241 @@ __device__ __forceinline__ bool tw_wait(uint64_t *b, uint32_t parity, unsigned l
   return true;
 }
 
+// the same wait, agreed by the whole warp (the warp then runs its .sync.aligned
+// tensor-memory instructions together, or leaves together)
+__device__ __forceinline__ bool tm_wait_warp(uint64_t *b, uint32_t parity, unsigned long long budget, int *err,
+                                             volatile int *abort) {
+  return __all_sync(0xffffffffu, tm_wait(b, parity, budget, err, abort));
+}
+
 __device__ __forceinline__ void tc_mbar_arrive(uint64_t *b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tc_smem(b)) : "memory");
 }
 
-__global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_constant__ TcArgs A) {
-  extern __shared__ __align__(1024) uint8_t tc_raw[];
+__device__ __forceinline__ void tm_expect(uint64_t *b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_smem(b)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tm_load2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          tc_smem(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(tc_smem(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tm_load3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar,
+                                          unsigned long long pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3, %4}], [%5], %6;" ::"r"(tc_smem(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(tc_smem(bar)), "l"(pol)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f16 with fp16 A and B: fp32 accumulator (bits 4-5 = 1),
+// A and B fp16 (bits 7-9, 10-12 = 0), both K-major, N >> 3 (bits 17-22), M >> 4 (24-28).
+__device__ __forceinline__ uint32_t tm_idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// MMA with the A operand in tensor memory (M = 128 rows in the 128 lanes, K = 16 as 8
+// columns of 16-bit pairs) and B in shared memory
+__device__ __forceinline__ void tm_mma(uint32_t tmem_d, uint32_t tmem_a, unsigned long long bd, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bd), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 16 registers into 16 consecutive TMEM columns of this warp's 32 lanes
+__device__ __forceinline__ void tm_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t tm_hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// bf16 bits -> fp16 bits (exact for values in the fp16 normal range)
+__device__ __forceinline__ uint16_t tm_bf2h(uint32_t b) { return __half_as_ushort(__float2half_rn(bf(b))); }
+
+// fp16 pair (lo, hi) of two fp32 values
+__device__ __forceinline__ uint32_t tm_h2(float a, float b) {
+  return (uint32_t)__half_as_ushort(__float2half_rn(a)) | ((uint32_t)__half_as_ushort(__float2half_rn(b)) << 16);
+}
+// the fp16 remainders of two fp32 values after their fp16 roundings
+__device__ __forceinline__ uint32_t tm_h2lo(float a, float b) {
+  return tm_h2(a - __half2float(__float2half_rn(a)), b - __half2float(__float2half_rn(b)));
+}
+
+// Row c of the min block's B tile: 16-bit position k holds hi(X_k) for k < GT and
+// lo(X_(k-GT)) for GT <= k < 2 GT (X = the column's GT group sums, src = nullptr: zeros).
+template <int GT>
+__device__ __forceinline__ void tm_bm_row(uint8_t *tile, int c, const float *src) {
+  float xv[GT];
+#pragma unroll
+  for (int g = 0; g < GT; g++) xv[g] = 0.f;
+  if (src) {
+    if constexpr (GT % 4 == 0) {
+#pragma unroll
+      for (int g = 0; g < GT; g += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(src + g);
+        xv[g] = v.x; xv[g + 1] = v.y; xv[g + 2] = v.z; xv[g + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int g = 0; g < GT; g += 2) {
+        const float2 v = *reinterpret_cast<const float2 *>(src + g);
+        xv[g] = v.x; xv[g + 1] = v.y;
+      }
+    }
+  }
+  uint32_t wv[32];
+#pragma unroll
+  for (int j = 0; j < GT / 2; j++) wv[j] = tm_h2(xv[2 * j], xv[2 * j + 1]);
+#pragma unroll
+  for (int j = 0; j < GT / 2; j++) wv[GT / 2 + j] = tm_h2lo(xv[2 * j], xv[2 * j + 1]);
+#pragma unroll
+  for (int j = GT; j < 32; j++) wv[j] = 0u;
+#pragma unroll
+  for (int ch = 0; ch < 8; ch++)
+    *reinterpret_cast<uint4 *>(tile + sw128(c, ch)) = make_uint4(wv[4 * ch], wv[4 * ch + 1], wv[4 * ch + 2], wv[4 * ch + 3]);
+}
+template <int GT>
+__device__ __forceinline__ void tm_bm_row_any(int G, uint8_t *tile, int c, const float *src) {
+  if (G == GT) tm_bm_row<GT>(tile, c, src);
+  else if constexpr (GT > 2) tm_bm_row_any<GT - 2>(G, tile, c, src);
+}
+
+// Row c of the LoRA block's B tile (rank RT): 16-bit position k holds hi(c t_g[k]) for
+// k < RT, lo(c t_g[k - RT]) for RT <= k < 2 RT, hi(c t_u[k - 2 RT]), lo(c t_u[k - 3 RT])
+// up to 4 RT (t = the token's A_g x, A_u x; nullptr: zeros).
+template <int RT>
+__device__ __forceinline__ void tm_bl_row(uint8_t *tile, int c, const float *t, float cs) {
+  float tg[RT], tu[RT];
+#pragma unroll
+  for (int q = 0; q < RT; q += 2) {
+    float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+    if (t) {
+      a = *reinterpret_cast<const float2 *>(t + q);
+      b = *reinterpret_cast<const float2 *>(t + RT + q);
+    }
+    tg[q] = cs * a.x; tg[q + 1] = cs * a.y;
+    tu[q] = cs * b.x; tu[q + 1] = cs * b.y;
+  }
+  uint32_t wv[32];
+#pragma unroll
+  for (int j = 0; j < RT / 2; j++) {
+    wv[j] = tm_h2(tg[2 * j], tg[2 * j + 1]);
+    wv[RT / 2 + j] = tm_h2lo(tg[2 * j], tg[2 * j + 1]);
+    wv[RT + j] = tm_h2(tu[2 * j], tu[2 * j + 1]);
+    wv[3 * RT / 2 + j] = tm_h2lo(tu[2 * j], tu[2 * j + 1]);
+  }
+#pragma unroll
+  for (int j = 2 * RT; j < 32; j++) wv[j] = 0u;
+#pragma unroll
+  for (int ch = 0; ch < 8; ch++)
+    *reinterpret_cast<uint4 *>(tile + sw128(c, ch)) = make_uint4(wv[4 * ch], wv[4 * ch + 1], wv[4 * ch + 2], wv[4 * ch + 3]);
+}
+template <int RT>
+__device__ __forceinline__ void tm_bl_row_any(int r, uint8_t *tile, int c, const float *t, float cs) {
+  if (r == RT) tm_bl_row<RT>(tile, c, t, cs);
+  else if constexpr (RT > 2) tm_bl_row_any<RT - 2>(r, tile, c, t, cs);
+}
+
+// this thread's weight row's scales and mins as fp16 into [group][row] (the epilogue
+// threads, one per row, two units ahead)
+__device__ __forceinline__ void tm_fill_scales(const TcArgs &A, const TmUnit &U, int G, int row, uint16_t (*sc)[128],
+                                               uint16_t (*mn)[128]) {
+  const uint8_t *base = U.shared ? A.shared : A.src.base(A.P.uexp[U.unit]);
+  const uint16_t *scl, *mnv;
+  if (A.mode == 0) {
+    const int i = 64 * U.mt + (row & 63);
+    const bool up = row >= 64;
+    scl = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.us : A.bl.gs)) + (size_t)i * G;
+    mnv = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.um : A.bl.gm)) + (size_t)i * G;
+  } else {
+    const int n = 128 * U.mt + row;
+    scl = reinterpret_cast<const uint16_t *>(base + A.bl.ds) + (size_t)n * G;
+    mnv = reinterpret_cast<const uint16_t *>(base + A.bl.dm) + (size_t)n * G;
+  }
+  if ((G & 7) == 0) {
+    uint4 s8[kTmMaxG / 8], m8[kTmMaxG / 8];
+#pragma unroll
+    for (int j = 0; j < kTmMaxG / 8; j++)
+      if (8 * j < G) {
+        s8[j] = *reinterpret_cast<const uint4 *>(scl + 8 * j);
+        m8[j] = *reinterpret_cast<const uint4 *>(mnv + 8 * j);
+      }
+#pragma unroll
+    for (int j = 0; j < kTmMaxG / 8; j++)
+      if (8 * j < G) {
+        const uint32_t sw[4] = {s8[j].x, s8[j].y, s8[j].z, s8[j].w}, mw[4] = {m8[j].x, m8[j].y, m8[j].z, m8[j].w};
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          sc[8 * j + 2 * e][row] = tm_bf2h(sw[e] & 0xFFFFu);
+          sc[8 * j + 2 * e + 1][row] = tm_bf2h(sw[e] >> 16);
+          mn[8 * j + 2 * e][row] = tm_bf2h(mw[e] & 0xFFFFu);
+          mn[8 * j + 2 * e + 1][row] = tm_bf2h(mw[e] >> 16);
+        }
+      }
+  } else {
+    for (int g = 0; g < G; g++) {
+      sc[g][row] = tm_bf2h(scl[g]);
+      mn[g][row] = tm_bf2h(mnv[g]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_constant__ TcArgs A) {
+  extern __shared__ __align__(1024) uint8_t tm_raw[];
   // the swizzled tiles need 1024-byte alignment
-  TwSmem &S = *reinterpret_cast<TwSmem *>((reinterpret_cast<uintptr_t>(tc_raw) + 1023) & ~(uintptr_t)1023);
+  TmSmem &S = *reinterpret_cast<TmSmem *>((reinterpret_cast<uintptr_t>(tm_raw) + 1023) & ~(uintptr_t)1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mtiles = A.mode == 0 ? A.I / 64 : A.d / 128;
-  const int tile = blockIdx.x / mtiles, mt = blockIdx.x % mtiles;
-  if (tile >= *A.ntiles) return;
-  const TcTile tl = A.tiles[tile];
-  const int U = A.P.U[0];
-  const bool shared = tl.unit == U;
-  const int cnt = shared ? A.T : A.P.ustart[tl.unit + 1] - A.P.ustart[tl.unit];
-  const int ncol = min(kTcN, cnt - tl.n0);
-  const int N = (ncol + 15) & ~15;            // MMA N: multiple of 16
-  const uint8_t *base = shared ? A.shared : A.src.base(A.P.uexp[tl.unit]);
+  const int total = *A.ntiles * mtiles;
   const int K = A.mode == 0 ? A.d : A.I;
   const int G = K / 64;
   const unsigned long long budget = A.timeout_ns;
+  // the LoRA up block runs on the gate/up units of the shared expert
+  const bool lora_blk = A.mode == 0 && A.Bg != nullptr;
 
-  // column bookkeeping: token, destination and combine weight of each column of this tile
-  for (int c = tid; c < kTcN; c += kTwThreads) {
-    int tok = -1, dst = -1;
-    float w = 0.f;
-    if (c < ncol) {
-      if (shared) {
-        tok = tl.n0 + c;
-        dst = A.mode == 0 ? A.T * A.k + tok : -1;             // grouped row of a
-        w = 1.f;
-      } else {
-        const int asg = A.P.assign[A.P.ustart[tl.unit] + tl.n0 + c];   // t * k + slot
-        tok = asg / A.k;
-        dst = A.mode == 0 ? A.P.ustart[tl.unit] + tl.n0 + c : asg;   // grouped row of a / gate index
-        if (A.mode == 1) w = A.gates[asg];
-      }
-    }
-    S.tok[c] = tok;
-    S.dst[c] = dst;
-    S.gw[c] = w;
-  }
   if (tid == 0) {
-    for (int s = 0; s < kTwBStages; s++) {
-      tc_mbar_init(&S.bfull[s], 33);   // the TMA's expect_tx arrival + 32 group-sum lanes
-      tc_mbar_init(&S.bempty[s], 8);
+    for (int s = 0; s < kTmBStages; s++) {
+      tc_mbar_init(&S.bfull[s], 1);
+      tc_mbar_init(&S.bempty[s], 1);
     }
-    for (int s = 0; s < kTwAStages; s++) {
-      tc_mbar_init(&S.afull[s], 2);
+    for (int s = 0; s < kTmCStages; s++) {
+      tc_mbar_init(&S.cfull[s], 1);
+      tc_mbar_init(&S.cempty[s], kTmConvWarps);
+    }
+    for (int s = 0; s < kTmAStages; s++) {
+      tc_mbar_init(&S.afull[s], kTmConvWarps);
       tc_mbar_init(&S.aempty[s], 1);
     }
-    for (int s = 0; s < kTwTBufs; s++) {
-      tc_mbar_init(&S.tfull[s], 1);
-      tc_mbar_init(&S.tempty[s], 8);
+    for (int s = 0; s < 2; s++) {
+      tc_mbar_init(&S.accfull[s], 2);
+      tc_mbar_init(&S.accempty[s], kTmEpiThreads / 32);
+      tc_mbar_init(&S.ufull[s], 32 + kTmEpiThreads);
+      tc_mbar_init(&S.uempty[s], kTmEpiThreads / 32);
+      tc_mbar_init(&S.drain[s], 1);
     }
-    tc_mbar_init(&S.pre, 64);
     S.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == kTwMmaWarp) {
+  if (warp == kTmMma0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_smem(&S.tmem)),
-                 "r"(kTwTBufs * kTcN)
+                 "r"(kTmCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -383,265 +600,343 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = S.tmem;
 
-  if (warp < kTwLoadWarps) {
-    // ---------------- loader: one TMA tile load per group + the columns' group sums -------
-    // the tile's tokens are consecutive rows of the grouped operand starting at row0; rows
-    // past the tensor's end arrive as zeros (their columns are never used)
-    const CUtensorMap *map = (A.mode == 0 && shared) ? &A.tmB[1] : &A.tmB[0];
-    const int row0 = shared ? (A.mode == 0 ? tl.n0 : A.T * A.k + tl.n0) : A.P.ustart[tl.unit] + tl.n0;
-    #pragma unroll 1
-    for (int g = 0; g < G; g++) {
-      const int bs = g % kTwBStages;
-      if (g >= kTwBStages &&
-          !tw_wait(&S.bempty[bs], (uint32_t)(((g / kTwBStages) - 1) & 1), budget, A.err, &S.abort))
-        break;
-      if (lane == 0) {
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_smem(&S.bfull[bs])),
-                     "r"(kTcN * 128)
-                     : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-                tc_smem(S.b[bs])),
-            "l"(map), "r"(g * 64), "r"(row0), "r"(tc_smem(&S.bfull[bs]))
-            : "memory");
-      }
-      for (int c = lane; c < N; c += 32) {
-        const int tok = S.tok[c];
-        if (tok < 0) continue;    // padding column: its sum is never used
-        const float *src = A.mode == 0 ? A.xsum + (size_t)tok * G : A.asum + (size_t)(row0 + c) * G;
-        tc_cp4(tc_smem(&S.xs[bs][c]), src + g);
-      }
-      tc_cp_arrive(&S.bfull[bs]);
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == kTwMmaWarp) {
-    // ---------------- one thread issues the MMAs ------------------------------------------
+  if (warp == kTmProdWarp) {
+    // ---------------- producer: code tiles and activation tiles ---------------------------
     if (lane == 0) {
-      const uint32_t idesc = tc_idesc(128, N);
-      int issued = 0;
-      #pragma unroll 1
-      for (int g = 0; g < G; g++) {
-        const int as = g % kTwAStages, bs = g % kTwBStages, tb = g % kTwTBufs;
-        if (!tw_wait(&S.afull[as], (uint32_t)((g / kTwAStages) & 1), budget, A.err, &S.abort)) break;
-        if (!tw_wait(&S.bfull[bs], (uint32_t)((g / kTwBStages) & 1), budget, A.err, &S.abort)) break;
-        if (g >= kTwTBufs && !tw_wait(&S.tempty[tb], (uint32_t)(((g / kTwTBufs) - 1) & 1), budget, A.err, &S.abort))
-          break;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t sa = tc_smem(S.a[as]), sb = tc_smem(S.b[bs]);
-        const uint32_t td = tmem + (uint32_t)(tb * kTcN);
-#pragma unroll
-        for (int kk = 0; kk < 4; kk++)   // K = 16 per instruction: 32 bytes along the swizzled row
-          tc_mma(td, tc_desc(sa + kk * 32), tc_desc(sb + kk * 32), idesc, kk ? 1u : 0u);
-        tc_commit(&S.tfull[tb]);
-        tc_commit(&S.aempty[as]);
-        issued = g + 1;
+      const unsigned long long pol_first = tc_policy_first();
+      const unsigned long long pol_keep = tc_policy_last();
+      int rg = 0, cc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+        const TmUnit U = tm_unit(A, u, mtiles);
+        // routed experts' codes are read by one or two token tiles (evict first); the
+        // shared expert's by every token tile of the call (keep)
+        const unsigned long long pol = U.shared ? pol_keep : pol_first;
+        const int z = U.shared ? 0 : A.P.uexp[U.unit];
+        const CUtensorMap *mapB = (A.mode == 0 && U.shared) ? &A.tmB[1] : &A.tmB[0];
+        const int brow = U.shared ? (A.mode == 0 ? U.n0 : A.T * A.k + U.n0) : A.P.ustart[U.unit] + U.n0;
+        for (int g0 = 0; g0 < G && ok; g0 += 4, cc++) {
+          const int cs = cc % kTmCStages;
+          if (cc >= kTmCStages &&
+              !(ok = tm_wait(&S.cempty[cs], (uint32_t)(((cc / kTmCStages) - 1) & 1), budget, A.err, &S.abort)))
+            break;
+          tm_expect(&S.cfull[cs], 128 * 128);
+          if (A.mode == 0) {
+            // gate rows 64 mt .. 64 mt + 63, then the up rows of the same intermediate units
+            const CUtensorMap *mg = U.shared ? &A.tmC[2] : &A.tmC[0];
+            const CUtensorMap *mu = U.shared ? &A.tmC[3] : &A.tmC[1];
+            tm_load3d(S.c[cs], mg, 32 * g0, 64 * U.mt, z, &S.cfull[cs], pol);
+            tm_load3d(S.c[cs] + 64 * 128, mu, 32 * g0, 64 * U.mt, z, &S.cfull[cs], pol);
+          } else {
+            tm_load3d(S.c[cs], U.shared ? &A.tmC[2] : &A.tmC[0], 32 * g0, 128 * U.mt, z, &S.cfull[cs], pol);
+          }
+          const int ng = min(4, G - g0);
+          for (int lg = 0; lg < ng; lg++, rg++) {
+            const int bs = rg % kTmBStages;
+            if (rg >= kTmBStages &&
+                !(ok = tm_wait(&S.bempty[bs], (uint32_t)(((rg / kTmBStages) - 1) & 1), budget, A.err, &S.abort)))
+              break;
+            tm_expect(&S.bfull[bs], kTmN * 128);
+            tm_load2d(S.b[bs], mapB, 64 * (g0 + lg), brow, &S.bfull[bs]);
+          }
+        }
       }
-      // after an abort, the MMAs in flight finish before TMEM is given back
-      if (issued > 0 && issued < G)
-        tc_wait_all(&S.tfull[(issued - 1) % kTwTBufs], (uint32_t)(((issued - 1) / kTwTBufs) & 1), budget, A.err);
+      if (!ok) {
+        // every tile load issued lands before the CTA may exit
+        for (int s = 0; s < kTmCStages; s++) {
+          const int n = cc / kTmCStages + (s < cc % kTmCStages ? 1 : 0);
+          if (n > 0) tc_wait_all(&S.cfull[s], (uint32_t)((n - 1) & 1), budget, A.err);
+        }
+        for (int s = 0; s < kTmBStages; s++) {
+          const int n = rg / kTmBStages + (s < rg % kTmBStages ? 1 : 0);
+          if (n > 0) tc_wait_all(&S.bfull[s], (uint32_t)((n - 1) & 1), budget, A.err);
+        }
+      }
     }
     __syncwarp();
-  } else if (warp < kTwFold0) {
-    // ---------------- converters: thread t owns weight rows t and t + 64 ------------------
-    // mode 0 -> gate rows i0..i0+63 then up rows i0..i0+63 (i0 = 64 mt); mode 1 -> down
-    // rows 128 mt .. 128 mt + 127
-    const int t = tid - kTwConv0 * 32;     // 0..63
-    const uint8_t *codes[2];
-    const uint16_t *scl[2], *mnv[2];
+  } else if (warp == kTmMma0 || warp == kTmMma1) {
+    // ---------------- the two MMA issuers -------------------------------------------------
+    // A-stage entries per unit: [min block] [LoRA block] group 0 .. G - 1.  Issuer 0 takes
+    // the extra blocks and the even groups, issuer 1 the odd groups, each both fp16 parts
+    // into its own accumulator.  Every stage has one owner, so an issuer waits on each of
+    // its barriers' phases in order: A stages 0, 1 belong to issuer 0 and stage 2 to issuer
+    // 1; B stage rg % kTmBStages carries real group rg, owned by issuer rg % 2 (every unit
+    // has an even number of K groups, kTmBStages is even).
+    if (lane == 0) {
+      const int part = warp == kTmMma0 ? 0 : 1;
+      int kown = 0, rg = 0, it = 0;
+      bool ok = true, any = false;
+      for (int u = blockIdx.x; u < total && ok; u += gridDim.x, it++) {
+        const TmUnit U = tm_unit(A, u, mtiles);
+        const uint32_t idesc = tm_idesc_f16(128, U.N);
+        const int ab = it & 1, slot = it & 1;
+        const uint32_t td = tmem + (uint32_t)((2 * part + ab) * kTmN);
+        const int nx = 1 + ((lora_blk && U.shared) ? 1 : 0);   // extra blocks of this unit
+        ok = (it < 2 || tm_wait(&S.accempty[ab], (uint32_t)(((it >> 1) - 1) & 1), budget, A.err, &S.abort)) &&
+             (part == 1 || tm_wait(&S.ufull[slot], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort));
+        if (!ok) break;
+        bool first = true;
+        for (int e = 0; e < nx + G; e++) {
+          const bool real = e >= nx;
+          const bool mine = real ? ((e - nx) & 1) == part : part == 0;
+          const int bs = rg % kTmBStages;
+          if (mine) {
+            const int as = part == 0 ? (kown & 1) : 2;
+            const uint32_t ph = (uint32_t)((part == 0 ? (kown >> 1) : kown) & 1);
+            ok = tm_wait(&S.afull[as], ph, budget, A.err, &S.abort) &&
+                 (!real || tm_wait(&S.bfull[bs], (uint32_t)((rg / kTmBStages) & 1), budget, A.err, &S.abort));
+            if (!ok) break;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t sb = tc_smem(real ? S.b[bs] : (e == 0 ? S.bm[slot] : S.bl[slot]));
+            const uint32_t ta = tmem + kTmACol + (uint32_t)(64 * as);
 #pragma unroll
-    for (int h = 0; h < 2; h++) {
-      const int r = t + 64 * h;
-      if (A.mode == 0) {
-        const int i = mt * 64 + (r & 63);
-        const bool up = r >= 64;
-        codes[h] = base + (up ? A.bl.uc : A.bl.gc) + (size_t)i * (A.d / 2);
-        scl[h] = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.us : A.bl.gs)) + (size_t)i * G;
-        mnv[h] = reinterpret_cast<const uint16_t *>(base + (up ? A.bl.um : A.bl.gm)) + (size_t)i * G;
-      } else {
-        const int n = mt * 128 + r;
-        codes[h] = base + A.bl.dc + (size_t)n * (A.I / 2);
-        scl[h] = reinterpret_cast<const uint16_t *>(base + A.bl.ds) + (size_t)n * G;
-        mnv[h] = reinterpret_cast<const uint16_t *>(base + A.bl.dm) + (size_t)n * G;
+            for (int kk = 0; kk < 4; kk++) {   // K = 16 per instruction: 8 TMEM columns of A, 32 bytes of B
+              tm_mma(td, ta + 8 * kk, tc_desc(sb + kk * 32), idesc, first ? 0u : 1u);   // s (q & 14)
+              first = false;
+              if (real) tm_mma(td, ta + 32 + 8 * kk, tc_desc(sb + kk * 32), idesc, 1u);  // s (q & 1)
+            }
+            any = true;
+            tc_commit(&S.aempty[as]);
+            if (real) tc_commit(&S.bempty[bs]);
+            kown++;
+          }
+          if (real) rg++;
+        }
+        if (!ok) break;
+        tc_commit(&S.accfull[ab]);
       }
-      // the row's scales and mins for the folders (rows of fewer than 16 bytes in 4-byte copies)
-      const int rb = G * 2;
-      if (rb % 16 == 0) {
-        for (int q = 0; q < rb / 16; q++) {
-          tc_cp16(tc_smem(S.sc + r * G + q * 8), scl[h] + q * 8, 16);
-          tc_cp16(tc_smem(S.mn + r * G + q * 8), mnv[h] + q * 8, 16);
-        }
-      } else {
-        for (int q = 0; q < rb / 4; q++) {
-          tc_cp4(tc_smem(S.sc + r * G + q * 2), scl[h] + q * 2);
-          tc_cp4(tc_smem(S.mn + r * G + q * 2), mnv[h] + q * 2);
-        }
+      // after an abort, the MMAs in flight finish before TMEM is given back
+      if (!ok && any) {
+        tc_commit(&S.drain[part]);
+        tc_wait_all(&S.drain[part], 0u, budget, A.err);
       }
     }
-    tc_cp_arrive(&S.pre);
-    // the rows' codes, kTwRawAhead groups in flight, one cp.async group per K group
-    const unsigned long long pol = tc_policy_first();
-    auto load_codes = [&](int g, int rs) {
-#pragma unroll
-      for (int h = 0; h < 2; h++) {
-        const int r = t + 64 * h;
-        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32), codes[h] + g * 32, 16, pol);
-        tc_cp16_hint(tc_smem(S.raw[rs] + r * 32 + 16), codes[h] + g * 32 + 16, 16, pol);
-      }
-    };
-    for (int g = 0; g < kTwRawAhead; g++) {
-      if (g < G) load_codes(g, g);
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    }
-    #pragma unroll 1
-    for (int g = 0; g < G; g++) {
-      const int as = g % kTwAStages, rs = g % kTwRawAhead;
-      asm volatile("cp.async.wait_group %0;" ::"n"(kTwRawAhead - 1) : "memory");   // own codes of g
-      if (g >= kTwAStages &&
-          !tw_wait(&S.aempty[as], (uint32_t)(((g / kTwAStages) - 1) & 1), budget, A.err, &S.abort))
+    __syncwarp();
+  } else if (warp == kTmUnitWarp) {
+    // ---------------- unit warp: bookkeeping, extra blocks' B tiles, scales ---------------
+    bool ok = true;
+    for (int u = blockIdx.x, it = 0; u < total && ok; u += gridDim.x, it++) {
+      const int slot = it & 1;
+      if (it >= 2 && !(ok = tm_wait_warp(&S.uempty[slot], (uint32_t)(((it >> 1) - 1) & 1), budget, A.err, &S.abort)))
         break;
-      // word j of a row's 32 code bytes = K elements 8 j .. 8 j + 7 = chunk j, unpacked in
-      // the permuted order (0,4,1,5,2,6,3,7) as bf16 128 + q
-      uint8_t *dstA = S.a[as];
-#pragma unroll
-      for (int h = 0; h < 2; h++) {
-        const int r = t + 64 * h;
-        const uint4 w0 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32);
-        const uint4 w1 = *reinterpret_cast<const uint4 *>(S.raw[rs] + r * 32 + 16);
-        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int j = 0; j < 8; j++) {
-          const uint32_t wd = ws[j];
-          const uint32_t p0 = (wd & 0x000F000Fu) | 0x43004300u;
-          const uint32_t p1 = ((wd >> 4) & 0x000F000Fu) | 0x43004300u;
-          const uint32_t p2 = ((wd >> 8) & 0x000F000Fu) | 0x43004300u;
-          const uint32_t p3 = ((wd >> 12) & 0x000F000Fu) | 0x43004300u;
-          *reinterpret_cast<uint4 *>(dstA + sw128(r, j)) = make_uint4(p0, p1, p2, p3);
+      const TmUnit U = tm_unit(A, u, mtiles);
+      const int row0 = U.shared ? (A.mode == 0 ? U.n0 : A.T * A.k + U.n0) : A.P.ustart[U.unit] + U.n0;
+      const bool lb = lora_blk && U.shared;
+      for (int c = lane; c < kTmN; c += 32) {
+        int tok = -1, dst = -1;
+        float w = 0.f;
+        if (c < U.ncol) {
+          if (U.shared) {
+            tok = U.n0 + c;
+            dst = A.mode == 0 ? A.T * A.k + tok : -1;             // grouped row of a
+            w = 1.f;
+          } else {
+            const int asg = A.P.assign[A.P.ustart[U.unit] + U.n0 + c];   // t * k + slot
+            tok = asg / A.k;
+            dst = A.mode == 0 ? A.P.ustart[U.unit] + U.n0 + c : asg;     // grouped row of a / gate index
+            if (A.mode == 1) w = A.gates[asg];
+          }
         }
+        S.tok[slot][c] = tok;
+        S.dst[slot][c] = dst;
+        S.gw[slot][c] = w;
+        // row c of the min block's B tile: the column's group sums (x by token for gate/up,
+        // a by grouped row for down) split hi | lo
+        const float *src = tok < 0 ? nullptr : (A.mode == 0 ? A.xsum + (size_t)tok * G : A.asum + (size_t)(row0 + c) * G);
+        tm_bm_row_any<kTmMaxG>(G, S.bm[slot], c, src);
+        // row c of the LoRA block's B tile: c t_g and c t_u split hi | lo
+        if (lb) tm_bl_row_any<kTmMaxR>(A.r, S.bl[slot], c, tok < 0 ? nullptr : A.lt + (size_t)tok * 3 * A.r, A.c);
       }
+      // the extra blocks' B tiles are read by the tensor core (async proxy)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) tc_mbar_arrive(&S.afull[as]);
-      // refill these rows' slots (their words are consumed above) with group g + kTwRawAhead
-      if (g + kTwRawAhead < G) load_codes(g + kTwRawAhead, rs);
-      asm volatile("cp.async.commit_group;" ::: "memory");
+      tc_mbar_arrive(&S.ufull[slot]);
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-  } else {
-    // ---------------- folders: TMEM -> registers, acc += s P + (m - 128 s) X -------------
-    const int fw = warp - kTwFold0;                 // 0..7
-    const int erow = 32 * (warp & 3) + lane;        // tile row = TMEM lane
-    const int cbeg = (fw >> 2) * (kTcN / 2);        // this warp's half of the columns
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    unsigned long long acc[kTcN / 4];               // 64 fp32 accumulators as packed pairs
-#pragma unroll
-    for (int i = 0; i < kTcN / 4; i++) acc[i] = 0ull;
-    bool ok = tw_wait(&S.pre, 0, budget, A.err, &S.abort);
-    #pragma unroll 1
-    for (int g = 0; g < G && ok; g++) {
-      const int tb = g % kTwTBufs, bs = g % kTwBStages;
-      ok = tw_wait(&S.tfull[tb], (uint32_t)((g / kTwTBufs) & 1), budget, A.err, &S.abort) &&
-           tw_wait(&S.bfull[bs], (uint32_t)((g / kTwBStages) & 1), budget, A.err, &S.abort);
-      if (!ok) break;
+  } else if (warp < kTmConv0) {
+    // ---------------- epilogue: TMEM -> SwiGLU / weighted combine --------------------------
+    const int q = warp & 3, row = 32 * q + lane, et = tid - kTmEpi0 * 32;   // et 0..127
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    // the rows' scales and mins of a unit, two units ahead (this thread: weight row `row`)
+    auto fill = [&](int it2) {
+      const int u2 = blockIdx.x + it2 * gridDim.x;
+      if (u2 >= total) return;
+      const TmUnit U2 = tm_unit(A, u2, mtiles);
+      tm_fill_scales(A, U2, G, row, S.sc[it2 & 1], S.mn[it2 & 1]);
+      tc_mbar_arrive(&S.ufull[it2 & 1]);
+    };
+    fill(0);
+    fill(1);
+    bool ok = true;
+    for (int u = blockIdx.x, it = 0; u < total && ok; u += gridDim.x, it++) {
+      const int ab = it & 1, slot = it & 1;
+      ok = tm_wait_warp(&S.accfull[ab], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort) &&
+           tm_wait_warp(&S.ufull[slot], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort);
+      {
+        // the four epilogue warps agree (named barrier 1) before any of them uses the
+        // exchange barriers below, so that none is left waiting for a warp that gave up
+        uint32_t bad;
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbarrier.red.or.pred q, 1, %2, p;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(bad)
+            : "r"((uint32_t)!ok), "r"(kTmEpiThreads)
+            : "memory");
+        if (bad) break;
+      }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const float s = bf(S.sc[erow * G + g]), m = fmaf(-128.f, s, bf(S.mn[erow * G + g]));
-      const unsigned long long s2 = pk2(s, s), m2 = pk2(m, m);
-      const float *xg = S.xs[bs] + cbeg;
-      const uint32_t taddr = lane_addr + (uint32_t)(tb * kTcN + cbeg);
-      if (cbeg < N) {
-        // this warp's 64 columns in one TMEM load (columns past N hold stale values that
-        // only reach accumulators of unused columns)
-        float v[64];
-        tc_ld64(taddr, v);
+      const TmUnit U = tm_unit(A, u, mtiles);
+      const uint32_t t0 = tmem + tl + (uint32_t)(ab * kTmN), t1 = tmem + tl + (uint32_t)((2 + ab) * kTmN);
+      if (A.mode == 0) {
+        // rows 0..63 gate, 64..127 up of intermediate units i = 64 mt + (row & 63)
+        const bool up = row >= 64;
+        for (int h64 = 0; h64 < U.N; h64 += 64) {
+          asm volatile("bar.sync 1, 128;" ::: "memory");   // the previous exchange has been read
 #pragma unroll
-        for (int cc = 0; cc < 64; cc += 4) {
-          const float4 x4 = *reinterpret_cast<const float4 *>(xg + cc);
-          unsigned long long &a0 = acc[cc / 2], &a1 = acc[cc / 2 + 1];
-          a0 = f2fma(m2, pk2(x4.x, x4.y), f2fma(s2, pk2(v[cc], v[cc + 1]), a0));
-          a1 = f2fma(m2, pk2(x4.z, x4.w), f2fma(s2, pk2(v[cc + 2], v[cc + 3]), a1));
+          for (int ch = 0; ch < 2; ch++) {
+            const int c0 = h64 + 32 * ch;
+            if (c0 < U.N) {
+              float v[32], w[32];
+              tc_ld32(t0 + c0, v);
+              tc_ld32(t1 + c0, w);
+              float *xr = S.xch[up ? 1 : 0] + (row & 63) * kTmXRow + 32 * ch;
+#pragma unroll
+              for (int j = 0; j < 32; j++) xr[j] = v[j] + w[j];
+            }
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          // a = bf16(silu(g) u): thread et takes unit et % 64 of every other column
+          const int iu = et & 63, ipos = kperm_pos(64 * U.mt + iu);
+          for (int j = et >> 6; j < 64; j += 2) {
+            const int c = h64 + j;
+            if (c >= U.ncol) break;
+            const int dst = S.dst[slot][c];
+            if (dst < 0) continue;
+            const float g = S.xch[0][iu * kTmXRow + j], uu = S.xch[1][iu * kTmXRow + j];
+            // the bf16 rounding point of a, stored as the same value in fp16 (the down
+            // GEMM's operand type)
+            const float av = __bfloat162float(__float2bfloat16_rn(g / (1.0f + expf(-g)) * uu));
+            A.ap_out[(size_t)dst * A.I + ipos] = __half_as_ushort(__float2half_rn(av));
+          }
+        }
+      } else {
+        float *yrow = A.yacc + 128 * U.mt + row;
+#pragma unroll
+        for (int ch = 0; ch < (kTmN + 31) / 32; ch++) {   // (columns past N are read, never used)
+          const int c0 = 32 * ch;
+          if (c0 < U.N) {
+            float v[32], w[32];
+            tc_ld32(t0 + c0, v);
+            tc_ld32(t1 + c0, w);
+#pragma unroll
+            for (int j = 0; j < 32; j++) {
+              const int c = c0 + j;
+              if (c >= U.ncol) continue;
+              const int tok = S.tok[slot][c];
+              if (tok < 0) continue;
+              asm volatile("red.global.add.f32 [%0], %1;" ::"l"(yrow + (size_t)tok * A.d),
+                           "f"(S.gw[slot][c] * (v[j] + w[j]))
+                           : "memory");
+            }
+          }
         }
       }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
-        tc_mbar_arrive(&S.tempty[tb]);
-        tc_mbar_arrive(&S.bempty[bs]);
+        tc_mbar_arrive(&S.accempty[ab]);
+        tc_mbar_arrive(&S.uempty[slot]);
       }
+      // every MMA of this unit has completed (accfull), so every converter is done with
+      // this slot's scales and mins
+      fill(it + 2);
     }
-    // every folder agrees before the epilogue (named barrier 1: the 8 folder warps)
-    {
-      uint32_t bad;
-      asm volatile(
-          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbarrier.red.or.pred q, 1, %2, p;\n\t"
-          "selp.u32 %0, 1, 0, q;\n\t}"
-          : "=r"(bad)
-          : "r"((uint32_t)!ok), "r"(256)
-          : "memory");
-      ok = bad == 0;
-    }
-    if (ok) {
-      // the tile's results go through shared memory as ex[row][column] with a row stride of
-      // kTcN + 1 floats, so that lanes on consecutive rows hit different banks both when
-      // writing (lane = row) and when reading (lane = row again, or four rows per lane)
-      constexpr int XS = kTcN + 1;
-      float *ex = reinterpret_cast<float *>(S.b[0]);   // 128 x XS floats (66 KB of the B ring)
-      if (A.mode == 0) {
-        // gate rows 0..63 and up rows 64..127 (with the shared expert's LoRA up branch);
-        // then all 256 folder threads form a = bf16(silu(g) u), thread t taking unit t % 64
-        // of four columns per pass
-        const int i = mt * 64 + (erow & 63);
-        const bool up = erow >= 64;
-        const bool lora = shared && A.Bg != nullptr;
-        float lb[kMaxR];
-        if (lora)
-          for (int q = 0; q < A.r; q++) lb[q] = bf((up ? A.Bu : A.Bg)[(size_t)i * A.r + q]);
+  } else {
+    // ---------------- converters: codes -> exact fp16 parts in TMEM ----------------------
+    const int q = warp & 3, h = (warp - kTmConv0) >> 2;
+    const int row = 32 * q + lane;              // weight row of the tile = TMEM lane
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    int gg = 0, cc = 0;
+    bool ok = true;
+    // one A-stage entry: this thread's 16 columns of part 0 (and of part 1 for a K group),
+    // into the next stage of the entry's issuer (stages 0, 1: issuer 0; stage 2: issuer 1)
+    int k0 = 0, k1 = 0;
+    auto put = [&](const uint32_t (&p1)[16], const uint32_t (&p2)[16], bool two, int owner) -> bool {
+      const int as = owner == 0 ? (k0 & 1) : 2;
+      const int n = owner == 0 ? (k0 >> 1) : k1;   // earlier uses of this stage
+      if (n > 0 && !tm_wait_warp(&S.aempty[as], (uint32_t)((n - 1) & 1), budget, A.err, &S.abort)) return false;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t ta = tmem + tl + kTmACol + (uint32_t)(64 * as + 16 * h);
+      tm_st16(ta, p1);
+      if (two) tm_st16(ta + 32, p2);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) tc_mbar_arrive(&S.afull[as]);
+      if (owner == 0) k0++;
+      else k1++;
+      gg++;
+      return true;
+    };
+    for (int u = blockIdx.x, it = 0; u < total && ok; u += gridDim.x, it++) {
+      const int slot = it & 1;
+      if (!(ok = tm_wait_warp(&S.ufull[slot], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort))) break;
+      const TmUnit U = tm_unit(A, u, mtiles);
+      uint32_t p1[16], p2[16];
+      // min block: element k of the row = m_(k mod G) for k < 2 G, else 0 (this thread's
+      // elements 32 h .. 32 h + 31)
 #pragma unroll
-        for (int cp = 0; cp < kTcN / 4; cp++) {
-          float v0 = __uint_as_float((uint32_t)acc[cp]), v1 = __uint_as_float((uint32_t)(acc[cp] >> 32));
-          const int c = cbeg + 2 * cp;
-          if (lora && c < ncol) {
-            for (int h2 = 0; h2 < 2; h2++) {
-              const int tok = S.tok[c + h2];
-              if (tok < 0) continue;
-              const float *t = A.lt + (size_t)tok * 3 * A.r + (up ? A.r : 0);
-              float la = 0.f;
-              for (int q = 0; q < A.r; q++) la = fmaf(lb[q], t[q], la);
-              if (h2 == 0) v0 = fmaf(A.c, la, v0);
-              else v1 = fmaf(A.c, la, v1);
+      for (int j = 0; j < 16; j++) {
+        const int k0 = 32 * h + 2 * j, k1 = k0 + 1;
+        const uint32_t v0 = k0 < 2 * G ? S.mn[slot][k0 < G ? k0 : k0 - G][row] : 0u;
+        const uint32_t v1 = k1 < 2 * G ? S.mn[slot][k1 < G ? k1 : k1 - G][row] : 0u;
+        p1[j] = v0 | (v1 << 16);
+      }
+      if (!(ok = put(p1, p2, false, 0))) break;
+      if (lora_blk && U.shared) {
+        // LoRA block: gate row i: B_g[i] at k < r and again at r <= k < 2 r; up row: B_u[i]
+        // at 2 r <= k < 3 r and again at 3 r <= k < 4 r
+        const int i = 64 * U.mt + (row & 63);
+        const bool up = row >= 64;
+        const uint16_t *Bm = (up ? A.Bu : A.Bg) + (size_t)i * A.r;
+        const int k0 = up ? 2 * A.r : 0;
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+          const int ka = 32 * h + 2 * j, kb = ka + 1;
+          const int qa = ka - k0, qb = kb - k0;   // index into the doubled B row
+          const uint32_t va = (qa >= 0 && qa < 2 * A.r) ? tm_bf2h(Bm[qa < A.r ? qa : qa - A.r]) : 0u;
+          const uint32_t vb = (qb >= 0 && qb < 2 * A.r) ? tm_bf2h(Bm[qb < A.r ? qb : qb - A.r]) : 0u;
+          p1[j] = va | (vb << 16);
+        }
+        if (!(ok = put(p1, p2, false, 0))) break;
+      }
+      for (int g0 = 0; g0 < G && ok; g0 += 4, cc++) {
+        const int cs = cc % kTmCStages, ng = min(4, G - g0);
+        if (!(ok = tm_wait_warp(&S.cfull[cs], (uint32_t)((cc / kTmCStages) & 1), budget, A.err, &S.abort))) break;
+#pragma unroll
+        for (int lg = 0; lg < 4; lg++) {
+          if (lg >= ng) break;
+          // half h of group g0 + lg of this row: 16 bytes = 32 codes
+          const uint4 w = *reinterpret_cast<const uint4 *>(S.c[cs] + sw128(row, 2 * lg + h));
+          if (lg == ng - 1) {
+            __syncwarp();
+            if (lane == 0) tc_mbar_arrive(&S.cempty[cs]);
+          }
+          const uint32_t sh = S.sc[slot][g0 + lg][row];
+          const uint32_t s2 = sh | (sh << 16);
+          const uint32_t c2 = tm_hfma2(s2, 0xE400E400u, 0u);   // -1024 s, exact
+          // word j holds K elements 8 j .. 8 j + 7; nibbles n and n + 4 form the fp16 pair
+          // of TMEM column 4 j + n (the K-permuted order of the activation operand):
+          // 1024 + (q & 14) and 1024 + (q & 1) as fp16, then (1024 + v) s - 1024 s = v s
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+#pragma unroll
+            for (int n = 0; n < 4; n++) {
+              const uint32_t sv = ws[j] >> (4 * n);
+              p1[4 * j + n] = tm_hfma2((sv & 0x000E000Eu) | 0x64006400u, s2, c2);
+              p2[4 * j + n] = tm_hfma2((sv & 0x00010001u) | 0x64006400u, s2, c2);
             }
           }
-          ex[erow * XS + c] = v0;
-          ex[erow * XS + c + 1] = v1;
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        const int ft = tid - kTwFold0 * 32, iu = ft & 63;
-        const int ipos = kperm_pos(mt * 64 + iu);
-        #pragma unroll 4
-        for (int c = ft >> 6; c < ncol; c += 4) {
-          const int dst = S.dst[c];
-          if (dst < 0) continue;
-          const float g = ex[iu * XS + c], u = ex[(64 + iu) * XS + c];
-          A.ap_out[(size_t)dst * A.I + ipos] = f2bf(g / (1.0f + expf(-g)) * u);   // bf16 rounding point of a
-        }
-      } else {
-        // gate-weighted values to shared memory, then four consecutive output rows of one
-        // column per thread, added into y with one vector reduction
-#pragma unroll
-        for (int cp = 0; cp < kTcN / 4; cp++) {
-          const int c = cbeg + 2 * cp;
-          ex[erow * XS + c] = S.gw[c] * __uint_as_float((uint32_t)acc[cp]);
-          ex[erow * XS + c + 1] = S.gw[c + 1] * __uint_as_float((uint32_t)(acc[cp] >> 32));
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        const int ft = tid - kTwFold0 * 32;
-        for (int it = ft; it < ncol * 32; it += 256) {
-          const int c = it >> 5, n4 = it & 31;
-          const int tok = S.tok[c];
-          if (tok < 0) continue;
-          const float y0 = ex[(4 * n4) * XS + c], y1 = ex[(4 * n4 + 1) * XS + c];
-          const float y2 = ex[(4 * n4 + 2) * XS + c], y3 = ex[(4 * n4 + 3) * XS + c];
-          float *dstp = A.yacc + (size_t)tok * A.d + mt * 128 + 4 * n4;
-          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dstp), "f"(y0), "f"(y1), "f"(y2), "f"(y3)
-                       : "memory");
+          if (!(ok = put(p1, p2, true, (g0 + lg) & 1))) break;
         }
       }
     }
@@ -649,8 +944,8 @@ __global__ void __launch_bounds__(kTwThreads, 1) k_moe_gemm_tc(const __grid_cons
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (warp == kTwMmaWarp)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTwTBufs * kTcN) : "memory");
+  if (warp == kTmMma0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmCols) : "memory");
 }
 
 // ---------------------------------------------------------------------------------------
@@ -817,7 +1112,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_rows(TcRowsArgs A) {
 // every group of 64 (natural order).  One thread per (row, group).
 // ---------------------------------------------------------------------------------------
 __global__ void k_perm_sums(const uint16_t *__restrict__ x, long long rows, int K, uint16_t *__restrict__ xp,
-                            float *__restrict__ sums) {
+                            float *__restrict__ sums, int in_f16) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int G = K / 64;
   if (i >= rows * G) return;
@@ -825,22 +1120,27 @@ __global__ void k_perm_sums(const uint16_t *__restrict__ x, long long rows, int 
   const int g = (int)(i % G);
   const uint4 *src = reinterpret_cast<const uint4 *>(x + r * K + g * 64);
   uint4 *dst = xp ? reinterpret_cast<uint4 *>(xp + r * K + g * 64) : nullptr;
+  // 16-bit element -> fp32 (bf16 or fp16 input), and a bf16 element as the same fp16 value
+  auto val = [&](uint32_t b) { return in_f16 ? __half2float(__ushort_as_half((uint16_t)b)) : bf(b); };
+  auto h16 = [&](uint32_t b) { return (uint32_t)__half_as_ushort(__float2half_rn(bf(b))); };
   float s = 0.f;
 #pragma unroll
   for (int q = 0; q < 8; q++) {
     const uint4 v = src[q];
     // natural elements 8q .. 8q+7 = (v.x lo, v.x hi, v.y lo, v.y hi, v.z lo, ...)
-    s += bf(v.x & 0xFFFFu);
-    s += bf(v.x >> 16);
-    s += bf(v.y & 0xFFFFu);
-    s += bf(v.y >> 16);
-    s += bf(v.z & 0xFFFFu);
-    s += bf(v.z >> 16);
-    s += bf(v.w & 0xFFFFu);
-    s += bf(v.w >> 16);
-    if (dst)   // permuted block (0,4,1,5,2,6,3,7)
-      dst[q] = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
-                          __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+    s += val(v.x & 0xFFFFu);
+    s += val(v.x >> 16);
+    s += val(v.y & 0xFFFFu);
+    s += val(v.y >> 16);
+    s += val(v.z & 0xFFFFu);
+    s += val(v.z >> 16);
+    s += val(v.w & 0xFFFFu);
+    s += val(v.w >> 16);
+    if (dst) {   // bf16 input -> the fp16 tensor-core operand, permuted block (0,4,1,5,2,6,3,7)
+      const uint32_t e0 = h16(v.x & 0xFFFFu), e1 = h16(v.x >> 16), e2 = h16(v.y & 0xFFFFu), e3 = h16(v.y >> 16);
+      const uint32_t e4 = h16(v.z & 0xFFFFu), e5 = h16(v.z >> 16), e6 = h16(v.w & 0xFFFFu), e7 = h16(v.w >> 16);
+      dst[q] = make_uint4(e0 | (e4 << 16), e1 | (e5 << 16), e2 | (e6 << 16), e3 | (e7 << 16));
+    }
   }
   sums[i] = s;
 }
@@ -855,8 +1155,9 @@ __global__ void k_group_rows(const uint16_t *__restrict__ xp, const int32_t *__r
   for (int i = threadIdx.x; i < d / 8; i += blockDim.x) dst[i] = src[i];
 }
 
-// t_d = Ad a_s from the K-permuted bf16 activations (one warp per token and rank row); the
-// shared expert's a rows are rows T k .. T k + T - 1 of the grouped a
+// t_d = Ad a_s from the K-permuted activations (fp16 holding the bf16 values of a; one warp
+// per token and rank row); the shared expert's a rows are rows T k .. T k + T - 1 of the
+// grouped a
 __global__ void k_lora_td(const uint16_t *__restrict__ Ad, const uint16_t *__restrict__ ap, int T, int I, int k,
                           int r, float *__restrict__ lt) {
   const int lane = threadIdx.x & 31;
@@ -865,7 +1166,8 @@ __global__ void k_lora_td(const uint16_t *__restrict__ Ad, const uint16_t *__res
   const int t = w / r, j = w % r;
   const uint16_t *as = ap + ((size_t)T * k + t) * I;
   float acc = 0.f;
-  for (int i = lane; i < I; i += 32) acc = fmaf(bf(Ad[(size_t)j * I + i]), bf(as[kperm_pos(i)]), acc);
+  for (int i = lane; i < I; i += 32)
+    acc = fmaf(bf(Ad[(size_t)j * I + i]), __half2float(__ushort_as_half(as[kperm_pos(i)])), acc);
   acc = warp_sum(acc);
   if (lane == 0) lt[((size_t)t * 3 + 2) * r + j] = acc;
 }
