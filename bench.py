@@ -49,9 +49,9 @@ KERNEL_TRAFFIC = {
                       "bytes to the 40-layer launch"),
     "prefill_t4096_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh",
                            "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "d088c3d2737d7eff", 343.6e6,
-                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 465.8 MB, "
-                          "down 221.4 MB, mean of the two"),
+                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "d60190184d9d6c48", 321.7e6,
+                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 425.5 MB, "
+                          "down 217.9 MB, mean of the two"),
 }
 
 
@@ -651,7 +651,7 @@ def run_prefill(args, dims, seed, ws, rank, local, T=4096):
         "metric": "MoE-stack prefill tokens/s on 1 B200 (4096-token chunk, 40 layers)", "value": tokens / (ms / 1e3),
         "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int4 weights as exact bf16 tensor-core operands (128+q), bf16 activations, fp32 accumulate",
+        "dtype": "int4 weights as two exact fp16 tensor-core operands (s(q&14), s(q&1)), bf16-valued fp16 activations, fp32 accumulate",
         "data": "synthetic (seeded)",
         "config": {"workload": "prefill_t4096_l40", "layers": dims.L, "tokens": T, "d": dims.d, "experts": dims.E,
                    "d_ff": dims.I, "top_k": dims.k, "parallelism": f"replicas x{ws}",
