@@ -50,11 +50,35 @@ __global__ void k_norm(const uint16_t *__restrict__ h, const float *__restrict__
   const uint16_t *hr = h + (size_t)t * d;
   const float *cr = chain ? chain + (size_t)t * d : nullptr;
   __shared__ double red[32];
-  double ss = 0.0;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    double v = (double)bf(hr[i]);
+  // the layer input (h, or bf16(h + chain)) of element i, in double
+  auto in = [&](int i, uint32_t hb) {
+    double v = (double)bf(hb);
     if (cr) v = (double)bf(d2bf(v + (double)cr[i]));
-    ss += v * v;
+    return v;
+  };
+  // fast path: 8 consecutive elements per thread held in registers (one read of h, 16-byte
+  // accesses); otherwise a strided pass per element
+  const bool vec = d % 8 == 0 && d / 8 <= (int)blockDim.x;
+  const int c8 = threadIdx.x;                   // this thread's 8-element chunk (fast path)
+  double v8[8];
+  double ss = 0.0;
+  if (vec) {
+    if (c8 < d / 8) {
+      const uint4 w = *reinterpret_cast<const uint4 *>(hr + 8 * c8);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        v8[2 * j] = in(8 * c8 + 2 * j, ws[j] & 0xFFFFu);
+        v8[2 * j + 1] = in(8 * c8 + 2 * j + 1, ws[j] >> 16);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; j++) ss += v8[j] * v8[j];
+    }
+  } else {
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+      const double v = in(i, hr[i]);
+      ss += v * v;
+    }
   }
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
@@ -66,12 +90,33 @@ __global__ void k_norm(const uint16_t *__restrict__ h, const float *__restrict__
   }
   __syncthreads();
   const double rinv = 1.0 / sqrt(red[0] / d + (double)eps);
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    double v = (double)bf(hr[i]);
-    if (cr) v = (double)bf(d2bf(v + (double)cr[i]));
-    const uint16_t b = d2bf(v * (double)bf(gamma[i]) * rinv);
-    xb[(size_t)t * d + i] = b;
-    xf[(size_t)t * d + i] = bf(b);
+  if (vec) {
+    if (c8 < d / 8) {
+      const uint4 gw = *reinterpret_cast<const uint4 *>(gamma + 8 * c8);
+      const uint32_t gs[4] = {gw.x, gw.y, gw.z, gw.w};
+      uint32_t ob[4];
+      float of[8];
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const uint16_t b0 = d2bf(v8[2 * j] * (double)bf(gs[j] & 0xFFFFu) * rinv);
+        const uint16_t b1 = d2bf(v8[2 * j + 1] * (double)bf(gs[j] >> 16) * rinv);
+        ob[j] = (uint32_t)b0 | ((uint32_t)b1 << 16);
+        of[2 * j] = bf(b0);
+        of[2 * j + 1] = bf(b1);
+      }
+      *reinterpret_cast<uint4 *>(xb + (size_t)t * d + 8 * c8) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+      if (xf) {
+        float4 *fo = reinterpret_cast<float4 *>(xf + (size_t)t * d + 8 * c8);
+        fo[0] = make_float4(of[0], of[1], of[2], of[3]);
+        fo[1] = make_float4(of[4], of[5], of[6], of[7]);
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < d; i += blockDim.x) {
+      const uint16_t b = d2bf(in(i, hr[i]) * (double)bf(gamma[i]) * rinv);
+      xb[(size_t)t * d + i] = b;
+      if (xf) xf[(size_t)t * d + i] = bf(b);
+    }
   }
 }
 

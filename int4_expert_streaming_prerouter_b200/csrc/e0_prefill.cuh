@@ -1165,9 +1165,26 @@ __global__ void k_lora_td(const uint16_t *__restrict__ Ad, const uint16_t *__res
   if (w >= T * r) return;
   const int t = w / r, j = w % r;
   const uint16_t *as = ap + ((size_t)T * k + t) * I;
+  const uint16_t *ad = Ad + (size_t)j * I;
   float acc = 0.f;
-  for (int i = lane; i < I; i += 32)
-    acc = fmaf(bf(Ad[(size_t)j * I + i]), __half2float(__ushort_as_half(as[kperm_pos(i)])), acc);
+  if (I % 8 == 0 && ((uintptr_t)ad & 15) == 0) {
+    // one 8-block per lane and step: a (fp16 holding its bf16 values) is stored in the
+    // block order (0,4,1,5,2,6,3,7), A_d in natural order
+    for (int b = lane; b < I / 8; b += 32) {
+      const uint4 aw = *reinterpret_cast<const uint4 *>(as + 8 * b), dw = *reinterpret_cast<const uint4 *>(ad + 8 * b);
+      const uint32_t av[4] = {aw.x, aw.y, aw.z, aw.w}, dv[4] = {dw.x, dw.y, dw.z, dw.w};
+#pragma unroll
+      for (int m = 0; m < 4; m++) {
+        // a word m holds elements m (low) and m + 4 (high); A_d word m / 2 holds 2 (m/2)..
+        const uint32_t d_lo = (m & 1) ? dv[m >> 1] >> 16 : dv[m >> 1] & 0xFFFFu;        // element m
+        const uint32_t d_hi = (m & 1) ? dv[2 + (m >> 1)] >> 16 : dv[2 + (m >> 1)] & 0xFFFFu;   // element m + 4
+        acc = fmaf(bf(d_lo), __half2float(__ushort_as_half((uint16_t)(av[m] & 0xFFFFu))), acc);
+        acc = fmaf(bf(d_hi), __half2float(__ushort_as_half((uint16_t)(av[m] >> 16))), acc);
+      }
+    }
+  } else {
+    for (int i = lane; i < I; i += 32) acc = fmaf(bf(ad[i]), __half2float(__ushort_as_half(as[kperm_pos(i)])), acc);
+  }
   acc = warp_sum(acc);
   if (lane == 0) lt[((size_t)t * 3 + 2) * r + j] = acc;
 }
