@@ -635,15 +635,19 @@ def run_prefill(args, dims, seed, ws, rank, local, T=4096):
     # the dominant kernel: the expert GEMMs' FLOPs over their own measured launch time
     achieved = flops * args.steps / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else flops / step_s / 1e12
     traffic, traffic_how = kernel_traffic("prefill_t4096_l40")
-    # end to end: the chunk's inputs from pinned host memory, its outputs back
+    # end to end through the C ABI with host buffers (e0_moe_prefill_stack_host): every
+    # layer's input copied in from pinned host memory and its output copied back, the
+    # copies of one layer beside the kernels of its neighbours
     h_host = h.cpu().pin_memory()
     y_host = torch.empty_like(h_host).pin_memory()
+    ctx.prefill_stack_host(h_host, y_host)   # untimed: the staging buffers are allocated on first use
+    ctx.host_io_wait()
+    torch.cuda.synchronize()
     e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_a.record(stream)
     for _ in range(args.steps):
-        h.copy_(h_host, non_blocking=True)
-        ctx.prefill_stack(h, y_out=y)
-        y_host.copy_(y, non_blocking=True)
+        ctx.prefill_stack_host(h_host, y_host)
+    ctx.host_io_wait()
     e_b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_a.elapsed_time(e_b), ws)

@@ -196,8 +196,9 @@ int e0_moe_stack_decode(e0_ctx *ctx, const void *h_in, int B, int step, void *y_
  * allocated. */
 int e0_moe_stack_decode_host(e0_ctx *ctx, const void *h_host, int B, int step, void *y_host, float *y_f32_host,
                              int streaming, int chained, void *stream);
-/* Make `stream` wait for every copy issued so far by e0_moe_stack_decode_host (no-op if
- * there was none).  Errors: INVALID_ARG (NULL context), CUDA. */
+/* Make `stream` wait for every copy issued so far by e0_moe_stack_decode_host and
+ * e0_moe_prefill_stack_host (no-op if there was none).  Errors: INVALID_ARG (NULL
+ * context), CUDA. */
 int e0_host_io_wait(e0_ctx *ctx, void *stream);
 
 /* Streaming decode mode ([G] "Sonuçlar": prerouter prefetch against fully reactive
@@ -219,6 +220,17 @@ int e0_stream_mode(e0_ctx *ctx, int reactive);
  * Errors: INVALID_ARG, CUDA. */
 int e0_moe_prefill_stack(e0_ctx *ctx, const void *h_in, int T, void *y_out, float *y_f32, int32_t *idx_out,
                          void *stream);
+
+/* e0_moe_prefill_stack with the input and outputs in host memory (pinned, so that the
+ * copies are asynchronous): h_host [L, T, d] bf16, y_host [L, T, d] bf16, y_f32_host
+ * [L, T, d] or NULL; idx_out [L, T, k] int32 device memory or NULL.  Layer l's input is
+ * copied in while layer l-1 computes and its outputs copied out while layer l+1 computes
+ * (two copy streams of the context, two alternating device staging buffers of max_tokens
+ * x d, allocated on the first call).  The outputs are complete after
+ * e0_host_io_wait(ctx, stream) and a synchronisation of `stream`; the host buffers must
+ * stay valid until then.  Errors: as e0_moe_prefill_stack, and OOM. */
+int e0_moe_prefill_stack_host(e0_ctx *ctx, const void *h_host, int T, void *y_host, float *y_f32_host,
+                              int32_t *idx_out, void *stream);
 
 /* Routing the last e0_moe_stack_decode used and predicted, copied to host memory:
  * idx [L, B, k] (routing used at that step), pred [L, B, k] (next step's routing; -1 for

@@ -73,6 +73,7 @@ _SIGS = {
     "e0_host_io_wait": (_I, [_P, _P]),
     "e0_get_routing": (_I, [_P, _I, _P, _P]),
     "e0_moe_prefill_stack": (_I, [_P, _P, _I, _P, _P, _P, _P]),
+    "e0_moe_prefill_stack_host": (_I, [_P, _P, _I, _P, _P, _P, _P]),
     "e0_get_stats": (_I, [_P, ctypes.POINTER(Stats)]),
     "e0_sync_status": (_I, [_P]),
     "e0_last_error": (ctypes.c_char_p, []),
@@ -282,6 +283,17 @@ class Context:
 
     def host_io_wait(self, stream=None):
         _check(lib().e0_host_io_wait(self._h, _stream(stream)))
+
+    def prefill_stack_host(self, h_host, y_host, y_f32_host=None, idx=None, stream=None):
+        """prefill_stack with pinned host tensors h_host, y_host [L, T, d] bf16 (y_f32_host
+        [L, T, d] fp32 or None; idx a CUDA int32 tensor [L, T, k] or None).  The library
+        overlaps each layer's copies with the neighbouring layers' kernels; the outputs are
+        complete after host_io_wait(stream) and a synchronisation of the stream."""
+        L, T, d = h_host.shape
+        assert not h_host.is_cuda and not y_host.is_cuda and (y_f32_host is None or not y_f32_host.is_cuda)
+        _check(lib().e0_moe_prefill_stack_host(self._h, _ptr(h_host), T, _ptr(y_host), _ptr(y_f32_host), _ptr(idx),
+                                               _stream(stream)))
+        return y_host
 
     def prefill_stack(self, h_in, y_out=None, y_f32=None, idx=None, stream=None):
         """h_in [L, T, d] bf16 -> y_out [L, T, d] bf16 (prediction-as-routing, one token ahead)."""

@@ -189,15 +189,22 @@ struct e0_ctx {
   e0_stats stats{};
   bool time_gemm = false;                          // profiling: event pairs around the GEMMs
   std::vector<std::pair<cudaEvent_t, cudaEvent_t>> gemm_ev;
-  // decode steps with host buffers (e0_moe_stack_decode_host): a copy stream and two
-  // alternating device staging buffers, ordered with the steps by events
+  // decode steps and prefill chunks with host buffers (e0_moe_stack_decode_host,
+  // e0_moe_prefill_stack_host): one copy stream for inputs and one for outputs (so that an
+  // input copy never queues behind the previous output copy, which waits for its kernels),
+  // and two alternating device staging buffers each, ordered with the compute by events
   struct HostIO {
-    cudaStream_t cs = nullptr;
-    cudaEvent_t in[2] = {}, out[2] = {}, done[2] = {}, tail = nullptr;
+    cudaStream_t cs = nullptr, ds = nullptr;   // host -> device, device -> host
+    cudaEvent_t in[2] = {}, out[2] = {}, done[2] = {}, tail = nullptr, tail2 = nullptr;
     uint16_t *h[2] = {}, *y[2] = {};
     float *yf[2] = {};
     bool used[2] = {};
     long long calls = 0;
+    // prefill chunks: per-layer staging (maxT x d each)
+    cudaEvent_t pin[2] = {}, pout[2] = {}, pdone[2] = {};
+    uint16_t *ph[2] = {}, *py[2] = {};
+    float *pyf[2] = {};
+    bool pused[2] = {};
   } io;
 };
 
@@ -248,13 +255,16 @@ extern "C" int e0_destroy(e0_ctx *C) {
     for (auto e : {r.c0, r.c1, r.w0, r.w1}) cudaEventDestroy(e);
   if (C->pool.side) cudaStreamDestroy(C->pool.side);
   for (int b = 0; b < 2; b++) {
-    for (cudaEvent_t e : {C->io.in[b], C->io.out[b], C->io.done[b]})
+    for (cudaEvent_t e : {C->io.in[b], C->io.out[b], C->io.done[b], C->io.pin[b], C->io.pout[b], C->io.pdone[b]})
       if (e) cudaEventDestroy(e);
-    for (void *m : {(void *)C->io.h[b], (void *)C->io.y[b], (void *)C->io.yf[b]})
+    for (void *m : {(void *)C->io.h[b], (void *)C->io.y[b], (void *)C->io.yf[b], (void *)C->io.ph[b],
+                    (void *)C->io.py[b], (void *)C->io.pyf[b]})
       if (m) cudaFree(m);
   }
-  if (C->io.tail) cudaEventDestroy(C->io.tail);
-  if (C->io.cs) cudaStreamDestroy(C->io.cs);
+  for (cudaEvent_t e : {C->io.tail, C->io.tail2})
+    if (e) cudaEventDestroy(e);
+  for (cudaStream_t st : {C->io.cs, C->io.ds})
+    if (st) cudaStreamDestroy(st);
   delete C;
   return E0_OK;
 }
@@ -1457,6 +1467,17 @@ extern "C" int e0_moe_stack_decode(e0_ctx *C, const void *h_in, int B, int step,
   return E0_OK;
 }
 
+// The two copy streams and their tail events (created on first use).
+static int host_io_streams(e0_ctx *C) {
+  auto &io = C->io;
+  if (io.cs) return E0_OK;
+  CK(cudaStreamCreateWithFlags(&io.cs, cudaStreamNonBlocking));
+  CK(cudaStreamCreateWithFlags(&io.ds, cudaStreamNonBlocking));
+  CK(cudaEventCreateWithFlags(&io.tail, cudaEventDisableTiming));
+  CK(cudaEventCreateWithFlags(&io.tail2, cudaEventDisableTiming));
+  return E0_OK;
+}
+
 // A decode step with the input and output in (pinned) host memory.  Step n uses staging
 // buffer n % 2: its input copy (copy stream) waits until step n-2's kernels have read the
 // buffer, the step (caller's stream) waits for the input copy and for step n-2's output
@@ -1470,8 +1491,9 @@ extern "C" int e0_moe_stack_decode_host(e0_ctx *C, const void *h_host, int B, in
     return fail(E0_ERR_INVALID_ARG, "e0_moe_stack_decode_host: bad arguments (B=%d, max %d)", B, C->maxT);
   auto &io = C->io;
   const size_t n = (size_t)C->L * C->maxT * C->dims.d_model, used = (size_t)C->L * B * C->dims.d_model;
-  if (!io.cs) {
-    CK(cudaStreamCreateWithFlags(&io.cs, cudaStreamNonBlocking));
+  int rc0;
+  if ((rc0 = host_io_streams(C))) return rc0;
+  if (!io.h[0]) {
     for (int b = 0; b < 2; b++) {
       CK(cudaEventCreateWithFlags(&io.in[b], cudaEventDisableTiming));
       CK(cudaEventCreateWithFlags(&io.out[b], cudaEventDisableTiming));
@@ -1479,7 +1501,6 @@ extern "C" int e0_moe_stack_decode_host(e0_ctx *C, const void *h_host, int B, in
       int rc;
       if ((rc = dalloc(&io.h[b], n)) || (rc = dalloc(&io.y[b], n))) return rc;
     }
-    CK(cudaEventCreateWithFlags(&io.tail, cudaEventDisableTiming));
   }
   if (y_f32_host && !io.yf[0]) {
     int rc;
@@ -1500,22 +1521,61 @@ extern "C" int e0_moe_stack_decode_host(e0_ctx *C, const void *h_host, int B, in
   io.calls++;
   CK(cudaEventRecord(io.out[b], s));
   if (rc) {
-    CK(cudaEventRecord(io.done[b], io.cs));
+    CK(cudaEventRecord(io.done[b], io.ds));
     return rc;
   }
-  CK(cudaStreamWaitEvent(io.cs, io.out[b], 0));
-  CK(cudaMemcpyAsync(y_host, io.y[b], used * 2, cudaMemcpyDeviceToHost, io.cs));
-  if (y_f32_host) CK(cudaMemcpyAsync(y_f32_host, io.yf[b], used * 4, cudaMemcpyDeviceToHost, io.cs));
-  CK(cudaEventRecord(io.done[b], io.cs));
+  CK(cudaStreamWaitEvent(io.ds, io.out[b], 0));
+  CK(cudaMemcpyAsync(y_host, io.y[b], used * 2, cudaMemcpyDeviceToHost, io.ds));
+  if (y_f32_host) CK(cudaMemcpyAsync(y_f32_host, io.yf[b], used * 4, cudaMemcpyDeviceToHost, io.ds));
+  CK(cudaEventRecord(io.done[b], io.ds));
   return E0_OK;
 }
 
-// Make `stream` wait for every copy that the host-buffer decode calls have issued.
+// Make `stream` wait for every copy that the host-buffer decode and prefill calls have
+// issued.
 extern "C" int e0_host_io_wait(e0_ctx *C, void *stream) {
   if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
   if (!C->io.cs) return E0_OK;
   CK(cudaEventRecord(C->io.tail, C->io.cs));
+  CK(cudaEventRecord(C->io.tail2, C->io.ds));
   CK(cudaStreamWaitEvent((cudaStream_t)stream, C->io.tail, 0));
+  CK(cudaStreamWaitEvent((cudaStream_t)stream, C->io.tail2, 0));
+  return E0_OK;
+}
+
+// One layer of a prefill chunk (see e0_moe_prefill_stack): h_l, y_l [T, d], yf_l [T, d]
+// or NULL, idx_l [T, k] or NULL.  Layer l reads the predictions layer l-1 made in the same
+// chunk (alternating buffers).
+static int prefill_layer(e0_ctx *C, int l, const uint16_t *h_l, int T, uint16_t *y_l, float *yf_l, int32_t *idx_l,
+                         cudaStream_t s) {
+  const int k = C->dims.top_k;
+  const bool predicted = l > 0 && C->heads[l - 1].w_lin != nullptr;
+  int32_t *pin = C->pf_buf + (size_t)((l + 1) & 1) * (C->maxT + 1) * k;   // written by layer l-1's head
+  int32_t *pout = C->pf_buf + (size_t)(l & 1) * (C->maxT + 1) * k;
+  LayerCall K{};
+  K.l = l; K.T = T; K.h = h_l;
+  K.route = predicted ? pin : nullptr;          // row t = prediction made on token t-1
+  K.full_mode = predicted ? 2 : 1;              // row 0 is -1: token 0 uses its own router
+  K.idx = idx_l ? idx_l : C->pf_idx + k;
+  K.gates = C->gates;
+  K.head = C->heads[l].w_lin != nullptr;
+  K.prev = nullptr;
+  K.pred = pout + k;                             // prediction of token t -> row t+1
+  K.y = y_l;
+  K.yf = yf_l;
+  int rc = layer_pre(C, K, s);
+  if (rc) return rc;
+  return layer_post(C, K, resident_src(C, l), s);
+}
+
+static int prefill_check(e0_ctx *C, const void *h, int T, const void *y) {
+  if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
+  if (!h || !y || T < 1 || T > C->maxT)
+    return fail(E0_ERR_INVALID_ARG, "prefill stack: bad arguments (T=%d, max %d)", T, C->maxT);
+  if (C->dims.head_hidden > 0 || C->dims.head_onehot)
+    return fail(E0_ERR_INVALID_ARG, "prefill stack supports the linear head without one-hot inputs");
+  for (int l = 0; l < C->L; l++)
+    if (!C->layers[l].experts) return fail(E0_ERR_INVALID_ARG, "layer %d has no resident experts", l);
   return E0_OK;
 }
 
@@ -1525,36 +1585,66 @@ extern "C" int e0_host_io_wait(e0_ctx *C, void *stream) {
 // inputs (the workloads' form).
 extern "C" int e0_moe_prefill_stack(e0_ctx *C, const void *h_in, int T, void *y_out, float *y_f32, int32_t *idx_out,
                                     void *stream) {
-  if (!C || !C->registered) return fail(E0_ERR_INVALID_ARG, "context missing or model not registered");
-  if (!h_in || !y_out || T < 1 || T > C->maxT)
-    return fail(E0_ERR_INVALID_ARG, "e0_moe_prefill_stack: bad arguments (T=%d, max %d)", T, C->maxT);
-  if (C->dims.head_hidden > 0 || C->dims.head_onehot)
-    return fail(E0_ERR_INVALID_ARG, "prefill stack supports the linear head without one-hot inputs");
-  for (int l = 0; l < C->L; l++)
-    if (!C->layers[l].experts) return fail(E0_ERR_INVALID_ARG, "layer %d has no resident experts", l);
+  int rc0;
+  if ((rc0 = prefill_check(C, h_in, T, y_out))) return rc0;
   cudaStream_t s = (cudaStream_t)stream;
   C->last = s;
-  const e0_dims &D = C->dims;
-  const int k = D.top_k;
-  const size_t ld = (size_t)T * D.d_model;
+  const size_t ld = (size_t)T * C->dims.d_model;
   for (int l = 0; l < C->L; l++) {
-    const bool predicted = l > 0 && C->heads[l - 1].w_lin != nullptr;
-    int32_t *pin = C->pf_buf + (size_t)((l + 1) & 1) * (C->maxT + 1) * k;   // written by layer l-1's head
-    int32_t *pout = C->pf_buf + (size_t)(l & 1) * (C->maxT + 1) * k;
-    LayerCall K{};
-    K.l = l; K.T = T; K.h = (const uint16_t *)h_in + l * ld;
-    K.route = predicted ? pin : nullptr;          // row t = prediction made on token t-1
-    K.full_mode = predicted ? 2 : 1;              // row 0 is -1: token 0 uses its own router
-    K.idx = idx_out ? idx_out + (size_t)l * T * k : C->pf_idx + k;
-    K.gates = C->gates;
-    K.head = C->heads[l].w_lin != nullptr;
-    K.prev = nullptr;
-    K.pred = pout + k;                             // prediction of token t -> row t+1
-    K.y = (uint16_t *)y_out + l * ld;
-    K.yf = y_f32 ? y_f32 + l * ld : nullptr;
-    int rc = layer_pre(C, K, s);
+    int rc = prefill_layer(C, l, (const uint16_t *)h_in + l * ld, T, (uint16_t *)y_out + l * ld,
+                           y_f32 ? y_f32 + l * ld : nullptr, idx_out ? idx_out + (size_t)l * T * C->dims.top_k : nullptr, s);
     if (rc) return rc;
-    if ((rc = layer_post(C, K, resident_src(C, l), s))) return rc;
+  }
+  return E0_OK;
+}
+
+// A prefill chunk with the input and output in (pinned) host memory: layer l's input is
+// copied in (input copy stream) while layer l-1 computes, and its output copied out
+// (output copy stream) while layer l+1 computes; two alternating device staging buffers,
+// ordered by events (the layers' inputs are independent, so the copies of every layer but
+// the first and the last hide behind the kernels).
+extern "C" int e0_moe_prefill_stack_host(e0_ctx *C, const void *h_host, int T, void *y_host, float *y_f32_host,
+                                         int32_t *idx_out, void *stream) {
+  int rc;
+  if ((rc = prefill_check(C, h_host, T, y_host))) return rc;
+  if ((rc = host_io_streams(C))) return rc;
+  auto &io = C->io;
+  const size_t cap = (size_t)C->maxT * C->dims.d_model, ld = (size_t)T * C->dims.d_model;
+  if (!io.ph[0]) {
+    for (int b = 0; b < 2; b++) {
+      CK(cudaEventCreateWithFlags(&io.pin[b], cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&io.pout[b], cudaEventDisableTiming));
+      CK(cudaEventCreateWithFlags(&io.pdone[b], cudaEventDisableTiming));
+      if ((rc = dalloc(&io.ph[b], cap)) || (rc = dalloc(&io.py[b], cap))) return rc;
+    }
+  }
+  if (y_f32_host && !io.pyf[0])
+    for (int b = 0; b < 2; b++)
+      if ((rc = dalloc(&io.pyf[b], cap))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  C->last = s;
+  for (int l = 0; l < C->L; l++) {
+    const int b = l & 1;
+    if (io.pused[b]) {
+      CK(cudaStreamWaitEvent(io.cs, io.pout[b], 0));   // the layer two back has read ph[b]
+      CK(cudaStreamWaitEvent(s, io.pdone[b], 0));      // py[b] of the layer two back is out
+    }
+    CK(cudaMemcpyAsync(io.ph[b], (const uint16_t *)h_host + l * ld, ld * 2, cudaMemcpyHostToDevice, io.cs));
+    CK(cudaEventRecord(io.pin[b], io.cs));
+    CK(cudaStreamWaitEvent(s, io.pin[b], 0));
+    rc = prefill_layer(C, l, io.ph[b], T, io.py[b], y_f32_host ? io.pyf[b] : nullptr,
+                       idx_out ? idx_out + (size_t)l * T * C->dims.top_k : nullptr, s);
+    io.pused[b] = true;
+    CK(cudaEventRecord(io.pout[b], s));
+    if (rc) {
+      CK(cudaEventRecord(io.pdone[b], io.ds));
+      return rc;
+    }
+    CK(cudaStreamWaitEvent(io.ds, io.pout[b], 0));
+    CK(cudaMemcpyAsync((uint16_t *)y_host + l * ld, io.py[b], ld * 2, cudaMemcpyDeviceToHost, io.ds));
+    if (y_f32_host)
+      CK(cudaMemcpyAsync(y_f32_host + l * ld, io.pyf[b], ld * 4, cudaMemcpyDeviceToHost, io.ds));
+    CK(cudaEventRecord(io.pdone[b], io.ds));
   }
   return E0_OK;
 }

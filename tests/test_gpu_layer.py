@@ -297,6 +297,38 @@ def test_prefill_stack_prediction_as_routing_shifted_one_token(cuda_ok):
     ctx.close()
 
 
+def test_prefill_stack_with_host_buffers_matches_the_device_call(cuda_ok):
+    """The host-buffer prefill (per-layer copies beside the neighbouring layers' kernels)
+    gives the routing and outputs of the device call on the same inputs, twice in a row
+    (the staging buffers alternate between layers and calls), and the oracle's."""
+    dims = Dims(d=256, E=16, I=128, k=4, r=8, L=3, head_layers=(0, 1))
+    ctx, _, _ = make_ctx(dims, 221, 256)
+    T = 96
+    hs = np.stack([synth.hidden(221 + n, 0, 1, T, dims.d)[0] for n in range(dims.L)])
+    idx_d = torch.empty((dims.L, T, dims.k), dtype=torch.int32, device="cuda")
+    yd32 = torch.empty((dims.L, T, dims.d), dtype=torch.float32, device="cuda")
+    ctx.prefill_stack(bf16_tensor(hs, "cuda"), y_f32=yd32, idx=idx_d)
+    ctx.sync_status()
+    h_host = bf16_tensor(hs, "cpu").pin_memory()
+    for call in range(2):
+        y_host = torch.empty((dims.L, T, dims.d), dtype=torch.bfloat16).pin_memory()
+        y32_host = torch.empty((dims.L, T, dims.d), dtype=torch.float32).pin_memory()
+        idx_h = torch.empty((dims.L, T, dims.k), dtype=torch.int32, device="cuda")
+        ctx.prefill_stack_host(h_host, y_host, y_f32_host=y32_host, idx=idx_h)
+        ctx.host_io_wait()
+        torch.cuda.synchronize()
+        ctx.sync_status()
+        assert torch.equal(idx_h.cpu(), idx_d.cpu()), call
+        # the expert combine adds in tile completion order: compare within the tolerance
+        for n in range(dims.L):
+            check_y(y32_host[n].numpy(), yd32[n].cpu().numpy().astype(np.float64), f"call {call} layer {n}")
+        yb = bf16_bits_to_np(y_host)
+        ref = oracle_layer(dims, 221, 0, hs[0], route=None, gpu_idx=idx_h.cpu().numpy()[0])
+        compare(dims, (yb[0], y32_host[0].numpy().astype(np.float64), idx_h.cpu().numpy()[0], np.zeros((T, dims.k))),
+                dict(ref, gates=np.zeros((T, dims.k))), f"call {call} layer 0 vs oracle")
+    ctx.close()
+
+
 def test_prefill_tensor_core_path_full_width_t4096(cuda_ok):
     """The benchmarked prefill chunk size on one full-width layer (d=2048, E=256, I=512,
     r=16, T=4096, about 64 tokens per routed expert), own-router routing, through the
