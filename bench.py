@@ -44,14 +44,14 @@ METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak
 KERNEL_TRAFFIC = {
     "decode_b1_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh",
                        "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "2e9b3dd381860134", 409.9e6,
-                      "4-layer capture (40.99 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
+                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "6c77dfd4624134ef", 408.5e6,
+                      "4-layer capture (40.85 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
                       "bytes to the 40-layer launch"),
     "prefill_t4096_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh",
                            "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "d60190184d9d6c48", 321.7e6,
-                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 425.5 MB, "
-                          "down 217.9 MB, mean of the two"),
+                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "42d0b551396104d8", 318.8e6,
+                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 422.9 MB, "
+                          "down 214.7 MB, mean of the two"),
 }
 
 
