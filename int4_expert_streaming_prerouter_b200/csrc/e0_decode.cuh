@@ -183,6 +183,16 @@ __host__ __device__ __forceinline__ void split_range(int N, int G, int c, int &a
 __host__ __device__ __forceinline__ int pair_index(int e) {   // uint16 index of element e
   return (e >> 3) * 8 + (e & 3) * 2 + ((e >> 2) & 1);
 }
+// uint16 index of element e of an N-element activation vector in the decode kernel's
+// tables: elements in pair_index order within each 8-element word, and within each
+// 512-element step of n words (64, or what is left) word w stored at (w & 1) n / 2 + (w >> 1),
+// so that the two B-fragment words of a row-pair step (w = 8 g + 2 t and 8 g + 2 t + 1) are
+// two lane-ordered 16-byte loads without bank conflicts
+__device__ __forceinline__ int pair_slot(int e, int N) {
+  const int w = e >> 3, s = w >> 6, wl = w & 63;
+  const int n = min(64, N / 8 - 64 * s);
+  return ((64 * s + (wl & 1) * (n >> 1) + (wl >> 1)) << 3) + (e & 3) * 2 + ((e >> 2) & 1);
+}
 __device__ __forceinline__ uint32_t nib_pair_bf16(uint32_t w, int j) {
   return ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
 }
@@ -205,6 +215,21 @@ __device__ __forceinline__ void pair_step(float (&d)[4], uint2 c0, uint2 c1, uin
                  vb.x, vb.y);
   mma_bf16_16816(d, nib_pair_bf16(c0.y, 2), nib_pair_bf16(c1.y, 2), nib_pair_bf16(c0.y, 3), nib_pair_bf16(c1.y, 3),
                  vb.z, vb.w);
+}
+// Sums over the warp of four per-lane values at once (a transposing butterfly, six
+// shuffles): lanes 0-7 return the sum of v0, lanes 8-15 of v1, 16-23 of v2, 24-31 of v3.
+__device__ __forceinline__ float warp_sum4(float v0, float v1, float v2, float v3, int lane) {
+  const bool hi = lane & 16;
+  float a = hi ? v2 : v0, b = hi ? v3 : v1;
+  a += __shfl_xor_sync(0xffffffffu, hi ? v0 : v2, 16);
+  b += __shfl_xor_sync(0xffffffffu, hi ? v1 : v3, 16);
+  const bool b8 = lane & 8;
+  float c = b8 ? b : a;
+  c += __shfl_xor_sync(0xffffffffu, b8 ? a : b, 8);
+  c += __shfl_xor_sync(0xffffffffu, c, 4);
+  c += __shfl_xor_sync(0xffffffffu, c, 2);
+  c += __shfl_xor_sync(0xffffffffu, c, 1);
+  return c;
 }
 // the diagonal lane's affine fold of group G of one row: s P + (m - 128 s) V
 __device__ __forceinline__ float group_fold(float P, const uint16_t *sc, const uint16_t *mn, int G, float V) {
@@ -261,6 +286,7 @@ __host__ __device__ __forceinline__ Item unpack_item(unsigned long long v) {
 // A range of gate/up units touches consecutive slots ("pieces"): at most kMaxPieces.
 constexpr int kMaxPieces = 4;
 constexpr int kDnMaxRows = 64;   // down rows per item (register accumulators per warp)
+static_assert(kMaxR <= 32, "the down items' LoRA terms take one lane each");
 
 // [s0, s1) = the part of [a, a + n) inside [lo, hi), relative to lo (empty: s0 = s1 = 0)
 __device__ __forceinline__ void sub_range(int a, int n, int lo, int hi, int &s0, int &s1) {
@@ -374,8 +400,8 @@ struct DecSmem {
     float yprev[D];                  //   the previous layer's y (fp32), in order + chained
     uint32_t stg[kDecMaxK * I];      //   routed a payloads as polled (a layer's first down item)
   };
-  alignas(16) uint16_t ap[(kDecMaxK + 1) * I];   // a of every slot, bf16 pairs (pair_index order)
-  alignas(16) uint16_t xp[D];        // x as bf16 pairs (pair_index order)
+  alignas(16) uint16_t ap[(kDecMaxK + 1) * I];   // a of every slot, bf16 pairs (pair_slot order)
+  alignas(16) uint16_t xp[D];        // x as bf16 pairs (pair_slot order)
   float asraw[I];                    // the shared expert's a (natural order, for t_d)
   float xg[D / 64];                  // sum of x over each group of 64
   float ag[(kDecMaxK + 1) * (I / 64)];     // sum of each slot's a over each group of 64
@@ -1016,14 +1042,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (i < D && !ab) {
           const uint16_t xb = d2bf_bits(hv[m] * (double)bf(gam[i]) * rinv);
           S.xn[i] = xb;
-          S.xp[pair_index(i)] = xb;
+          S.xp[pair_slot(i, D)] = xb;
         }
       }
       cbar();
       // the group sums that every gate/up row of the layer uses with its minima
       #pragma unroll 1
       for (int G = warp; G < D / 64 && !ab; G += kDecCW) {
-        const float v = warp_sum(bf(S.xp[pair_index(64 * G + lane)]) + bf(S.xp[pair_index(64 * G + 32 + lane)]));
+        const float v = warp_sum(bf(S.xp[pair_slot(64 * G + lane, D)]) + bf(S.xp[pair_slot(64 * G + 32 + lane, D)]));
         if (lane == 0) S.xg[G] = v;
       }
       cbar();
@@ -1127,10 +1153,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
           // shorter than a step) feed zeros and fold nothing
           const int G = 8 * st + g8;
           const bool gv = G < NG;
-          const int wi = 64 * st + 8 * g8 + 2 * t4;  // code / activation word of this lane
+          const int wi = 64 * st + 8 * g8 + 2 * t4;  // code word of this lane (natural order)
+          const int nw = min(64, D / 8 - 64 * st);   // activation words of this step
           const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
           const uint2 z2 = make_uint2(0u, 0u);
-          const uint4 va = gv ? xw[wi] : z4, vb = gv ? xw[wi + 1] : z4;
+          const uint4 va = gv ? xw[64 * st + lane] : z4, vb = gv ? xw[64 * st + nw / 2 + lane] : z4;
           const float V = gv ? S.xg[G] : 0.f;
           float d[4];
           pair_step(d, gv ? ld_code2(A.gc + 4 * wi) : z2, gv ? ld_code2(A.uc + 4 * wi) : z2, va, vb);
@@ -1146,16 +1173,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
             }
           }
         }
-        ag0 = warp_sum(own ? ag0 : 0.f);
-        au0 = warp_sum(own ? au0 : 0.f);
-        if (two) {
-          ag1 = warp_sum(own ? ag1 : 0.f);
-          au1 = warp_sum(own ? au1 : 0.f);
-        }
-        if (lane == 0) {
-          publish(u0, ag0, au0);
-          if (two) publish(u1, ag1, au1);
-        }
+        // the four row sums at once: lane 0 gets u0's gate and up sums, lane 16 u1's
+        const float v = warp_sum4(own ? ag0 : 0.f, own ? au0 : 0.f, own ? ag1 : 0.f, own ? au1 : 0.f, lane);
+        const float vu = __shfl_down_sync(0xffffffffu, v, 8);
+        if (lane == 0) publish(u0, v, vu);
+        if (lane == 16 && two) publish(u1, v, vu);
       }
       if (ct == 0) stamp(P, l, TR_GU_DONE);
     } else {
@@ -1182,7 +1204,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
 #pragma unroll 1
           for (int i = ct; i < k * I; i += kDecConsumers) {
             const int j = i / I, e = i - j * I;
-            S.ap[j * I + pair_index(e)] = (uint16_t)(S.stg[i] & 0xFFFFu);
+            S.ap[j * I + pair_slot(e, I)] = (uint16_t)(S.stg[i] & 0xFFFFu);
           }
           if (ct == 0) stamp(P, l, TR_A_POLL);
           const int sbd = dn_bd(k);
@@ -1212,7 +1234,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
             }
             const uint16_t a16 = f2bf(g / (1.0f + expf(-g)) * u);
             S.asraw[i] = bf(a16);
-            S.ap[k * I + pair_index(i)] = a16;
+            S.ap[k * I + pair_slot(i, I)] = a16;
           }
           if (ct == 0) {
             float lg[kMaxK], mx = -INFINITY, sum = 0.f;
@@ -1234,8 +1256,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         // the group sums that every down row of the layer uses with its minima
         #pragma unroll 1
         for (int G = warp; G < (k + 1) * NGI && !ab; G += kDecCW) {
-          const float v = warp_sum(bf(S.ap[(G / NGI) * I + pair_index((G % NGI) * 64 + lane)]) +
-                                   bf(S.ap[(G / NGI) * I + pair_index((G % NGI) * 64 + 32 + lane)]));
+          const float v = warp_sum(bf(S.ap[(G / NGI) * I + pair_slot((G % NGI) * 64 + lane, I)]) +
+                                   bf(S.ap[(G / NGI) * I + pair_slot((G % NGI) * 64 + 32 + lane, I)]));
           if (lane == 0) S.ag[G] = v;
         }
         if (!ab && lora) {
@@ -1287,7 +1309,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
               const int G = 8 * st + g8;
               const bool gv = G < NGI;
               const int wi = 64 * st + 8 * g8 + 2 * t4;
-              const uint4 va = gv ? aw[j * (I / 8) + wi] : z4, vb = gv ? aw[j * (I / 8) + wi + 1] : z4;
+              const int nw = min(64, I / 8 - 64 * st);
+              const uint4 va = gv ? aw[j * (I / 8) + 64 * st + lane] : z4;
+              const uint4 vb = gv ? aw[j * (I / 8) + 64 * st + nw / 2 + lane] : z4;
               const float V = gv ? S.ag[j * NGI + G] : 0.f;
               float d[4];
 #pragma unroll
@@ -1305,25 +1329,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
             for (int q4 = 0; q4 < 4; q4++) y4[q4] = j < k ? fmaf(gj, f4[q4], y4[q4]) : y4[q4] + f4[q4];
           }
           // the shared expert's LoRA down branch c * (Bd t_d) of each row, its r terms
-          // spread over the lanes, then one warp sum per row
+          // spread over the lanes; then the four row sums at once (lane 8 q4 gets row
+          // r0 + q4), stored by four lanes
           const uint16_t *bd = lora ? reinterpret_cast<const uint16_t *>(S.ring + S.seg_off[slot][dn_bd(k)]) : nullptr;
+          float v4[4];
 #pragma unroll
           for (int q4 = 0; q4 < 4; q4++) {
-            if (q4 >= 2 && !pair2) break;
-            float v = own ? y4[q4] : 0.f;
-            if (lora && rv[q4]) {
-              float lo = 0.f;
-              #pragma unroll 1
-              for (int jj = lane; jj < r; jj += 32) lo = fmaf(bf(bd[(r0 + q4) * r + jj]), S.td[jj], lo);
-              v = fmaf(P.c, lo, v);
-            }
-            v = warp_sum(v);
-            if (lane == 0 && rv[q4]) {
-              const int n = ia + r0 + q4;
-              st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(v));
-              P.y[(size_t)l * D + n] = f2bf(v);
-              if (P.yf) P.yf[(size_t)l * D + n] = v;
-            }
+            float v = own && rv[q4] ? y4[q4] : 0.f;
+            if (lora && rv[q4] && lane < r)    // r <= kMaxR <= 32: one term per lane
+              v = fmaf(P.c, bf(bd[(r0 + q4) * r + lane]) * S.td[lane], v);
+            v4[q4] = v;
+          }
+          const float v = warp_sum4(v4[0], v4[1], v4[2], v4[3], lane);
+          const int q4 = lane >> 3;
+          if ((lane & 7) == 0 && r0 + q4 < in) {
+            const int n = ia + r0 + q4;
+            st_tag(P.t_y + (size_t)l * D + n, tag, __float_as_uint(v));
+            P.y[(size_t)l * D + n] = f2bf(v);
+            if (P.yf) P.yf[(size_t)l * D + n] = v;
           }
         }
       }
