@@ -49,9 +49,9 @@ KERNEL_TRAFFIC = {
                       "bytes to the 40-layer launch"),
     "prefill_t4096_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh",
                            "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "42d0b551396104d8", 318.8e6,
-                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 422.9 MB, "
-                          "down 214.7 MB, mean of the two"),
+                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "0a3a65b0cbfbbc46", 318.4e6,
+                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 422.6 MB, "
+                          "down 214.2 MB, mean of the two"),
 }
 
 

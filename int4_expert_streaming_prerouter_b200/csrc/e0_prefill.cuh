@@ -299,6 +299,8 @@ constexpr int kTmAStages = 3;      // A operand stages in TMEM (64 columns: both
 constexpr int kTmMaxG = 32;        // K <= 2048
 constexpr int kTmMaxR = 16;        // LoRA rank of the extra block (4 r <= 64)
 constexpr int kTmXRow = 65;        // epilogue exchange row stride in floats (conflict-free scalar access)
+constexpr int kTmDRow = 132;       // down combine exchange: floats per column (128 rows + pad, 16-byte rows)
+static_assert(32 * kTmDRow <= 2 * 64 * kTmXRow, "down combine exchange fits the gate/up one");
 constexpr uint32_t kTmACol = 4 * kTmN, kTmCols = 512;
 static_assert(kTmACol + kTmAStages * 64 <= kTmCols, "TMEM budget");
 static_assert((kTmN * 128) % 1024 == 0 && kTmN % 16 == 0, "tile rows");
@@ -310,13 +312,14 @@ struct TmSmem {
   uint8_t bl[2][kTmN * 128];           // LoRA block B tiles: c t_g hi | lo | c t_u hi | lo
   uint16_t sc[2][kTmMaxG][128];        // fp16 scales [group][row], per unit slot
   uint16_t mn[2][kTmMaxG][128];        // fp16 mins
-  float xch[2][64 * kTmXRow];          // epilogue exchange: gate and up values of 64 columns
+  alignas(16) float xch[2][64 * kTmXRow];   // epilogue exchange: gate and up values of 64 columns,
+                                            // or (down) 32 columns x 128 rows, [column][row + pad]
   int tok[2][kTmN];                    // token of each column (-1: padding)
   int dst[2][kTmN];                    // a row (gate/up) or gate index (down) of each column
   float gw[2][kTmN];                   // combine weight of each column (down)
   uint64_t bfull[kTmBStages], bempty[kTmBStages], cfull[kTmCStages], cempty[kTmCStages];
   uint64_t afull[kTmAStages], aempty[kTmAStages];
-  uint64_t accfull[2], accempty[2], ufull[2], uempty[2], drain[2];
+  uint64_t accfull[2], accempty[2], ufull[2], uempty[2], sfull[2], drain[2];
   uint32_t tmem;
   volatile int abort;
 };
@@ -582,7 +585,8 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
     for (int s = 0; s < 2; s++) {
       tc_mbar_init(&S.accfull[s], 2);
       tc_mbar_init(&S.accempty[s], kTmEpiThreads / 32);
-      tc_mbar_init(&S.ufull[s], 32 + kTmEpiThreads);
+      tc_mbar_init(&S.ufull[s], 32);               // the unit warp's bookkeeping and B tiles
+      tc_mbar_init(&S.sfull[s], kTmEpiThreads);    // the rows' scales and mins
       tc_mbar_init(&S.uempty[s], kTmEpiThreads / 32);
       tc_mbar_init(&S.drain[s], 1);
     }
@@ -656,9 +660,9 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
     __syncwarp();
   } else if (warp == kTmMma0 || warp == kTmMma1) {
     // ---------------- the two MMA issuers -------------------------------------------------
-    // A-stage entries per unit: [min block] [LoRA block] group 0 .. G - 1.  Issuer 0 takes
-    // the extra blocks and the even groups, issuer 1 the odd groups, each both fp16 parts
-    // into its own accumulator.  Every stage has one owner, so an issuer waits on each of
+    // A-stage entries per unit: group 0 .. G - 1, [min block] [LoRA block].  Issuer 0 takes
+    // the even groups and the extra blocks (whose B tiles the unit warp fills while the
+    // groups run), issuer 1 the odd groups, each both fp16 parts into its own accumulator.  Every stage has one owner, so an issuer waits on each of
     // its barriers' phases in order: A stages 0, 1 belong to issuer 0 and stage 2 to issuer
     // 1; B stage rg % kTmBStages carries real group rg, owned by issuer rg % 2 (every unit
     // has an even number of K groups, kTmBStages is even).
@@ -672,14 +676,15 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
         const int ab = it & 1, slot = it & 1;
         const uint32_t td = tmem + (uint32_t)((2 * part + ab) * kTmN);
         const int nx = 1 + ((lora_blk && U.shared) ? 1 : 0);   // extra blocks of this unit
-        ok = (it < 2 || tm_wait(&S.accempty[ab], (uint32_t)(((it >> 1) - 1) & 1), budget, A.err, &S.abort)) &&
-             (part == 1 || tm_wait(&S.ufull[slot], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort));
+        ok = it < 2 || tm_wait(&S.accempty[ab], (uint32_t)(((it >> 1) - 1) & 1), budget, A.err, &S.abort);
         if (!ok) break;
         bool first = true;
-        for (int e = 0; e < nx + G; e++) {
-          const bool real = e >= nx;
-          const bool mine = real ? ((e - nx) & 1) == part : part == 0;
+        for (int e = 0; e < G + nx; e++) {
+          const bool real = e < G;
+          const bool mine = real ? (e & 1) == part : part == 0;
           const int bs = rg % kTmBStages;
+          if (e == G && part == 0 && !(ok = tm_wait(&S.ufull[slot], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort)))
+            break;
           if (mine) {
             const int as = part == 0 ? (kown & 1) : 2;
             const uint32_t ph = (uint32_t)((part == 0 ? (kown >> 1) : kown) & 1);
@@ -687,7 +692,7 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
                  (!real || tm_wait(&S.bfull[bs], (uint32_t)((rg / kTmBStages) & 1), budget, A.err, &S.abort));
             if (!ok) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t sb = tc_smem(real ? S.b[bs] : (e == 0 ? S.bm[slot] : S.bl[slot]));
+            const uint32_t sb = tc_smem(real ? S.b[bs] : (e == G ? S.bm[slot] : S.bl[slot]));
             const uint32_t ta = tmem + kTmACol + (uint32_t)(64 * as);
 #pragma unroll
             for (int kk = 0; kk < 4; kk++) {   // K = 16 per instruction: 8 TMEM columns of A, 32 bytes of B
@@ -761,7 +766,7 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
       if (u2 >= total) return;
       const TmUnit U2 = tm_unit(A, u2, mtiles);
       tm_fill_scales(A, U2, G, row, S.sc[it2 & 1], S.mn[it2 & 1]);
-      tc_mbar_arrive(&S.ufull[it2 & 1]);
+      tc_mbar_arrive(&S.sfull[it2 & 1]);
     };
     fill(0);
     fill(1);
@@ -818,24 +823,34 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
           }
         }
       } else {
-        float *yrow = A.yacc + 128 * U.mt + row;
-#pragma unroll
-        for (int ch = 0; ch < (kTmN + 31) / 32; ch++) {   // (columns past N are read, never used)
+        // the gate-weighted combine into y: per chunk of 32 columns the 128 x 32 values go
+        // through shared memory ([column][row], rows padded to kTmDRow), so that each thread
+        // adds four consecutive rows of one token with one vector reduction (a quarter of
+        // the L2 atomic operations of per-element reductions)
+        float *xb = &S.xch[0][0];
+        for (int ch = 0; ch < (kTmN + 31) / 32; ch++) {
           const int c0 = 32 * ch;
-          if (c0 < U.N) {
+          if (c0 >= U.N) break;                             // block-uniform
+          asm volatile("bar.sync 1, 128;" ::: "memory");   // the previous chunk has been read
+          {
             float v[32], w[32];
-            tc_ld32(t0 + c0, v);
+            tc_ld32(t0 + c0, v);                           // (columns past N are read, never used)
             tc_ld32(t1 + c0, w);
 #pragma unroll
-            for (int j = 0; j < 32; j++) {
-              const int c = c0 + j;
-              if (c >= U.ncol) continue;
-              const int tok = S.tok[slot][c];
-              if (tok < 0) continue;
-              asm volatile("red.global.add.f32 [%0], %1;" ::"l"(yrow + (size_t)tok * A.d),
-                           "f"(S.gw[slot][c] * (v[j] + w[j]))
-                           : "memory");
-            }
+            for (int j = 0; j < 32; j++) xb[j * kTmDRow + row] = v[j] + w[j];
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll 2
+          for (int i = et; i < 32 * 32; i += 128) {
+            const int j = i >> 5, r4 = 4 * (i & 31), c = c0 + j;
+            if (c >= U.ncol) continue;
+            const int tok = S.tok[slot][c];
+            if (tok < 0) continue;
+            const float g = S.gw[slot][c];
+            const float4 val = *reinterpret_cast<const float4 *>(xb + j * kTmDRow + r4);
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(A.yacc + (size_t)tok * A.d + 128 * U.mt + r4),
+                         "f"(g * val.x), "f"(g * val.y), "f"(g * val.z), "f"(g * val.w)
+                         : "memory");
           }
         }
       }
@@ -878,36 +893,9 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
     };
     for (int u = blockIdx.x, it = 0; u < total && ok; u += gridDim.x, it++) {
       const int slot = it & 1;
-      if (!(ok = tm_wait_warp(&S.ufull[slot], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort))) break;
+      if (!(ok = tm_wait_warp(&S.sfull[slot], (uint32_t)((it >> 1) & 1), budget, A.err, &S.abort))) break;
       const TmUnit U = tm_unit(A, u, mtiles);
       uint32_t p1[16], p2[16];
-      // min block: element k of the row = m_(k mod G) for k < 2 G, else 0 (this thread's
-      // elements 32 h .. 32 h + 31)
-#pragma unroll
-      for (int j = 0; j < 16; j++) {
-        const int k0 = 32 * h + 2 * j, k1 = k0 + 1;
-        const uint32_t v0 = k0 < 2 * G ? S.mn[slot][k0 < G ? k0 : k0 - G][row] : 0u;
-        const uint32_t v1 = k1 < 2 * G ? S.mn[slot][k1 < G ? k1 : k1 - G][row] : 0u;
-        p1[j] = v0 | (v1 << 16);
-      }
-      if (!(ok = put(p1, p2, false, 0))) break;
-      if (lora_blk && U.shared) {
-        // LoRA block: gate row i: B_g[i] at k < r and again at r <= k < 2 r; up row: B_u[i]
-        // at 2 r <= k < 3 r and again at 3 r <= k < 4 r
-        const int i = 64 * U.mt + (row & 63);
-        const bool up = row >= 64;
-        const uint16_t *Bm = (up ? A.Bu : A.Bg) + (size_t)i * A.r;
-        const int k0 = up ? 2 * A.r : 0;
-#pragma unroll
-        for (int j = 0; j < 16; j++) {
-          const int ka = 32 * h + 2 * j, kb = ka + 1;
-          const int qa = ka - k0, qb = kb - k0;   // index into the doubled B row
-          const uint32_t va = (qa >= 0 && qa < 2 * A.r) ? tm_bf2h(Bm[qa < A.r ? qa : qa - A.r]) : 0u;
-          const uint32_t vb = (qb >= 0 && qb < 2 * A.r) ? tm_bf2h(Bm[qb < A.r ? qb : qb - A.r]) : 0u;
-          p1[j] = va | (vb << 16);
-        }
-        if (!(ok = put(p1, p2, false, 0))) break;
-      }
       for (int g0 = 0; g0 < G && ok; g0 += 4, cc++) {
         const int cs = cc % kTmCStages, ng = min(4, G - g0);
         if (!(ok = tm_wait_warp(&S.cfull[cs], (uint32_t)((cc / kTmCStages) & 1), budget, A.err, &S.abort))) break;
@@ -938,6 +926,34 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
           }
           if (!(ok = put(p1, p2, true, (g0 + lg) & 1))) break;
         }
+      }
+      // the extra blocks last (issuer 0 takes them after its groups)
+      // min block: element k of the row = m_(k mod G) for k < 2 G, else 0 (this thread's
+      // elements 32 h .. 32 h + 31)
+#pragma unroll
+      for (int j = 0; j < 16; j++) {
+        const int k0 = 32 * h + 2 * j, k1 = k0 + 1;
+        const uint32_t v0 = k0 < 2 * G ? S.mn[slot][k0 < G ? k0 : k0 - G][row] : 0u;
+        const uint32_t v1 = k1 < 2 * G ? S.mn[slot][k1 < G ? k1 : k1 - G][row] : 0u;
+        p1[j] = v0 | (v1 << 16);
+      }
+      if (!ok || !(ok = put(p1, p2, false, 0))) break;
+      if (lora_blk && U.shared) {
+        // LoRA block: gate row i: B_g[i] at k < r and again at r <= k < 2 r; up row: B_u[i]
+        // at 2 r <= k < 3 r and again at 3 r <= k < 4 r
+        const int i = 64 * U.mt + (row & 63);
+        const bool up = row >= 64;
+        const uint16_t *Bm = (up ? A.Bu : A.Bg) + (size_t)i * A.r;
+        const int k0 = up ? 2 * A.r : 0;
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+          const int ka = 32 * h + 2 * j, kb = ka + 1;
+          const int qa = ka - k0, qb = kb - k0;   // index into the doubled B row
+          const uint32_t va = (qa >= 0 && qa < 2 * A.r) ? tm_bf2h(Bm[qa < A.r ? qa : qa - A.r]) : 0u;
+          const uint32_t vb = (qb >= 0 && qb < 2 * A.r) ? tm_bf2h(Bm[qb < A.r ? qb : qb - A.r]) : 0u;
+          p1[j] = va | (vb << 16);
+        }
+        if (!(ok = put(p1, p2, false, 0))) break;
       }
     }
   }
