@@ -44,14 +44,14 @@ METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak
 KERNEL_TRAFFIC = {
     "decode_b1_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh",
                        "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "5d29fd26c49bd4f6", 408.7e6,
+                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "2bcbd1df81abb2f2", 408.7e6,
                       "4-layer capture (40.87 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
                       "bytes to the 40-layer launch"),
     "prefill_t4096_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh",
                            "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "0a3a65b0cbfbbc46", 318.4e6,
-                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 422.6 MB, "
-                          "down 214.2 MB, mean of the two"),
+                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "64b04da2e4d9a4f4", 319.0e6,
+                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 423.4 MB, "
+                          "down 214.6 MB, mean of the two"),
 }
 
 

@@ -516,7 +516,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   const e0_layer &Y = C->layers[K.l];
   const size_t nx = (size_t)K.T * D.d_model;
   const long long xg = (long long)K.T * (D.d_model / 64);
-  k_perm_sums<<<(unsigned)((xg + 255) / 256), 256, 0, s>>>(C->xb, K.T, D.d_model, C->xp, C->xsum, 0);
+  k_perm_sums<<<(unsigned)((8 * xg + 255) / 256), 256, 0, s>>>(C->xb, K.T, D.d_model, C->xp, C->xsum, 0);
   CKL("k_perm_sums(x)");
   k_tc_tiles<<<1, 32, 0, s>>>(C->plan, K.T, C->tiles, C->ntiles, C->tile_cap);
   CKL("k_tc_tiles");
@@ -554,7 +554,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
     g0 = g1 = nullptr;
   }
   const long long ag = (long long)K.T * (D.top_k + 1) * (D.d_ff / 64);
-  k_perm_sums<<<(unsigned)((ag + 255) / 256), 256, 0, s>>>(C->ap, (long long)K.T * (D.top_k + 1), D.d_ff, nullptr,
+  k_perm_sums<<<(unsigned)((8 * ag + 255) / 256), 256, 0, s>>>(C->ap, (long long)K.T * (D.top_k + 1), D.d_ff, nullptr,
                                                           C->asum, 1);
   CKL("k_perm_sums(a)");
   if (Y.lora_Ad) {
@@ -580,7 +580,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
     C->gemm_ev.push_back({g0, g1});
   }
   k_tc_finish<<<K.T, 256, 0, s>>>(C->yacc, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
-                                                           D.d_model, D.lora_rank, D.lora_scale, K.y, K.yf);
+                                  D.d_model, D.lora_rank, D.lora_scale, K.y, K.yf);
   CKL("k_tc_finish");
   return E0_OK;
 }

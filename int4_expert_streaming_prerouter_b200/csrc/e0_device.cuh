@@ -46,7 +46,19 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
 // Round a double to the nearest bfloat16 (ties to even) directly, without passing
 // through binary32: a bfloat16 keeps 8 significant bits, so for |v| in [2^(e-1), 2^e)
 // the spacing is 2^(e-8) (2^-133 below the smallest normal).
+// Results in the normal range take the integer form of the same rounding on the double's
+// bits: add 2^44 - 1 plus the kept lowest bit (bit 45) and keep the top 16 bits of the
+// re-biased exponent and 7 mantissa bits (a mantissa carry moves into the exponent).
 __device__ __forceinline__ uint16_t d2bf(double v) {
+  unsigned long long b = (unsigned long long)__double_as_longlong(v);
+  const int eb = (int)((b >> 52) & 0x7FF) - 1023 + 127;   // binary32 biased exponent
+  if (eb >= 1 && eb <= 254) {
+    b += (1ull << 44) - 1 + ((b >> 45) & 1ull);
+    const int e2 = (int)((b >> 52) & 0x7FF) - 1023 + 127;
+    const uint32_t sgn = (uint32_t)(b >> 63) << 15;
+    if (e2 >= 255) return (uint16_t)(sgn | 0x7F80u);      // rounds past the largest: infinity
+    return (uint16_t)(sgn | ((uint32_t)e2 << 7) | (uint32_t)((b >> 45) & 0x7Full));
+  }
   if (v == 0.0) return (uint16_t)((unsigned long long)__double_as_longlong(v) >> 48);
   int e = ilogb(v) + 1;
   if (e < -125) e = -125;

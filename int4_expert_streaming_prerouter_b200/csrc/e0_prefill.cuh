@@ -1125,24 +1125,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_rows(TcRowsArgs A) {
 
 // ---------------------------------------------------------------------------------------
 // Operand preparation: the K-permuted bf16 copy of x (or nullptr) and the fp32 sum of
-// every group of 64 (natural order).  One thread per (row, group).
+// every group of 64 (natural order).  Eight threads per (row, group), one 16-byte word
+// each (a warp reads four whole groups), the group sum reduced over the eight.
 // ---------------------------------------------------------------------------------------
 __global__ void k_perm_sums(const uint16_t *__restrict__ x, long long rows, int K, uint16_t *__restrict__ xp,
                             float *__restrict__ sums, int in_f16) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int G = K / 64;
-  if (i >= rows * G) return;
-  const long long r = i / G;
-  const int g = (int)(i % G);
-  const uint4 *src = reinterpret_cast<const uint4 *>(x + r * K + g * 64);
-  uint4 *dst = xp ? reinterpret_cast<uint4 *>(xp + r * K + g * 64) : nullptr;
+  const long long rg = i >> 3;            // (row, group)
+  const int q = (int)(i & 7);             // this thread's word of the group
+  const bool live = rg < rows * G;        // whole octets are live or not (blockDim % 8 == 0)
+  const long long r = live ? rg / G : 0;
+  const int g = live ? (int)(rg % G) : 0;
   // 16-bit element -> fp32 (bf16 or fp16 input), and a bf16 element as the same fp16 value
   auto val = [&](uint32_t b) { return in_f16 ? __half2float(__ushort_as_half((uint16_t)b)) : bf(b); };
   auto h16 = [&](uint32_t b) { return (uint32_t)__half_as_ushort(__float2half_rn(bf(b))); };
   float s = 0.f;
-#pragma unroll
-  for (int q = 0; q < 8; q++) {
-    const uint4 v = src[q];
+  if (live) {
+    const uint4 v = reinterpret_cast<const uint4 *>(x + r * K + g * 64)[q];
     // natural elements 8q .. 8q+7 = (v.x lo, v.x hi, v.y lo, v.y hi, v.z lo, ...)
     s += val(v.x & 0xFFFFu);
     s += val(v.x >> 16);
@@ -1152,13 +1152,16 @@ __global__ void k_perm_sums(const uint16_t *__restrict__ x, long long rows, int 
     s += val(v.z >> 16);
     s += val(v.w & 0xFFFFu);
     s += val(v.w >> 16);
-    if (dst) {   // bf16 input -> the fp16 tensor-core operand, permuted block (0,4,1,5,2,6,3,7)
+    if (xp) {   // bf16 input -> the fp16 tensor-core operand, permuted block (0,4,1,5,2,6,3,7)
       const uint32_t e0 = h16(v.x & 0xFFFFu), e1 = h16(v.x >> 16), e2 = h16(v.y & 0xFFFFu), e3 = h16(v.y >> 16);
       const uint32_t e4 = h16(v.z & 0xFFFFu), e5 = h16(v.z >> 16), e6 = h16(v.w & 0xFFFFu), e7 = h16(v.w >> 16);
-      dst[q] = make_uint4(e0 | (e4 << 16), e1 | (e5 << 16), e2 | (e6 << 16), e3 | (e7 << 16));
+      reinterpret_cast<uint4 *>(xp + r * K + g * 64)[q] =
+          make_uint4(e0 | (e4 << 16), e1 | (e5 << 16), e2 | (e6 << 16), e3 | (e7 << 16));
     }
   }
-  sums[i] = s;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (live && q == 0) sums[rg] = s;
 }
 
 // x rows in expert-grouped order: row p of xg = the permuted x row of the token of
