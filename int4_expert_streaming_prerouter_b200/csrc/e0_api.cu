@@ -1311,7 +1311,7 @@ static int phased_launch(e0_ctx *C, const PhParams &P, cudaStream_t s) {
   PHL(ph_launch(k_ph_norm<D>, L * B, 256, 0, s, false, P), "k_ph_norm");
   PHL(ph_launch(k_ph_rows<D>, P.nblocks, 32 * PhRowsCfg<D>::NW, 0, s, pdl, P), "k_ph_rows");
   PHL(ph_launch(k_ph_route, L, 256, 0, s, pdl, P), "k_ph_route");
-  PHL(ph_launch(k_ph_gateup<D, I>, L * Umax * (I / 8), 32 * (D / 256), 0, s, pdl, P), "k_ph_gateup");
+  PHL(ph_launch(k_ph_gateup<D, I>, L * Umax * (I / 8 / kPhGuBlocks), 32 * (D / 256), 0, s, pdl, P), "k_ph_gateup");
   PHL(ph_launch(k_ph_tdsum<I>, L * B, 256, 0, s, pdl, P), "k_ph_tdsum");
   PHL(ph_launch(k_ph_down<D, I>, L * (D / 16), 32 * (I / 64), ph_dn_smem<D, I>(B, P.k), s, pdl, P), "k_ph_down");
 #undef PHL

@@ -454,27 +454,29 @@ __global__ void __launch_bounds__(256) k_ph_route(PhParams P) {
 
 // ---------------------------------------------------------------------------------------
 // KC: gate/up + SwiGLU.  One CTA per (layer, expert of the layer's plan or the shared
-// expert, 8 intermediate indices i0..i0+7); several CTAs are resident per SM and each
-// warp issues all of its weight loads at once.  MMA row g is the gate row i0 + g, row
-// g + 8 the up row i0 + g; warp w takes groups 4w .. 4w + 3 of K.  Lane (g, t) holds bytes
-// 8 t .. 8 t + 7 of each of its rows' groups (16 codes: nibbles j and j + 4 of a word form
-// the bf16 pair {128 + q_j, 128 + q_(j+4)}) and the same 16 activations of token g in pair
-// order.  The warps' partial sums are added in order.  The shared expert's g and u go out
-// before its LoRA and activation, which the next kernel applies.
+// expert, kPhGuBlocks blocks of 8 intermediate indices): while a block's products are
+// formed, the next block's weights are already in flight.  MMA row g is the gate row
+// i0 + g, row g + 8 the up row i0 + g; warp w takes groups 4w .. 4w + 3 of K.  Lane (g, t)
+// holds bytes 8 t .. 8 t + 7 of each of its rows' groups (16 codes: nibbles j and j + 4 of a
+// word form the bf16 pair {128 + q_j, 128 + q_(j+4)}) and the same 16 activations of token
+// g in pair order.  The warps' partial sums are added in order.  The shared expert's g and
+// u go out before its LoRA and activation, which the next kernel applies.
 // ---------------------------------------------------------------------------------------
+constexpr int kPhGuBlocks = 4;   // blocks of 8 intermediate indices per gate/up CTA
 template <int D, int I>
 __global__ void __launch_bounds__(32 * (D / 256)) k_ph_gateup(PhParams P) {
-  constexpr int NG = D / 64, NW = NG / 4, O = I / 8;
+  constexpr int NG = D / 64, NW = NG / 4, O = I / 8, OC = O / kPhGuBlocks;
   static_assert(NG % 4 == 0, "D must be a multiple of 256");
+  static_assert(O % kPhGuBlocks == 0, "I / 8 must be a multiple of the blocks per CTA");
   ph_launch_next();
   const int Umax = min(P.B * P.k, P.E) + 1;
-  const int o = blockIdx.x % O, u = (blockIdx.x / O) % Umax, l = blockIdx.x / (O * Umax);
+  const int oc = blockIdx.x % OC, u = (blockIdx.x / OC) % Umax, l = blockIdx.x / (OC * Umax);
   const PhLayer &Y = P.layers[l];
   const bool pred = ph_predicted(P, l);
   const int k = P.k, E = P.E;
   __shared__ int s_e;
   __shared__ int s_slot[kPhMaxB];
-  __shared__ float part[NW][32][4];
+  __shared__ float part[2][NW][32][4];
   if (!pred) ph_wait_prev();
   if (threadIdx.x < kPhMaxB) {
     // this CTA's expert and, per token, the slot it was routed to the expert in
@@ -490,74 +492,91 @@ __global__ void __launch_bounds__(32 * (D / 256)) k_ph_gateup(PhParams P) {
   const Blob bl = blob_of(D, I);
   const uint8_t *base = e == E ? Y.shared : Y.experts + (size_t)ph_clamp_e(e, E) * bl.bytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int i = o * 8 + g, G0 = warp * 4;
-  uint2 cg[4], cu[4];
+  const int G0 = warp * 4;
+  // one block's weights of this lane: codes of its gate and up rows, their scales and minima
+  struct W {
+    uint2 cg[4], cu[4], sg, mg, su, mu;
+  };
+  auto load = [&](int o, W &w) {
+    const int i = o * 8 + g;
 #pragma unroll
-  for (int q = 0; q < 4; q++) {
-    cg[q] = ldg_nc64(base + bl.gc + (size_t)i * (D / 2) + 32 * (G0 + q) + 8 * t);
-    cu[q] = ldg_nc64(base + bl.uc + (size_t)i * (D / 2) + 32 * (G0 + q) + 8 * t);
-  }
-  const uint2 sg = ldg_nc64(base + bl.gs + ((size_t)i * NG + G0) * 2);
-  const uint2 mg = ldg_nc64(base + bl.gm + ((size_t)i * NG + G0) * 2);
-  const uint2 su = ldg_nc64(base + bl.us + ((size_t)i * NG + G0) * 2);
-  const uint2 mu = ldg_nc64(base + bl.um + ((size_t)i * NG + G0) * 2);
+    for (int q = 0; q < 4; q++) {
+      w.cg[q] = ldg_nc64(base + bl.gc + (size_t)i * (D / 2) + 32 * (G0 + q) + 8 * t);
+      w.cu[q] = ldg_nc64(base + bl.uc + (size_t)i * (D / 2) + 32 * (G0 + q) + 8 * t);
+    }
+    w.sg = ldg_nc64(base + bl.gs + ((size_t)i * NG + G0) * 2);
+    w.mg = ldg_nc64(base + bl.gm + ((size_t)i * NG + G0) * 2);
+    w.su = ldg_nc64(base + bl.us + ((size_t)i * NG + G0) * 2);
+    w.mu = ldg_nc64(base + bl.um + ((size_t)i * NG + G0) * 2);
+  };
+  W cur, nxt;
+  load(oc * kPhGuBlocks, cur);
   if (pred) ph_wait_prev();
   const size_t tg = (size_t)l * kPhMaxB;
   const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-  float ag0 = 0.f, ag1 = 0.f, au0 = 0.f, au1 = 0.f;
 #pragma unroll
-  for (int q = 0; q < 4; q++) {
-    const int G = G0 + q;
-    uint4 xa = z4, xb = z4;
-    if (g < P.B) {
-      const uint16_t *xr = P.xp + (tg + g) * D + 64 * G + 16 * t;
-      xa = *reinterpret_cast<const uint4 *>(xr);
-      xb = *reinterpret_cast<const uint4 *>(xr + 8);
-    }
-    const float X0 = 2 * t < P.B ? P.xs[(tg + 2 * t) * NG + G] : 0.f;
-    const float X1 = 2 * t + 1 < P.B ? P.xs[(tg + 2 * t + 1) * NG + G] : 0.f;
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    mma_bf16_16816(d, nib_pair_bf16(cg[q].x, 0), nib_pair_bf16(cu[q].x, 0), nib_pair_bf16(cg[q].x, 1),
-                   nib_pair_bf16(cu[q].x, 1), xa.x, xa.y);
-    mma_bf16_16816(d, nib_pair_bf16(cg[q].x, 2), nib_pair_bf16(cu[q].x, 2), nib_pair_bf16(cg[q].x, 3),
-                   nib_pair_bf16(cu[q].x, 3), xa.z, xa.w);
-    mma_bf16_16816(d, nib_pair_bf16(cg[q].y, 0), nib_pair_bf16(cu[q].y, 0), nib_pair_bf16(cg[q].y, 1),
-                   nib_pair_bf16(cu[q].y, 1), xb.x, xb.y);
-    mma_bf16_16816(d, nib_pair_bf16(cg[q].y, 2), nib_pair_bf16(cu[q].y, 2), nib_pair_bf16(cg[q].y, 3),
-                   nib_pair_bf16(cu[q].y, 3), xb.z, xb.w);
-    const uint32_t wsg = q < 2 ? sg.x : sg.y, wmg = q < 2 ? mg.x : mg.y;
-    const uint32_t wsu = q < 2 ? su.x : su.y, wmu = q < 2 ? mu.x : mu.y;
-    const float s_g = (q & 1) ? bf_hi(wsg) : bf_lo(wsg), m_g = (q & 1) ? bf_hi(wmg) : bf_lo(wmg);
-    const float s_u = (q & 1) ? bf_hi(wsu) : bf_lo(wsu), m_u = (q & 1) ? bf_hi(wmu) : bf_lo(wmu);
-    const float mp_g = fmaf(-128.f, s_g, m_g), mp_u = fmaf(-128.f, s_u, m_u);
-    ag0 = ph_fold(ag0, s_g, mp_g, d[0], X0);
-    ag1 = ph_fold(ag1, s_g, mp_g, d[1], X1);
-    au0 = ph_fold(au0, s_u, mp_u, d[2], X0);
-    au1 = ph_fold(au1, s_u, mp_u, d[3], X1);
-  }
-  part[warp][lane][0] = ag0;
-  part[warp][lane][1] = ag1;
-  part[warp][lane][2] = au0;
-  part[warp][lane][3] = au1;
-  __syncthreads();
-  for (int tid = threadIdx.x; tid < 8 * P.B; tid += blockDim.x) {
-    const int ii = tid % 8, n = tid / 8;
-    const int src = 4 * ii + n / 2, hh = n & 1;
-    float gs = 0.f, us = 0.f;
+  for (int ob = 0; ob < kPhGuBlocks; ob++) {
+    const int o = oc * kPhGuBlocks + ob;
+    if (ob + 1 < kPhGuBlocks) load(o + 1, nxt);
+    float ag0 = 0.f, ag1 = 0.f, au0 = 0.f, au1 = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; w++) {
-      gs += part[w][src][hh];
-      us += part[w][src][2 + hh];
+    for (int q = 0; q < 4; q++) {
+      const int G = G0 + q;
+      uint4 xa = z4, xb = z4;
+      if (g < P.B) {
+        const uint16_t *xr = P.xp + (tg + g) * D + 64 * G + 16 * t;
+        xa = *reinterpret_cast<const uint4 *>(xr);
+        xb = *reinterpret_cast<const uint4 *>(xr + 8);
+      }
+      const float X0 = 2 * t < P.B ? P.xs[(tg + 2 * t) * NG + G] : 0.f;
+      const float X1 = 2 * t + 1 < P.B ? P.xs[(tg + 2 * t + 1) * NG + G] : 0.f;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_bf16_16816(d, nib_pair_bf16(cur.cg[q].x, 0), nib_pair_bf16(cur.cu[q].x, 0), nib_pair_bf16(cur.cg[q].x, 1),
+                     nib_pair_bf16(cur.cu[q].x, 1), xa.x, xa.y);
+      mma_bf16_16816(d, nib_pair_bf16(cur.cg[q].x, 2), nib_pair_bf16(cur.cu[q].x, 2), nib_pair_bf16(cur.cg[q].x, 3),
+                     nib_pair_bf16(cur.cu[q].x, 3), xa.z, xa.w);
+      mma_bf16_16816(d, nib_pair_bf16(cur.cg[q].y, 0), nib_pair_bf16(cur.cu[q].y, 0), nib_pair_bf16(cur.cg[q].y, 1),
+                     nib_pair_bf16(cur.cu[q].y, 1), xb.x, xb.y);
+      mma_bf16_16816(d, nib_pair_bf16(cur.cg[q].y, 2), nib_pair_bf16(cur.cu[q].y, 2), nib_pair_bf16(cur.cg[q].y, 3),
+                     nib_pair_bf16(cur.cu[q].y, 3), xb.z, xb.w);
+      const uint32_t wsg = q < 2 ? cur.sg.x : cur.sg.y, wmg = q < 2 ? cur.mg.x : cur.mg.y;
+      const uint32_t wsu = q < 2 ? cur.su.x : cur.su.y, wmu = q < 2 ? cur.mu.x : cur.mu.y;
+      const float s_g = (q & 1) ? bf_hi(wsg) : bf_lo(wsg), m_g = (q & 1) ? bf_hi(wmg) : bf_lo(wmg);
+      const float s_u = (q & 1) ? bf_hi(wsu) : bf_lo(wsu), m_u = (q & 1) ? bf_hi(wmu) : bf_lo(wmu);
+      const float mp_g = fmaf(-128.f, s_g, m_g), mp_u = fmaf(-128.f, s_u, m_u);
+      ag0 = ph_fold(ag0, s_g, mp_g, d[0], X0);
+      ag1 = ph_fold(ag1, s_g, mp_g, d[1], X1);
+      au0 = ph_fold(au0, s_u, mp_u, d[2], X0);
+      au1 = ph_fold(au1, s_u, mp_u, d[3], X1);
     }
-    const int iidx = o * 8 + ii;
-    const size_t tn = tg + n;
-    if (e == E) {
-      P.gus[tn * 2 * I + iidx] = gs;
-      P.gus[tn * 2 * I + I + iidx] = us;
-    } else {
-      const int sl = s_slot[n];
-      if (sl >= 0) P.a[(tn * (k + 1) + sl) * I + pair_index(iidx)] = f2bf(gs / (1.0f + expf(-gs)) * us);
+    // partial sums double-buffered: the reduction of block ob - 1 (same buffer two blocks
+    // back) finished before this block's barrier
+    float (*pt)[32][4] = part[ob & 1];
+    pt[warp][lane][0] = ag0;
+    pt[warp][lane][1] = ag1;
+    pt[warp][lane][2] = au0;
+    pt[warp][lane][3] = au1;
+    __syncthreads();
+    for (int tid = threadIdx.x; tid < 8 * P.B; tid += blockDim.x) {
+      const int ii = tid % 8, n = tid / 8;
+      const int src = 4 * ii + n / 2, hh = n & 1;
+      float gs = 0.f, us = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; w++) {
+        gs += pt[w][src][hh];
+        us += pt[w][src][2 + hh];
+      }
+      const int iidx = o * 8 + ii;
+      const size_t tn = tg + n;
+      if (e == E) {
+        P.gus[tn * 2 * I + iidx] = gs;
+        P.gus[tn * 2 * I + I + iidx] = us;
+      } else {
+        const int sl = s_slot[n];
+        if (sl >= 0) P.a[(tn * (k + 1) + sl) * I + pair_index(iidx)] = f2bf(gs / (1.0f + expf(-gs)) * us);
+      }
     }
+    if (ob + 1 < kPhGuBlocks) cur = nxt;
   }
 }
 
