@@ -221,6 +221,16 @@ int e0_stream_mode(e0_ctx *ctx, int reactive);
 int e0_moe_prefill_stack(e0_ctx *ctx, const void *h_in, int T, void *y_out, float *y_f32, int32_t *idx_out,
                          void *stream);
 
+/* Combine order of the tensor-core prefill path (e0_moe_layer_forward and the prefill
+ * stacks from 64 tokens).  0 (default): the down GEMM adds each expert's gate-weighted
+ * rows into the fp32 output with vector reductions in completion order, so the last bits
+ * of y can differ between runs.  1: each (expert slot, token) contribution is stored once
+ * in its own plane ([k + 1, max_tokens, d] fp32 of device memory, allocated on the first
+ * call with on = 1 and kept until e0_destroy) and the planes are summed in slot order
+ * (routed slots 0..k-1, then the shared expert), so y is bit-reproducible; it reads and
+ * writes (k + 1) * T * d * 4 more bytes per layer.  Errors: INVALID_ARG, OOM. */
+int e0_prefill_fixed_order(e0_ctx *ctx, int on);
+
 /* e0_moe_prefill_stack with the input and outputs in host memory (pinned, so that the
  * copies are asynchronous): h_host [L, T, d] bf16, y_host [L, T, d] bf16, y_f32_host
  * [L, T, d] or NULL; idx_out [L, T, k] int32 device memory or NULL.  Layer l's input is

@@ -88,6 +88,7 @@ _SIGS = {
     "e0_debug_force_general": (_I, [_P, _I]),
     "e0_debug_decode_trace": (_I, [_P, _P]),
     "e0_debug_prefill_path": (_I, [_P, _I]),
+    "e0_prefill_fixed_order": (_I, [_P, _I]),
     "e0_debug_decode_mode": (_I, [_P, _I]),
     "e0_debug_decode_flat": (_I, [_P, _I]),
     "e0_debug_time_gemm": (_I, [_P, _I]),
@@ -357,6 +358,11 @@ class Context:
 
     def debug_prefill_path(self, mode: int):
         _check(lib().e0_debug_prefill_path(self._h, mode))
+
+    def prefill_fixed_order(self, on: bool):
+        """Tensor-core prefill combine in slot order (bit-reproducible y) instead of
+        completion-order reductions."""
+        _check(lib().e0_prefill_fixed_order(self._h, int(on)))
 
     def debug_force_general(self, on: bool):
         _check(lib().e0_debug_force_general(self._h, int(on)))

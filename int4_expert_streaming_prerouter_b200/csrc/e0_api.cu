@@ -178,6 +178,8 @@ struct e0_ctx {
   uint16_t *xp = nullptr, *ap = nullptr, *xg = nullptr;
   float *xsum = nullptr, *asum = nullptr;
   float *yacc = nullptr;
+  float *ypart = nullptr;            // fixed-order prefill combine: [k + 1][maxT][d] (on request)
+  bool pf_det = false;
   TcTile *tiles = nullptr;
   int *ntiles = nullptr;
   int tile_cap = 0;
@@ -238,7 +240,7 @@ extern "C" int e0_destroy(e0_ctx *C) {
   }
   void *bufs[] = {C->xb, C->xf, C->logits, C->hlog, C->lt, C->gates, C->idx, C->a, C->plan_mem,
                   C->yscratch, C->pred_tab, C->hist_tab, C->err, C->h1pre, C->h1, C->pool.mem, C->pool.slot_of,
-                  C->pool.slot_tag, C->xp, C->ap, C->xg, C->xsum, C->asum, C->yacc, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
+                  C->pool.slot_tag, C->xp, C->ap, C->xg, C->xsum, C->asum, C->yacc, C->ypart, C->tiles, C->ntiles, C->pf_buf, C->pf_idx};
   for (void *b : bufs)
     if (b) cudaFree(b);
   decode_free(C->dec);
@@ -562,7 +564,8 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
                                                            D.top_k, D.lora_rank, C->lt);
     CKL("k_lora_td");
   }
-  CK(cudaMemsetAsync(C->yacc, 0, nx * sizeof(float), s));
+  if (!C->pf_det) CK(cudaMemsetAsync(C->yacc, 0, nx * sizeof(float), s));
+  A.ypart = C->pf_det ? C->ypart : nullptr;   // every (slot, token, row) is written once
   A.mode = 1;
   if ((rc = tmap_bf16_rows(&A.tmB[0], C->ap, D.d_ff, (long long)K.T * (D.top_k + 1), true)) ||
       (rc = tmap_codes(&A.tmC[0], ex + C->bl.dc, D.d_ff / 2, D.d_model, D.n_experts, bb, 128)) ||
@@ -579,7 +582,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
     cudaEventRecord(g1, s);
     C->gemm_ev.push_back({g0, g1});
   }
-  k_tc_finish<<<K.T, 256, 0, s>>>(C->yacc, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
+  k_tc_finish<<<K.T, 256, 0, s>>>(C->yacc, A.ypart, D.top_k + 1, (const uint16_t *)Y.lora_Bd, C->lt, K.T,
                                   D.d_model, D.lora_rank, D.lora_scale, K.y, K.yf);
   CKL("k_tc_finish");
   return E0_OK;
@@ -1725,6 +1728,17 @@ extern "C" int e0_debug_decode_trace(e0_ctx *C, unsigned long long *buf) {
 
 // Select the expert path of e0_moe_layer_forward: 0 = tensor cores from kTcMinTokens
 // tokens (default), 1 = CUDA-core kernels, 2 = tensor cores whenever the context has them.
+extern "C" int e0_prefill_fixed_order(e0_ctx *C, int on) {
+  if (!C) return fail(E0_ERR_INVALID_ARG, "NULL context");
+  if (on && !C->ypart) {
+    const size_t n = (size_t)(C->dims.top_k + 1) * C->maxT * C->dims.d_model;
+    int rc = dalloc(&C->ypart, n);
+    if (rc) return rc;
+  }
+  C->pf_det = on != 0;
+  return E0_OK;
+}
+
 extern "C" int e0_debug_prefill_path(e0_ctx *C, int mode) {
   if (!C || mode < 0 || mode > 2) return fail(E0_ERR_INVALID_ARG, "bad prefill path");
   C->prefill_path = mode;

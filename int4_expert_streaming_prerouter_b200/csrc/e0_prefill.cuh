@@ -59,6 +59,7 @@ struct TcArgs {
   const float *lt;          // [T, 3, r]
   const float *gates;       // [T, k] (mode 1)
   float *yacc;              // [T, d] (mode 1)
+  float *ypart;             // [k + 1][T, d] (mode 1, fixed-order combine) or nullptr
   int *err;
   unsigned long long timeout_ns;
 };
@@ -848,9 +849,17 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
             if (tok < 0) continue;
             const float g = S.gw[slot][c];
             const float4 val = *reinterpret_cast<const float4 *>(xb + j * kTmDRow + r4);
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(A.yacc + (size_t)tok * A.d + 128 * U.mt + r4),
-                         "f"(g * val.x), "f"(g * val.y), "f"(g * val.z), "f"(g * val.w)
-                         : "memory");
+            if (A.ypart) {
+              // fixed-order combine: this (slot, token) contribution stored once, in its own
+              // plane (routed slot = assignment mod k, the shared expert's plane k)
+              const int dst = S.dst[slot][c], sp = dst >= 0 ? dst % A.k : A.k;
+              *reinterpret_cast<float4 *>(A.ypart + ((size_t)sp * A.T + tok) * A.d + 128 * U.mt + r4) =
+                  make_float4(g * val.x, g * val.y, g * val.z, g * val.w);
+            } else {
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(A.yacc + (size_t)tok * A.d + 128 * U.mt + r4),
+                           "f"(g * val.x), "f"(g * val.y), "f"(g * val.z), "f"(g * val.w)
+                           : "memory");
+            }
           }
         }
       }
@@ -1208,18 +1217,26 @@ __global__ void k_lora_td(const uint16_t *__restrict__ Ad, const uint16_t *__res
   if (lane == 0) lt[((size_t)t * 3 + 2) * r + j] = acc;
 }
 
-// y = yacc + c Bd t_d  -> fp32 and bf16 outputs.  One block per token: t_d in shared
-// memory, each thread a strided set of output rows n with its B_d row in 16-byte loads.
-__global__ void k_tc_finish(const float *__restrict__ yacc, const uint16_t *__restrict__ Bd,
-                            const float *__restrict__ lt, int T, int d, int r, float c, uint16_t *__restrict__ y,
-                            float *__restrict__ yf) {
+// y = yacc + c Bd t_d  -> fp32 and bf16 outputs; with ypart (the fixed-order combine), the
+// accumulated value is instead the sum of the token's nslot planes in plane order.  One
+// block per token: t_d in shared memory, each thread a strided set of output rows n with
+// its B_d row in 16-byte loads.
+__global__ void k_tc_finish(const float *__restrict__ yacc, const float *__restrict__ ypart, int nslot,
+                            const uint16_t *__restrict__ Bd, const float *__restrict__ lt, int T, int d, int r,
+                            float c, uint16_t *__restrict__ y, float *__restrict__ yf) {
   const int t = blockIdx.x;
   __shared__ float td[kMaxR];
   if (Bd && threadIdx.x < r) td[threadIdx.x] = lt[((size_t)t * 3 + 2) * r + threadIdx.x];
   __syncthreads();
   for (int n = threadIdx.x; n < d; n += blockDim.x) {
     const size_t i = (size_t)t * d + n;
-    float v = yacc[i];
+    float v;
+    if (ypart) {
+      v = 0.f;
+      for (int j = 0; j < nslot; j++) v += ypart[((size_t)j * T + t) * d + n];
+    } else {
+      v = yacc[i];
+    }
     if (Bd) {
       float lo = 0.f;
       if (r % 8 == 0 && ((uintptr_t)Bd & 15) == 0) {
