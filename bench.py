@@ -44,13 +44,13 @@ METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak
 KERNEL_TRAFFIC = {
     "decode_b1_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh",
                        "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "2bcbd1df81abb2f2", 408.7e6,
-                      "4-layer capture (40.87 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
+                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "994f0bc761d25bc1", 408.5e6,
+                      "4-layer capture (40.85 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
                       "bytes to the 40-layer launch"),
     "prefill_t4096_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh",
                            "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "9e40ce84ee4cb9bd", 318.7e6,
-                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 422.6 MB, "
+                           "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "83ec15cef93f05d6", 319.5e6,
+                          "k_moe_gemm_tc DRAM bytes per launch on one full-width layer (T=4096): gate/up 424.3 MB, "
                           "down 214.8 MB, mean of the two"),
 }
 

@@ -291,7 +291,7 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
   if ((rc = dalloc(&C->xb, T * d)) || (rc = dalloc(&C->xf, T * d)) || (rc = dalloc(&C->logits, T * E)) ||
       (rc = dalloc(&C->hlog, T * E)) || (rc = dalloc(&C->lt, T * 3 * r)) || (rc = dalloc(&C->gates, T * k)) ||
       (rc = dalloc(&C->idx, T * k)) || (rc = dalloc(&C->a, T * (k + 1) * I)) ||
-      (rc = dalloc(&C->plan_mem, 1 + E + E + 1 + T * k)) || (rc = dalloc(&C->yscratch, 2 * T * d)) ||
+      (rc = dalloc(&C->plan_mem, 1 + E + E + 1 + 2 * T * k)) || (rc = dalloc(&C->yscratch, 2 * T * d)) ||
       (rc = dalloc(&C->pred_tab, 2 * (n_layers + 1) * T * k)) ||
       (rc = dalloc(&C->hist_tab, 2 * n_layers * T * k)) || (rc = dalloc(&C->err, 4)) ||
       (dims->head_hidden > 0 && ((rc = dalloc(&C->h1pre, T * dims->head_hidden)) ||
@@ -330,6 +330,7 @@ extern "C" int e0_create(const e0_dims *dims, int n_layers, int max_tokens, e0_c
   C->plan.uexp = C->plan_mem + 1;
   C->plan.ustart = C->plan_mem + 1 + E;
   C->plan.assign = C->plan_mem + 2 + 2 * E;
+  C->plan.pos = C->plan.assign + T * k;
   cudaMemset(C->pred_tab, 0xFF, 2 * (n_layers + 1) * T * k * sizeof(int32_t));
   cudaMemset(C->hist_tab, 0xFF, 2 * n_layers * T * k * sizeof(int32_t));
   cudaMemset(C->err, 0, 16);
@@ -518,13 +519,13 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   const e0_layer &Y = C->layers[K.l];
   const size_t nx = (size_t)K.T * D.d_model;
   const long long xg = (long long)K.T * (D.d_model / 64);
-  k_perm_sums<<<(unsigned)((8 * xg + 255) / 256), 256, 0, s>>>(C->xb, K.T, D.d_model, C->xp, C->xsum, 0);
+  // the permuted x rows, their group sums, and the routed tokens' rows in expert-grouped
+  // order (each tile's tokens consecutive)
+  k_perm_sums<<<(unsigned)((8 * xg + 255) / 256), 256, 0, s>>>(C->xb, K.T, D.d_model, C->xp, C->xsum, 0,
+                                                          C->plan.pos, D.top_k, C->xg);
   CKL("k_perm_sums(x)");
   k_tc_tiles<<<1, 32, 0, s>>>(C->plan, K.T, C->tiles, C->ntiles, C->tile_cap);
   CKL("k_tc_tiles");
-  // the routed tokens' x rows in expert-grouped order (each tile's tokens consecutive)
-  k_group_rows<<<K.T * D.top_k, std::min(256, D.d_model / 8), 0, s>>>(C->xp, C->plan.assign, D.top_k, D.d_model, C->xg);
-  CKL("k_group_rows");
   TcArgs A{};
   int rc;
   if ((rc = tmap_bf16_rows(&A.tmB[0], C->xg, D.d_model, (long long)K.T * D.top_k, true)) ||
@@ -557,7 +558,7 @@ static int layer_post_tc(e0_ctx *C, const LayerCall &K, const ExpertSrc &src, cu
   }
   const long long ag = (long long)K.T * (D.top_k + 1) * (D.d_ff / 64);
   k_perm_sums<<<(unsigned)((8 * ag + 255) / 256), 256, 0, s>>>(C->ap, (long long)K.T * (D.top_k + 1), D.d_ff, nullptr,
-                                                          C->asum, 1);
+                                                          C->asum, 1, nullptr, 0, nullptr);
   CKL("k_perm_sums(a)");
   if (Y.lora_Ad) {
     k_lora_td<<<(K.T * D.lora_rank + 7) / 8, 256, 0, s>>>((const uint16_t *)Y.lora_Ad, C->ap, K.T, D.d_ff,

@@ -377,6 +377,7 @@ struct Plan {
   int32_t *uexp;    // [E]
   int32_t *ustart;  // [E + 1]
   int32_t *assign;  // [T * k]  entries t * k + j
+  int32_t *pos;     // [T * k]  grouped position of entry t * k + j (-1: invalid expert), or nullptr
 };
 
 // Counting sort by expert, stable in (token, slot) order: each of the 32 warps owns a
@@ -446,6 +447,9 @@ __global__ void __launch_bounds__(1024) k_plan(const int32_t *__restrict__ idx, 
     if (ok) {
       const int rank = __popc(peers & ((1u << lane) - 1u));
       P.assign[cnt[warp][e] + rank] = a;
+      if (P.pos) P.pos[a] = cnt[warp][e] + rank;
+    } else if (P.pos && a < a1) {
+      P.pos[a] = -1;
     }
     __syncwarp();
     // the lowest lane of each peer group advances its expert's offset

@@ -1135,10 +1135,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_tc_rows(TcRowsArgs A) {
 // ---------------------------------------------------------------------------------------
 // Operand preparation: the K-permuted bf16 copy of x (or nullptr) and the fp32 sum of
 // every group of 64 (natural order).  Eight threads per (row, group), one 16-byte word
-// each (a warp reads four whole groups), the group sum reduced over the eight.
+// each (a warp reads four whole groups), the group sum reduced over the eight.  With `pos`
+// (x rows only), each permuted word also goes to the expert-grouped rows of the row's
+// k assignments (xg row pos[r k + j]), so that each routed expert's tokens are consecutive.
 // ---------------------------------------------------------------------------------------
 __global__ void k_perm_sums(const uint16_t *__restrict__ x, long long rows, int K, uint16_t *__restrict__ xp,
-                            float *__restrict__ sums, int in_f16) {
+                            float *__restrict__ sums, int in_f16, const int32_t *__restrict__ pos, int k,
+                            uint16_t *__restrict__ xg) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int G = K / 64;
   const long long rg = i >> 3;            // (row, group)
@@ -1164,23 +1167,18 @@ __global__ void k_perm_sums(const uint16_t *__restrict__ x, long long rows, int 
     if (xp) {   // bf16 input -> the fp16 tensor-core operand, permuted block (0,4,1,5,2,6,3,7)
       const uint32_t e0 = h16(v.x & 0xFFFFu), e1 = h16(v.x >> 16), e2 = h16(v.y & 0xFFFFu), e3 = h16(v.y >> 16);
       const uint32_t e4 = h16(v.z & 0xFFFFu), e5 = h16(v.z >> 16), e6 = h16(v.w & 0xFFFFu), e7 = h16(v.w >> 16);
-      reinterpret_cast<uint4 *>(xp + r * K + g * 64)[q] =
-          make_uint4(e0 | (e4 << 16), e1 | (e5 << 16), e2 | (e6 << 16), e3 | (e7 << 16));
+      const uint4 pw = make_uint4(e0 | (e4 << 16), e1 | (e5 << 16), e2 | (e6 << 16), e3 | (e7 << 16));
+      reinterpret_cast<uint4 *>(xp + r * K + g * 64)[q] = pw;
+      if (pos)
+        for (int j = 0; j < k; j++) {
+          const int p = pos[r * k + j];
+          if (p >= 0) reinterpret_cast<uint4 *>(xg + (size_t)p * K + g * 64)[q] = pw;
+        }
     }
   }
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (live && q == 0) sums[rg] = s;
-}
-
-// x rows in expert-grouped order: row p of xg = the permuted x row of the token of
-// assignment assign[p] (t * k + slot).  One block per row, one 16-byte chunk per thread.
-__global__ void k_group_rows(const uint16_t *__restrict__ xp, const int32_t *__restrict__ assign, int k, int d,
-                             uint16_t *__restrict__ xg) {
-  const int p = blockIdx.x, t = assign[p] / k;
-  const uint4 *src = reinterpret_cast<const uint4 *>(xp + (size_t)t * d);
-  uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)p * d);
-  for (int i = threadIdx.x; i < d / 8; i += blockDim.x) dst[i] = src[i];
 }
 
 // t_d = Ad a_s from the K-permuted activations (fp16 holding the bf16 values of a; one warp
