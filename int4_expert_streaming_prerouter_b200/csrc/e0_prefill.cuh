@@ -258,7 +258,7 @@ __global__ void k_tc_tiles(Plan P, int T, TcTile *tiles, int *ntiles, int cap) {
 // scale and min of the row's group g, q in 0..15) and q = (q & 14) + (q & 1):
 //   sum_k w_k x_k = sum_k s (q_k & 14) x_k + sum_k s (q_k & 1) x_k + sum_g m_g X_g,
 // X_g = sum_{k in g} x_k.  s (q & 14) = 2 s (q >> 1) has at most 8 + 3 significant bits and
-// s (q & 1) is 0 or s, so both are exact fp16 values (for 2^-15 <= |s| < 64; the pages'
+// s (q & 1) is 0 or s, so both are exact fp16 values (for 2^-13 <= |s| < 64; the pages'
 // scales are ~1e-2), and x (bf16) is an exact fp16 value in its range, so the tensor core
 // forms every product exactly and accumulates in fp32.  The min term is one more K = 64
 // block per unit: A = the row's mins (exact in fp16) twice, B = each column's group sums
@@ -919,18 +919,26 @@ __global__ void __launch_bounds__(kTmThreads, 1) k_moe_gemm_tc(const __grid_cons
           }
           const uint32_t sh = S.sc[slot][g0 + lg][row];
           const uint32_t s2 = sh | (sh << 16);
-          const uint32_t c2 = tm_hfma2(s2, 0xE400E400u, 0u);   // -1024 s, exact
+          const uint32_t c2 = tm_hfma2(s2, 0xE400E400u, 0u);    // -1024 s, exact
+          const uint32_t s16 = tm_hfma2(s2, 0x2C002C00u, 0u);   // s / 16, exact for |s| >= 2^-13
+          const uint32_t c16 = tm_hfma2(s2, 0xD400D400u, 0u);   // -64 s, exact
           // word j holds K elements 8 j .. 8 j + 7; nibbles n and n + 4 form the fp16 pair
-          // of TMEM column 4 j + n (the K-permuted order of the activation operand):
-          // 1024 + (q & 14) and 1024 + (q & 1) as fp16, then (1024 + v) s - 1024 s = v s
+          // of TMEM column 4 j + n (the K-permuted order of the activation operand).  A
+          // nibble in bits 0-3 of its half gives 1024 + (q & 14) and 1024 + (q & 1) as fp16,
+          // then (1024 + v) s - 1024 s = v s; one in bits 4-7 is masked in place, giving
+          // 1024 + 16 v, then (1024 + 16 v)(s / 16) - 64 s = v s (one rounding, exact as
+          // before); nibbles 2 and 3 are those of the word shifted right by 8
           const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int j = 0; j < 4; j++) {
 #pragma unroll
-            for (int n = 0; n < 4; n++) {
-              const uint32_t sv = ws[j] >> (4 * n);
+            for (int hb = 0; hb < 2; hb++) {
+              const uint32_t sv = hb ? ws[j] >> 8 : ws[j];
+              const int n = 2 * hb;
               p1[4 * j + n] = tm_hfma2((sv & 0x000E000Eu) | 0x64006400u, s2, c2);
               p2[4 * j + n] = tm_hfma2((sv & 0x00010001u) | 0x64006400u, s2, c2);
+              p1[4 * j + n + 1] = tm_hfma2((sv & 0x00E000E0u) | 0x64006400u, s16, c16);
+              p2[4 * j + n + 1] = tm_hfma2((sv & 0x00100010u) | 0x64006400u, s16, c16);
             }
           }
           if (!(ok = put(p1, p2, true, (g0 + lg) & 1))) break;
