@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(256) k_ph_route(PhParams P) {
 // g in pair order.  The warps' partial sums are added in order.  The shared expert's g and
 // u go out before its LoRA and activation, which the next kernel applies.
 // ---------------------------------------------------------------------------------------
-constexpr int kPhGuBlocks = 4;   // blocks of 8 intermediate indices per gate/up CTA
+constexpr int kPhGuBlocks = 8;   // blocks of 8 intermediate indices per gate/up CTA
 template <int D, int I>
 __global__ void __launch_bounds__(32 * (D / 256)) k_ph_gateup(PhParams P) {
   constexpr int NG = D / 64, NW = NG / 4, O = I / 8, OC = O / kPhGuBlocks;
