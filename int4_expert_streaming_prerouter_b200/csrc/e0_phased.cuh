@@ -46,7 +46,7 @@ constexpr int kPhMaxB = 8;                       // tokens per pass of the kerne
 constexpr int kPhGroups = 8;                     // passes per step: up to 64 streams
 constexpr int kPhMaxU = kPhMaxB * kMaxK + 1;     // distinct routed experts + the shared one
 constexpr int kPhMaxH = 512;                     // full-head hidden width on this path
-constexpr int kPhBatch = 5;                      // experts whose down rows a warp loads at once
+constexpr int kPhBatch = 3;                      // experts whose down rows a warp loads at once
 constexpr int kPlanInts = 1 + kPhMaxU;           // U, then the expert list
 
 struct PhLayer {
