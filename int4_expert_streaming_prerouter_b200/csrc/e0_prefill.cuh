@@ -6,13 +6,15 @@
 //             the shared expert adds c * B (A x) to g and u first;
 //   down:     Y_e = Dq(W_d) A_e^T, y[t] += w_{t,j} Y_e[:, t]  (w = 1 for the shared expert).
 //
-// B200 design.  The int4 codes are expanded exactly into bf16 128 + q (one mask and one OR
-// per two weights) and each K group of 64 is one tensor-core accumulation; the affine
-// dequantisation is folded once per group and output on the CUDA cores.  The expanded
-// weights go from registers straight into tensor memory, the A operand of tcgen05.mma, so
-// shared memory carries only raw codes and activation tiles, both by TMA.  Persistent
-// warp-specialised CTAs overlap code/activation loads, conversion, MMAs, folds and the
-// epilogues of consecutive work units (details at k_moe_gemm_tc).
+// B200 design.  Each int4 weight s q + m enters the tensor core as two exact fp16 parts,
+// s (q & 14) and s (q & 1), formed by half-precision FMAs on the masked code bits, so every
+// product with the (fp16-held) bf16 activations is exact and accumulates in fp32 with no
+// per-group fold; the min term and the shared expert's LoRA up branch are extra K blocks
+// of the same accumulation.  The expanded weights go from registers straight into tensor
+// memory, the A operand of tcgen05.mma, so shared memory carries only raw codes and
+// activation tiles, both by TMA.  Persistent warp-specialised CTAs overlap code/activation
+// loads, conversion, MMAs and the epilogues of consecutive work units (details at
+// k_moe_gemm_tc).
 #pragma once
 #include <cuda.h>
 #include <cuda_fp16.h>
