@@ -51,7 +51,8 @@ enum {
   E0_ERR_STAGING = -4,       /* an expert copy into the HBM pool could not be issued */
   E0_ERR_SLOT_MISMATCH = -5, /* a kernel found a pool slot holding another expert */
   E0_ERR_TIMEOUT = -6,       /* a bounded device-side wait gave up */
-  E0_ERR_DEVICE = -7         /* a kernel rejected its data (index out of range, duplicate) */
+  E0_ERR_DEVICE = -7         /* a kernel rejected its data (index out of range, duplicate,
+                                an activation beyond the one-launch decode's fp16 operand range) */
 };
 
 typedef struct e0_ctx e0_ctx;

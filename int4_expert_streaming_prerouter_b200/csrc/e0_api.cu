@@ -1709,6 +1709,9 @@ extern "C" int e0_sync_status(e0_ctx *C) {
   if (err & (DERR_INDEX | DERR_DUP))
     return fail(E0_ERR_DEVICE, "routing rejected on the device (%s)",
                 (err & DERR_INDEX) ? "expert index out of range" : "duplicate expert in a token");
+  if (err & kDerrRange)
+    return fail(E0_ERR_DEVICE, "one-launch decode: an activation beyond the fp16 operand range (|v| >= 65520); "
+                               "e0_debug_force_general(ctx, 1) runs such steps on the per-layer kernels");
   return E0_OK;
 }
 

@@ -16,8 +16,8 @@
 //     known a whole token ahead, the producer runs ahead of the data dependencies and keeps
 //     HBM busy while the consumers wait for other CTAs.
 //   * Consumers (11 warps) compute the int4 dot products on the tensor cores as row pairs
-//     that share one activation vector (mma.sync m16n8k16 bf16 with the codes expanded to
-//     128 + q and the group scale/min folded per group of 64), the SwiGLU, the LoRA branch
+//     that share one activation vector (mma.sync m16n8k16 fp16 with the codes masked in
+//     place as fp16 subnormals and the group scale/min folded per group of 64), the SwiGLU, the LoRA branch
 //     and the weighted combine.
 //   * CTAs exchange results (a, y, LoRA intermediates, logits) through global memory as
 //     64-bit words {32-bit tag, payload} written with one relaxed store; a reader polls the
@@ -83,6 +83,10 @@ struct DecodeParams {
   const unsigned long long *sched;  // [G][kMaxItems] item lists (pack_item), built on the host
   const int *sched_n;               // [G] items per CTA
 };
+
+// Error bit of this kernel alone (beside the DERR_ bits): an activation outside the range of
+// the fp16 tensor-core operand; the step's outputs are then not valid.
+constexpr int kDerrRange = 16;
 
 // Timeline stamps of the optional trace (one row of 16 per CTA and layer).
 enum : int {
@@ -168,17 +172,20 @@ __host__ __device__ __forceinline__ void split_range(int N, int G, int c, int &a
 // A warp takes two rows r0, r1 that share the activation vector v and walks their K in
 // steps of 512 (eight groups of 64).  In a step, lane (g, t) (g = lane / 4, t = lane % 4)
 // holds code words 8 g + 2 t and 8 g + 2 t + 1 of the step of both rows (16 codes of
-// group g each).  Word nibbles n0..n7 (elements 8 w .. 8 w + 7) become the bf16 pairs
-// {128 + n_j, 128 + n_(j+4)}, j = 0..3, exact, with one mask and one OR each.  In the
-// m16n8k16 MMA, row g is r0 restricted to group g, row g + 8 is r1 restricted to group g,
-// and column g is v restricted to group g, paired in the same element order, so the
-// diagonal entries D[g][g] and D[g + 8][g] are P = sum (128 + q) v over group g of r0 and
-// of r1 (the other entries are not used).  Four MMAs cover a step.  The lane that holds
-// the diagonal (t = g / 2) folds the group's affine weights w = s q + m into its partial
-// sum as s P + (m - 128 s) V, V = sum v over the group; a warp sum finishes each row.
+// group g each).  Word nibbles n0..n7 (elements 8 w .. 8 w + 7) become the fp16 pairs
+// {n_j, n_(j+4)}, j = 0..3, masked in place (subnormals q 2^-24 for even j, q 2^-20 for
+// odd j; one shift per word brings j = 2, 3 down), exact.  In the m16n8k16 MMA, row g is
+// r0 restricted to group g, row g + 8 is r1 restricted to group g, and column g is v
+// restricted to group g, paired in the same element order, with v's odd elements held
+// as v / 16, so the diagonal entries D[g][g] and D[g + 8][g] are P = 2^-24 sum q v over
+// group g of r0 and of r1 (the other entries are not used).  Four MMAs cover a step.  The
+// lane that holds the diagonal (t = g / 2) folds the group's affine weights w = s q + m
+// into its partial sum as s 2^24 P + m V, V = sum v over the group; a warp sum finishes
+// each row.
 //
-// v lives in shared memory as bf16 pairs in the same order: word w of v is the uint4
-// {v0|v4, v1|v5, v2|v6, v3|v7} of elements 8 w .. 8 w + 7 (low half first).
+// v lives in shared memory as fp16 pairs in the same order: word w of v is the uint4
+// {v0|v4, v1|v5, v2|v6, v3|v7} of elements 8 w .. 8 w + 7 (low half first), odd elements
+// divided by 16 (act_f16).
 // ---------------------------------------------------------------------------------------
 __host__ __device__ __forceinline__ int pair_index(int e) {   // uint16 index of element e
   return (e >> 3) * 8 + (e & 3) * 2 + ((e >> 2) & 1);
@@ -193,6 +200,18 @@ __device__ __forceinline__ int pair_slot(int e, int N) {
   const int n = min(64, N / 8 - 64 * s);
   return ((64 * s + (wl & 1) * (n >> 1) + (wl >> 1)) << 3) + (e & 3) * 2 + ((e >> 2) & 1);
 }
+// Code word w (elements 8 w .. 8 w + 7, element 8 w + j in bits 4 j .. 4 j + 3) -> the four
+// fp16 operand pairs {j, j + 4}, masked in place: a nibble pair at bits 0-3 / 16-19 reads as
+// the fp16 subnormals q 2^-24, one at bits 4-7 / 20-23 as q 2^-20, both exact.  Five integer
+// instructions per word, no offset to remove afterwards.
+__device__ __forceinline__ void nib_f16(uint32_t w, uint32_t &e0, uint32_t &e1, uint32_t &e2, uint32_t &e3) {
+  const uint32_t h = w >> 8;
+  e0 = w & 0x000F000Fu;   // elements 0, 4: q 2^-24
+  e1 = w & 0x00F000F0u;   // elements 1, 5: q 2^-20
+  e2 = h & 0x000F000Fu;   // elements 2, 6: q 2^-24
+  e3 = h & 0x00F000F0u;   // elements 3, 7: q 2^-20
+}
+// bf16 form (the phased kernels): word nibbles j, j + 4 -> the exact bf16 pair {128 + q_j, 128 + q_(j+4)}
 __device__ __forceinline__ uint32_t nib_pair_bf16(uint32_t w, int j) {
   return ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
 }
@@ -203,18 +222,36 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// The fp16 operand of activation element e (v a bf16 value): v for even e, v / 16 for odd e,
+// so that with the codes above every product is q v 2^-24.  Exact for 2^-13 <= |v| < 65520
+// (even e) or 16 * 65520 (odd e); below 2^-13 fp16 keeps v to 2^-20 absolute.  `bad` is set
+// when a finite v overflows.
+__device__ __forceinline__ uint16_t act_f16(float v, int e, bool &bad) {
+  const uint16_t b = __half_as_ushort(__float2half_rn((e & 1) ? v * 0.0625f : v));
+  bad |= (b & 0x7FFFu) == 0x7C00u && fabsf(v) <= 3.0e38f;
+  return b;
+}
 // one 512-wide step: c0, c1 the two code words of rows r0, r1; va, vb the activation
-// words 8 g + 2 t and 8 g + 2 t + 1 of the step
+// words 8 g + 2 t and 8 g + 2 t + 1 of the step (fp16 operands as act_f16 forms them);
+// the diagonal entries come out as 2^-24 sum q v over the lane's group
 __device__ __forceinline__ void pair_step(float (&d)[4], uint2 c0, uint2 c1, uint4 va, uint4 vb) {
   d[0] = d[1] = d[2] = d[3] = 0.f;
-  mma_bf16_16816(d, nib_pair_bf16(c0.x, 0), nib_pair_bf16(c1.x, 0), nib_pair_bf16(c0.x, 1), nib_pair_bf16(c1.x, 1),
-                 va.x, va.y);
-  mma_bf16_16816(d, nib_pair_bf16(c0.x, 2), nib_pair_bf16(c1.x, 2), nib_pair_bf16(c0.x, 3), nib_pair_bf16(c1.x, 3),
-                 va.z, va.w);
-  mma_bf16_16816(d, nib_pair_bf16(c0.y, 0), nib_pair_bf16(c1.y, 0), nib_pair_bf16(c0.y, 1), nib_pair_bf16(c1.y, 1),
-                 vb.x, vb.y);
-  mma_bf16_16816(d, nib_pair_bf16(c0.y, 2), nib_pair_bf16(c1.y, 2), nib_pair_bf16(c0.y, 3), nib_pair_bf16(c1.y, 3),
-                 vb.z, vb.w);
+  uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+  nib_f16(c0.x, a0, a1, a2, a3);
+  nib_f16(c1.x, b0, b1, b2, b3);
+  mma_f16_16816(d, a0, b0, a1, b1, va.x, va.y);
+  mma_f16_16816(d, a2, b2, a3, b3, va.z, va.w);
+  nib_f16(c0.y, a0, a1, a2, a3);
+  nib_f16(c1.y, b0, b1, b2, b3);
+  mma_f16_16816(d, a0, b0, a1, b1, vb.x, vb.y);
+  mma_f16_16816(d, a2, b2, a3, b3, vb.z, vb.w);
 }
 // Sums over the warp of four per-lane values at once (a transposing butterfly, six
 // shuffles): lanes 0-7 return the sum of v0, lanes 8-15 of v1, 16-23 of v2, 24-31 of v3.
@@ -231,10 +268,9 @@ __device__ __forceinline__ float warp_sum4(float v0, float v1, float v2, float v
   c += __shfl_xor_sync(0xffffffffu, c, 1);
   return c;
 }
-// the diagonal lane's affine fold of group G of one row: s P + (m - 128 s) V
+// the diagonal lane's affine fold of group G of one row: s 2^24 P + m V (P = 2^-24 sum q v)
 __device__ __forceinline__ float group_fold(float P, const uint16_t *sc, const uint16_t *mn, int G, float V) {
-  const float s = bf(sc[G]);
-  return fmaf(s, P, fmaf(-128.f, s, bf(mn[G])) * V);
+  return fmaf(bf(sc[G]) * 16777216.f, P, bf(mn[G]) * V);
 }
 __device__ __forceinline__ uint2 ld_code2(const uint8_t *p) { return *reinterpret_cast<const uint2 *>(p); }
 
@@ -949,6 +985,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
   Ctl C{P.timeout_ns, P.err, &S.abort};
   int q = 0;
   bool ab = false;
+  bool range_bad = false;   // an activation outside the fp16 operand range (act_f16)
 
   if (c == P.stall_cta) {
     // test hook: wait for a word that is never written, so that the timeout path runs
@@ -1042,14 +1079,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         if (i < D && !ab) {
           const uint16_t xb = d2bf_bits(hv[m] * (double)bf(gam[i]) * rinv);
           S.xn[i] = xb;
-          S.xp[pair_slot(i, D)] = xb;
+          S.xp[pair_slot(i, D)] = act_f16(bf(xb), i, range_bad);
         }
       }
       cbar();
       // the group sums that every gate/up row of the layer uses with its minima
       #pragma unroll 1
       for (int G = warp; G < D / 64 && !ab; G += kDecCW) {
-        const float v = warp_sum(bf(S.xp[pair_slot(64 * G + lane, D)]) + bf(S.xp[pair_slot(64 * G + 32 + lane, D)]));
+        const float v = warp_sum(bf(S.xn[64 * G + lane]) + bf(S.xn[64 * G + 32 + lane]));
         if (lane == 0) S.xg[G] = v;
       }
       cbar();
@@ -1204,7 +1241,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
 #pragma unroll 1
           for (int i = ct; i < k * I; i += kDecConsumers) {
             const int j = i / I, e = i - j * I;
-            S.ap[j * I + pair_slot(e, I)] = (uint16_t)(S.stg[i] & 0xFFFFu);
+            S.ap[j * I + pair_slot(e, I)] = act_f16(bf(S.stg[i] & 0xFFFFu), e, range_bad);
           }
           if (ct == 0) stamp(P, l, TR_A_POLL);
           const int sbd = dn_bd(k);
@@ -1234,7 +1271,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
             }
             const uint16_t a16 = f2bf(g / (1.0f + expf(-g)) * u);
             S.asraw[i] = bf(a16);
-            S.ap[k * I + pair_slot(i, I)] = a16;
+            S.ap[k * I + pair_slot(i, I)] = act_f16(bf(a16), i, range_bad);
           }
           if (ct == 0) {
             float lg[kMaxK], mx = -INFINITY, sum = 0.f;
@@ -1256,8 +1293,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         // the group sums that every down row of the layer uses with its minima
         #pragma unroll 1
         for (int G = warp; G < (k + 1) * NGI && !ab; G += kDecCW) {
-          const float v = warp_sum(bf(S.ap[(G / NGI) * I + pair_slot((G % NGI) * 64 + lane, I)]) +
-                                   bf(S.ap[(G / NGI) * I + pair_slot((G % NGI) * 64 + 32 + lane, I)]));
+          // from the natural-order values: the routed slots' bf16 payloads, then a_s
+          const int j = G / NGI, e0 = (G % NGI) * 64 + lane;
+          const float v = warp_sum(j < k ? bf(S.stg[j * I + e0] & 0xFFFFu) + bf(S.stg[j * I + e0 + 32] & 0xFFFFu)
+                                         : S.asraw[e0] + S.asraw[e0 + 32]);
           if (lane == 0) S.ag[G] = v;
         }
         if (!ab && lora) {
@@ -1356,6 +1395,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty[slot]);
   }
+  if (range_bad) atomicOr(P.err, kDerrRange);
   ab = cbar_or(ab);
   if (ab) return;
   // ---- end of step: CTA c records layer c's routing and runs layer c's head top-k; every

@@ -208,6 +208,28 @@ def test_one_launch_decode_bounded_wait_reports_timeout(cuda_ok):
     ctx.close()
 
 
+def test_one_launch_decode_reports_activations_beyond_fp16(cuda_ok):
+    """The one-launch kernel holds activations as fp16 tensor-core operands: a finite
+    activation beyond that range latches a device error instead of a silent infinity, and
+    once the input is back in range the context decodes correctly again."""
+    import int4_expert_streaming_prerouter_b200 as e0
+    ctx, lys, _ = build(SMALL, 95, 4)
+    ctx.debug_decode_mode(1)
+    gamma = lys[1]["norm_w"]
+    saved = gamma.clone()
+    gamma.fill_(2.0e5)     # |x| = |RMSNorm(h)| * 2e5 reaches well past 65520 (finite in bf16)
+    h = bf16_tensor(synth.hidden(95, 0, SMALL.L, 1, SMALL.d), "cuda")
+    ctx.stack_decode(h, 0)
+    with pytest.raises(e0.E0Error) as ei:
+        ctx.sync_status()
+    assert ei.value.status == "DEVICE"
+    gamma.copy_(saved)
+    gpu = run_steps(ctx, SMALL, 95, 1, 2)
+    ref = oracle_steps(SMALL, 95, 1, 2, gpu[2], gpu[3])
+    compare_steps(SMALL, gpu, ref)
+    ctx.close()
+
+
 @pytest.mark.parametrize("B", [1, 5])
 def test_graph_replay_decode_matches_oracle(cuda_ok, B):
     """The decode step replayed as a captured CUDA graph of the per-layer kernels."""
