@@ -44,8 +44,8 @@ METRIC = "MoE-stack decode tokens/s on 1 B200; achieved HBM GB/s vs ~8 TB/s peak
 KERNEL_TRAFFIC = {
     "decode_b1_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_decode.cuh",
                        "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",
-                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "2dc2a9d34f7c17a6", 408.7e6,
-                      "4-layer capture (40.87 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
+                       "int4_expert_streaming_prerouter_b200/csrc/e0_device.cuh"), "5c7d623b5c947fb3", 408.6e6,
+                      "4-layer capture (40.86 MB DRAM per launch for 40.67 MB algorithmic) scaled by algorithmic "
                       "bytes to the 40-layer launch"),
     "prefill_t4096_l40": (("int4_expert_streaming_prerouter_b200/csrc/e0_prefill.cuh",
                            "int4_expert_streaming_prerouter_b200/csrc/e0_kernels.cuh",

@@ -1147,7 +1147,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
       if (ct == 0) stamp(P, l, TR_GU_FULL);
       constexpr int NG = D / 64, NS = (NG + 7) / 8;   // groups per row, 512-wide steps
       const int g8 = lane >> 2, t4 = lane & 3;
-      const bool own = t4 == (g8 >> 1);               // this lane holds the diagonal
+      // Rotated columns: in step st the B column n carries the activation of group
+      // pg(n) = 2 (((n >> 1) - st) & 3) + (n & 1) of the step (parity kept, so the loads
+      // stay free of bank conflicts), which puts row g's diagonal in lane (g, t) exactly
+      // when st % 4 == sown = (t - g / 2) % 4: every lane holds one useful gate and one
+      // useful up sum per four steps and folds them once, instead of every lane folding
+      // every step for the eight lanes that hold a diagonal.
+      const int sown = (t4 - (g8 >> 1)) & 3;
       const int slot0 = ia / I;
       // unit u = global unit ia + u: slot es = (ia + u) / I, index i = (ia + u) % I; its
       // piece p is the slot's order among the item's slots, its row the index minus the
@@ -1183,35 +1189,47 @@ __global__ void __launch_bounds__(kDecThreads, 1) k_decode(DecodeParams P) {
         const int u1 = u0 + kDecCW;
         const bool two = u1 < in;                      // warp-uniform
         const UnitRows A = unit_rows(u0), B = unit_rows(two ? u1 : u0);
-        float ag0 = 0.f, au0 = 0.f, ag1 = 0.f, au1 = 0.f;
+        float ag0 = 0.f, au0 = 0.f, ag1 = 0.f, au1 = 0.f;   // folded sums
+        float kg0 = 0.f, ku0 = 0.f, kg1 = 0.f, ku1 = 0.f;   // this lane's diagonal of the chunk
 #pragma unroll
         for (int st = 0; st < NS; st++) {
           // every lane takes part in the MMAs; lanes past the row's last group (rows
-          // shorter than a step) feed zeros and fold nothing
-          const int G = 8 * st + g8;
-          const bool gv = G < NG;
+          // shorter than a step) feed zeros, and so do column lanes past it
+          const bool gv = 8 * st + g8 < NG;
+          const int pg = 2 * (((g8 >> 1) - st) & 3) + (g8 & 1);   // group of this lane's B column
+          const bool bv = 8 * st + pg < NG;
           const int wi = 64 * st + 8 * g8 + 2 * t4;  // code word of this lane (natural order)
           const int nw = min(64, D / 8 - 64 * st);   // activation words of this step
           const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
           const uint2 z2 = make_uint2(0u, 0u);
-          const uint4 va = gv ? xw[64 * st + lane] : z4, vb = gv ? xw[64 * st + nw / 2 + lane] : z4;
-          const float V = gv ? S.xg[G] : 0.f;
+          const uint4 va = bv ? xw[64 * st + 4 * pg + t4] : z4, vb = bv ? xw[64 * st + nw / 2 + 4 * pg + t4] : z4;
+          const bool mine = (st & 3) == sown;
           float d[4];
           pair_step(d, gv ? ld_code2(A.gc + 4 * wi) : z2, gv ? ld_code2(A.uc + 4 * wi) : z2, va, vb);
-          if (gv) {
-            ag0 += group_fold((g8 & 1) ? d[1] : d[0], A.gs, A.gm, G, V);
-            au0 += group_fold((g8 & 1) ? d[3] : d[2], A.us, A.um, G, V);
-          }
+          kg0 = mine ? ((g8 & 1) ? d[1] : d[0]) : kg0;
+          ku0 = mine ? ((g8 & 1) ? d[3] : d[2]) : ku0;
           if (two) {
             pair_step(d, gv ? ld_code2(B.gc + 4 * wi) : z2, gv ? ld_code2(B.uc + 4 * wi) : z2, va, vb);
-            if (gv) {
-              ag1 += group_fold((g8 & 1) ? d[1] : d[0], B.gs, B.gm, G, V);
-              au1 += group_fold((g8 & 1) ? d[3] : d[2], B.us, B.um, G, V);
+            kg1 = mine ? ((g8 & 1) ? d[1] : d[0]) : kg1;
+            ku1 = mine ? ((g8 & 1) ? d[3] : d[2]) : ku1;
+          }
+          if ((st & 3) == 3 || st == NS - 1) {
+            // end of a chunk of four steps: fold this lane's group of the chunk
+            const int G = 8 * ((st & ~3) + sown) + g8;
+            if (G < NG) {
+              const float V = S.xg[G];
+              ag0 += group_fold(kg0, A.gs, A.gm, G, V);
+              au0 += group_fold(ku0, A.us, A.um, G, V);
+              if (two) {
+                ag1 += group_fold(kg1, B.gs, B.gm, G, V);
+                au1 += group_fold(ku1, B.us, B.um, G, V);
+              }
             }
+            kg0 = ku0 = kg1 = ku1 = 0.f;
           }
         }
         // the four row sums at once: lane 0 gets u0's gate and up sums, lane 16 u1's
-        const float v = warp_sum4(own ? ag0 : 0.f, own ? au0 : 0.f, own ? ag1 : 0.f, own ? au1 : 0.f, lane);
+        const float v = warp_sum4(ag0, au0, ag1, au1, lane);
         const float vu = __shfl_down_sync(0xffffffffu, v, 8);
         if (lane == 0) publish(u0, v, vu);
         if (lane == 16 && two) publish(u1, v, vu);
