@@ -181,7 +181,8 @@ __host__ __device__ __forceinline__ void split_range(int N, int G, int c, int &a
 // group g of r0 and of r1 (the other entries are not used).  Four MMAs cover a step.  The
 // lane that holds the diagonal (t = g / 2) folds the group's affine weights w = s q + m
 // into its partial sum as s 2^24 P + m V, V = sum v over the group; a warp sum finishes
-// each row.
+// each row.  (The gate/up loop rotates the column groups from step to step so that the
+// diagonals, and with them the folds, spread over all four lanes of a group row.)
 //
 // v lives in shared memory as fp16 pairs in the same order: word w of v is the uint4
 // {v0|v4, v1|v5, v2|v6, v3|v7} of elements 8 w .. 8 w + 7 (low half first), odd elements
