@@ -179,7 +179,11 @@ int e0_stage_experts(e0_ctx *ctx, int layer, const int32_t *host_idx, int n, voi
  * routing into the context.  step == 0 starts a new sequence.  streaming = 1 serves the
  * routed experts from the pool (e0_stream_register), 0 from the resident weights.
  * chained = 1 feeds bf16(h_N + y_{N-1}) to layer N (a dependency check); 0 feeds h_N.
- * Errors: INVALID_ARG, STAGING, CUDA; DEVICE/SLOT_MISMATCH are latched. */
+ * Errors: INVALID_ARG, STAGING, CUDA; DEVICE/SLOT_MISMATCH are latched.  The one-launch
+ * kernel (B = 1, resident experts) holds activations as fp16 tensor-core operands: a
+ * finite activation at or beyond 65520 in magnitude latches DEVICE and the step's
+ * outputs are not valid (e0_debug_force_general takes such models through the per-layer
+ * kernels). */
 int e0_moe_stack_decode(e0_ctx *ctx, const void *h_in, int B, int step, void *y_out, float *y_f32,
                         int streaming, int chained, void *stream);
 
